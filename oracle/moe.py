@@ -1,0 +1,289 @@
+"""Routing, permutation, grouped expert MLP (forward and backward) — fp64 oracle.
+
+Test infrastructure only (see the package docstring). Pages and sections followed:
+
+* routing and combine — "Efficient MoE training for biological foundation models"
+  (sitech.ge, introduction and section "Grouped experts instead of a Python loop"):
+  each token is sent to a few experts and their outputs are weighted by the routing
+  weights, which the fused GroupedMLP kernel applies itself;
+* grouping — same section, and news.bpdata.com section 1): tokens are grouped per
+  expert and the grouped GEMM takes per-expert token counts (``split_sizes``); the
+  result equals running every expert in a loop. "NeMo AutoModel" (seventnews.com,
+  section on Transformers v5 expert back-ends): ``grouped_mm`` runs on tokens sorted by
+  expert;
+* fused chain — news.bpdata.com section 3): GroupedLinear -> ScaledSwiGLU ->
+  GroupedLinear; sitech.ge section "Reducing memory and quantisation cost": the
+  backward pass has a fused counterpart.
+
+Readings where the pages are silent:
+  * router input is fp32 logits [T, E]; softmax over all E experts; the k experts with
+    the largest logits are selected (ties -> lower expert index), slot j holds the
+    j-th largest; with ``renorm`` the k selected probabilities are divided by their sum;
+  * permutation is a stable counting sort of the T*k slots (flat slot s = t*k + j) by
+    expert: ``row_map[s]`` is the slot's row in the expert-contiguous order, rows of one
+    expert keep ascending slot order; ``split_sizes[e]`` counts them, ``offsets`` is
+    their exclusive prefix sum (length E+1);
+  * w1[e] is [H, 2F] with gate columns [0, F) and up columns [F, 2F); w2[e] is [F, H];
+  * ScaledSwiGLU: a = SiLU(gate) * up * p with SiLU(z) = z / (1 + exp(-z)) and p the
+    slot's routing probability; the probability is applied there only, so the combine
+    that follows sums the k expert outputs with weight 1;
+  * the BF16 path stores ``a`` in bf16 (round to nearest even) before fc2; the oracle
+    reproduces that rounding when ``a_round="bf16"``; everything else stays fp64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import mxfp8
+
+
+# ----------------------------------------------------------------------------- helpers
+def round_to_bf16(v) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value, ties to even (fp64 result)."""
+    v = np.asarray(v, dtype=np.float64)
+    _, ex = np.frexp(v)                             # |v| in [2**(ex-1), 2**ex)
+    q = np.ldexp(1.0, np.maximum(ex.astype(np.int64) - 8, -133))   # bf16 spacing
+    return np.where(v == 0.0, v, np.rint(v / q) * q)
+
+
+def silu(z):
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def silu_grad(z):
+    """d/dz SiLU(z) = s(z) * (1 + z * (1 - s(z))) with s the logistic sigmoid."""
+    z = np.asarray(z, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def f64(t) -> np.ndarray:
+    """Any CPU tensor or array as float64 numpy."""
+    if hasattr(t, "detach"):
+        import torch
+        return t.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------- routing
+def route(logits, k: int, renorm: bool = True):
+    """Top-k router softmax. Returns idx int32 [T, k] and prob float64 [T, k]."""
+    lg = f64(logits)
+    T, E = lg.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    m = lg.max(axis=1, keepdims=True)
+    ex = np.exp(lg - m)
+    soft = ex / ex.sum(axis=1, keepdims=True)
+    # stable sort of the negated logits: largest first, equal logits keep index order
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+    prob = np.take_along_axis(soft, order, axis=1)
+    if renorm:
+        prob = prob / prob.sum(axis=1, keepdims=True)
+    return order.astype(np.int32), prob
+
+
+# ------------------------------------------------------------------------- permutation
+def permute_index(idx, E: int):
+    """Stable counting sort of the flat slots by expert.
+
+    Returns row_map int32 [T*k], split_sizes int32 [E], offsets int32 [E+1].
+    """
+    flat = np.asarray(idx, dtype=np.int64).reshape(-1)
+    if flat.size and (flat.min() < 0 or flat.max() >= E):
+        raise ValueError("expert index out of range")
+    split_sizes = np.bincount(flat, minlength=E).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(split_sizes)])
+    order = np.argsort(flat, kind="stable")          # slots in expert-contiguous order
+    row_map = np.empty(flat.size, dtype=np.int64)
+    row_map[order] = np.arange(flat.size)
+    return row_map.astype(np.int32), split_sizes.astype(np.int32), offsets.astype(np.int32)
+
+
+def permute_rows(x, row_map, k: int) -> np.ndarray:
+    """xp[row_map[t*k + j]] = x[t] (works on any dtype; rows are copied unchanged)."""
+    x = np.asarray(x)
+    row_map = np.asarray(row_map, dtype=np.int64)
+    R = row_map.size
+    xp = np.empty((R,) + x.shape[1:], dtype=x.dtype)
+    xp[row_map] = np.repeat(x, k, axis=0)
+    return xp
+
+
+def permute_probs(prob, row_map) -> np.ndarray:
+    pp = np.empty(np.asarray(row_map).size, dtype=np.float64)
+    pp[np.asarray(row_map, dtype=np.int64)] = f64(prob).reshape(-1)
+    return pp
+
+
+def unpermute(yp, row_map, T: int, k: int, prob=None) -> np.ndarray:
+    """out[t] = sum_j w_tj * yp[row_map[t*k + j]], w = 1 unless ``prob`` is given."""
+    yp = f64(yp)
+    rm = np.asarray(row_map, dtype=np.int64).reshape(T, k)
+    out = np.zeros((T,) + yp.shape[1:], dtype=np.float64)
+    for j in range(k):
+        w = 1.0 if prob is None else f64(prob)[:, j][:, None]
+        out += w * yp[rm[:, j]]
+    return out
+
+
+# -------------------------------------------------------------------- expert MLP (fwd)
+def _round_a(a, a_round):
+    if a_round is None or a_round == "f64":
+        return a
+    if a_round == "bf16":
+        return round_to_bf16(a)
+    if a_round == "mxfp8":
+        codes, scales = mxfp8.quantize_blocks_last_axis(a)
+        return mxfp8.dequantize_blocks_last_axis(codes, scales)
+    raise ValueError(a_round)
+
+
+def moe_forward_per_token(x, idx, prob, w1, w2, a_round="bf16", tokens=None) -> np.ndarray:
+    """Definition of the layer, one token at a time, no permutation.
+
+    out[t] = sum_j ( SiLU(x_t W1g_e) * (x_t W1u_e) * p_tj ) W2_e, with e = idx[t, j].
+    ``tokens`` restricts the computation to those token indices (rows of the result
+    follow that order).
+    """
+    x = f64(x)
+    idx = np.asarray(idx, dtype=np.int64)
+    prob = f64(prob)
+    w1 = f64(w1) if not isinstance(w1, list) else w1
+    w2 = f64(w2) if not isinstance(w2, list) else w2
+    F = w2[0].shape[0]
+    toks = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    out = np.zeros((toks.size, x.shape[1]), dtype=np.float64)
+    for n, t in enumerate(toks):
+        for j in range(idx.shape[1]):
+            e = idx[t, j]
+            h = x[t] @ w1[e]
+            a = silu(h[:F]) * h[F:] * prob[t, j]
+            out[n] += _round_a(a, a_round) @ w2[e]
+    return out
+
+
+def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm, a_round="bf16"):
+    """The per-expert loop over expert-contiguous rows (grouped GEMM semantics).
+
+    Returns (yp [R,H], h [R,2F], a [R,F]) in float64; ``a`` carries the path rounding.
+    """
+    xp = f64(xp)
+    w1 = f64(w1)
+    w2 = f64(w2)
+    pp = f64(probs_perm)
+    R, H = xp.shape
+    F = w2.shape[1]
+    yp = np.zeros((R, w2.shape[2]), dtype=np.float64)
+    hh = np.zeros((R, 2 * F), dtype=np.float64)
+    aa = np.zeros((R, F), dtype=np.float64)
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        h = xp[rows] @ w1[e]
+        a = _round_a(silu(h[:, :F]) * h[:, F:] * pp[rows, None], a_round)
+        yp[rows] = a @ w2[e]
+        hh[rows] = h
+        aa[rows] = a
+        start += n
+    if start != R:
+        raise ValueError("split_sizes must sum to the number of rows")
+    return yp, hh, aa
+
+
+def grouped_mlp_bwd(dy_perm, xp, split_sizes, w1, w2, probs_perm, a_round="bf16"):
+    """Analytic gradient of :func:`grouped_mlp_fwd` with respect to xp, w1, w2, probs_perm.
+
+    Per expert e (rows of the group, a = SiLU(g) * u * p):
+        da = dy W2_e^T;  dg = da * p * u * SiLU'(g);  du = da * p * SiLU(g);
+        dp = sum_f da * SiLU(g) * u;  dW2_e = a^T dy;  dxp = [dg|du] W1_e^T;
+        dW1_e = xp^T [dg|du].
+    Returns (dxp [R,H], dw1 [E,H,2F], dw2 [E,F,H], dprobs_perm [R], dh [R,2F]).
+    """
+    dy = f64(dy_perm)
+    xp = f64(xp)
+    w1 = f64(w1)
+    w2 = f64(w2)
+    pp = f64(probs_perm)
+    R, H = xp.shape
+    E, F = w2.shape[0], w2.shape[1]
+    dxp = np.zeros_like(xp)
+    dw1 = np.zeros_like(w1)
+    dw2 = np.zeros_like(w2)
+    dpp = np.zeros(R, dtype=np.float64)
+    dhh = np.zeros((R, 2 * F), dtype=np.float64)
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        h = xp[rows] @ w1[e]
+        g, u = h[:, :F], h[:, F:]
+        p = pp[rows, None]
+        a = _round_a(silu(g) * u * p, a_round)
+        da = dy[rows] @ w2[e].T
+        dg = da * p * u * silu_grad(g)
+        du = da * p * silu(g)
+        dpp[rows] = np.sum(da * silu(g) * u, axis=1)
+        dh = np.concatenate([dg, du], axis=1)
+        dw2[e] = a.T @ dy[rows]
+        dxp[rows] = dh @ w1[e].T
+        dw1[e] = xp[rows].T @ dh
+        dhh[rows] = dh
+        start += n
+    return dxp, dw1, dw2, dpp, dhh
+
+
+def moe_backward_tokens(dx_perm, dprobs_perm, row_map, T: int, k: int):
+    """dx[t] = sum_j dxp[row_map[t*k+j]];  dprob[t, j] = dprobs_perm[row_map[t*k+j]]."""
+    dx = unpermute(dx_perm, row_map, T, k)
+    dprob = f64(dprobs_perm)[np.asarray(row_map, dtype=np.int64)].reshape(T, k)
+    return dx, dprob
+
+
+# ------------------------------------------------------------------ MXFP8 expert MLP
+def quantize_weights_kmajor(w, along: str):
+    """MXFP8 codes of stacked expert weights, transposed so the contraction axis is last.
+
+    ``w1`` [E, H, 2F] quantised along H gives codes [E, 2F, H] (``along="rows"``);
+    the same call serves w2 [E, F, H] along F, giving [E, H, F].
+    """
+    if along != "rows":
+        raise ValueError(along)
+    return mxfp8.quantize(f64(w), axis=1, transpose_out=True)
+
+
+def grouped_mlp_fwd_mxfp8(xp_codes, xp_scales, split_sizes, w1_codes, w1_scales, w2_codes,
+                          w2_scales, probs_perm, a_codes=None, a_scales=None):
+    """MXFP8 forward on quantised operands, computed in float64.
+
+    xp codes [R,H] / scales [R,H/32] (blocks along H); w1 codes [E,2F,H] / scales
+    [E,2F,H/32]; w2 codes [E,H,F] / scales [E,H,F/32]. The fc1 epilogue output
+    a = SiLU(g)*u*p is quantised along F with the same rule, unless ``a_codes`` /
+    ``a_scales`` (an externally produced quantised ``a``) are given, in which case fc2
+    runs on those. Returns (yp [R,H], a_codes, a_scales, h [R,2F]).
+    """
+    xq = mxfp8.dequantize_blocks_last_axis(xp_codes, xp_scales)
+    w1q = mxfp8.dequantize_blocks_last_axis(w1_codes, w1_scales)     # [E, 2F, H]
+    w2q = mxfp8.dequantize_blocks_last_axis(w2_codes, w2_scales)     # [E, H, F]
+    pp = f64(probs_perm)
+    R = xq.shape[0]
+    E, H, F = w2q.shape
+    h_all = np.zeros((R, 2 * F))
+    a_all = np.zeros((R, F))
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        h = xq[rows] @ w1q[e].T
+        h_all[rows] = h
+        a_all[rows] = silu(h[:, :F]) * h[:, F:] * pp[rows, None]
+        start += n
+    if a_codes is None:
+        a_codes, a_scales = mxfp8.quantize_blocks_last_axis(a_all)
+    aq = mxfp8.dequantize_blocks_last_axis(a_codes, a_scales)
+    yp = np.zeros((R, H))
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        yp[rows] = aq[rows] @ w2q[e].T
+        start += n
+    return yp, a_codes, a_scales, h_all

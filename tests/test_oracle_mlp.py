@@ -1,0 +1,166 @@
+"""Pins of the oracle's grouped expert MLP (forward and backward)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe, mxfp8
+
+
+def _layer(T, H, F, E, k, seed=0, empty=()):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(T, H))
+    lg = rng.normal(size=(T, E))
+    for e in empty:
+        lg[:, e] -= 100.0
+    w1 = rng.normal(0, 0.3, size=(E, H, 2 * F))
+    w2 = rng.normal(0, 0.3, size=(E, F, H))
+    idx, prob = moe.route(lg, k)
+    return x, idx, prob, w1, w2
+
+
+def _grouped_layer(x, idx, prob, w1, w2, a_round):
+    T, k = idx.shape
+    E = w1.shape[0]
+    row_map, split, _ = moe.permute_index(idx, E)
+    xp = moe.permute_rows(x, row_map, k)
+    pp = moe.permute_probs(prob, row_map)
+    yp, _, _ = moe.grouped_mlp_fwd(xp, split, w1, w2, pp, a_round)
+    return moe.unpermute(yp, row_map, T, k)
+
+
+@pytest.mark.parametrize("a_round", ["f64", "bf16"])
+@pytest.mark.parametrize("T,H,F,E,k,empty", [(16, 8, 6, 4, 2, (1,)), (40, 12, 8, 6, 3, (0, 5)),
+                                             (9, 4, 3, 1, 1, ())])
+def test_per_token_definition_equals_grouped_loop(T, H, F, E, k, empty, a_round):
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=T, empty=empty)
+    ref = moe.moe_forward_per_token(x, idx, prob, w1, w2, a_round)
+    got = _grouped_layer(x, idx, prob, w1, w2, a_round)
+    assert np.max(np.abs(got - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def _pure_python_layer(x, idx, prob, w1, w2):
+    """Brute force with scalar loops only (no numpy linear algebra)."""
+    T, H = x.shape
+    F = w2.shape[1]
+    out = [[0.0] * H for _ in range(T)]
+    for t in range(T):
+        for j in range(idx.shape[1]):
+            e = int(idx[t, j])
+            h = [sum(float(x[t, i]) * float(w1[e, i, c]) for i in range(H)) for c in range(2 * F)]
+            a = [h[f] / (1.0 + math.exp(-h[f])) * h[F + f] * float(prob[t, j]) for f in range(F)]
+            for o in range(H):
+                out[t][o] += sum(a[f] * float(w2[e, f, o]) for f in range(F))
+    return np.array(out)
+
+
+def test_brute_force_tiny_with_empty_expert():
+    x, idx, prob, w1, w2 = _layer(8, 5, 4, 4, 2, seed=3, empty=(2,))
+    assert not np.any(idx == 2)
+    ref = _pure_python_layer(x, idx, prob, w1, w2)
+    got = _grouped_layer(x, idx, prob, w1, w2, "f64")
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_single_expert_reduces_to_dense_swiglu_mlp():
+    # E=1, k=1: p = 1 and the layer is the textbook SwiGLU MLP, checked with torch fp64
+    x, idx, prob, w1, w2 = _layer(32, 16, 12, 1, 1, seed=9)
+    assert np.all(prob == 1.0)
+    xt, w1t, w2t = (torch.from_numpy(a) for a in (x, w1[0], w2[0]))
+    ref = (torch.nn.functional.silu(xt @ w1t[:, :12]) * (xt @ w1t[:, 12:])) @ w2t
+    got = _grouped_layer(x, idx, prob, w1, w2, "f64")
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_round_to_bf16_matches_torch_cast():
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.normal(size=5000), rng.normal(size=5000) * 1e-30,
+                        rng.normal(size=5000) * 1e20, [0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]])
+    v32 = v.astype(np.float32)
+    ref = torch.from_numpy(v32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(moe.round_to_bf16(v32.astype(np.float64)), ref)
+
+
+def _torch_layer_grads(x, idx, prob, w1, w2, dy):
+    """Autograd of the per-expert loop written with torch fp64 ops."""
+    T, k = idx.shape
+    E, F = w2.shape[0], w2.shape[1]
+    row_map, split, _ = moe.permute_index(idx, E)
+    xp = torch.tensor(moe.permute_rows(x, row_map, k), requires_grad=True)
+    pp = torch.tensor(moe.permute_probs(prob, row_map), requires_grad=True)
+    w1t = torch.tensor(w1, requires_grad=True)
+    w2t = torch.tensor(w2, requires_grad=True)
+    outs = []
+    s = 0
+    for e, n in enumerate(split):
+        h = xp[s:s + n] @ w1t[e]
+        a = torch.nn.functional.silu(h[:, :F]) * h[:, F:] * pp[s:s + n, None]
+        outs.append(a @ w2t[e])
+        s += n
+    yp = torch.cat(outs)
+    dyp = torch.tensor(moe.permute_rows(dy, row_map, k))
+    (yp * dyp).sum().backward()
+    return xp.grad.numpy(), w1t.grad.numpy(), w2t.grad.numpy(), pp.grad.numpy(), split, dyp.numpy(), \
+        xp.detach().numpy(), pp.detach().numpy(), row_map
+
+
+@pytest.mark.parametrize("T,H,F,E,k", [(12, 6, 4, 3, 2), (30, 8, 8, 5, 3)])
+def test_backward_matches_torch_autograd(T, H, F, E, k):
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=T + 1, empty=(E - 1,))
+    dy = np.random.default_rng(4).normal(size=(T, H))
+    gx, gw1, gw2, gp, split, dyp, xp, pp, row_map = _torch_layer_grads(x, idx, prob, w1, w2, dy)
+    dxp, dw1, dw2, dpp, _ = moe.grouped_mlp_bwd(dyp, xp, split, w1, w2, pp, a_round="f64")
+    for got, ref in ((dxp, gx), (dw1, gw1), (dw2, gw2), (dpp, gp)):
+        np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+    assert np.all(dw1[E - 1] == 0) and np.all(dw2[E - 1] == 0)    # empty expert: zero grads
+    dx, dprob = moe.moe_backward_tokens(dxp, dpp, row_map, T, k)
+    assert dx.shape == (T, H) and dprob.shape == (T, k)
+
+
+def test_backward_matches_finite_differences():
+    T, H, F, E, k = 6, 4, 3, 2, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=21)
+    row_map, split, _ = moe.permute_index(idx, E)
+    xp = moe.permute_rows(x, row_map, k)
+    pp = moe.permute_probs(prob, row_map)
+    dy = np.random.default_rng(8).normal(size=xp.shape)
+
+    def loss(xp_, w1_, w2_, pp_):
+        yp, _, _ = moe.grouped_mlp_fwd(xp_, split, w1_, w2_, pp_, a_round="f64")
+        return float(np.sum(yp * dy))
+
+    dxp, dw1, dw2, dpp, _ = moe.grouped_mlp_bwd(dy, xp, split, w1, w2, pp, a_round="f64")
+    eps = 1e-6
+    for arr, grad, at in ((xp, dxp, (3, 2)), (w1, dw1, (1, 2, 5)), (w2, dw2, (0, 1, 3)), (pp, dpp, (4,))):
+        args = [xp, w1, w2, pp]
+        pos = [a is arr for a in args].index(True)
+        plus = [a.copy() for a in args]
+        minus = [a.copy() for a in args]
+        plus[pos][at] += eps
+        minus[pos][at] -= eps
+        fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+        assert abs(fd - grad[at]) <= 1e-7 * max(1.0, abs(fd))
+
+
+def test_mxfp8_grouped_equals_per_token_on_quantised_operands():
+    T, H, F, E, k = 24, 64, 64, 3, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=31)
+    xc, xs = mxfp8.quantize(x, axis=0)
+    w1c, w1s = moe.quantize_weights_kmajor(w1, "rows")           # [E, 2F, H]
+    w2c, w2s = moe.quantize_weights_kmajor(w2, "rows")           # [E, H, F]
+    row_map, split, _ = moe.permute_index(idx, E)
+    xpc = moe.permute_rows(xc, row_map, k)
+    xps = moe.permute_rows(xs, row_map, k)
+    pp = moe.permute_probs(prob, row_map)
+    yp, ac, asc, _ = moe.grouped_mlp_fwd_mxfp8(xpc, xps, split, w1c, w1s, w2c, w2s, pp)
+    got = moe.unpermute(yp, row_map, T, k)
+    # definition (per token) on the dequantised operands with `a` rounded to MXFP8
+    xq = mxfp8.dequantize(xc, xs, axis=0)
+    w1q = np.swapaxes(mxfp8.dequantize_blocks_last_axis(w1c, w1s), 1, 2)
+    w2q = np.swapaxes(mxfp8.dequantize_blocks_last_axis(w2c, w2s), 1, 2)
+    ref = moe.moe_forward_per_token(xq, idx, prob, w1q, w2q, a_round="mxfp8")
+    assert np.max(np.abs(got - ref)) <= 1e-12 * np.max(np.abs(ref))
+    # feeding the layer's own quantised `a` back in reproduces the same output
+    yp2, _, _, _ = moe.grouped_mlp_fwd_mxfp8(xpc, xps, split, w1c, w1s, w2c, w2s, pp, ac, asc)
+    assert np.array_equal(yp, yp2)
