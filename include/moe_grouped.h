@@ -1,0 +1,205 @@
+/*
+ * moe_grouped.h — C ABI of the B200 (sm_100a) MoE expert-MLP hot path.
+ *
+ * The path: top-k router softmax -> stable permutation of tokens into expert-contiguous
+ * rows with per-expert counts (split_sizes) -> grouped GEMM fc1 (gate|up) with the
+ * ScaledSwiGLU epilogue (SiLU(gate) * up * routing probability) -> grouped GEMM fc2 ->
+ * unpermute and combine of the k expert outputs of every token; plus the backward
+ * dgrad/wgrad grouped GEMMs, and an MXFP8 variant (E4M3 values, one E8M0 scale per 32
+ * consecutive values along K).
+ *
+ * Pages: "Efficient MoE training for biological foundation models" — sitech.ge,
+ * sections "Grouped experts instead of a Python loop" and "Reducing memory and
+ * quantisation cost"; news.bpdata.com, sections 1) to 3).
+ *
+ * Conventions shared by every call:
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller allocates and
+ *     owns every buffer. The library never allocates device memory in these calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every call only enqueues work on it and returns; nothing synchronises the host.
+ *   - bf16 tensors are passed as uint16_t* (raw bfloat16 bits); all tensors are dense
+ *     row-major with the logical shapes given below.
+ *   - Return value: a moe_status_t. Argument errors are reported synchronously before
+ *     anything is launched. Errors found by kernels (bad expert index, split sizes that
+ *     do not add up, a wait that ran out of time) set a device error word that
+ *     moe_device_status() reads. CUDA launch errors return MOE_ERR_CUDA.
+ *   - Sizes: T tokens, E experts (1..1024), k experts per token (1..min(E,32)),
+ *     H hidden size, F expert FFN size, R = T*k routed rows.
+ */
+#ifndef MOE_GROUPED_H
+#define MOE_GROUPED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, k > E, workspace too small */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but unsupported shape (e.g. H % 256 != 0) */
+  MOE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_CHECK = 4,  /* a kernel detected bad data (see moe_device_status) */
+  MOE_ERR_TIMEOUT = 5        /* a kernel wait exceeded its time budget */
+} moe_status_t;
+
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_precision_t;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
+MOE_API int moe_device_status(void* stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+MOE_API uint64_t moe_launch_count(void);
+
+/*
+ * moe_route — top-k router softmax.
+ * Pages: sitech.ge introduction and news.bpdata.com "dense vs MoE": every token is sent
+ * to a few experts whose outputs are weighted by routing weights.
+ * Computes, per token t, the softmax of logits[t, :] over all E experts (fp32), selects
+ * the k largest logits (equal logits: lower expert index first) in descending order and
+ * writes their experts and probabilities; with renorm != 0 the k probabilities are
+ * divided by their sum.
+ *   logits [T, E] fp32 (input); idx [T, k] int32 (output); prob [T, k] fp32 (output).
+ */
+MOE_API int moe_route(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* prob, void* stream);
+
+/* Bytes of device scratch moe_permute needs (per-block expert histograms). */
+MOE_API size_t moe_permute_workspace_size(int T, int k, int E);
+
+/*
+ * moe_permute — stable permutation of the T*k routed slots into expert-contiguous rows.
+ * Pages: sitech.ge "Grouped experts instead of a Python loop" and news.bpdata.com
+ * section 1): tokens are grouped per expert and the grouped GEMM receives the per-expert
+ * token counts (split_sizes); NeMo AutoModel page, Transformers v5 back-ends: grouped_mm
+ * runs on tokens sorted by expert.
+ * Slot s = t*k + j (token t, choice j). Within an expert, rows keep ascending slot order.
+ *   x [T, H] bf16 (input); idx [T, k] int32 (input, values in [0, E));
+ *   prob [T, k] fp32 (input, may be NULL when probs_perm is NULL);
+ *   precision MOE_BF16: xp [R, H] bf16, xp_scale ignored (may be NULL);
+ *   precision MOE_MXFP8: xp [R, H] E4M3 codes (uint8), xp_scale [R, H/32] E8M0 codes,
+ *     each row quantised along H in blocks of 32 (H % 32 == 0);
+ *   row_map [R] int32 (output): row of slot s in xp;
+ *   probs_perm [R] fp32 (output, may be NULL): probs_perm[row_map[s]] = prob[s];
+ *   split_sizes [E] int32 (output); offsets [E+1] int32 (output, exclusive prefix sum);
+ *   workspace: device scratch of at least moe_permute_workspace_size(T, k, E) bytes.
+ * Requires H % 8 == 0 (bf16) or H % 32 == 0 (MXFP8). An index outside [0, E) sets
+ * MOE_ERR_DEVICE_CHECK in the device error word and its slot gets row_map = -1.
+ */
+MOE_API int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
+                int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                int32_t* split_sizes, int32_t* offsets, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_permute_rows — the data movement of moe_permute alone, for a tensor that follows
+ * an existing row_map (e.g. the gradient of the layer output in the backward pass):
+ * dst[row_map[t*k + j]] = src[t]. src [T, H] bf16, dst [R, H] bf16, H % 8 == 0.
+ */
+MOE_API int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, int k, uint16_t* dst, void* stream);
+
+/*
+ * moe_unpermute — combine of the k expert outputs of every token.
+ * Pages: sitech.ge "Grouped experts instead of a Python loop": the routing weights are
+ * applied inside the GroupedMLP kernel, so the combine adds the k rows with weight 1;
+ * pass `prob` to weight them here instead (when the MLP ran without probabilities).
+ *   out[t] = sum_{j<k} w_tj * yp[row_map[t*k + j]], w = prob[t, j] or 1 if prob == NULL,
+ *   accumulated in fp32 in slot order and rounded once to bf16.
+ *   yp [R, H] bf16; row_map [R]; prob [T, k] fp32 or NULL; out [T, H] bf16. H % 8 == 0.
+ */
+MOE_API int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const float* prob, int T, int H, int k,
+                  uint16_t* out, void* stream);
+
+/*
+ * mxfp8_quantize — MXFP8 quantisation of a batch of bf16 matrices in[batch, rows, cols].
+ * Pages: news.bpdata.com section 2) and sitech.ge "Reducing memory and quantisation
+ * cost": one scale per block of 32 consecutive values; 16-bit masters are quantised
+ * every step (section 3).
+ * Per block of 32 values with amax = max|v|: scale X = 2^(floor(log2 amax) - 8) stored
+ * as E8M0 (exponent clamped to [-127, 127]; amax == 0 gives code 0); elements are
+ * v / X rounded to nearest-even E4M3, saturating at +-448.
+ *   axis 0: blocks along cols (cols % 32 == 0): codes [batch, rows, cols],
+ *           scales [batch, rows, cols/32]; transpose_out must be 0.
+ *   axis 1: blocks along rows (rows % 32 == 0).
+ *           transpose_out = 1: codes [batch, cols, rows], scales [batch, cols, rows/32]
+ *             (the transposed matrix quantised along its rows: K-major weights);
+ *           transpose_out = 0: codes [batch, rows, cols], scales [batch, rows/32, cols].
+ */
+MOE_API int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out,
+                   uint8_t* codes, uint8_t* scales, void* stream);
+
+/* Bytes of scratch grouped_mlp_fwd needs (the fc1 output `a` when saved == NULL). */
+MOE_API size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int training);
+
+/* Bytes of the buffer grouped_mlp_fwd fills for the backward pass (training mode):
+ * h = [gate | up] pre-activations [R, 2F] bf16, then a [R, F] bf16. */
+MOE_API size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision);
+
+/*
+ * grouped_mlp_fwd — fc1 (gate|up) -> ScaledSwiGLU -> fc2 over expert-contiguous rows.
+ * Pages: news.bpdata.com section 1) (grouped GEMM with split_sizes, equal to the
+ * per-expert loop) and section 3) (GroupedLinear -> ScaledSwiGLU -> GroupedLinear fused
+ * into one pattern); sitech.ge "Grouped experts instead of a Python loop" (routing
+ * weights applied inside the GroupedMLP kernel).
+ * For every expert e with rows [off_e, off_e + split_sizes[e]):
+ *   h = xp_e @ w1[e]            (K = H, N = 2F; gate = h[:, :F], up = h[:, F:])
+ *   a = SiLU(gate) * up * p     (p = probs_perm of the row, 1 if probs_perm == NULL)
+ *   yp_e = a @ w2[e]            (K = F, N = H)
+ * MOE_BF16: xp [R, H] bf16, w1 [E, H, 2F] bf16, w2 [E, F, H] bf16; scales ignored;
+ *   a is rounded to bf16 before fc2; fp32 accumulation.
+ * MOE_MXFP8: xp [R, H] E4M3 + xp_scale [R, H/32]; w1 [E, 2F, H] E4M3 + w1_scale
+ *   [E, 2F, H/32]; w2 [E, H, F] E4M3 + w2_scale [E, H, F/32] (weights as produced by
+ *   mxfp8_quantize(axis=1, transpose_out=1)); the fc1 epilogue quantises a along F.
+ * split_sizes [E] int32 on the device (no host synchronisation happens); R = sum.
+ * yp [R, H] bf16 output. saved: NULL for inference, else a buffer of
+ * grouped_mlp_saved_size() bytes that receives h and a for grouped_mlp_bwd.
+ * ws: scratch of grouped_mlp_workspace_size() bytes.
+ * Requires H % 64 == 0 and F % 128 == 0.
+ */
+MOE_API int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
+                    const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                    const float* probs_perm, int precision, uint16_t* yp, void* saved, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* Bytes of scratch grouped_mlp_bwd needs (dh [R, 2F] bf16 and dprob partial sums). */
+MOE_API size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision);
+
+/*
+ * grouped_mlp_bwd — backward of grouped_mlp_fwd (the "counterpart in the backward
+ * pass" of sitech.ge "Reducing memory and quantisation cost").
+ * For every expert e (a = SiLU(g) * u * p, with g, u, a from `saved`):
+ *   da = dy_e @ w2[e]^T;  dg = da*p*u*SiLU'(g);  du = da*p*SiLU(g);
+ *   dprobs_perm = sum_f da*SiLU(g)*u;  dw2[e] = a_e^T @ dy_e;
+ *   dxp_e = [dg | du] @ w1[e]^T;  dw1[e] = xp_e^T @ [dg | du].
+ * dy_perm [R, H] bf16 (the layer-output gradient permuted with moe_permute_rows);
+ * xp [R, H] bf16; w1 [E, H, 2F] bf16; w2 [E, F, H] bf16; probs_perm [R] fp32 or NULL;
+ * saved: the buffer filled by grouped_mlp_fwd in training mode.
+ * Outputs: dxp [R, H] bf16, dw1 [E, H, 2F] bf16, dw2 [E, F, H] bf16 (experts with no rows
+ * get zeros), dprobs_perm [R] fp32 (may be NULL). Only MOE_BF16 is supported.
+ */
+MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
+                    const void* w1, const void* w2, const float* probs_perm, int precision, const void* saved,
+                    uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * moe_gather_slots — dst[s] = src[row_map[s]] for s < R (fp32): brings per-row values
+ * (e.g. dprobs_perm) back to token/slot order [T, k].
+ */
+MOE_API int moe_gather_slots(const float* src, const int32_t* row_map, int R, float* dst, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_GROUPED_H */

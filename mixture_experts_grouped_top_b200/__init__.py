@@ -1,0 +1,229 @@
+"""B200 (sm_100a) MoE expert-MLP hot path: Python binding of the C ABI in include/moe_grouped.h.
+
+Every function here only marshals arguments (torch CUDA tensors -> device pointers and
+the current CUDA stream) and calls the function of the same name in libmoe_grouped.so;
+all computation runs in the library's CUDA kernels. Output and scratch buffers are
+allocated here with torch when the caller does not pass them (the library itself never
+allocates). There is no CPU fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+BF16 = 0
+MXFP8 = 1
+_PREC = {"bf16": BF16, "mxfp8": MXFP8, BF16: BF16, MXFP8: MXFP8}
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+          4: "MOE_ERR_DEVICE_CHECK", 5: "MOE_ERR_TIMEOUT"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+def lib():
+    return _lib.load()
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(name: str, rc: int):
+    if rc != 0:
+        raise MoEError(name, rc)
+
+
+def _need(t, dtype, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------------ status helpers
+def moe_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return lib().moe_device_status(_stream(stream))
+
+
+def moe_launch_count() -> int:
+    return int(lib().moe_launch_count())
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+# ------------------------------------------------------------------------ routing
+def moe_route(logits, k: int, renorm: bool = True, idx=None, prob=None, stream=None):
+    _need(logits, torch.float32, "logits")
+    T, E = logits.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device) if idx is None else idx
+    prob = torch.empty((T, k), dtype=torch.float32, device=logits.device) if prob is None else prob
+    _check("moe_route", lib().moe_route(_p(logits), T, E, k, int(bool(renorm)), _p(idx), _p(prob), _stream(stream)))
+    return idx, prob
+
+
+def moe_permute_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_permute_workspace_size(T, k, E))
+
+
+def moe_permute(x, idx, prob, E: int, precision="bf16", out=None, workspace=None, stream=None):
+    """Permute tokens into expert-contiguous rows. Returns a dict with xp, xp_scale
+    (MXFP8 only), row_map, probs_perm (None when prob is None), split_sizes, offsets."""
+    _need(x, torch.bfloat16, "x")
+    _need(idx, torch.int32, "idx")
+    prec = _PREC[precision]
+    T, H = x.shape
+    k = idx.shape[1]
+    R = T * k
+    dev = x.device
+    o = dict(out or {})
+    if "xp" not in o:
+        o["xp"] = torch.empty((R, H), dtype=torch.bfloat16 if prec == BF16 else torch.uint8, device=dev)
+    if prec == MXFP8 and "xp_scale" not in o:
+        o["xp_scale"] = torch.empty((R, H // 32), dtype=torch.uint8, device=dev)
+    o.setdefault("row_map", torch.empty(R, dtype=torch.int32, device=dev))
+    if prob is not None:
+        o.setdefault("probs_perm", torch.empty(R, dtype=torch.float32, device=dev))
+    o.setdefault("split_sizes", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    ws_bytes = moe_permute_workspace_size(T, k, E)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    rc = lib().moe_permute(_p(x), _p(idx), _p(prob), T, H, E, k, prec, _p(o["xp"]), _p(o.get("xp_scale")),
+                           _p(o["row_map"]), _p(o.get("probs_perm")), _p(o["split_sizes"]), _p(o["offsets"]),
+                           _p(workspace), workspace.numel(), _stream(stream))
+    _check("moe_permute", rc)
+    o.setdefault("xp_scale", None)
+    o.setdefault("probs_perm", None)
+    return o
+
+
+def moe_permute_rows(src, row_map, k: int, out=None, stream=None):
+    _need(src, torch.bfloat16, "src")
+    T, H = src.shape
+    out = torch.empty((T * k, H), dtype=torch.bfloat16, device=src.device) if out is None else out
+    _check("moe_permute_rows", lib().moe_permute_rows(_p(src), _p(row_map), T, H, k, _p(out), _stream(stream)))
+    return out
+
+
+def moe_unpermute(yp, row_map, T: int, k: int, prob=None, out=None, stream=None):
+    _need(yp, torch.bfloat16, "yp")
+    H = yp.shape[1]
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=yp.device) if out is None else out
+    _check("moe_unpermute",
+           lib().moe_unpermute(_p(yp), _p(row_map), _p(prob), T, H, k, _p(out), _stream(stream)))
+    return out
+
+
+def moe_gather_slots(src, row_map, out=None, stream=None):
+    R = row_map.numel()
+    out = torch.empty(R, dtype=torch.float32, device=src.device) if out is None else out
+    _check("moe_gather_slots", lib().moe_gather_slots(_p(src), _p(row_map), R, _p(out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------------- MXFP8
+def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, scales=None, stream=None):
+    """Quantise bf16 [batch, rows, cols] (or [rows, cols]). Returns (codes, scales) uint8."""
+    _need(x, torch.bfloat16, "x")
+    squeeze = x.dim() == 2
+    x3 = x.unsqueeze(0) if squeeze else x
+    B, rows, cols = x3.shape
+    dev = x.device
+    if axis == 0:
+        cshape, sshape = (B, rows, cols), (B, rows, cols // 32)
+    elif transpose_out:
+        cshape, sshape = (B, cols, rows), (B, cols, rows // 32)
+    else:
+        cshape, sshape = (B, rows, cols), (B, rows // 32, cols)
+    codes = torch.empty(cshape, dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty(sshape, dtype=torch.uint8, device=dev) if scales is None else scales
+    rc = lib().mxfp8_quantize(_p(x3), B, rows, cols, axis, int(bool(transpose_out)), _p(codes), _p(scales),
+                              _stream(stream))
+    _check("mxfp8_quantize", rc)
+    if squeeze:
+        return codes.reshape(cshape[1:]), scales.reshape(sshape[1:])
+    return codes, scales
+
+
+# ------------------------------------------------------------- grouped expert MLP
+def grouped_mlp_workspace_size(E, R, H, F, precision="bf16", training=False) -> int:
+    return int(lib().grouped_mlp_workspace_size(E, R, H, F, _PREC[precision], int(bool(training))))
+
+
+def grouped_mlp_saved_size(E, R, H, F, precision="bf16") -> int:
+    return int(lib().grouped_mlp_saved_size(E, R, H, F, _PREC[precision]))
+
+
+def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm=None, precision="bf16", xp_scale=None, w1_scale=None,
+                    w2_scale=None, yp=None, saved=None, training=False, workspace=None, F=None, stream=None):
+    """fc1 (gate|up) -> ScaledSwiGLU -> fc2 over expert-contiguous rows.
+
+    BF16: w1 [E, H, 2F], w2 [E, F, H] bf16. MXFP8: xp/w1/w2 are E4M3 codes with scales
+    (w1 [E, 2F, H], w2 [E, H, F]). Returns (yp, saved); ``saved`` is None unless
+    ``training`` (or a saved buffer is passed).
+    """
+    prec = _PREC[precision]
+    R, H = xp.shape
+    E = split_sizes.numel()
+    if F is None:
+        F = w2.shape[1] if prec == BF16 else w2.shape[2]
+    dev = xp.device
+    yp = torch.empty((R, H), dtype=torch.bfloat16, device=dev) if yp is None else yp
+    if training and saved is None:
+        saved = torch.empty(grouped_mlp_saved_size(E, R, H, F, precision), dtype=torch.uint8, device=dev)
+    ws_bytes = grouped_mlp_workspace_size(E, R, H, F, precision, saved is not None)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    rc = lib().grouped_mlp_fwd(_p(xp), _p(xp_scale), _p(split_sizes), E, R, H, F, _p(w1), _p(w1_scale), _p(w2),
+                               _p(w2_scale), _p(probs_perm), prec, _p(yp), _p(saved), _p(workspace),
+                               workspace.numel(), _stream(stream))
+    _check("grouped_mlp_fwd", rc)
+    return yp, saved
+
+
+def grouped_mlp_bwd_workspace_size(E, R, H, F, precision="bf16") -> int:
+    return int(lib().grouped_mlp_bwd_workspace_size(E, R, H, F, _PREC[precision]))
+
+
+def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precision="bf16", dxp=None, dw1=None,
+                    dw2=None, dprobs_perm=None, workspace=None, stream=None):
+    """Backward of grouped_mlp_fwd. Returns (dxp, dw1, dw2, dprobs_perm)."""
+    prec = _PREC[precision]
+    R, H = dy_perm.shape
+    E = split_sizes.numel()
+    F = w2.shape[1]
+    dev = dy_perm.device
+    dxp = torch.empty((R, H), dtype=torch.bfloat16, device=dev) if dxp is None else dxp
+    dw1 = torch.empty((E, H, 2 * F), dtype=torch.bfloat16, device=dev) if dw1 is None else dw1
+    dw2 = torch.empty((E, F, H), dtype=torch.bfloat16, device=dev) if dw2 is None else dw2
+    if dprobs_perm is None and probs_perm is not None:
+        dprobs_perm = torch.empty(R, dtype=torch.float32, device=dev)
+    ws_bytes = grouped_mlp_bwd_workspace_size(E, R, H, F, precision)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    rc = lib().grouped_mlp_bwd(_p(dy_perm), _p(split_sizes), E, R, H, F, _p(xp), _p(w1), _p(w2), _p(probs_perm),
+                               prec, _p(saved), _p(dxp), _p(dw1), _p(dw2), _p(dprobs_perm), _p(workspace),
+                               workspace.numel(), _stream(stream))
+    _check("grouped_mlp_bwd", rc)
+    return dxp, dw1, dw2, dprobs_perm
+
+
+from .layer import MoEExpertLayer, moe_layer_forward  # noqa: E402,F401

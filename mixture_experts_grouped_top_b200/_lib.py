@@ -1,0 +1,57 @@
+"""ctypes loader for libmoe_grouped.so and the argument/return types of every C entry point."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_grouped.so")
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/moe_grouped.h
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_device_status": (_i, [_vp]),
+    "moe_launch_count": (ctypes.c_uint64, []),
+    "moe_route": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_permute_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_rows": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_unpermute": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "mxfp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "grouped_mlp_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "grouped_mlp_saved_size": (_sz, [_i, _i, _i, _i, _i]),
+    "grouped_mlp_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "grouped_mlp_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "grouped_mlp_bwd": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                             _vp]),
+    "moe_gather_slots": (_i, [_vp, _vp, _i, _vp, _vp]),
+}
+
+_lock = threading.Lock()
+_handle = None
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+def load() -> ctypes.CDLL:
+    """Load the CUDA library (once). Raises LibraryMissing if it has not been built."""
+    global _handle
+    with _lock:
+        if _handle is not None:
+            return _handle
+        if not os.path.exists(LIB_PATH):
+            raise LibraryMissing(
+                f"{LIB_PATH} is not built; run `python -m mixture_experts_grouped_top_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _handle = h
+        return h

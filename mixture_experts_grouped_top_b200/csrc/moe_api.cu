@@ -1,0 +1,456 @@
+// Host side of the C ABI declared in include/moe_grouped.h: argument validation,
+// tensor-map construction, launch configuration and the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_grouped.h"
+#include "grouped_gemm_sm100.cuh"
+#include "token_kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "moe_grouped: launch failed: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+inline void count_launch(int n = 1) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+struct DeviceProps {
+  int sm_count = 0;
+};
+
+DeviceProps& device_props() {
+  static DeviceProps props[64];
+  static std::once_flag flags[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::call_once(flags[dev], [dev]() {
+    cudaDeviceGetAttribute(&props[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (props[dev].sm_count <= 0) props[dev].sm_count = 148;
+  });
+  return props[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D tiled tensor map with 128-byte swizzle: dims {d0 (contiguous), d1, d2},
+// byte strides of d1 and d2, box {box0, box1, 1}.
+int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (stride1 & 15) || (stride2 & 15)) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fprintf(stderr, "moe_grouped: cuTensorMapEncodeTiled failed (%d)\n", (int)r);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// bf16 matrix [rows, cols] (row-major) as a TMA source. K-major operand: box {64 cols, box_rows}.
+int tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, cols, rows, 1, cols * 2, rows * cols * 2, 64, box_rows);
+}
+// bf16 stacked matrices [batch, rows, cols] as a TMA source with box {64 cols, box_rows}.
+int tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, cols, rows, batch, cols * 2, rows * cols * 2, 64,
+                   box_rows);
+}
+
+template <bool A_MN, bool B_MN, bool KG, int EPI>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+  auto kern = grouped_gemm_bf16_kernel<A_MN, B_MN, KG, EPI>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  const int grid = device_props().sm_count;
+  kern<<<grid, gg::kThreads, gg::kSmemBytes, st>>>(ta, tb, p);
+  count_launch();
+  return launch_status();
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+GemmParams base_params(const int32_t* split_sizes, int E) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.E = E;
+  p.split_sizes = split_sizes;
+  p.timeout_ns = gg::kTimeoutNs;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_device_status(void* stream) {
+  cudaStream_t st = as_stream(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (h) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (h & DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (h) return MOE_ERR_DEVICE_CHECK;
+  return MOE_OK;
+}
+
+int moe_route(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* prob, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!logits || !idx || !prob) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int threads = 256, wpb = threads / 32;
+  const int grid = std::min((T + wpb - 1) / wpb, device_props().sm_count * 16);
+  const int vpl = (E + 31) / 32;
+#define MOE_ROUTE_CASE(V) \
+  case V: route_topk_kernel<V><<<grid, threads, 0, st>>>(logits, T, E, k, renorm, idx, prob); break;
+  switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : vpl <= 8 ? 8 : vpl <= 16 ? 16 : 32) {
+    MOE_ROUTE_CASE(1)
+    MOE_ROUTE_CASE(2)
+    MOE_ROUTE_CASE(4)
+    MOE_ROUTE_CASE(8)
+    MOE_ROUTE_CASE(16)
+    MOE_ROUTE_CASE(32)
+  }
+#undef MOE_ROUTE_CASE
+  count_launch();
+  return launch_status();
+}
+
+size_t moe_permute_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  const size_t R = (size_t)T * k;
+  const size_t nblk = (R + kPermuteChunk - 1) / kPermuteChunk;
+  return align_up(std::max<size_t>(nblk, 1) * E * sizeof(int32_t), 256);
+}
+
+int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, int k, uint16_t* dst, void* stream) {
+  if (T < 0 || H < 8 || (H % 8) || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!src || !row_map || !dst) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int grid = std::min((T + 7) / 8, device_props().sm_count * 8);
+  permute_rows_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(src), T, H / 8, k, row_map,
+                                                 reinterpret_cast<uint4*>(dst));
+  count_launch();
+  return launch_status();
+}
+
+int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k, int precision,
+                void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm, int32_t* split_sizes,
+                int32_t* offsets, void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32 || H < 8) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_BF16 && (H % 8)) return MOE_ERR_UNSUPPORTED;
+  if (precision == MOE_MXFP8 && (H % 32)) return MOE_ERR_UNSUPPORTED;
+  if (!split_sizes || !offsets) return MOE_ERR_INVALID_ARG;
+  if (probs_perm && !prob) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const long long R = (long long)T * k;
+  if (R > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (!x || !idx || !xp || !row_map || !workspace)) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_MXFP8 && T > 0 && !xp_scale) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe_permute_workspace_size(T, k, E)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 15) return MOE_ERR_INVALID_ARG;
+  if (R == 0) {
+    // no rows: every expert is empty
+    if (cudaMemsetAsync(split_sizes, 0, E * sizeof(int32_t), st) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const int nblk = (int)((R + kPermuteChunk - 1) / kPermuteChunk);
+  int32_t* counts = reinterpret_cast<int32_t*>(workspace);
+  permute_hist_kernel<<<nblk, kPermuteThreads, E * sizeof(int32_t), st>>>(idx, (int)R, E, counts);
+  const int P = std::max(1, 1024 / E);
+  permute_scan_kernel<<<1, 1024, (size_t)(P * E + E) * sizeof(int32_t), st>>>(counts, nblk, E, (int)R, split_sizes,
+                                                                                offsets);
+  static std::once_flag once;
+  std::call_once(once, []() {
+    cudaFuncSetAttribute(permute_rowmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * kMaxExperts * 4);
+  });
+  permute_rowmap_kernel<<<nblk, kPermuteThreads, (size_t)(kPermuteThreads / 32) * E * sizeof(int32_t), st>>>(
+      idx, prob, (int)R, E, counts, row_map, probs_perm);
+  const int grid = std::min((T + 7) / 8, device_props().sm_count * 8);
+  if (precision == MOE_BF16) {
+    permute_rows_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), T, H / 8, k, row_map,
+                                                   reinterpret_cast<uint4*>(xp));
+  } else {
+    permute_rows_mxfp8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), T, H, k, row_map,
+                                                    reinterpret_cast<uint8_t*>(xp), xp_scale);
+  }
+  count_launch(4);
+  return launch_status();
+}
+
+int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const float* prob, int T, int H, int k, uint16_t* out,
+                  void* stream) {
+  if (T < 0 || H < 8 || (H % 8) || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!yp || !row_map || !out) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(yp) | reinterpret_cast<uintptr_t>(out)) & 15) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int grid = std::min((T + 7) / 8, device_props().sm_count * 8);
+  unpermute_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(yp), row_map, prob, T, H / 8, k,
+                                              reinterpret_cast<uint4*>(out));
+  count_launch();
+  return launch_status();
+}
+
+int moe_gather_slots(const float* src, const int32_t* row_map, int R, float* dst, void* stream) {
+  if (R < 0) return MOE_ERR_INVALID_ARG;
+  if (R == 0) return MOE_OK;
+  if (!src || !row_map || !dst) return MOE_ERR_INVALID_ARG;
+  const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
+  gather_slots_f32_kernel<<<grid, 256, 0, as_stream(stream)>>>(src, row_map, R, dst);
+  count_launch();
+  return launch_status();
+}
+
+int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out, uint8_t* codes,
+                   uint8_t* scales, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+  if (axis != 0 && axis != 1) return MOE_ERR_INVALID_ARG;
+  if (axis == 0 && transpose_out) return MOE_ERR_INVALID_ARG;
+  if ((long long)batch * rows * cols == 0) return MOE_OK;
+  if (!in || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (axis == 0) {
+    if (cols % 32) return MOE_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(in) & 15) || (reinterpret_cast<uintptr_t>(codes) & 7))
+      return MOE_ERR_INVALID_ARG;
+    const long long nvec = (long long)batch * rows * cols / 8;
+    const long long want = (nvec + 255) / 256;
+    const int grid = (int)std::min<long long>(want, (long long)device_props().sm_count * 16);
+    quant_rows_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(in), nvec, cols, codes, scales);
+  } else {
+    if (rows % 32) return MOE_ERR_UNSUPPORTED;
+    if (transpose_out && (reinterpret_cast<uintptr_t>(codes) & 15)) return MOE_ERR_INVALID_ARG;
+    if (batch > 65535 || rows / 32 > 65535) return MOE_ERR_UNSUPPORTED;
+    dim3 grid((cols + 255) / 256, rows / 32, batch);
+    quant_cols_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in), rows, cols, transpose_out,
+                                            codes, scales);
+  }
+  count_launch();
+  return launch_status();
+}
+
+size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int training) {
+  (void)E;
+  (void)H;
+  if (R < 0 || F < 0) return 0;
+  if (training) return 256;  // `a` lives in the saved buffer
+  if (precision == MOE_MXFP8) return align_up((size_t)R * F + (size_t)R * (F / 32), 256) + 256;
+  return align_up((size_t)R * F * 2, 256) + 256;
+}
+
+size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision) {
+  (void)E;
+  (void)H;
+  if (R < 0 || F < 0) return 0;
+  if (precision == MOE_MXFP8) return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
+  return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
+}
+
+int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
+                    const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                    const float* probs_perm, int precision, uint16_t* yp, void* saved, void* ws, size_t ws_bytes,
+                    void* stream) {
+  (void)xp_scale;
+  (void)w1_scale;
+  (void)w2_scale;
+  if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  if (precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (R == 0) return MOE_OK;
+  if (!xp || !split_sizes || !w1 || !w2 || !yp || !ws) return MOE_ERR_INVALID_ARG;
+  const int training = saved != nullptr;
+  if (ws_bytes < grouped_mlp_workspace_size(E, R, H, F, precision, training)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+
+  uint16_t* h_buf = nullptr;
+  uint16_t* a_buf = reinterpret_cast<uint16_t*>(ws);
+  if (training) {
+    h_buf = reinterpret_cast<uint16_t*>(saved);
+    a_buf = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256));
+  }
+  CUtensorMap ta, tb;
+  int rc;
+  // fc1: A = xp [R, H] (K-major), B = w1 [E, H, 2F] (N contiguous: MN-major)
+  if ((rc = tmap_bf16_2d(&ta, xp, R, H, gg::BM))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, 64))) return rc;
+  GemmParams p1 = base_params(split_sizes, E);
+  p1.M = R;
+  p1.N = F;
+  p1.K = H;
+  p1.out = a_buf;
+  p1.ldo = F;
+  p1.out2 = h_buf;
+  p1.ldo2 = 2 * F;
+  p1.probs = probs_perm;
+  p1.F = F;
+  if ((rc = launch_gemm<false, true, false, EPI_SWIGLU>(ta, tb, p1, st))) return rc;
+  // fc2: A = a [R, F] (K-major), B = w2 [E, F, H] (MN-major)
+  if ((rc = tmap_bf16_2d(&ta, a_buf, R, F, gg::BM))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, 64))) return rc;
+  GemmParams p2 = base_params(split_sizes, E);
+  p2.M = R;
+  p2.N = H;
+  p2.K = F;
+  p2.out = yp;
+  p2.ldo = H;
+  return launch_gemm<false, true, false, EPI_STORE>(ta, tb, p2, st);
+}
+
+size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision) {
+  (void)E;
+  (void)H;
+  (void)precision;
+  if (R < 0 || F < 0) return 0;
+  const size_t nparts = (size_t)(F + gg::BN - 1) / gg::BN;
+  return align_up((size_t)R * 2 * F * 2, 256) + align_up(nparts * R * 4, 256) + 256;
+}
+
+int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
+                    const void* w1, const void* w2, const float* probs_perm, int precision, const void* saved,
+                    uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws, size_t ws_bytes,
+                    void* stream) {
+  if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
+  if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  if (precision != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!split_sizes || !w1 || !w2 || !dw1 || !dw2) return MOE_ERR_INVALID_ARG;
+  if (R > 0 && (!dy_perm || !xp || !saved || !dxp || !ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < grouped_mlp_bwd_workspace_size(E, R, H, F, precision)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (R == 0) {
+    if (cudaMemsetAsync(dw1, 0, (size_t)E * H * 2 * F * 2, st) != cudaSuccess ||
+        cudaMemsetAsync(dw2, 0, (size_t)E * F * H * 2, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const uint16_t* h_buf = reinterpret_cast<const uint16_t*>(saved);
+  const uint16_t* a_buf =
+      reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256));
+  uint16_t* dh = reinterpret_cast<uint16_t*>(ws);
+  float* dpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + align_up((size_t)R * 2 * F * 2, 256));
+  const int nparts = (F + gg::BN - 1) / gg::BN;
+
+  CUtensorMap ta, tb;
+  int rc;
+  // fc2 dgrad + SwiGLU backward: A = dy [R, H] (K-major), B = w2 [E, F, H] read as [E, N=F, K=H] (K-major)
+  if ((rc = tmap_bf16_2d(&ta, dy_perm, R, H, gg::BM))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, gg::BN))) return rc;
+  GemmParams p = base_params(split_sizes, E);
+  p.M = R;
+  p.N = F;
+  p.K = H;
+  p.out2 = dh;
+  p.ldo2 = 2 * F;
+  p.probs = probs_perm;
+  p.aux = h_buf;
+  p.ld_aux = 2 * F;
+  p.dprob_part = dpart;
+  p.F = F;
+  if ((rc = launch_gemm<false, false, false, EPI_DSWIGLU>(ta, tb, p, st))) return rc;
+  if (dprobs_perm) {
+    const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
+    reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
+    count_launch();
+    if ((rc = launch_status())) return rc;
+  }
+  // fc2 wgrad: dw2[e] = a_e^T dy_e. A = a [R, F] (rows = K, MN-major), B = dy [R, H] (MN-major)
+  if ((rc = tmap_bf16_2d(&ta, a_buf, R, F, 64))) return rc;
+  if ((rc = tmap_bf16_2d(&tb, dy_perm, R, H, 64))) return rc;
+  p = base_params(split_sizes, E);
+  p.M = F;
+  p.N = H;
+  p.out = dw2;
+  p.ldo = H;
+  p.out_batch = (long long)F * H;
+  if ((rc = launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st))) return rc;
+  // fc1 dgrad: dxp = dh w1[e]^T. A = dh [R, 2F] (K-major), B = w1 [E, H, 2F] read as [E, N=H, K=2F] (K-major)
+  if ((rc = tmap_bf16_2d(&ta, dh, R, 2 * F, gg::BM))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, gg::BN))) return rc;
+  p = base_params(split_sizes, E);
+  p.M = R;
+  p.N = H;
+  p.K = 2 * F;
+  p.out = dxp;
+  p.ldo = H;
+  if ((rc = launch_gemm<false, false, false, EPI_STORE>(ta, tb, p, st))) return rc;
+  // fc1 wgrad: dw1[e] = xp_e^T dh_e. A = xp [R, H] (MN-major), B = dh [R, 2F] (MN-major)
+  if ((rc = tmap_bf16_2d(&ta, xp, R, H, 64))) return rc;
+  if ((rc = tmap_bf16_2d(&tb, dh, R, 2 * F, 64))) return rc;
+  p = base_params(split_sizes, E);
+  p.M = H;
+  p.N = 2 * F;
+  p.out = dw1;
+  p.ldo = 2 * F;
+  p.out_batch = (long long)H * 2 * F;
+  return launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st);
+}
+
+}  // extern "C"

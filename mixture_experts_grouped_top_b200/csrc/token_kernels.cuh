@@ -1,0 +1,449 @@
+// Token-side kernels of the MoE expert-MLP path: top-k router softmax, the stable
+// expert-contiguous permutation (index build + data movement, with an optional fused
+// MXFP8 row quantisation), the unpermute/combine, and the standalone MXFP8 quantiser.
+//
+// Pages: "Efficient MoE training for biological foundation models" (sitech.ge section
+// "Grouped experts instead of a Python loop"; news.bpdata.com sections 1-2): tokens are
+// routed to a few experts, grouped per expert with per-expert counts (split_sizes), and
+// MXFP8 keeps one scale per 32 consecutive values.
+#pragma once
+#include <cuda_fp8.h>
+
+#include "ptx_sm100.cuh"
+
+namespace moe {
+
+constexpr int kPermuteChunk = 1024;   // slots per block in the index build
+constexpr int kPermuteThreads = 256;  // 8 warps, 128 consecutive slots per warp
+constexpr int kMaxExperts = 1024;
+
+// ------------------------------------------------------------------------ routing
+// One warp per token. Softmax over all E logits in fp32, then the k largest logits
+// (ties -> lower expert index) in descending order; with renorm the k probabilities
+// are divided by their sum.
+template <int VPL>  // logits held per lane: ceil(E / 32)
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                         int renorm, int32_t* __restrict__ idx,
+                                                         float* __restrict__ prob) {
+  const int lane = threadIdx.x & 31;
+  const int warps_per_block = blockDim.x >> 5;
+  for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
+    const float* row = logits + (size_t)t * E;
+    float v[VPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (e < E) ? row[e] : -INFINITY;
+      m = fmaxf(m, v[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (lane + 32 * i < E) s += expf(v[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+
+    uint32_t taken = 0;
+    float psum = 0.f;
+    float pk = 0.f;   // lane j (< k) keeps probability j
+    int ek = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+          bv = v[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      const float p = expf(bv - m) / s;
+      psum += p;
+      if (lane == j) {
+        pk = p;
+        ek = be;
+      }
+    }
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = ek;
+      prob[(size_t)t * k + lane] = renorm ? pk / psum : pk;
+    }
+  }
+}
+
+// ------------------------------------------------------------- permutation index
+// Pass 1: per-block expert histogram of a chunk of kPermuteChunk consecutive slots.
+__global__ void __launch_bounds__(kPermuteThreads) permute_hist_kernel(const int32_t* __restrict__ idx, int R,
+                                                                       int E, int32_t* __restrict__ counts) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int s0 = blockIdx.x * kPermuteChunk;
+  for (int i = threadIdx.x; i < kPermuteChunk; i += blockDim.x) {
+    const int s = s0 + i;
+    if (s < R) {
+      const int e = idx[s];
+      if (e >= 0 && e < E)
+        atomicAdd(&hist[e], 1);
+      else
+        flag_error(DEVERR_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// Pass 2 (one block of 1024 threads, E <= 1024): split_sizes, offsets, and the first
+// row of every (block, expert) pair, written over the counts. Threads form a [P][E]
+// grid (P = 1024 / E) that splits the blocks into P contiguous ranges.
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ counts, int nblk, int E, int R,
+                                                            int32_t* __restrict__ split_sizes,
+                                                            int32_t* __restrict__ offsets) {
+  extern __shared__ int32_t sm[];
+  __shared__ int32_t wsum[32];
+  const int P = max(1, (int)blockDim.x / E);
+  int32_t* part = sm;          // [P][E] partial sums, then their exclusive prefix over p
+  int32_t* off = sm + P * E;   // [E] first row of each expert
+  const int per = (nblk + P - 1) / P;
+  for (int tid = threadIdx.x; tid < E * P; tid += blockDim.x) {
+    const int p = tid / E, e = tid % E;
+    int acc = 0;
+    for (int b = p * per; b < min(nblk, (p + 1) * per); ++b) acc += counts[(size_t)b * E + e];
+    part[p * E + e] = acc;
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  int tot = 0;
+  if (e < E) {
+    for (int p = 0; p < P; ++p) {
+      const int c = part[p * E + e];
+      part[p * E + e] = tot;
+      tot += c;
+    }
+    split_sizes[e] = tot;
+  }
+  // block-wide exclusive scan of tot over e
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < (int)(blockDim.x >> 5)) ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    wsum[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - tot + (warp > 0 ? wsum[warp - 1] : 0);
+  if (e < E) {
+    off[e] = excl;
+    offsets[e] = excl;
+    if (e == E - 1) {
+      offsets[E] = excl + tot;
+      if (excl + tot != R) flag_error(DEVERR_SPLIT_SUM);
+    }
+  }
+  __syncthreads();
+  for (int tid = threadIdx.x; tid < E * P; tid += blockDim.x) {
+    const int p = tid / E, ee = tid % E;
+    int base = off[ee] + part[p * E + ee];
+    for (int b = p * per; b < min(nblk, (p + 1) * per); ++b) {
+      const int c = counts[(size_t)b * E + ee];
+      counts[(size_t)b * E + ee] = base;
+      base += c;
+    }
+  }
+}
+
+// Pass 3: stable ranks inside the block. Warp w owns slots [w*128, w*128+128) of the
+// chunk; ranks follow slot order: earlier warps, then earlier lanes/iterations.
+__global__ void __launch_bounds__(kPermuteThreads) permute_rowmap_kernel(const int32_t* __restrict__ idx,
+                                                                         const float* __restrict__ prob, int R,
+                                                                         int E, const int32_t* __restrict__ base,
+                                                                         int32_t* __restrict__ row_map,
+                                                                         float* __restrict__ probs_perm) {
+  constexpr int kWarps = kPermuteThreads / 32;
+  constexpr int kPerWarp = kPermuteChunk / kWarps;   // 128
+  extern __shared__ int32_t cnt[];                   // [kWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int s_warp = blockIdx.x * kPermuteChunk + warp * kPerWarp;
+  const unsigned lt = (1u << lane) - 1u;
+  // count this warp's slots per expert
+  for (int it = 0; it < kPerWarp; it += 32) {
+    const int s = s_warp + it + lane;
+    int e = (s < R) ? idx[s] : -1;
+    if (e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt) == 0) cnt[warp * E + e] += __popc(peers);
+  }
+  __syncthreads();
+  // exclusive prefix across warps, seeded with the block's starting row per expert
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = base[(size_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int it = 0; it < kPerWarp; it += 32) {
+    const int s = s_warp + it + lane;
+    int e = (s < R) ? idx[s] : -1;
+    if (e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int row = cnt[warp * E + e] + __popc(peers & lt);
+      row_map[s] = row;
+      if (probs_perm) probs_perm[row] = prob[s];
+    } else if (s < R) {
+      row_map[s] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) cnt[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------ permutation data
+// xp[row_map[t*k + j]] = x[t] for j < k. One warp per token, 16-byte vectors.
+__global__ void __launch_bounds__(256) permute_rows_bf16_kernel(const uint4* __restrict__ x, int T, int H8, int k,
+                                                                const int32_t* __restrict__ row_map,
+                                                                uint4* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int rows[8];
+    const int kk = min(k, 8);
+    for (int j = 0; j < kk; ++j) rows[j] = row_map[(size_t)t * k + j];
+    const uint4* src = x + (size_t)t * H8;
+    for (int c = lane; c < H8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      for (int j = 0; j < kk; ++j)
+        if (rows[j] >= 0) xp[(size_t)rows[j] * H8 + c] = v;
+    }
+    for (int j = 8; j < k; ++j) {   // k > 8: rare, plain loop
+      const int r = row_map[(size_t)t * k + j];
+      if (r < 0) continue;
+      for (int c = lane; c < H8; c += 32) xp[(size_t)r * H8 + c] = __ldg(src + c);
+    }
+  }
+}
+
+// Quantise 8 consecutive bf16 values held by one lane of a 4-lane group (one 32-value
+// block per group): amax over the group, E8M0 code = max(biased_exp(amax) - 8, 0),
+// elements scaled by 2^(127 - code) (exact) and converted with round-to-nearest-even,
+// saturating to +-448.
+__device__ __forceinline__ uint2 mxfp8_quant8(const uint4 v, uint8_t* scale_out) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+  float f[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p = __bfloat1622float2(h[i]);
+    f[2 * i] = p.x;
+    f[2 * i + 1] = p.y;
+    amax = fmaxf(amax, fmaxf(fabsf(p.x), fabsf(p.y)));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+  const int code = max(bexp - 8, 0);
+  *scale_out = (uint8_t)code;
+  const float inv = __uint_as_float((uint32_t)(254 - code) << 23);   // 2^(127 - code)
+  uint32_t w[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const __nv_fp8x2_storage_t lo =
+        __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i] * inv, f[4 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi =
+        __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i + 2] * inv, f[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+    w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// MXFP8 permute: quantise each token row along H once, write codes/scales to its k rows.
+// Every lane of a warp runs the same number of iterations (the 4-lane shuffles inside
+// the quantiser need the whole warp); lanes past the row end work on zeros.
+__global__ void __launch_bounds__(256) permute_rows_mxfp8_kernel(const uint4* __restrict__ x, int T, int H, int k,
+                                                                 const int32_t* __restrict__ row_map,
+                                                                 uint8_t* __restrict__ xq,
+                                                                 uint8_t* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int H8 = H >> 3;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    const uint4* src = x + (size_t)t * H8;
+    for (int c0 = 0; c0 < H8; c0 += 32) {
+      const int c = c0 + lane;
+      const bool live = c < H8;   // H8 is a multiple of 4: a 4-lane group is all live or all dead
+      uint8_t sc;
+      const uint2 q = mxfp8_quant8(live ? __ldg(src + c) : make_uint4(0, 0, 0, 0), &sc);
+      if (!live) continue;
+      for (int j = 0; j < k; ++j) {
+        const int r = row_map[(size_t)t * k + j];
+        if (r < 0) continue;
+        *reinterpret_cast<uint2*>(xq + (size_t)r * H + (size_t)c * 8) = q;
+        if ((lane & 3) == 0) xs[(size_t)r * (H >> 5) + (c >> 2)] = sc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- unpermute/combine
+// out[t] = sum_j w_tj * yp[row_map[t*k+j]] (w = 1 without prob), fp32 accumulation in
+// slot order, rounded once to bf16.
+__global__ void __launch_bounds__(256) unpermute_bf16_kernel(const uint4* __restrict__ yp,
+                                                             const int32_t* __restrict__ row_map,
+                                                             const float* __restrict__ prob, int T, int H8, int k,
+                                                             uint4* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    for (int c = lane; c < H8; c += 32) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int j = 0; j < k; ++j) {
+        const int r = row_map[(size_t)t * k + j];
+        if (r < 0) continue;
+        const float w = prob ? prob[(size_t)t * k + j] : 1.0f;
+        const uint4 v = __ldg(yp + (size_t)r * H8 + c);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 p = __bfloat1622float2(h[i]);
+          acc[2 * i] = fmaf(w, p.x, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(w, p.y, acc[2 * i + 1]);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      out[(size_t)t * H8 + c] = o;
+    }
+  }
+}
+
+// dprob[t, j] = dprobs_perm[row_map[t*k + j]]
+__global__ void gather_slots_f32_kernel(const float* __restrict__ src, const int32_t* __restrict__ row_map, int R,
+                                        float* __restrict__ dst) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < R; s += gridDim.x * blockDim.x) {
+    const int r = row_map[s];
+    dst[s] = (r >= 0) ? src[r] : 0.f;
+  }
+}
+
+// ------------------------------------------------------------ MXFP8 quantiser
+// axis 0: blocks of 32 along the columns of each row. 4 lanes per block.
+__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ in, long long nvec, int cols,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  // nvec = rows * cols / 8; vector v covers columns [8*(v % (cols/8)), +8) of row v / (cols/8)
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // the loop runs while the warp's first vector is in range, so all 32 lanes stay
+  // together for the shuffles; nvec is a multiple of 4, so groups are all live or all dead
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v - (threadIdx.x & 31) < nvec; v += stride) {
+    const bool live = v < nvec;
+    uint8_t sc;
+    const uint2 q = mxfp8_quant8(live ? __ldg(in + v) : make_uint4(0, 0, 0, 0), &sc);
+    if (live) {
+      *reinterpret_cast<uint2*>(codes + v * 8) = q;
+      if ((threadIdx.x & 3) == 0) scales[v >> 2] = sc;
+    }
+  }
+}
+
+// axis 1: blocks of 32 along the rows of each column. A block of 256 threads handles a
+// 32 x 256 tile of one batch matrix [rows, cols]; thread j owns column c0 + j.
+// transpose_out: codes [cols, rows], scales [cols, rows/32]; else codes [rows, cols],
+// scales [rows/32, cols].
+__global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols,
+                                                         int transpose_out, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ scales) {
+  __shared__ __align__(16) uint8_t tile[32][256 + 16];
+  const int b = blockIdx.z;
+  const int r0 = blockIdx.y * 32;
+  const int c0 = blockIdx.x * 256;
+  const int j = threadIdx.x;
+  const int c = c0 + j;
+  const __nv_bfloat16* src = in + (size_t)b * rows * cols;
+  uint8_t* dst = codes + (size_t)b * rows * cols;
+  uint8_t* sdst = scales + (size_t)b * (rows / 32) * cols;
+  float f[32];
+  float amax = 0.f;
+  if (c < cols) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      f[i] = __bfloat162float(src[(size_t)(r0 + i) * cols + c]);
+      amax = fmaxf(amax, fabsf(f[i]));
+    }
+  }
+  const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+  const int code = max(bexp - 8, 0);
+  const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+  if (c < cols) {
+    if (transpose_out) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i] * inv, f[4 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(f[4 * i + 2] * inv, f[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+      }
+      uint4* o = reinterpret_cast<uint4*>(dst + (size_t)c * rows + r0);
+      o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      sdst[(size_t)c * (rows / 32) + (r0 / 32)] = (uint8_t)code;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const __nv_fp8x2_storage_t p =
+            __nv_cvt_float2_to_fp8x2(make_float2(f[i] * inv, f[i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        tile[i][j] = (uint8_t)(p & 0xFF);
+        tile[i + 1][j] = (uint8_t)(p >> 8);
+      }
+      sdst[(size_t)(r0 / 32) * cols + c] = (uint8_t)code;
+    }
+  }
+  if (!transpose_out) {
+    __syncthreads();
+    // 32 rows x 256 bytes: each thread writes 32 bytes of one row
+    const int row = threadIdx.x >> 3, part = threadIdx.x & 7;
+    const int cc = c0 + part * 32;
+    if (cc < cols) {
+      const int n = min(32, cols - cc);
+      uint8_t* o = dst + (size_t)(r0 + row) * cols + cc;
+      for (int i = 0; i < n; ++i) o[i] = tile[row][part * 32 + i];
+    }
+  }
+}
+
+}  // namespace moe

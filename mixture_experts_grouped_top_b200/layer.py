@@ -1,0 +1,113 @@
+"""One MoE expert-MLP layer on preallocated device buffers, sequencing the C-ABI calls.
+
+forward:  moe_route -> moe_permute -> grouped_mlp_fwd -> moe_unpermute
+backward: moe_permute_rows(grad_out) -> grouped_mlp_bwd -> moe_unpermute(dxp) -> moe_gather_slots
+
+All arithmetic runs in libmoe_grouped.so; this module only owns buffers and call order.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (BF16, MXFP8, _PREC, grouped_mlp_bwd, grouped_mlp_bwd_workspace_size, grouped_mlp_fwd,
+               grouped_mlp_saved_size, grouped_mlp_workspace_size, moe_gather_slots, moe_permute,
+               moe_permute_rows, moe_permute_workspace_size, moe_route, moe_unpermute, mxfp8_quantize)
+
+
+class MoEExpertLayer:
+    def __init__(self, T: int, H: int, F: int, E: int, k: int, precision="bf16", training: bool = False,
+                 renorm: bool = True, device="cuda"):
+        self.T, self.H, self.F, self.E, self.k = T, H, F, E, k
+        self.R = T * k
+        self.prec = _PREC[precision]
+        self.precision = "bf16" if self.prec == BF16 else "mxfp8"
+        self.training = training
+        self.renorm = renorm
+        dev = torch.device(device)
+        self.device = dev
+        R = self.R
+        u8, i32, f32, bf = torch.uint8, torch.int32, torch.float32, torch.bfloat16
+        self.idx = torch.empty((T, k), dtype=i32, device=dev)
+        self.prob = torch.empty((T, k), dtype=f32, device=dev)
+        self.perm = {
+            "xp": torch.empty((R, H), dtype=bf if self.prec == BF16 else u8, device=dev),
+            "row_map": torch.empty(R, dtype=i32, device=dev),
+            "probs_perm": torch.empty(R, dtype=f32, device=dev),
+            "split_sizes": torch.empty(E, dtype=i32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=i32, device=dev),
+        }
+        if self.prec == MXFP8:
+            self.perm["xp_scale"] = torch.empty((R, H // 32), dtype=u8, device=dev)
+        self.perm_ws = torch.empty(max(moe_permute_workspace_size(T, k, E), 1), dtype=u8, device=dev)
+        self.yp = torch.empty((R, H), dtype=bf, device=dev)
+        self.out = torch.empty((T, H), dtype=bf, device=dev)
+        self.mlp_ws = torch.empty(grouped_mlp_workspace_size(E, R, H, F, self.precision, training), dtype=u8,
+                                  device=dev)
+        self.saved = (torch.empty(grouped_mlp_saved_size(E, R, H, F, self.precision), dtype=u8, device=dev)
+                      if training else None)
+        self.w1 = self.w2 = None
+        self.w1_scale = self.w2_scale = None
+        self._bwd = None
+
+    # --------------------------------------------------------------- weights
+    def set_weights(self, w1: torch.Tensor, w2: torch.Tensor, stream=None):
+        """w1 [E, H, 2F] and w2 [E, F, H] bf16 masters on the device. The MXFP8 layer
+        quantises them here (once per optimizer step) into K-major E4M3 codes."""
+        self.w1_master, self.w2_master = w1, w2
+        if self.prec == BF16:
+            self.w1, self.w2 = w1, w2
+        else:
+            self.w1, self.w1_scale = mxfp8_quantize(w1, axis=1, transpose_out=True, stream=stream)
+            self.w2, self.w2_scale = mxfp8_quantize(w2, axis=1, transpose_out=True, stream=stream)
+
+    # --------------------------------------------------------------- forward
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, stream=None) -> torch.Tensor:
+        moe_route(logits, self.k, self.renorm, idx=self.idx, prob=self.prob, stream=stream)
+        moe_permute(x, self.idx, self.prob, self.E, self.precision, out=self.perm, workspace=self.perm_ws,
+                    stream=stream)
+        grouped_mlp_fwd(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2, self.perm["probs_perm"],
+                        self.precision, xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
+                        w2_scale=self.w2_scale, yp=self.yp, saved=self.saved, workspace=self.mlp_ws, F=self.F,
+                        stream=stream)
+        moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
+        return self.out
+
+    # -------------------------------------------------------------- backward
+    def _alloc_bwd(self):
+        T, H, F, E, R = self.T, self.H, self.F, self.E, self.R
+        dev, bf = self.device, torch.bfloat16
+        self._bwd = {
+            "dy_perm": torch.empty((R, H), dtype=bf, device=dev),
+            "dxp": torch.empty((R, H), dtype=bf, device=dev),
+            "dw1": torch.empty((E, H, 2 * F), dtype=bf, device=dev),
+            "dw2": torch.empty((E, F, H), dtype=bf, device=dev),
+            "dprobs_perm": torch.empty(R, dtype=torch.float32, device=dev),
+            "dx": torch.empty((T, H), dtype=bf, device=dev),
+            "dprob": torch.empty((T, self.k), dtype=torch.float32, device=dev),
+            "ws": torch.empty(grouped_mlp_bwd_workspace_size(E, R, H, F, self.precision), dtype=torch.uint8,
+                              device=dev),
+        }
+
+    def backward(self, grad_out: torch.Tensor, stream=None):
+        """Gradients of the last forward: returns (dx [T,H], dw1, dw2, dprob [T,k])."""
+        if not self.training:
+            raise RuntimeError("layer was built without training=True")
+        if self._bwd is None:
+            self._alloc_bwd()
+        b = self._bwd
+        moe_permute_rows(grad_out, self.perm["row_map"], self.k, out=b["dy_perm"], stream=stream)
+        grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], self.perm["xp"], self.w1, self.w2,
+                        self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"], dw1=b["dw1"],
+                        dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream)
+        moe_unpermute(b["dxp"], self.perm["row_map"], self.T, self.k, out=b["dx"], stream=stream)
+        moe_gather_slots(b["dprobs_perm"], self.perm["row_map"], out=b["dprob"].view(-1), stream=stream)
+        return b["dx"], b["dw1"], b["dw2"], b["dprob"]
+
+
+def moe_layer_forward(x, logits, w1, w2, k: int, precision="bf16", stream=None):
+    """One-shot forward of a layer (allocates its buffers; use MoEExpertLayer to reuse them)."""
+    T, H = x.shape
+    E, _, F2 = w1.shape
+    layer = MoEExpertLayer(T, H, F2 // 2, E, k, precision, device=x.device)
+    layer.set_weights(w1, w2, stream=stream)
+    return layer.forward(x, logits, stream=stream), layer

@@ -287,3 +287,33 @@ def grouped_mlp_fwd_mxfp8(xp_codes, xp_scales, split_sizes, w1_codes, w1_scales,
         yp[rows] = aq[rows] @ w2q[e].T
         start += n
     return yp, a_codes, a_scales, h_all
+
+
+def moe_forward_sampled(x, idx, prob, w1, w2, tokens, a_round="bf16") -> np.ndarray:
+    """The per-token definition restricted to ``tokens``, computed expert by expert.
+
+    Same sum as :func:`moe_forward_per_token` (the k terms of a token are added in slot
+    order j = 0..k-1), but each expert's weights are converted to float64 once, so the
+    full-size layers fit in host memory. ``w1``/``w2`` may be bf16 CPU tensors.
+    """
+    toks = np.asarray(tokens, dtype=np.int64)
+    idx = np.asarray(idx, dtype=np.int64)[toks]
+    prob = f64(prob)[toks]
+    xs = f64(x[toks]) if hasattr(x, "detach") else f64(x)[toks]
+    E = w1.shape[0]
+    F = w2.shape[1]
+    terms = np.zeros((idx.shape[1], toks.size, xs.shape[1]), dtype=np.float64)
+    for e in range(E):
+        sel = np.nonzero(idx == e)
+        if sel[0].size == 0:
+            continue
+        w1e = f64(w1[e])
+        w2e = f64(w2[e])
+        n, j = sel
+        h = xs[n] @ w1e
+        a = _round_a(silu(h[:, :F]) * h[:, F:] * prob[n, j][:, None], a_round)
+        terms[j, n] = a @ w2e
+    out = np.zeros((toks.size, xs.shape[1]), dtype=np.float64)
+    for j in range(idx.shape[1]):
+        out += terms[j]
+    return out

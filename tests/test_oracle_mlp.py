@@ -164,3 +164,11 @@ def test_mxfp8_grouped_equals_per_token_on_quantised_operands():
     # feeding the layer's own quantised `a` back in reproduces the same output
     yp2, _, _, _ = moe.grouped_mlp_fwd_mxfp8(xpc, xps, split, w1c, w1s, w2c, w2s, pp, ac, asc)
     assert np.array_equal(yp, yp2)
+
+
+def test_sampled_forward_equals_per_token_definition():
+    x, idx, prob, w1, w2 = _layer(30, 8, 6, 4, 2, seed=41)
+    toks = np.array([0, 3, 7, 29])
+    ref = moe.moe_forward_per_token(x, idx, prob, w1, w2, "bf16", tokens=toks)
+    got = moe.moe_forward_sampled(x, idx, prob, w1, w2, toks, "bf16")
+    assert np.max(np.abs(got - ref)) <= 1e-13 * np.max(np.abs(ref))
