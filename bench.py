@@ -182,11 +182,13 @@ def run_ours(args, world, rank, local):
     launches0 = mb.moe_launch_count()
     with ClockSampler(local, os.path.join(ROOT, "gpurun_out", "clocks.csv")
                       if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None) as clocks:
+        wall0 = time.perf_counter()
         t0.record(stream)
         for i in range(K):
             step(mlp_events[i])
         t1.record(stream)
         torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
     launches = mb.moe_launch_count() - launches0
     barrier(world)
     ms = t0.elapsed_time(t1) / K
@@ -225,7 +227,11 @@ def run_ours(args, world, rank, local):
     e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # a timed region of a second or more runs under the power cap: compare with the
+    # sustained GEMM peak; a shorter one with the burst peak
+    regime = "sustained" if wall >= 1.0 else "burst"
+    key = "bf16_tflops_sustained" if regime == "sustained" else "bf16_tflops"
+    peak = peaks.get(key, FALLBACK_PEAKS[key])
     achieved = flops / (mlp_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -254,7 +260,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"kernel": "grouped_mlp_fwd (fc1 gate|up + ScaledSwiGLU, fc2: two tcgen05 grouped GEMMs)",
                      "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_src} bf16 sustained", "traffic": None,
+                     "peak_source": f"{peak_src} bf16 {regime} (timed region {wall:.2f} s)", "traffic": None,
                      "avg_launch_ms": round(mlp_ms, 4)},
     }
     cl = clocks.summary()
