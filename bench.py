@@ -16,6 +16,7 @@ path); the step time is the max over ranks and `value` counts all ranks' work.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -141,6 +142,8 @@ def run_ours(args, world, rank, local):
     import mixture_experts_grouped_top_b200 as mb
 
     cfg = workloads.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_T{args.tokens}", T=args.tokens)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     d = workloads.make_layer_inputs(cfg, seed=rank_seed(cfg.seed, rank), with_grad=cfg.passes == "fwd+bwd")
@@ -329,6 +332,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs on a smaller batch)")
     ap.add_argument("--cpu-baseline-tokens", type=int, default=256)
     ap.add_argument("--reference-tokens", type=int, default=64)
     args = ap.parse_args(argv)
