@@ -101,6 +101,36 @@ MOE_API int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob
                 int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
                 int32_t* split_sizes, int32_t* offsets, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Largest per-block histogram table moe_permute_noalloc can hold, in int32 entries:
+ * ceil(T*k / 1024) * E must not exceed it (e.g. T*k <= 2,097,152 with E = 128). */
+#define MOE_PERMUTE_NOALLOC_MAX_COUNTS 262144
+
+/*
+ * moe_permute_noalloc — moe_permute for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it is the same stable permutation as
+ * moe_permute (same arguments, same outputs, bit for bit) minus the workspace argument.
+ *
+ * Who needs it: hosts that must not allocate once they are running — an inference
+ * server or embedded runtime that plans all device memory at start-up and forbids
+ * cudaMalloc afterwards (it can fail under memory pressure and it synchronises the
+ * device), or a plain C caller with no caching allocator that would otherwise pay a
+ * cudaMalloc/cudaFree pair around every call. The caller still allocates and passes all
+ * inputs and outputs; only the scratch table is provided by the library.
+ *
+ * Scratch: a fixed table of MOE_PERMUTE_NOALLOC_MAX_COUNTS int32 (1 MiB) in static
+ * device memory that every GPU which loads the library holds until the process exits.
+ * Sizes that need more return MOE_ERR_UNSUPPORTED (with a message on stderr) before
+ * anything is launched. This call never calls cudaMalloc, cudaFree or any allocating
+ * routine. The first call on each device looks up the table's device address (with that
+ * device current); make that first call before any stream capture. All calls share the
+ * one table and it keeps the last call's contents (every entry a call reads is written
+ * by the same call first), so calls whose GPU work overlaps — on two streams, or from
+ * two host threads — race on it and must be serialised by the caller.
+ */
+MOE_API int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
+                                int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                                int32_t* split_sizes, int32_t* offsets, void* stream);
+
 /*
  * moe_permute_rows — the data movement of moe_permute alone, for a tensor that follows
  * an existing row_map (e.g. the gradient of the layer output in the backward pass):

@@ -115,6 +115,22 @@ def moe_permute(x, idx, prob, E: int, precision="bf16", out=None, workspace=None
     return o
 
 
+def moe_permute_noalloc(x, idx, prob, E: int, precision="bf16", out=None, stream=None):
+    """moe_permute with the library's static scratch table instead of a workspace (for
+    callers that must not allocate device memory); outputs as moe_permute."""
+    _need(x, torch.bfloat16, "x")
+    _need(idx, torch.int32, "idx")
+    prec = _PREC[precision]
+    T, H = x.shape
+    k = idx.shape[1]
+    o = dict(out)   # every output buffer is passed by the caller
+    rc = lib().moe_permute_noalloc(_p(x), _p(idx), _p(prob), T, H, E, k, prec, _p(o["xp"]), _p(o.get("xp_scale")),
+                                   _p(o["row_map"]), _p(o.get("probs_perm")), _p(o["split_sizes"]),
+                                   _p(o["offsets"]), _stream(stream))
+    _check("moe_permute_noalloc", rc)
+    return o
+
+
 def moe_permute_rows(src, row_map, k: int, out=None, stream=None):
     _need(src, torch.bfloat16, "src")
     T, H = src.shape

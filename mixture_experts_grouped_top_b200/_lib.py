@@ -19,6 +19,7 @@ SIGNATURES = {
     "moe_route": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute_rows": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_unpermute": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "mxfp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),

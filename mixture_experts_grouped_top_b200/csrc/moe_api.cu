@@ -454,3 +454,48 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free permutation: moe_permute with its histogram table in static device
+// memory instead of a caller workspace (see moe_permute_noalloc in the header).
+namespace {
+
+static __device__ __align__(256) int32_t g_permute_scratch[MOE_PERMUTE_NOALLOC_MAX_COUNTS];
+
+// Device address of g_permute_scratch on the current device, looked up once per device
+// with that device current (host code cannot use the symbol itself as a pointer).
+int32_t* permute_scratch_on_current_device() {
+  static int32_t* ptr[64];
+  static cudaError_t err[64];
+  static std::once_flag once[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev]() {
+    void* p = nullptr;
+    err[dev] = cudaGetSymbolAddress(&p, g_permute_scratch);
+    ptr[dev] = static_cast<int32_t*>(p);
+  });
+  return err[dev] == cudaSuccess ? ptr[dev] : nullptr;
+}
+
+}  // namespace
+
+extern "C" int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E,
+                                   int k, int precision, void* xp, uint8_t* xp_scale, int32_t* row_map,
+                                   float* probs_perm, int32_t* split_sizes, int32_t* offsets, void* stream) {
+  if (T < 0 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_permute_workspace_size(T, k, E);
+  if (need > sizeof(int32_t) * (size_t)MOE_PERMUTE_NOALLOC_MAX_COUNTS) {
+    fprintf(stderr,
+            "moe_permute_noalloc: T*k=%lld with E=%d needs %zu bytes of scratch; the static table holds %zu "
+            "(ceil(T*k/1024)*E must be <= %d)\n",
+            (long long)T * k, E, need, sizeof(int32_t) * (size_t)MOE_PERMUTE_NOALLOC_MAX_COUNTS,
+            MOE_PERMUTE_NOALLOC_MAX_COUNTS);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  int32_t* scratch = permute_scratch_on_current_device();
+  if (!scratch) return MOE_ERR_CUDA;
+  return moe_permute(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, split_sizes, offsets,
+                     scratch, sizeof(int32_t) * (size_t)MOE_PERMUTE_NOALLOC_MAX_COUNTS, stream);
+}
+
