@@ -156,20 +156,35 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     prec = cfg.precision
 
-    def step(ev_mlp=None):
+    training = cfg.passes == "fwd+bwd"
+
+    def step(ev=None):
+        """One pass of the path; `ev` = 4 events bracketing the grouped-GEMM calls."""
         mb.moe_route(logits, cfg.k, True, idx=layer.idx, prob=layer.prob)
         mb.moe_permute(x, layer.idx, layer.prob, cfg.E, prec, out=layer.perm, workspace=layer.perm_ws)
-        if ev_mlp is not None:
-            ev_mlp[0].record(stream)
+        if ev is not None:
+            ev[0].record(stream)
         mb.grouped_mlp_fwd(layer.perm["xp"], layer.perm["split_sizes"], layer.w1, layer.w2,
                            layer.perm["probs_perm"], prec, xp_scale=layer.perm.get("xp_scale"),
                            w1_scale=layer.w1_scale, w2_scale=layer.w2_scale, yp=layer.yp, saved=layer.saved,
                            workspace=layer.mlp_ws, F=cfg.F)
-        if ev_mlp is not None:
-            ev_mlp[1].record(stream)
+        if ev is not None:
+            ev[1].record(stream)
         mb.moe_unpermute(layer.yp, layer.perm["row_map"], cfg.T, cfg.k, out=layer.out)
-        if grad is not None:
-            layer.backward(grad)
+        if training:
+            if layer._bwd is None:
+                layer._alloc_bwd()
+            b = layer._bwd
+            mb.moe_permute_rows(grad, layer.perm["row_map"], cfg.k, out=b["dy_perm"])
+            if ev is not None:
+                ev[2].record(stream)
+            mb.grouped_mlp_bwd(b["dy_perm"], layer.perm["split_sizes"], layer.perm["xp"], layer.w1, layer.w2,
+                               layer.perm["probs_perm"], layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"], dw2=b["dw2"],
+                               dprobs_perm=b["dprobs_perm"], workspace=b["ws"])
+            if ev is not None:
+                ev[3].record(stream)
+            mb.moe_unpermute(b["dxp"], layer.perm["row_map"], cfg.T, cfg.k, out=b["dx"])
+            mb.moe_gather_slots(b["dprobs_perm"], layer.perm["row_map"], out=b["dprob"].view(-1))
 
     for _ in range(args.warmup):
         step()
@@ -178,7 +193,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device error during warm-up")
 
     K = args.steps
-    mlp_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    mlp_events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -196,7 +211,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     ms = t0.elapsed_time(t1) / K
     ms_max = max_over_ranks(ms, world)
-    mlp_ms = statistics.mean(a.elapsed_time(b) for a, b in mlp_events)
+    mlp_ms = statistics.mean(ev[0].elapsed_time(ev[1]) + (ev[2].elapsed_time(ev[3]) if training else 0.0)
+                             for ev in mlp_events)
     if mb.moe_device_status() != 0:
         raise RuntimeError("device error during the timed region")
 
@@ -205,16 +221,25 @@ def run_ours(args, world, rank, local):
     tokens_s = world * cfg.T / (ms_max * 1e-3)
 
     # ------------------------------------------------ end to end through host buffers
+    # every step: pinned host -> device copies of the step's inputs, the path, and a
+    # device -> host read of its result (the layer output; with backward also dx)
     x_h = d["x"].pin_memory()
     lg_h = d["logits"].pin_memory()
+    g_h = d["grad_out"].pin_memory() if training else None
     out_h = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    dx_h = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() if training else None
     xd, lgd = torch.empty_like(x), torch.empty_like(logits)
+    gd = torch.empty_like(grad) if training else None
 
     def e2e_step():
         xd.copy_(x_h, non_blocking=True)
         lgd.copy_(lg_h, non_blocking=True)
         out = layer.forward(xd, lgd)
         out_h.copy_(out, non_blocking=True)
+        if training:
+            gd.copy_(g_h, non_blocking=True)
+            dx = layer.backward(gd)[0]
+            dx_h.copy_(dx, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -228,6 +253,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world)
     e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
+    h2d = x.numel() * 2 + logits.numel() * 4 + (grad.numel() * 2 if training else 0)
+    d2h = cfg.T * cfg.H * 2 * (2 if training else 1)
 
     peaks, peak_src = load_peaks()
     # a timed region of a second or more runs under the power cap: compare with the
@@ -235,6 +262,11 @@ def run_ours(args, world, rank, local):
     regime = "sustained" if wall >= 1.0 else "burst"
     key = "bf16_tflops_sustained" if regime == "sustained" else "bf16_tflops"
     peak = peaks.get(key, FALLBACK_PEAKS[key])
+    peak_note = f"{peak_src} bf16 {regime}"
+    if prec == "mxfp8":
+        # no measured MXFP8 figure: the measured bf16 one times the nominal dense ratio 4.5/2.25
+        peak = 2.0 * peak
+        peak_note = f"{peak_src} bf16 {regime} x 2 (nominal MXFP8/BF16 dense ratio)"
     achieved = flops / (mlp_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -257,13 +289,13 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"dp{world} replicas" if world > 1 else "single GPU"},
         "tokens_per_s": round(tokens_s, 1),
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
-                "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
-                "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
-        "roofline": {"kernel": "grouped_mlp_fwd (fc1 gate|up + ScaledSwiGLU, fc2: two tcgen05 grouped GEMMs)",
+        "roofline": {"kernel": ("grouped_mlp_fwd + grouped_mlp_bwd (the six tcgen05 grouped GEMMs)" if training
+                               else "grouped_mlp_fwd (fc1 gate|up + ScaledSwiGLU, fc2: two tcgen05 grouped GEMMs)"),
                      "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_src} bf16 {regime} (timed region {wall:.2f} s)", "traffic": None,
+                     "peak_source": f"{peak_note} (timed region {wall:.2f} s)", "traffic": None,
                      "avg_launch_ms": round(mlp_ms, 4)},
     }
     cl = clocks.summary()

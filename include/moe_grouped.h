@@ -53,6 +53,10 @@ typedef enum {
 
 typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_precision_t;
 
+/* Flag OR-ed into grouped_mlp_fwd's `precision`: write yp as fp32 [R, H] instead of bf16
+ * (the fc2 accumulator without the bf16 storage rounding). */
+#define MOE_OUT_F32 0x100
+
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int status);
 
@@ -150,6 +154,15 @@ MOE_API int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T,
 MOE_API int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const float* prob, int T, int H, int k,
                   uint16_t* out, void* stream);
 
+/* Scale layouts of mxfp8_quantize's output. PLAIN is the [rows, K/32] grid. MMA arranges
+ * the scales of a K-major matrix [N, K] (N and K multiples of 128) in the 512-byte atoms
+ * the block-scaled tensor-core instruction consumes: atom (g, j) holds rows
+ * [128 g, 128 g + 128) and K blocks [4 j, 4 j + 4) at byte offset (g * K/128 + j) * 512;
+ * inside it, row r's four bytes form the 32-bit word (r % 32) * 4 + r / 32, byte
+ * (block % 4). Stacked expert matrices [E, N, K] number their row groups e * N/128 + n/128. */
+#define MOE_SCALES_PLAIN 0
+#define MOE_SCALES_MMA 1
+
 /*
  * mxfp8_quantize — MXFP8 quantisation of a batch of bf16 matrices in[batch, rows, cols].
  * Pages: news.bpdata.com section 2) and sitech.ge "Reducing memory and quantisation
@@ -164,15 +177,19 @@ MOE_API int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const floa
  *           transpose_out = 1: codes [batch, cols, rows], scales [batch, cols, rows/32]
  *             (the transposed matrix quantised along its rows: K-major weights);
  *           transpose_out = 0: codes [batch, rows, cols], scales [batch, rows/32, cols].
+ *   scale_layout: MOE_SCALES_PLAIN, or MOE_SCALES_MMA (axis 1 with transpose_out only;
+ *           rows and cols multiples of 128) for weights handed to grouped_mlp_fwd.
  */
 MOE_API int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out,
-                   uint8_t* codes, uint8_t* scales, void* stream);
+                           int scale_layout, uint8_t* codes, uint8_t* scales, void* stream);
 
 /* Bytes of scratch grouped_mlp_fwd needs (the fc1 output `a` when saved == NULL). */
 MOE_API size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int training);
 
 /* Bytes of the buffer grouped_mlp_fwd fills for the backward pass (training mode):
- * h = [gate | up] pre-activations [R, 2F] bf16, then a [R, F] bf16. */
+ * h = [gate | up] pre-activations [R, 2F] bf16, then a: [R, F] bf16 (MOE_BF16) or
+ * [R, F] E4M3 codes followed by their scale atoms (MOE_MXFP8); each part starts on a
+ * 256-byte boundary. */
 MOE_API size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision);
 
 /*
@@ -187,18 +204,22 @@ MOE_API size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision)
  *   yp_e = a @ w2[e]            (K = F, N = H)
  * MOE_BF16: xp [R, H] bf16, w1 [E, H, 2F] bf16, w2 [E, F, H] bf16; scales ignored;
  *   a is rounded to bf16 before fc2; fp32 accumulation.
- * MOE_MXFP8: xp [R, H] E4M3 + xp_scale [R, H/32]; w1 [E, 2F, H] E4M3 + w1_scale
- *   [E, 2F, H/32]; w2 [E, H, F] E4M3 + w2_scale [E, H, F/32] (weights as produced by
- *   mxfp8_quantize(axis=1, transpose_out=1)); the fc1 epilogue quantises a along F.
+ * MOE_MXFP8: xp [R, H] E4M3 + xp_scale [R, H/32] (plain, as moe_permute writes it);
+ *   w1 [E, 2F, H] E4M3 and w2 [E, H, F] E4M3 with their scales in the MOE_SCALES_MMA
+ *   layout (as produced by mxfp8_quantize(axis=1, transpose_out=1, MOE_SCALES_MMA));
+ *   the fc1 epilogue quantises a along F (blocks of 32) and keeps its scales as MMA
+ *   atoms whose row groups are the 128-row tiles of each expert (sum over earlier
+ *   experts of ceil(n_e/128), then the tile index); requires H % 128 == 0.
  * split_sizes [E] int32 on the device (no host synchronisation happens); R = sum.
- * yp [R, H] bf16 output. saved: NULL for inference, else a buffer of
+ * yp [R, H] bf16 output (fp32 when MOE_OUT_F32 is OR-ed into precision).
+ * saved: NULL for inference, else a buffer of
  * grouped_mlp_saved_size() bytes that receives h and a for grouped_mlp_bwd.
  * ws: scratch of grouped_mlp_workspace_size() bytes.
  * Requires H % 64 == 0 and F % 128 == 0.
  */
 MOE_API int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
                     const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
-                    const float* probs_perm, int precision, uint16_t* yp, void* saved, void* ws, size_t ws_bytes,
+                    const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
                     void* stream);
 
 /* Bytes of scratch grouped_mlp_bwd needs (dh [R, 2F] bf16 and dprob partial sums). */

@@ -16,6 +16,7 @@ from . import _lib
 
 BF16 = 0
 MXFP8 = 1
+OUT_F32 = 0x100
 _PREC = {"bf16": BF16, "mxfp8": MXFP8, BF16: BF16, MXFP8: MXFP8}
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
@@ -156,8 +157,19 @@ def moe_gather_slots(src, row_map, out=None, stream=None):
 
 
 # ------------------------------------------------------------------------- MXFP8
-def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, scales=None, stream=None):
-    """Quantise bf16 [batch, rows, cols] (or [rows, cols]). Returns (codes, scales) uint8."""
+SCALES_PLAIN = 0
+SCALES_MMA = 1
+
+
+def mma_scale_bytes(groups: int, K: int) -> int:
+    return groups * (K // 128) * 512
+
+
+def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, scales=None, mma_scales=False,
+                   stream=None):
+    """Quantise bf16 [batch, rows, cols] (or [rows, cols]). Returns (codes, scales) uint8.
+    With ``mma_scales`` (axis 1, transpose_out) the scales come in the MMA atom layout
+    (a flat uint8 tensor) that grouped_mlp_fwd expects for weights."""
     _need(x, torch.bfloat16, "x")
     squeeze = x.dim() == 2
     x3 = x.unsqueeze(0) if squeeze else x
@@ -169,13 +181,15 @@ def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, sc
         cshape, sshape = (B, cols, rows), (B, cols, rows // 32)
     else:
         cshape, sshape = (B, rows, cols), (B, rows // 32, cols)
+    if mma_scales:
+        sshape = (B * cols * rows // 32,)
     codes = torch.empty(cshape, dtype=torch.uint8, device=dev) if codes is None else codes
     scales = torch.empty(sshape, dtype=torch.uint8, device=dev) if scales is None else scales
-    rc = lib().mxfp8_quantize(_p(x3), B, rows, cols, axis, int(bool(transpose_out)), _p(codes), _p(scales),
-                              _stream(stream))
+    rc = lib().mxfp8_quantize(_p(x3), B, rows, cols, axis, int(bool(transpose_out)),
+                              SCALES_MMA if mma_scales else SCALES_PLAIN, _p(codes), _p(scales), _stream(stream))
     _check("mxfp8_quantize", rc)
     if squeeze:
-        return codes.reshape(cshape[1:]), scales.reshape(sshape[1:])
+        return codes.reshape(cshape[1:]), (scales if mma_scales else scales.reshape(sshape[1:]))
     return codes, scales
 
 
@@ -189,7 +203,8 @@ def grouped_mlp_saved_size(E, R, H, F, precision="bf16") -> int:
 
 
 def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm=None, precision="bf16", xp_scale=None, w1_scale=None,
-                    w2_scale=None, yp=None, saved=None, training=False, workspace=None, F=None, stream=None):
+                    w2_scale=None, yp=None, saved=None, training=False, workspace=None, F=None, out_f32=False,
+                    stream=None):
     """fc1 (gate|up) -> ScaledSwiGLU -> fc2 over expert-contiguous rows.
 
     BF16: w1 [E, H, 2F], w2 [E, F, H] bf16. MXFP8: xp/w1/w2 are E4M3 codes with scales
@@ -202,14 +217,16 @@ def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm=None, precision="bf16", 
     if F is None:
         F = w2.shape[1] if prec == BF16 else w2.shape[2]
     dev = xp.device
-    yp = torch.empty((R, H), dtype=torch.bfloat16, device=dev) if yp is None else yp
+    if yp is None:
+        yp = torch.empty((R, H), dtype=torch.float32 if out_f32 else torch.bfloat16, device=dev)
     if training and saved is None:
         saved = torch.empty(grouped_mlp_saved_size(E, R, H, F, precision), dtype=torch.uint8, device=dev)
     ws_bytes = grouped_mlp_workspace_size(E, R, H, F, precision, saved is not None)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     rc = lib().grouped_mlp_fwd(_p(xp), _p(xp_scale), _p(split_sizes), E, R, H, F, _p(w1), _p(w1_scale), _p(w2),
-                               _p(w2_scale), _p(probs_perm), prec, _p(yp), _p(saved), _p(workspace),
+                               _p(w2_scale), _p(probs_perm), prec | (OUT_F32 if out_f32 else 0), _p(yp), _p(saved),
+                               _p(workspace),
                                workspace.numel(), _stream(stream))
     _check("grouped_mlp_fwd", rc)
     return yp, saved

@@ -1,0 +1,383 @@
+// Persistent grouped GEMM for MXFP8 operands on sm_100a: E4M3 A and B, one E8M0 scale
+// per 32 consecutive K values of every row, fp32 accumulation in tensor memory
+// (tcgen05.mma kind::mxf8f6f4.block_scale, M=128, N=256, K=32 per instruction).
+//
+// Pages: "Efficient MoE training for biological foundation models" (news.bpdata.com
+// section 2: MXFP8 keeps one scale per block of 32 consecutive values and Blackwell
+// tensor cores consume it directly; section 3: the fused GroupedLinear -> ScaledSwiGLU ->
+// GroupedLinear chain with quantisation fused into it).
+//
+// Same tile walk and warp roles as the BF16 kernel (grouped_gemm_sm100.cuh). What is
+// specific to block scaling:
+//   * scales travel with every 128-wide k-block as 512-byte atoms (128 rows x 4 scale
+//     bytes, row r of the group at word (r % 32) * 4 + r / 32, the layout tcgen05.cp
+//     expects), already arranged so in global memory (mma_scale_offset): the producer
+//     fetches one atom for A and two for B with bulk copies on the stage's barrier;
+//   * the MMA thread moves the atoms into tensor memory with tcgen05.cp (32 lanes x 16 B,
+//     replicated to the four sub-partitions), then issues the four K=32 MMAs of the
+//     stage, selecting scale byte kk of each word through the scale-factor ids;
+//   * two 256-column accumulators plus 12 scale columns exceed the 512 tensor-memory
+//     columns, so the accumulators overlap: acc0 = columns [0, 256), acc1 = [224, 480),
+//     scales at [480, 492). The epilogue drains the shared 32-column strip first and
+//     signals `tovl`; the next tile's MMAs wait for that strip (and for the full drain
+//     of the tile two back) instead of the whole previous epilogue.
+#pragma once
+#include "grouped_gemm_sm100.cuh"
+#include "token_kernels.cuh"
+
+namespace moe {
+
+namespace mx {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;                       // fp8: 128 bytes of K per row (one swizzle span)
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kABytes = BM * BK;              // 16 KB
+constexpr int kBBytes = BN * BK;              // 32 KB
+constexpr int kSfaBytes = 512;                // 128 rows x 4 scale bytes
+constexpr int kSfbBytes = 1024;               // 256 rows x 4 scale bytes
+constexpr int kMaxE = 1024;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kAcc1Col = 224;
+constexpr uint32_t kSfaCol = 480;
+constexpr uint32_t kSfbCol = 484;
+constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kStages * (kSfaBytes + kSfbBytes) + 1024 +
+                           2 * (kMaxE + 1) * 4;
+}  // namespace mx
+
+enum MxEpiKind : int {
+  MXEPI_STORE = 0,      // out[row, col] = bf16(acc)
+  MXEPI_SWIGLU_Q = 1,   // a = SiLU(g) * u * p quantised to MXFP8 along the columns (+ bf16 h)
+};
+
+struct MxGemmParams {
+  GemmParams g;               // E, M (rows R), N (output cols), K, split_sizes, out, ldo, out2/ldo2 (h), probs, F
+  const uint8_t* a_atoms;     // A scales as atoms, row groups = expert tiles (sum of ceil(n_e/128))
+  const uint8_t* b_atoms;     // B scales as atoms, row groups = e * (b_rows / 128) + row / 128
+  int b_rows;                 // rows of each expert's B (2F for fc1, H for fc2)
+  uint8_t* out_atoms;         // MXEPI_SWIGLU_Q: scales of `a` as atoms for the next GEMM (K = F)
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(mx::kThreads, 1)
+    grouped_gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const MxGemmParams mp) {
+  using namespace mx;
+  const GemmParams& p = mp.g;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kStages * kABytes;
+  uint8_t* sSfa = sB + kStages * kBBytes;
+  uint8_t* sSfb = sSfa + kStages * kSfaBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSfb + kStages * kSfbBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = bars + 2 * kStages + 2;
+  uint64_t* tovl = bars + 2 * kStages + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
+  int32_t* tile_off = row_off + (kMaxE + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const int NT = (EPI == MXEPI_SWIGLU_Q) ? (p.N / 128) : (p.N + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(tovl, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 3) {
+    int carry_r = 0, carry_t = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? p.split_sizes[e] : 0;
+      const int tiles = (e < E) ? ((n + BM - 1) / BM) * NT : 0;
+      int ir = n, it = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yt = __shfl_up_sync(0xffffffffu, it, o);
+        if (lane >= o) {
+          ir += yr;
+          it += yt;
+        }
+      }
+      if (e < E) {
+        row_off[e] = carry_r + ir - n;
+        tile_off[e] = carry_t + it - tiles;
+      }
+      carry_r += __shfl_sync(0xffffffffu, ir, 31);
+      carry_t += __shfl_sync(0xffffffffu, it, 31);
+    }
+    if (lane == 0) {
+      row_off[E] = carry_r;
+      tile_off[E] = carry_t;
+    }
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  TileWalker<false> walk{row_off, tile_off, E, 0, NT, p.K};
+  // the walker's k-block count assumes 64-wide blocks; MXFP8 uses 128-wide ones
+  const int num_kb = p.K / BK;
+  const int total = walk.total();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      const int KB4 = p.K / 128;
+      const int bgroups = mp.b_rows / 128;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = walk.decode(t);
+        const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
+        const size_t ga = (size_t)(tile_off[ti.e] / NT + ti.m_blk);          // A row group (expert tile)
+        const size_t gb0 = (size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? n0 / 128 : n0 / 128);
+        size_t gb1 = (size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? (p.F + n0) / 128 : n0 / 128 + 1);
+        if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const int k0 = kb * BK;
+          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes + kSfaBytes + kSfbBytes);
+          tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
+          uint8_t* b_dst = sB + stage * kBBytes;
+          if (EPI == MXEPI_SWIGLU_Q) {
+            tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
+            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, p.F + n0, ti.e);
+          } else {
+            tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
+            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, n0 + 128, ti.e);
+          }
+          bulk_load(sSfa + stage * kSfaBytes, mp.a_atoms + (ga * KB4 + kb) * 512, 512, &full[stage]);
+          bulk_load(sSfb + stage * kSfbBytes, mp.b_atoms + (gb0 * KB4 + kb) * 512, 512, &full[stage]);
+          bulk_load(sSfb + stage * kSfbBytes + 512, mp.b_atoms + (gb1 * KB4 + kb) * 512, 512, &full[stage]);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        int st = stage, ph = phase;
+        for (int i = 0; i < min(issued, kStages); ++i) {
+          if (--st < 0) {
+            st = kStages - 1;
+            ph ^= 1;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[st], ph) && global_timer_ns() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int lt = 0;
+    bool ok = true;
+    const uint32_t sfa_t = tmem_base + kSfaCol;
+    const uint32_t sfb_t = tmem_base + kSfbCol;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+      if (lt > 0 && !mbar_wait_bounded(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (acc ? kAcc1Col : 0u);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sfa_s = smem_u32(sSfa + stage * kSfaBytes);
+          const uint32_t sfb_s = smem_u32(sSfb + stage * kSfbBytes);
+          tmem_cp_32x128b_warpx4(sfa_t, make_sdesc(sfa_s, 0, 128, 0));
+          tmem_cp_32x128b_warpx4(sfb_t, make_sdesc(sfb_s, 0, 128, 0));
+          tmem_cp_32x128b_warpx4(sfb_t + 4, make_sdesc(sfb_s + kSfaBytes, 0, 128, 0));
+          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            const uint64_t adesc = make_sdesc(a_addr + kk * 32, 16, 1024, 2);
+            const uint64_t bdesc = make_sdesc(b_addr + kk * 32, 16, 1024, 2);
+            const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk);
+            mma_mxf8_ss(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30),
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&tfull[acc]);
+      __syncwarp();
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp - 4;
+    const int r_local = q * 32 + lane;
+    int lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const TileInfo ti = walk.decode(t);
+      const int acc = lt & 1;
+      if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (acc ? kAcc1Col : 0u) + ((uint32_t)(q * 32) << 16);
+      const bool row_ok = r_local < ti.rows;
+      const long long row = ti.row0 + r_local;
+      uint32_t sc_word = 0;   // SwiGLU: this row's four scale bytes (k-blocks 4*n_blk..+3 of the next GEMM)
+
+      if (EPI == MXEPI_STORE) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        const int n0 = ti.n_blk * BN;
+        const int first = acc ? 0 : 7;   // the 32-column strip shared with the other accumulator
+#pragma unroll 1
+        for (int it = 0; it < 8; ++it) {
+          const int c = (it == 0) ? first : (acc ? it : it - 1);
+          uint32_t v0[16], v1[16];
+          tmem_ld_32x32b_x16(t_row + c * 32, v0);
+          tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
+          tmem_wait_ld();
+          if (it == 0) {
+            tc_fence_before();
+            mbar_arrive(tovl);
+          }
+          if (row_ok && n0 + c * 32 < p.N && p.out_f32) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + row * p.ldo + n0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dst[i] = make_uint4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
+              dst[4 + i] = make_uint4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
+            }
+          } else if (row_ok && n0 + c * 32 < p.N) {
+            uint4 o[4];
+            uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              ow[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+              ow[8 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = o[i];
+          }
+        }
+      } else {
+        // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
+        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+        const int n0 = ti.n_blk * 128;
+        uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
+        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
+        const int first = acc ? 0 : 3;
+#pragma unroll 1
+        for (int it = 0; it < 4; ++it) {
+          const int c = (it == 0) ? first : (acc ? it : it - 1);
+          uint32_t g0[16], g1[16], u0[16], u1[16];
+          tmem_ld_32x32b_x16(t_row + c * 32, g0);
+          tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
+          tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
+          tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
+          tmem_wait_ld();
+          if (it == 0) {
+            tc_fence_before();
+            mbar_arrive(tovl);
+          }
+          if (row_ok) {
+            float a[32];
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              a[i] = silu_f(__uint_as_float(g0[i])) * __uint_as_float(u0[i]) * pr;
+              a[16 + i] = silu_f(__uint_as_float(g1[i])) * __uint_as_float(u1[i]) * pr;
+              amax = fmaxf(amax, fmaxf(fabsf(a[i]), fabsf(a[16 + i])));
+            }
+            const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+            const int code = max(bexp - 8, 0);
+            const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] *= inv;
+            uint32_t w0[4], w1[4];
+            pack_e4m3x16(a, w0);
+            pack_e4m3x16(a + 16, w1);
+            uint4* dst = reinterpret_cast<uint4*>(a_codes + row * p.ldo + n0 + c * 32);
+            dst[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+            dst[1] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+            sc_word |= (uint32_t)code << (8 * c);
+            if (hout) {
+              uint4 hg[4], hu[4];
+              uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
+              uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                hgw[i] = pack_bf16x2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1]));
+                hgw[8 + i] = pack_bf16x2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1]));
+                huw[i] = pack_bf16x2(__uint_as_float(u0[2 * i]), __uint_as_float(u0[2 * i + 1]));
+                huw[8 + i] = pack_bf16x2(__uint_as_float(u1[2 * i]), __uint_as_float(u1[2 * i + 1]));
+              }
+              uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c * 32);
+              uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                hd[i] = hg[i];
+                hd2[i] = hu[i];
+              }
+            }
+          }
+        }
+      }
+      if (EPI == MXEPI_SWIGLU_Q) {
+        // rows past the expert's end store zero scales
+        const size_t g = (size_t)(tile_off[ti.e] / NT + ti.m_blk);
+        *reinterpret_cast<uint32_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk, p.N / 128)) =
+            sc_word;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -66,6 +66,7 @@ struct GemmParams {
   long long ld_aux;
   float* dprob_part;           // DSwiGLU: [ceil(N/256)][R] partial sums
   int F;                       // SwiGLU / DSwiGLU: width of the gate half
+  int out_f32;                 // EPI_STORE: write fp32 instead of bf16
   uint64_t timeout_ns;
 };
 
@@ -361,14 +362,20 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
           tmem_ld_32x32b_x16(t_row + c, v);
           tmem_wait_ld();
           if (row_ok && n0 + c < p.N) {
-            uint4 o[2];
-            uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+            if (EPI == EPI_STORE && p.out_f32) {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c);
-            dst[0] = o[0];
-            dst[1] = o[1];
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint4 o[2];
+              uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c);
+              dst[0] = o[0];
+              dst[1] = o[1];
+            }
           }
         }
       } else if (EPI == EPI_SWIGLU) {

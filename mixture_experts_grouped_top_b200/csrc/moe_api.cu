@@ -8,7 +8,8 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/moe_grouped.h"
+#include "moe_grouped.h"
+#include "grouped_gemm_mxf8_sm100.cuh"
 #include "grouped_gemm_sm100.cuh"
 #include "token_kernels.cuh"
 
@@ -112,7 +113,33 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
   return launch_status();
 }
 
+// E4M3 codes [batch, rows, cols] as a TMA source with box {128 bytes of K, box_rows}.
+int tmap_u8_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, cols, rows, batch, cols, rows * cols, 128, box_rows);
+}
+
+template <int EPI>
+int launch_gemm_mx(const CUtensorMap& ta, const CUtensorMap& tb, const MxGemmParams& p, cudaStream_t st) {
+  auto kern = grouped_gemm_mxf8_kernel<EPI>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mx::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  const int grid = device_props().sm_count;
+  kern<<<grid, mx::kThreads, mx::kSmemBytes, st>>>(ta, tb, p);
+  count_launch();
+  return launch_status();
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bytes of MMA scale atoms for R expert-contiguous rows of K values: at most R/128 + E
+// row groups (one partial group per expert), K/128 atoms of 512 bytes each.
+size_t mma_atoms_bytes(int E, int R, int K) {
+  return align_up(((size_t)R / 128 + (size_t)E) * (size_t)(K / 128) * 512, 256);
+}
 
 GemmParams base_params(const int32_t* split_sizes, int E) {
   GemmParams p;
@@ -269,11 +296,14 @@ int moe_gather_slots(const float* src, const int32_t* row_map, int R, float* dst
   return launch_status();
 }
 
-int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out, uint8_t* codes,
-                   uint8_t* scales, void* stream) {
+int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out,
+                   int scale_layout, uint8_t* codes, uint8_t* scales, void* stream) {
   if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
   if (axis != 0 && axis != 1) return MOE_ERR_INVALID_ARG;
   if (axis == 0 && transpose_out) return MOE_ERR_INVALID_ARG;
+  if (scale_layout != MOE_SCALES_PLAIN && scale_layout != MOE_SCALES_MMA) return MOE_ERR_INVALID_ARG;
+  if (scale_layout == MOE_SCALES_MMA && !(axis == 1 && transpose_out)) return MOE_ERR_INVALID_ARG;
+  if (scale_layout == MOE_SCALES_MMA && ((rows % 128) || (cols % 128))) return MOE_ERR_UNSUPPORTED;
   if ((long long)batch * rows * cols == 0) return MOE_OK;
   if (!in || !codes || !scales) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
@@ -291,7 +321,7 @@ int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, 
     if (batch > 65535 || rows / 32 > 65535) return MOE_ERR_UNSUPPORTED;
     dim3 grid((cols + 255) / 256, rows / 32, batch);
     quant_cols_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in), rows, cols, transpose_out,
-                                            codes, scales);
+                                            scale_layout == MOE_SCALES_MMA, codes, scales);
   }
   count_launch();
   return launch_status();
@@ -301,8 +331,13 @@ size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int
   (void)E;
   (void)H;
   if (R < 0 || F < 0) return 0;
-  if (training) return 256;  // `a` lives in the saved buffer
-  if (precision == MOE_MXFP8) return align_up((size_t)R * F + (size_t)R * (F / 32), 256) + 256;
+  if (training && precision != MOE_MXFP8) return 256;  // `a` lives in the saved buffer
+  if (precision == MOE_MXFP8) {
+    // xp scale atoms, plus `a` codes and scale atoms unless they live in the saved buffer
+    const size_t xa = mma_atoms_bytes(E, R, H);
+    if (training) return xa + 256;
+    return xa + align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F) + 256;
+  }
   return align_up((size_t)R * F * 2, 256) + 256;
 }
 
@@ -310,26 +345,98 @@ size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision) {
   (void)E;
   (void)H;
   if (R < 0 || F < 0) return 0;
-  if (precision == MOE_MXFP8) return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
+  if (precision == MOE_MXFP8)
+    return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F);
   return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
 }
 
+}  // extern "C"
+
+namespace {
+
+int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H,
+                          int F, const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                          const float* probs_perm, void* yp, int out_f32, void* saved, void* ws, cudaStream_t st) {
+  if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  if (!xp_scale || !w1_scale || !w2_scale) return MOE_ERR_INVALID_ARG;
+  // workspace: xp scale atoms [, a codes, a scale atoms]; training keeps a in `saved`
+  uint8_t* xp_atoms = reinterpret_cast<uint8_t*>(ws);
+  uint8_t* a_codes = xp_atoms + mma_atoms_bytes(E, R, H);
+  uint16_t* h_buf = nullptr;
+  if (saved) {
+    h_buf = reinterpret_cast<uint16_t*>(saved);
+    a_codes = reinterpret_cast<uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256);
+  }
+  uint8_t* a_atoms = a_codes + align_up((size_t)R * F, 256);
+  {
+    const long long words = ((long long)R / 128 + E) * (H / 128) * 128;
+    const int grid = (int)std::min<long long>((words + 255) / 256, (long long)device_props().sm_count * 8);
+    scales_to_atoms_kernel<<<grid, 256, 2 * (E + 1) * sizeof(int32_t), st>>>(
+        xp_scale, split_sizes, E, H / 32, (long long)R / 128 + E, reinterpret_cast<uint32_t*>(xp_atoms));
+    count_launch();
+    int rc0 = launch_status();
+    if (rc0) return rc0;
+  }
+  CUtensorMap ta, tb;
+  int rc;
+  // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
+  if ((rc = tmap_u8_3d(&ta, xp, 1, R, H, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, w1, E, 2 * F, H, 128))) return rc;
+  MxGemmParams p1;
+  p1.g = base_params(split_sizes, E);
+  p1.g.M = R;
+  p1.g.N = F;
+  p1.g.K = H;
+  p1.g.out = a_codes;
+  p1.g.ldo = F;
+  p1.g.out2 = h_buf;
+  p1.g.ldo2 = 2 * F;
+  p1.g.probs = probs_perm;
+  p1.g.F = F;
+  p1.a_atoms = xp_atoms;
+  p1.b_atoms = w1_scale;
+  p1.b_rows = 2 * F;
+  p1.out_atoms = a_atoms;
+  if ((rc = launch_gemm_mx<MXEPI_SWIGLU_Q>(ta, tb, p1, st))) return rc;
+  // fc2: A = a codes [R, F], B = w2 codes [E, H, F]
+  if ((rc = tmap_u8_3d(&ta, a_codes, 1, R, F, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, w2, E, H, F, 128))) return rc;
+  MxGemmParams p2;
+  p2.g = base_params(split_sizes, E);
+  p2.g.M = R;
+  p2.g.N = H;
+  p2.g.K = F;
+  p2.g.out = yp;
+  p2.g.ldo = H;
+  p2.g.out_f32 = out_f32;
+  p2.a_atoms = a_atoms;
+  p2.b_atoms = w2_scale;
+  p2.b_rows = H;
+  p2.out_atoms = nullptr;
+  return launch_gemm_mx<MXEPI_STORE>(ta, tb, p2, st);
+}
+
+}  // namespace
+
+extern "C" {
+
 int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
                     const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
-                    const float* probs_perm, int precision, uint16_t* yp, void* saved, void* ws, size_t ws_bytes,
+                    const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
                     void* stream) {
-  (void)xp_scale;
-  (void)w1_scale;
-  (void)w2_scale;
+  const int out_f32 = (precision & MOE_OUT_F32) ? 1 : 0;
+  precision &= ~MOE_OUT_F32;
   if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
   if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
   if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
-  if (precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
   if (R == 0) return MOE_OK;
   if (!xp || !split_sizes || !w1 || !w2 || !yp || !ws) return MOE_ERR_INVALID_ARG;
   const int training = saved != nullptr;
   if (ws_bytes < grouped_mlp_workspace_size(E, R, H, F, precision, training)) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
+  if (precision == MOE_MXFP8)
+    return grouped_mlp_fwd_mxfp8(xp, xp_scale, split_sizes, E, R, H, F, w1, w1_scale, w2, w2_scale, probs_perm, yp,
+                                 out_f32, saved, ws, st);
 
   uint16_t* h_buf = nullptr;
   uint16_t* a_buf = reinterpret_cast<uint16_t*>(ws);
@@ -362,6 +469,7 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   p2.K = F;
   p2.out = yp;
   p2.ldo = H;
+  p2.out_f32 = out_f32;
   return launch_gemm<false, true, false, EPI_STORE>(ta, tb, p2, st);
 }
 

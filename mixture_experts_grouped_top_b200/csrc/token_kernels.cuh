@@ -360,6 +360,81 @@ __global__ void gather_slots_f32_kernel(const float* __restrict__ src, const int
   }
 }
 
+// ------------------------------------------------------ MMA scale-atom layout
+// The block-scaled MMA reads its scales from tensor memory, filled by tcgen05.cp from a
+// 512-byte shared-memory atom per 128 rows x 4 k-blocks (4 x 32 K values): row r of the
+// group is the 32-bit word (r % 32) * 4 + r / 32 and k-block kb its byte kb % 4. Keeping
+// scales in global memory already arranged as these atoms lets a GEMM stage fetch its
+// scales with one bulk copy per 128 rows. Atom (g, j) covers row group g and k-blocks
+// [4j, 4j+4); atoms of one row group are consecutive: offset (g * KB4 + j) * 512.
+__host__ __device__ __forceinline__ size_t mma_scale_offset(size_t group, int r, int kb, int kb4_per_row) {
+  return ((group * (size_t)kb4_per_row + (size_t)(kb >> 2)) * 128 + (size_t)((r & 31) * 4 + (r >> 5))) * 4 +
+         (size_t)(kb & 3);
+}
+
+// Plain [R, K/32] scales of expert-contiguous rows -> MMA atoms grouped per expert tile:
+// row group g = (sum over e' < e of ceil(n_e' / 128)) + m for rows [off_e + 128 m, +128) of
+// expert e; rows past the expert's end get zero scales. One thread per (group, row,
+// 4-k-block word). Each block rebuilds the expert prefix tables from split_sizes.
+__global__ void __launch_bounds__(256) scales_to_atoms_kernel(const uint8_t* __restrict__ plain,
+                                                              const int32_t* __restrict__ split_sizes, int E, int KS,
+                                                              long long max_groups, uint32_t* __restrict__ atoms) {
+  extern __shared__ int32_t tabs[];   // [E+1] row offsets, [E+1] group offsets
+  int32_t* roff = tabs;
+  int32_t* goff = tabs + E + 1;
+  if (threadIdx.x < 32) {   // warp prefix sums of split_sizes and of their 128-row groups
+    const int lane = threadIdx.x;
+    int cr = 0, cg = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? split_sizes[e] : 0;
+      const int gn = (n + 127) / 128;
+      int ir = n, ig = gn;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yg = __shfl_up_sync(0xffffffffu, ig, o);
+        if (lane >= o) {
+          ir += yr;
+          ig += yg;
+        }
+      }
+      if (e < E) {
+        roff[e] = cr + ir - n;
+        goff[e] = cg + ig - gn;
+      }
+      cr += __shfl_sync(0xffffffffu, ir, 31);
+      cg += __shfl_sync(0xffffffffu, ig, 31);
+    }
+    if (lane == 0) {
+      roff[E] = cr;
+      goff[E] = cg;
+    }
+  }
+  __syncthreads();
+  const int KB4 = KS / 4;
+  const long long total = (long long)goff[E] * KB4 * 128;
+  (void)max_groups;
+  for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < total;
+       w += (long long)gridDim.x * blockDim.x) {
+    const int word = (int)(w % 128);
+    const long long gj = w / 128;
+    const int j = (int)(gj % KB4);
+    const int g = (int)(gj / KB4);
+    int lo = 0, hi = E - 1;   // expert whose groups contain g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (goff[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int r = (word & 3) * 32 + (word >> 2);   // inverse of (r % 32) * 4 + r / 32
+    const int l = (g - goff[e]) * 128 + r;
+    uint32_t v = 0;
+    if (l < roff[e + 1] - roff[e]) v = *reinterpret_cast<const uint32_t*>(plain + (size_t)(roff[e] + l) * KS + 4 * j);
+    atoms[w] = v;
+  }
+}
+
 // ------------------------------------------------------------ MXFP8 quantiser
 // axis 0: blocks of 32 along the columns of each row. 4 lanes per block.
 __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ in, long long nvec, int cols,
@@ -384,7 +459,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
 // transpose_out: codes [cols, rows], scales [cols, rows/32]; else codes [rows, cols],
 // scales [rows/32, cols].
 __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols,
-                                                         int transpose_out, uint8_t* __restrict__ codes,
+                                                         int transpose_out, int mma_scales,
+                                                         uint8_t* __restrict__ codes,
                                                          uint8_t* __restrict__ scales) {
   __shared__ __align__(16) uint8_t tile[32][256 + 16];
   const int b = blockIdx.z;
@@ -421,7 +497,12 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __
       uint4* o = reinterpret_cast<uint4*>(dst + (size_t)c * rows + r0);
       o[0] = make_uint4(w[0], w[1], w[2], w[3]);
       o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      sdst[(size_t)c * (rows / 32) + (r0 / 32)] = (uint8_t)code;
+      if (mma_scales) {
+        // scale atoms of the transposed matrix [cols, rows]: see mma_scale_offset
+        scales[mma_scale_offset((size_t)b * (cols / 128) + c / 128, c % 128, r0 / 32, rows / 128)] = (uint8_t)code;
+      } else {
+        sdst[(size_t)c * (rows / 32) + (r0 / 32)] = (uint8_t)code;
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {

@@ -57,8 +57,8 @@ class MoEExpertLayer:
         if self.prec == BF16:
             self.w1, self.w2 = w1, w2
         else:
-            self.w1, self.w1_scale = mxfp8_quantize(w1, axis=1, transpose_out=True, stream=stream)
-            self.w2, self.w2_scale = mxfp8_quantize(w2, axis=1, transpose_out=True, stream=stream)
+            self.w1, self.w1_scale = mxfp8_quantize(w1, axis=1, transpose_out=True, mma_scales=True, stream=stream)
+            self.w2, self.w2_scale = mxfp8_quantize(w2, axis=1, transpose_out=True, mma_scales=True, stream=stream)
 
     # --------------------------------------------------------------- forward
     def forward(self, x: torch.Tensor, logits: torch.Tensor, stream=None) -> torch.Tensor:

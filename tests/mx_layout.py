@@ -1,0 +1,33 @@
+"""Test-side conversion between the plain [rows, K/32] scale grid and the MMA atom layout
+(512-byte atoms of 128 rows x 4 k-blocks; row r is word (r % 32) * 4 + r // 32)."""
+import numpy as np
+
+_WORD = np.array([(r % 32) * 4 + r // 32 for r in range(128)])
+
+
+def plain_to_atoms(plain):
+    """[G*128, KS] uint8 -> flat atoms (row group g = row // 128)."""
+    plain = np.asarray(plain, dtype=np.uint8)
+    rows, ks = plain.shape
+    g, kb4 = rows // 128, ks // 4
+    src = plain.reshape(g, 128, kb4, 4).transpose(0, 2, 1, 3)          # [g, j, r, byte]
+    out = np.empty((g, kb4, 128, 4), dtype=np.uint8)
+    out[:, :, _WORD, :] = src
+    return out.reshape(-1)
+
+
+def atoms_to_plain(atoms, groups, ks):
+    a = np.asarray(atoms, dtype=np.uint8)[: groups * (ks // 4) * 512].reshape(groups, ks // 4, 128, 4)
+    return a[:, :, _WORD, :].transpose(0, 2, 1, 3).reshape(groups * 128, ks)
+
+
+def tile_atoms_to_plain(atoms, split_sizes, ks):
+    """Atoms whose row groups are each expert's 128-row tiles -> plain [R, ks] (tails dropped)."""
+    split = [int(n) for n in split_sizes]
+    groups = sum((n + 127) // 128 for n in split)
+    padded = atoms_to_plain(atoms, groups, ks)
+    out, g = [], 0
+    for n in split:
+        out.append(padded[g * 128: g * 128 + n])
+        g += (n + 127) // 128
+    return np.concatenate(out) if out else np.zeros((0, ks), np.uint8), padded, groups

@@ -66,8 +66,10 @@ def test_other_entry_points_reject_bad_arguments():
                              None, 0, None) == 1                                       # E = 0
     assert h.grouped_mlp_bwd(None, None, 4, 16, 128, 256, None, None, None, None, 1, None, None, None, None,
                              None, None, 0, None) == 2                                 # MXFP8 backward
-    assert h.mxfp8_quantize(None, 1, 4, 33, 0, 0, None, None, None) == 1               # null input
-    assert h.mxfp8_quantize(None, 1, 4, 64, 0, 1, None, None, None) == 1               # transpose with axis 0
+    assert h.mxfp8_quantize(None, 1, 4, 33, 0, 0, 0, None, None, None) == 1            # null input
+    assert h.mxfp8_quantize(None, 1, 4, 64, 0, 1, 0, None, None, None) == 1            # transpose with axis 0
+    assert h.mxfp8_quantize(None, 1, 128, 128, 0, 0, 1, None, None, None) == 1         # MMA scales need axis 1
+    assert h.mxfp8_quantize(None, 1, 96, 128, 1, 1, 1, None, None, None) == 2          # ... and 128-multiples
     assert h.moe_unpermute(None, None, None, 4, 12, 2, None, None) == 1                # H % 8
     assert h.moe_permute(None, None, None, 4, 64, 4, 8, 0, None, None, None, None, None, None, None, 0,
                          None) == 1                                                    # k > E
@@ -77,7 +79,7 @@ def test_zero_token_calls_are_noops():
     h = moe_b200.lib()
     assert h.moe_route(None, 0, 4, 2, 1, None, None, None) == 0
     assert h.moe_unpermute(None, None, None, 0, 64, 2, None, None) == 0
-    assert h.mxfp8_quantize(None, 0, 32, 64, 1, 1, None, None, None) == 0
+    assert h.mxfp8_quantize(None, 0, 32, 64, 1, 1, 0, None, None, None) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

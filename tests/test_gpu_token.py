@@ -132,6 +132,17 @@ def test_quantize_axis1_bit_exact(B, rows, cols, transpose):
     _status_ok()
 
 
+@pytest.mark.parametrize("B,rows,cols", [(2, 128, 256), (3, 256, 384), (8, 512, 128)])
+def test_quantize_mma_scale_layout_bit_exact(B, rows, cols):
+    from tests.mx_layout import plain_to_atoms
+    rng = np.random.default_rng(rows + 7 * cols)
+    x = torch.from_numpy((rng.standard_normal((B, rows, cols), dtype=np.float32) * 0.02)).to(torch.bfloat16)
+    codes, atoms = mb.mxfp8_quantize(x.to(DEV), axis=1, transpose_out=True, mma_scales=True)
+    rc, rs = oq.quantize(om.f64(x), axis=1, transpose_out=True)          # [B, cols, rows], [B, cols, rows/32]
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(atoms.cpu().numpy(), plain_to_atoms(rs.reshape(B * cols, rows // 32)))
+
+
 def test_quantize_golden_block_and_edges():
     # the hand-worked block of tests/golden/mxfp8_block.txt (values exact in bf16 except 0.1)
     from tests.golden import load
