@@ -152,6 +152,8 @@ def run_ours(args, world, rank, local):
     w1, w2 = d["w1"].to(dev), d["w2"].to(dev)
     layer.set_weights(w1, w2)
     x, logits = d["x"].to(dev), d["logits"].to(dev)
+    if cfg.passes == "fwd+bwd" and cfg.precision == "mxfp8":
+        layer.xp_bf16 = torch.empty((cfg.R, cfg.H), dtype=torch.bfloat16, device=dev)
     grad = d["grad_out"].to(dev) if "grad_out" in d else None
     stream = torch.cuda.current_stream(dev)
     prec = cfg.precision
@@ -160,6 +162,8 @@ def run_ours(args, world, rank, local):
 
     def step(ev=None):
         """One pass of the path; `ev` = 4 events bracketing the grouped-GEMM calls."""
+        if training and prec == "mxfp8":
+            layer.set_weights(w1, w2)   # a training step re-quantises the bf16 masters
         mb.moe_route(logits, cfg.k, True, idx=layer.idx, prob=layer.prob)
         mb.moe_permute(x, layer.idx, layer.prob, cfg.E, prec, out=layer.perm, workspace=layer.perm_ws)
         if ev is not None:
@@ -178,7 +182,10 @@ def run_ours(args, world, rank, local):
             mb.moe_permute_rows(grad, layer.perm["row_map"], cfg.k, out=b["dy_perm"])
             if ev is not None:
                 ev[2].record(stream)
-            mb.grouped_mlp_bwd(b["dy_perm"], layer.perm["split_sizes"], layer.perm["xp"], layer.w1, layer.w2,
+            if prec == "mxfp8":
+                mb.moe_permute_rows(x, layer.perm["row_map"], cfg.k, out=layer.xp_bf16)
+            xp_b = layer.perm["xp"] if prec == "bf16" else layer.xp_bf16
+            mb.grouped_mlp_bwd(b["dy_perm"], layer.perm["split_sizes"], xp_b, w1, w2,
                                layer.perm["probs_perm"], layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"], dw2=b["dw2"],
                                dprobs_perm=b["dprobs_perm"], workspace=b["ws"])
             if ev is not None:

@@ -177,8 +177,9 @@ MOE_API int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const floa
  *           transpose_out = 1: codes [batch, cols, rows], scales [batch, cols, rows/32]
  *             (the transposed matrix quantised along its rows: K-major weights);
  *           transpose_out = 0: codes [batch, rows, cols], scales [batch, rows/32, cols].
- *   scale_layout: MOE_SCALES_PLAIN, or MOE_SCALES_MMA (axis 1 with transpose_out only;
- *           rows and cols multiples of 128) for weights handed to grouped_mlp_fwd.
+ *   scale_layout: MOE_SCALES_PLAIN, or MOE_SCALES_MMA (axis 1 with transpose_out, or
+ *           axis 0 without; rows and cols multiples of 128) for weights handed to the
+ *           block-scaled GEMMs.
  */
 MOE_API int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, int transpose_out,
                            int scale_layout, uint8_t* codes, uint8_t* scales, void* stream);
@@ -222,26 +223,56 @@ MOE_API int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32
                     const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
                     void* stream);
 
-/* Bytes of scratch grouped_mlp_bwd needs (dh [R, 2F] bf16 and dprob partial sums). */
+/* Bytes of scratch grouped_mlp_bwd needs: dh [R, 2F] bf16 and dprob partial sums; for
+ * MOE_MXFP8 also the recomputed a [R, F] bf16 and every quantised GEMM operand. */
 MOE_API size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision);
+
+/* Byte offset, inside grouped_mlp_bwd's workspace, of part 0 (dh = [dg | du] [R, 2F]
+ * bf16) or part 1 (MOE_MXFP8 only: the recomputed a [R, F] bf16); (size_t)-1 otherwise.
+ * The parts hold the last call's values after it completes. */
+MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part);
 
 /*
  * grouped_mlp_bwd — backward of grouped_mlp_fwd (the "counterpart in the backward
  * pass" of sitech.ge "Reducing memory and quantisation cost").
- * For every expert e (a = SiLU(g) * u * p, with g, u, a from `saved`):
+ * For every expert e (a = SiLU(g) * u * p, with g, u from `saved`):
  *   da = dy_e @ w2[e]^T;  dg = da*p*u*SiLU'(g);  du = da*p*SiLU(g);
  *   dprobs_perm = sum_f da*SiLU(g)*u;  dw2[e] = a_e^T @ dy_e;
  *   dxp_e = [dg | du] @ w1[e]^T;  dw1[e] = xp_e^T @ [dg | du].
  * dy_perm [R, H] bf16 (the layer-output gradient permuted with moe_permute_rows);
- * xp [R, H] bf16; w1 [E, H, 2F] bf16; w2 [E, F, H] bf16; probs_perm [R] fp32 or NULL;
- * saved: the buffer filled by grouped_mlp_fwd in training mode.
+ * xp [R, H] bf16 (the permuted layer input, bf16 also on the MXFP8 path);
+ * w1 [E, H, 2F] bf16; w2 [E, F, H] bf16 (the masters); probs_perm [R] fp32 or NULL;
+ * saved: the buffer filled by grouped_mlp_fwd in training mode (same precision).
  * Outputs: dxp [R, H] bf16, dw1 [E, H, 2F] bf16, dw2 [E, F, H] bf16 (experts with no rows
- * get zeros), dprobs_perm [R] fp32 (may be NULL). Only MOE_BF16 is supported.
+ * get zeros), dprobs_perm [R] fp32 (may be NULL).
+ * MOE_MXFP8: all four GEMMs run on MXFP8 operands quantised along their own contraction
+ * axis (blocks of 32): dy and dh along columns for the data gradients, and dy, a
+ * (recomputed from h), dh and xp along rows — in 32-row blocks restarting at every
+ * expert's first row — for the weight gradients; the weights are re-quantised along
+ * their other axis. Requires H % 128 == 0 for MOE_MXFP8.
  */
-MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
-                    const void* w1, const void* w2, const float* probs_perm, int precision, const void* saved,
-                    uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws, size_t ws_bytes,
-                    void* stream);
+MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
+                            const void* xp, const void* w1, const void* w2, const float* probs_perm, int precision,
+                            const void* saved, uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * mxfp8_quantize_grouped — MXFP8 quantisation of expert-contiguous rows along the rows:
+ * for every column, blocks of 32 consecutive rows that restart at each expert's first row
+ * (the last block of an expert covers its remaining rows, as if zero-padded). This is the
+ * operand layout of the weight-gradient GEMMs (contraction over an expert's rows).
+ *   in [R, C] bf16, C % 128 == 0; split_sizes [E] on the device (sum = R);
+ *   codes [R, C] E4M3 (same layout as in);
+ *   atoms: scales in the MMA atom layout, numbered per expert: expert e owns
+ *     KG_e = ceil(n_e/128) k-groups; the atom of column group cg (128 columns) and k-group
+ *     kg sits at byte (kgoff_e * C/128 + cg * KG_e + kg) * 512, kgoff_e = sum of KG over
+ *     earlier experts; inside an atom, column c's word is (c % 32) * 4 + (c % 128) / 32
+ *     and block j its byte j % 4; bytes of blocks past an expert's end are zero.
+ *     Size: mxfp8_grouped_atoms_bytes(E, R, C).
+ */
+MOE_API int mxfp8_quantize_grouped(const uint16_t* in, int R, int C, const int32_t* split_sizes, int E,
+                                   uint8_t* codes, uint8_t* atoms, void* stream);
+MOE_API size_t mxfp8_grouped_atoms_bytes(int E, int R, int C);
 
 /*
  * moe_gather_slots — dst[s] = src[row_map[s]] for s < R (fp32): brings per-row values

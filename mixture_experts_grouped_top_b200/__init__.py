@@ -193,6 +193,20 @@ def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, sc
     return codes, scales
 
 
+def mxfp8_quantize_grouped(x, split_sizes, codes=None, atoms=None, stream=None):
+    """Quantise expert-contiguous rows x [R, C] along the rows (32-row blocks restarting
+    at every expert). Returns (codes [R, C] uint8, scale atoms (flat uint8))."""
+    _need(x, torch.bfloat16, "x")
+    R, C = x.shape
+    E = split_sizes.numel()
+    codes = torch.empty((R, C), dtype=torch.uint8, device=x.device) if codes is None else codes
+    if atoms is None:
+        atoms = torch.zeros(int(lib().mxfp8_grouped_atoms_bytes(E, R, C)), dtype=torch.uint8, device=x.device)
+    _check("mxfp8_quantize_grouped", lib().mxfp8_quantize_grouped(_p(x), R, C, _p(split_sizes), E, _p(codes),
+                                                                   _p(atoms), _stream(stream)))
+    return codes, atoms
+
+
 # ------------------------------------------------------------- grouped expert MLP
 def grouped_mlp_workspace_size(E, R, H, F, precision="bf16", training=False) -> int:
     return int(lib().grouped_mlp_workspace_size(E, R, H, F, _PREC[precision], int(bool(training))))
@@ -236,9 +250,14 @@ def grouped_mlp_bwd_workspace_size(E, R, H, F, precision="bf16") -> int:
     return int(lib().grouped_mlp_bwd_workspace_size(E, R, H, F, _PREC[precision]))
 
 
+def grouped_mlp_bwd_workspace_offset(E, R, H, F, precision, part) -> int:
+    return int(lib().grouped_mlp_bwd_workspace_offset(E, R, H, F, _PREC[precision], part))
+
+
 def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precision="bf16", dxp=None, dw1=None,
                     dw2=None, dprobs_perm=None, workspace=None, stream=None):
-    """Backward of grouped_mlp_fwd. Returns (dxp, dw1, dw2, dprobs_perm)."""
+    """Backward of grouped_mlp_fwd. Returns (dxp, dw1, dw2, dprobs_perm). xp, w1 and w2
+    are bf16 on both paths (the MXFP8 path quantises what it needs)."""
     prec = _PREC[precision]
     R, H = dy_perm.shape
     E = split_sizes.numel()

@@ -29,6 +29,9 @@ SIGNATURES = {
     "grouped_mlp_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "grouped_mlp_bwd": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                              _vp]),
+    "grouped_mlp_bwd_workspace_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "mxfp8_quantize_grouped": (_i, [_vp, _i, _i, _vp, _i, _vp, _vp, _vp]),
+    "mxfp8_grouped_atoms_bytes": (_sz, [_i, _i, _i]),
     "moe_gather_slots": (_i, [_vp, _vp, _i, _vp, _vp]),
 }
 

@@ -43,23 +43,28 @@ constexpr uint32_t kAcc1Col = 224;
 constexpr uint32_t kSfaCol = 480;
 constexpr uint32_t kSfbCol = 484;
 constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kStages * (kSfaBytes + kSfbBytes) + 1024 +
-                           2 * (kMaxE + 1) * 4;
+                           3 * (kMaxE + 1) * 4;
 }  // namespace mx
 
 enum MxEpiKind : int {
-  MXEPI_STORE = 0,      // out[row, col] = bf16(acc)
+  MXEPI_STORE = 0,      // out[row, col] = bf16(acc) (fp32 with out_f32)
   MXEPI_SWIGLU_Q = 1,   // a = SiLU(g) * u * p quantised to MXFP8 along the columns (+ bf16 h)
+  MXEPI_DSWIGLU = 2,    // SwiGLU backward from da = acc and the saved h: dh, recomputed a (bf16), dprob partials
+  MXEPI_WGRAD = 3,      // K-grouped: out[e, m, n] = bf16(acc), zeros for an expert without rows
 };
 
 struct MxGemmParams {
   GemmParams g;               // E, M (rows R), N (output cols), K, split_sizes, out, ldo, out2/ldo2 (h), probs, F
-  const uint8_t* a_atoms;     // A scales as atoms, row groups = expert tiles (sum of ceil(n_e/128))
-  const uint8_t* b_atoms;     // B scales as atoms, row groups = e * (b_rows / 128) + row / 128
+  // M-grouped: A scale atoms grouped per expert tile (sum of ceil(n_e/128)), B scale atoms
+  // grouped e * (b_rows / 128) + row / 128. K-grouped (MN-major codes [R, M] and [R, N]):
+  // atoms per expert, k-group and column group, as quant_cols_grouped_kernel writes them.
+  const uint8_t* a_atoms;
+  const uint8_t* b_atoms;
   int b_rows;                 // rows of each expert's B (2F for fc1, H for fc2)
   uint8_t* out_atoms;         // MXEPI_SWIGLU_Q: scales of `a` as atoms for the next GEMM (K = F)
 };
 
-template <int EPI>
+template <bool KGROUP, int EPI>
 __global__ void __launch_bounds__(mx::kThreads, 1)
     grouped_gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const MxGemmParams mp) {
@@ -81,10 +86,12 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
+  int32_t* kg_off = tile_off + (kMaxE + 1);   // K-grouped: k-groups (128 rows) of earlier experts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
   const int NT = (EPI == MXEPI_SWIGLU_Q) ? (p.N / 128) : (p.N + BN - 1) / BN;
+  const int MT = KGROUP ? (p.M + BM - 1) / BM : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -104,31 +111,37 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 3) {
-    int carry_r = 0, carry_t = 0;
+    int carry_r = 0, carry_t = 0, carry_k = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
       const int n = (e < E) ? p.split_sizes[e] : 0;
-      const int tiles = (e < E) ? ((n + BM - 1) / BM) * NT : 0;
-      int ir = n, it = tiles;
+      const int tiles = (e < E) ? (KGROUP ? MT * NT : ((n + BM - 1) / BM) * NT) : 0;
+      const int kgs = (n + BK - 1) / BK;
+      int ir = n, it = tiles, ik = kgs;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int yr = __shfl_up_sync(0xffffffffu, ir, o);
         const int yt = __shfl_up_sync(0xffffffffu, it, o);
+        const int yk = __shfl_up_sync(0xffffffffu, ik, o);
         if (lane >= o) {
           ir += yr;
           it += yt;
+          ik += yk;
         }
       }
       if (e < E) {
         row_off[e] = carry_r + ir - n;
         tile_off[e] = carry_t + it - tiles;
+        kg_off[e] = carry_k + ik - kgs;
       }
       carry_r += __shfl_sync(0xffffffffu, ir, 31);
       carry_t += __shfl_sync(0xffffffffu, it, 31);
+      carry_k += __shfl_sync(0xffffffffu, ik, 31);
     }
     if (lane == 0) {
       row_off[E] = carry_r;
       tile_off[E] = carry_t;
+      kg_off[E] = carry_k;
     }
   }
   if (warp == 2) {
@@ -140,9 +153,9 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  TileWalker<false> walk{row_off, tile_off, E, 0, NT, p.K};
+  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K};
   // the walker's k-block count assumes 64-wide blocks; MXFP8 uses 128-wide ones
-  const int num_kb = p.K / BK;
+  auto kblocks = [&](const TileInfo& ti) { return KGROUP ? (ti.rows + BK - 1) / BK : p.K / BK; };
   const int total = walk.total();
 
   if (warp == 0) {
@@ -152,15 +165,24 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      const int KB4 = p.K / 128;
+      const int KB4 = KGROUP ? 0 : p.K / 128;
       const int bgroups = mp.b_rows / 128;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const TileInfo ti = walk.decode(t);
+        const int num_kb = kblocks(ti);
         const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
-        const size_t ga = (size_t)(tile_off[ti.e] / NT + ti.m_blk);          // A row group (expert tile)
-        const size_t gb0 = (size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? n0 / 128 : n0 / 128);
-        size_t gb1 = (size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? (p.F + n0) / 128 : n0 / 128 + 1);
-        if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+        size_t ga, gb0, gb1;   // first atom of A's and of B's two 128-row halves (k-group 0)
+        if (KGROUP) {
+          const size_t kg = (size_t)(ti.rows + BK - 1) / BK;
+          ga = (size_t)kg_off[ti.e] * (p.M / 128) + (size_t)ti.m_blk * kg;
+          gb0 = (size_t)kg_off[ti.e] * (p.N / 128) + (size_t)(n0 / 128) * kg;
+          gb1 = (n0 + 128 < p.N) ? gb0 + kg : gb0;
+        } else {
+          ga = (size_t)(tile_off[ti.e] / NT + ti.m_blk) * KB4;          // A row group (expert tile)
+          gb0 = ((size_t)ti.e * bgroups + n0 / 128) * KB4;
+          gb1 = ((size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? (p.F + n0) / 128 : n0 / 128 + 1)) * KB4;
+          if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+        }
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
             ok = false;
@@ -168,18 +190,20 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           }
           const int k0 = kb * BK;
           mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes + kSfaBytes + kSfbBytes);
-          tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
           uint8_t* b_dst = sB + stage * kBBytes;
-          if (EPI == MXEPI_SWIGLU_Q) {
-            tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
-            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, p.F + n0, ti.e);
+          if (KGROUP) {
+            // MN-major codes: box {128 columns, 128 rows} at the expert's k-th row block
+            tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], ti.m_blk * BM, ti.row0 + k0, 0);
+            tma_load_3d(b_dst, &tmB, &full[stage], n0, ti.row0 + k0, 0);
+            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], n0 + 128, ti.row0 + k0, 0);
           } else {
+            tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
             tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
-            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, n0 + 128, ti.e);
+            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, EPI == MXEPI_SWIGLU_Q ? p.F + n0 : n0 + 128, ti.e);
           }
-          bulk_load(sSfa + stage * kSfaBytes, mp.a_atoms + (ga * KB4 + kb) * 512, 512, &full[stage]);
-          bulk_load(sSfb + stage * kSfbBytes, mp.b_atoms + (gb0 * KB4 + kb) * 512, 512, &full[stage]);
-          bulk_load(sSfb + stage * kSfbBytes + 512, mp.b_atoms + (gb1 * KB4 + kb) * 512, 512, &full[stage]);
+          bulk_load(sSfa + stage * kSfaBytes, mp.a_atoms + (ga + kb) * 512, 512, &full[stage]);
+          bulk_load(sSfb + stage * kSfbBytes, mp.b_atoms + (gb0 + kb) * 512, 512, &full[stage]);
+          bulk_load(sSfb + stage * kSfbBytes + 512, mp.b_atoms + (gb1 + kb) * 512, 512, &full[stage]);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -209,6 +233,8 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
     const uint32_t sfa_t = tmem_base + kSfaCol;
     const uint32_t sfb_t = tmem_base + kSfbCol;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      const TileInfo ti = walk.decode(t);
+      const int num_kb = kblocks(ti);
       const int acc = lt & 1;
       if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
       if (lt > 0 && !mbar_wait_bounded(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
@@ -220,6 +246,18 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           break;
         }
         tc_fence_after();
+        if (KGROUP && (kb + 1) * BK > ti.rows) {
+          // clip the contraction at the expert's last row: zero K-rows >= valid (128-byte lines)
+          const int valid = ti.rows - kb * BK;
+          const int per = (BK - valid) * 8;   // 16-byte vectors per 128-row operand block
+          for (int i = lane; i < 3 * per; i += 32) {
+            const int blk = i / per, r = i % per;
+            uint8_t* base = (blk == 0) ? sA + stage * kABytes : sB + stage * kBBytes + (blk - 1) * BM * BK;
+            *reinterpret_cast<uint4*>(base + valid * 128 + r * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
         if (lane == 0) {
           const uint32_t sfa_s = smem_u32(sSfa + stage * kSfaBytes);
           const uint32_t sfb_s = smem_u32(sSfb + stage * kSfbBytes);
@@ -230,9 +268,13 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
-            const uint64_t adesc = make_sdesc(a_addr + kk * 32, 16, 1024, 2);
-            const uint64_t bdesc = make_sdesc(b_addr + kk * 32, 16, 1024, 2);
-            const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk);
+            // K-major: next 32 K values are 32 bytes further in each 128-byte row;
+            // MN-major: 32 rows further (4 x 8-row swizzle atoms), halves of B 16 KB apart
+            const uint64_t adesc = KGROUP ? make_sdesc(a_addr + kk * 4096, BM * BK, 1024, 2)
+                                          : make_sdesc(a_addr + kk * 32, 16, 1024, 2);
+            const uint64_t bdesc = KGROUP ? make_sdesc(b_addr + kk * 4096, BM * BK, 1024, 2)
+                                          : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
+            const uint32_t idesc = make_idesc_mxf8(BM, BN, KGROUP, KGROUP, kk, kk);
             mma_mxf8_ss(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30),
                         (kb > 0 || kk > 0) ? 1u : 0u);
           }
@@ -245,7 +287,12 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
         }
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(&tfull[acc]);
+      if (lane == 0) {
+        if (num_kb > 0)
+          mma_commit(&tfull[acc]);
+        else
+          mbar_arrive(&tfull[acc]);
+      }
       __syncwarp();
     }
   } else if (warp >= 4) {
@@ -263,9 +310,21 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       const long long row = ti.row0 + r_local;
       uint32_t sc_word = 0;   // SwiGLU: this row's four scale bytes (k-blocks 4*n_blk..+3 of the next GEMM)
 
-      if (EPI == MXEPI_STORE) {
+      if (EPI == MXEPI_STORE || EPI == MXEPI_WGRAD) {
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const int n0 = ti.n_blk * BN;
+        long long orow;
+        bool ok_row;
+        bool zero = false;
+        if (EPI == MXEPI_WGRAD) {
+          const int m = ti.m_blk * BM + r_local;
+          ok_row = m < p.M;
+          orow = (long long)ti.e * p.out_batch + (long long)m * p.ldo;
+          zero = ti.rows == 0;
+        } else {
+          ok_row = row_ok;
+          orow = row * p.ldo;
+        }
         const int first = acc ? 0 : 7;   // the 32-column strip shared with the other accumulator
 #pragma unroll 1
         for (int it = 0; it < 8; ++it) {
@@ -278,26 +337,95 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
             tc_fence_before();
             mbar_arrive(tovl);
           }
-          if (row_ok && n0 + c * 32 < p.N && p.out_f32) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + row * p.ldo + n0 + c * 32);
+          if (ok_row && n0 + c * 32 < p.N && p.out_f32) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               dst[i] = make_uint4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
               dst[4 + i] = make_uint4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
             }
-          } else if (row_ok && n0 + c * 32 < p.N) {
+          } else if (ok_row && n0 + c * 32 < p.N) {
             uint4 o[4];
             uint32_t* ow = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              ow[i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-              ow[8 + i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+              ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+              ow[8 + i] = zero ? 0u : pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
             }
-            uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = o[i];
           }
         }
+      } else if (EPI == MXEPI_DSWIGLU) {
+        // acc = da for columns [n0, n0+256) of F. With h = [g | u] from the forward:
+        // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u; a = SiLU(g) u p is
+        // recomputed (bf16) for the fc2 weight gradient.
+        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
+        __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
+        __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        const int n0 = ti.n_blk * BN;
+        const int first = acc ? 0 : 7;
+        float dp = 0.f;
+#pragma unroll 1
+        for (int it = 0; it < 8; ++it) {
+          const int c = (it == 0) ? first : (acc ? it : it - 1);
+          uint32_t v0[16], v1[16];
+          tmem_ld_32x32b_x16(t_row + c * 32, v0);
+          tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
+          tmem_wait_ld();
+          if (it == 0) {
+            tc_fence_before();
+            mbar_arrive(tovl);
+          }
+          const int col = n0 + c * 32;
+          if (row_ok && col < p.N) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const int cc = col + 16 * half;
+              const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + cc);
+              const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + cc);
+              uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
+              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
+              const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
+              uint4 og[2], ou[2], oa[2];
+              uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
+              uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
+              uint32_t* oaw = reinterpret_cast<uint32_t*>(oa);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float2 gg2 = __bfloat1622float2(g2[i]);
+                const float2 uu2 = __bfloat1622float2(u2[i]);
+                const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
+                float dg[2], du[2], av[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const float da = __uint_as_float(half ? v1[2 * i + j] : v0[2 * i + j]);
+                  const float sg = 1.0f / (1.0f + expf(-gs[j]));
+                  const float sl = gs[j] * sg;
+                  dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+                  du[j] = da * pr * sl;
+                  av[j] = sl * us[j] * pr;
+                  dp = fmaf(da, sl * us[j], dp);
+                }
+                ogw[i] = pack_bf16x2(dg[0], dg[1]);
+                ouw[i] = pack_bf16x2(du[0], du[1]);
+                oaw[i] = pack_bf16x2(av[0], av[1]);
+              }
+              uint4* d0 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + cc);
+              uint4* d1 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + cc);
+              uint4* d2 = reinterpret_cast<uint4*>(a_out + row * p.ldo + cc);
+              d0[0] = og[0];
+              d0[1] = og[1];
+              d1[0] = ou[0];
+              d1[1] = ou[1];
+              d2[0] = oa[0];
+              d2[1] = oa[1];
+            }
+          }
+        }
+        if (row_ok) p.dprob_part[(long long)ti.n_blk * p.M + row] = dp;
       } else {
         // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
         const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;

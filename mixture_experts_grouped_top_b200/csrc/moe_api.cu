@@ -118,9 +118,9 @@ int tmap_u8_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, u
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, cols, rows, batch, cols, rows * cols, 128, box_rows);
 }
 
-template <int EPI>
+template <bool KG, int EPI>
 int launch_gemm_mx(const CUtensorMap& ta, const CUtensorMap& tb, const MxGemmParams& p, cudaStream_t st) {
-  auto kern = grouped_gemm_mxf8_kernel<EPI>;
+  auto kern = grouped_gemm_mxf8_kernel<KG, EPI>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&]() {
@@ -135,11 +135,48 @@ int launch_gemm_mx(const CUtensorMap& ta, const CUtensorMap& tb, const MxGemmPar
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+int quant_rows_launch(const void* in, long long rows, int cols, int mma, uint8_t* codes, uint8_t* scales,
+                      cudaStream_t st) {
+  const long long nvec = rows * cols / 8;
+  const int grid = (int)std::min<long long>((nvec + 255) / 256, (long long)device_props().sm_count * 16);
+  quant_rows_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(in), nvec, cols, mma, codes, scales);
+  count_launch();
+  return launch_status();
+}
+
+int quant_cols_grouped_launch(const void* in, int R, int C, const int32_t* split_sizes, int E, uint8_t* codes,
+                              uint8_t* atoms, cudaStream_t st) {
+  const int blocks32 = R / 32 + E;   // upper bound of sum(ceil(n_e / 32))
+  dim3 grid(std::min(blocks32, device_props().sm_count * 32), (C + 255) / 256);
+  quant_cols_grouped_kernel<<<grid, 256, 3 * (E + 1) * sizeof(int32_t), st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(in), C, split_sizes, E, codes, atoms);
+  count_launch();
+  return launch_status();
+}
+
+int scales_to_atoms_launch(const uint8_t* plain, const int32_t* split_sizes, int E, int R, int K, uint8_t* atoms,
+                           cudaStream_t st) {
+  const long long words = ((long long)R / 128 + E) * (K / 128) * 128;
+  const int grid = (int)std::min<long long>((words + 255) / 256, (long long)device_props().sm_count * 8);
+  scales_to_atoms_kernel<<<grid, 256, 2 * (E + 1) * sizeof(int32_t), st>>>(
+      plain, split_sizes, E, K / 32, (long long)R / 128 + E, reinterpret_cast<uint32_t*>(atoms));
+  count_launch();
+  return launch_status();
+}
+
 // Bytes of MMA scale atoms for R expert-contiguous rows of K values: at most R/128 + E
 // row groups (one partial group per expert), K/128 atoms of 512 bytes each.
 size_t mma_atoms_bytes(int E, int R, int K) {
   return align_up(((size_t)R / 128 + (size_t)E) * (size_t)(K / 128) * 512, 256);
 }
+
+// Launch helpers used by the MXFP8 backward (all asynchronous on `st`).
+int quant_rows_launch(const void* in, long long rows, int cols, int mma, uint8_t* codes, uint8_t* scales,
+                      cudaStream_t st);
+int quant_cols_grouped_launch(const void* in, int R, int C, const int32_t* split_sizes, int E, uint8_t* codes,
+                              uint8_t* atoms, cudaStream_t st);
+int scales_to_atoms_launch(const uint8_t* plain, const int32_t* split_sizes, int E, int R, int K, uint8_t* atoms,
+                           cudaStream_t st);
 
 GemmParams base_params(const int32_t* split_sizes, int E) {
   GemmParams p;
@@ -302,7 +339,8 @@ int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, 
   if (axis != 0 && axis != 1) return MOE_ERR_INVALID_ARG;
   if (axis == 0 && transpose_out) return MOE_ERR_INVALID_ARG;
   if (scale_layout != MOE_SCALES_PLAIN && scale_layout != MOE_SCALES_MMA) return MOE_ERR_INVALID_ARG;
-  if (scale_layout == MOE_SCALES_MMA && !(axis == 1 && transpose_out)) return MOE_ERR_INVALID_ARG;
+  if (scale_layout == MOE_SCALES_MMA && !((axis == 1 && transpose_out) || (axis == 0 && !transpose_out)))
+    return MOE_ERR_INVALID_ARG;
   if (scale_layout == MOE_SCALES_MMA && ((rows % 128) || (cols % 128))) return MOE_ERR_UNSUPPORTED;
   if ((long long)batch * rows * cols == 0) return MOE_OK;
   if (!in || !codes || !scales) return MOE_ERR_INVALID_ARG;
@@ -314,7 +352,8 @@ int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, 
     const long long nvec = (long long)batch * rows * cols / 8;
     const long long want = (nvec + 255) / 256;
     const int grid = (int)std::min<long long>(want, (long long)device_props().sm_count * 16);
-    quant_rows_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(in), nvec, cols, codes, scales);
+    quant_rows_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(in), nvec, cols,
+                                            scale_layout == MOE_SCALES_MMA, codes, scales);
   } else {
     if (rows % 32) return MOE_ERR_UNSUPPORTED;
     if (transpose_out && (reinterpret_cast<uintptr_t>(codes) & 15)) return MOE_ERR_INVALID_ARG;
@@ -368,17 +407,9 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
     a_codes = reinterpret_cast<uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256);
   }
   uint8_t* a_atoms = a_codes + align_up((size_t)R * F, 256);
-  {
-    const long long words = ((long long)R / 128 + E) * (H / 128) * 128;
-    const int grid = (int)std::min<long long>((words + 255) / 256, (long long)device_props().sm_count * 8);
-    scales_to_atoms_kernel<<<grid, 256, 2 * (E + 1) * sizeof(int32_t), st>>>(
-        xp_scale, split_sizes, E, H / 32, (long long)R / 128 + E, reinterpret_cast<uint32_t*>(xp_atoms));
-    count_launch();
-    int rc0 = launch_status();
-    if (rc0) return rc0;
-  }
   CUtensorMap ta, tb;
   int rc;
+  if ((rc = scales_to_atoms_launch(xp_scale, split_sizes, E, R, H, xp_atoms, st))) return rc;
   // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
   if ((rc = tmap_u8_3d(&ta, xp, 1, R, H, mx::BM))) return rc;
   if ((rc = tmap_u8_3d(&tb, w1, E, 2 * F, H, 128))) return rc;
@@ -397,7 +428,7 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p1.b_atoms = w1_scale;
   p1.b_rows = 2 * F;
   p1.out_atoms = a_atoms;
-  if ((rc = launch_gemm_mx<MXEPI_SWIGLU_Q>(ta, tb, p1, st))) return rc;
+  if ((rc = launch_gemm_mx<false, MXEPI_SWIGLU_Q>(ta, tb, p1, st))) return rc;
   // fc2: A = a codes [R, F], B = w2 codes [E, H, F]
   if ((rc = tmap_u8_3d(&ta, a_codes, 1, R, F, mx::BM))) return rc;
   if ((rc = tmap_u8_3d(&tb, w2, E, H, F, 128))) return rc;
@@ -413,7 +444,7 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p2.b_atoms = w2_scale;
   p2.b_rows = H;
   p2.out_atoms = nullptr;
-  return launch_gemm_mx<MXEPI_STORE>(ta, tb, p2, st);
+  return launch_gemm_mx<false, MXEPI_STORE>(ta, tb, p2, st);
 }
 
 }  // namespace
@@ -473,14 +504,181 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   return launch_gemm<false, true, false, EPI_STORE>(ta, tb, p2, st);
 }
 
-size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision) {
-  (void)E;
-  (void)H;
-  (void)precision;
-  if (R < 0 || F < 0) return 0;
-  const size_t nparts = (size_t)(F + gg::BN - 1) / gg::BN;
-  return align_up((size_t)R * 2 * F * 2, 256) + align_up(nparts * R * 4, 256) + 256;
+}  // extern "C"
+
+namespace {
+
+// Backward workspace parts (each 256-byte aligned, in this order):
+//   0 dh bf16 [R, 2F];  1 a bf16 [R, F] (MXFP8 only: recomputed for the fc2 weight gradient);
+//   2 dprob partial sums [ceil(F/256)][R] fp32;  MXFP8 only, quantised operands:
+//   3 w2 codes [E, F, H] + scale atoms;  4 w1 codes [E, H, 2F] + atoms;
+//   5 dy codes [R, H] + plain scales + atoms (along H);  6 dy codes + atoms (along rows);
+//   7 a codes [R, F] + atoms (rows);  8 dh codes [R, 2F] + plain scales + atoms (along 2F);
+//   9 dh codes + atoms (rows);  10 xp codes [R, H] + atoms (rows).
+size_t bwd_part_bytes(int part, int E, int R, int H, int F) {
+  const size_t r = (size_t)R, e = (size_t)E, h = (size_t)H, f = (size_t)F;
+  switch (part) {
+    case 0: return align_up(r * 2 * f * 2, 256);
+    case 1: return align_up(r * f * 2, 256);
+    case 2: return align_up((size_t)((F + gg::BN - 1) / gg::BN) * r * 4, 256);
+    case 3: return align_up(e * f * h, 256) + align_up(e * f * h / 32, 256);
+    case 4: return align_up(e * h * 2 * f, 256) + align_up(e * h * 2 * f / 32, 256);
+    case 5: return align_up(r * h, 256) + align_up(r * h / 32, 256) + mma_atoms_bytes(E, R, H);
+    case 6: return align_up(r * h, 256) + mma_atoms_bytes(E, R, H);
+    case 7: return align_up(r * f, 256) + mma_atoms_bytes(E, R, F);
+    case 8: return align_up(r * 2 * f, 256) + align_up(r * 2 * f / 32, 256) + mma_atoms_bytes(E, R, 2 * F);
+    case 9: return align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F);
+    case 10: return align_up(r * h, 256) + mma_atoms_bytes(E, R, H);
+    default: return 0;
+  }
 }
+
+size_t bwd_part_offset(int part, int E, int R, int H, int F, int precision) {
+  size_t off = 0;
+  for (int i = 0; i < part; ++i) {
+    if (precision != MOE_MXFP8 && i == 1) continue;
+    off += bwd_part_bytes(i, E, R, H, F);
+  }
+  return off;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision) {
+  if (R < 0 || F < 0 || E < 1) return 0;
+  return bwd_part_offset(precision == MOE_MXFP8 ? 11 : 3, E, R, H, F, precision) + 256;
+}
+
+size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part) {
+  if (R < 0 || F < 0 || E < 1 || part < 0 || part > 1) return (size_t)-1;
+  if (part == 1 && precision != MOE_MXFP8) return (size_t)-1;
+  return bwd_part_offset(part, E, R, H, F, precision);
+}
+
+}  // extern "C"
+
+namespace {
+
+int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
+                          const void* xp, const void* w1, const void* w2, const float* probs_perm, const void* saved,
+                          uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws,
+                          cudaStream_t st) {
+  if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  auto part = [&](int i) { return base + bwd_part_offset(i, E, R, H, F, MOE_MXFP8); };
+  uint16_t* dh = reinterpret_cast<uint16_t*>(part(0));
+  uint16_t* a_bf = reinterpret_cast<uint16_t*>(part(1));
+  float* dpart = reinterpret_cast<float*>(part(2));
+  const size_t efh = (size_t)E * F * H;
+  uint8_t* w2q = part(3);
+  uint8_t* w2a = w2q + align_up(efh, 256);
+  uint8_t* w1q = part(4);
+  uint8_t* w1a = w1q + align_up(efh * 2, 256);
+  uint8_t* dyr = part(5);
+  uint8_t* dyr_s = dyr + align_up((size_t)R * H, 256);
+  uint8_t* dyr_a = dyr_s + align_up((size_t)R * H / 32, 256);
+  uint8_t* dyc = part(6);
+  uint8_t* dyc_a = dyc + align_up((size_t)R * H, 256);
+  uint8_t* ac = part(7);
+  uint8_t* ac_a = ac + align_up((size_t)R * F, 256);
+  uint8_t* dhr = part(8);
+  uint8_t* dhr_s = dhr + align_up((size_t)R * 2 * F, 256);
+  uint8_t* dhr_a = dhr_s + align_up((size_t)R * 2 * F / 32, 256);
+  uint8_t* dhc = part(9);
+  uint8_t* dhc_a = dhc + align_up((size_t)R * 2 * F, 256);
+  uint8_t* xc = part(10);
+  uint8_t* xc_a = xc + align_up((size_t)R * H, 256);
+  const uint16_t* h_saved = reinterpret_cast<const uint16_t*>(saved);
+  const int nparts = (F + gg::BN - 1) / gg::BN;
+  int rc;
+  // weights along their other axis (the masters change every optimizer step)
+  if ((rc = quant_rows_launch(w2, (long long)E * F, H, 1, w2q, w2a, st))) return rc;
+  if ((rc = quant_rows_launch(w1, (long long)E * H, 2 * F, 1, w1q, w1a, st))) return rc;
+  // dy along H (fc2 dgrad) and along rows (fc2 wgrad)
+  if ((rc = quant_rows_launch(dy_perm, R, H, 0, dyr, dyr_s, st))) return rc;
+  if ((rc = scales_to_atoms_launch(dyr_s, split_sizes, E, R, H, dyr_a, st))) return rc;
+  if ((rc = quant_cols_grouped_launch(dy_perm, R, H, split_sizes, E, dyc, dyc_a, st))) return rc;
+  CUtensorMap ta, tb;
+  // fc2 dgrad + SwiGLU backward: A = dy codes [R, H], B = w2 codes [E, F, H] (N = F)
+  if ((rc = tmap_u8_3d(&ta, dyr, 1, R, H, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, w2q, E, F, H, 128))) return rc;
+  MxGemmParams p;
+  p.g = base_params(split_sizes, E);
+  p.g.M = R;
+  p.g.N = F;
+  p.g.K = H;
+  p.g.out = a_bf;
+  p.g.ldo = F;
+  p.g.out2 = dh;
+  p.g.ldo2 = 2 * F;
+  p.g.aux = h_saved;
+  p.g.ld_aux = 2 * F;
+  p.g.probs = probs_perm;
+  p.g.dprob_part = dpart;
+  p.g.F = F;
+  p.a_atoms = dyr_a;
+  p.b_atoms = w2a;
+  p.b_rows = F;
+  p.out_atoms = nullptr;
+  if ((rc = launch_gemm_mx<false, MXEPI_DSWIGLU>(ta, tb, p, st))) return rc;
+  if (dprobs_perm) {
+    const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
+    reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
+    count_launch();
+    if ((rc = launch_status())) return rc;
+  }
+  // operands of the remaining GEMMs
+  if ((rc = quant_cols_grouped_launch(a_bf, R, F, split_sizes, E, ac, ac_a, st))) return rc;
+  if ((rc = quant_rows_launch(dh, R, 2 * F, 0, dhr, dhr_s, st))) return rc;
+  if ((rc = scales_to_atoms_launch(dhr_s, split_sizes, E, R, 2 * F, dhr_a, st))) return rc;
+  if ((rc = quant_cols_grouped_launch(dh, R, 2 * F, split_sizes, E, dhc, dhc_a, st))) return rc;
+  if ((rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc, xc_a, st))) return rc;
+  // fc2 wgrad: dw2[e] = a_e^T dy_e (MN-major codes, contraction over the expert's rows)
+  if ((rc = tmap_u8_3d(&ta, ac, 1, R, F, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, dyc, 1, R, H, mx::BM))) return rc;
+  p.g = base_params(split_sizes, E);
+  p.g.M = F;
+  p.g.N = H;
+  p.g.out = dw2;
+  p.g.ldo = H;
+  p.g.out_batch = (long long)F * H;
+  p.a_atoms = ac_a;
+  p.b_atoms = dyc_a;
+  p.b_rows = H;
+  if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
+  // fc1 dgrad: dxp = dh w1[e]^T. A = dh codes [R, 2F], B = w1 codes [E, H, 2F] (N = H)
+  if ((rc = tmap_u8_3d(&ta, dhr, 1, R, 2 * F, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, w1q, E, H, 2 * F, 128))) return rc;
+  p.g = base_params(split_sizes, E);
+  p.g.M = R;
+  p.g.N = H;
+  p.g.K = 2 * F;
+  p.g.out = dxp;
+  p.g.ldo = H;
+  p.a_atoms = dhr_a;
+  p.b_atoms = w1a;
+  p.b_rows = H;
+  if ((rc = launch_gemm_mx<false, MXEPI_STORE>(ta, tb, p, st))) return rc;
+  // fc1 wgrad: dw1[e] = xp_e^T dh_e
+  if ((rc = tmap_u8_3d(&ta, xc, 1, R, H, mx::BM))) return rc;
+  if ((rc = tmap_u8_3d(&tb, dhc, 1, R, 2 * F, mx::BM))) return rc;
+  p.g = base_params(split_sizes, E);
+  p.g.M = H;
+  p.g.N = 2 * F;
+  p.g.out = dw1;
+  p.g.ldo = 2 * F;
+  p.g.out_batch = (long long)H * 2 * F;
+  p.a_atoms = xc_a;
+  p.b_atoms = dhc_a;
+  p.b_rows = 2 * F;
+  return launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st);
+}
+
+}  // namespace
+
+extern "C" {
 
 int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
                     const void* w1, const void* w2, const float* probs_perm, int precision, const void* saved,
@@ -488,7 +686,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
                     void* stream) {
   if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
   if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
-  if (precision != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
   if (!split_sizes || !w1 || !w2 || !dw1 || !dw2) return MOE_ERR_INVALID_ARG;
   if (R > 0 && (!dy_perm || !xp || !saved || !dxp || !ws)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < grouped_mlp_bwd_workspace_size(E, R, H, F, precision)) return MOE_ERR_INVALID_ARG;
@@ -499,11 +697,14 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
       return MOE_ERR_CUDA;
     return MOE_OK;
   }
+  if (precision == MOE_MXFP8)
+    return grouped_mlp_bwd_mxfp8(dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
+                                 dprobs_perm, ws, st);
   const uint16_t* h_buf = reinterpret_cast<const uint16_t*>(saved);
   const uint16_t* a_buf =
       reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256));
-  uint16_t* dh = reinterpret_cast<uint16_t*>(ws);
-  float* dpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + align_up((size_t)R * 2 * F * 2, 256));
+  uint16_t* dh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + bwd_part_offset(0, E, R, H, F, MOE_BF16));
+  float* dpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + bwd_part_offset(2, E, R, H, F, MOE_BF16));
   const int nparts = (F + gg::BN - 1) / gg::BN;
 
   CUtensorMap ta, tb;
@@ -605,5 +806,19 @@ extern "C" int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const 
   if (!scratch) return MOE_ERR_CUDA;
   return moe_permute(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, split_sizes, offsets,
                      scratch, sizeof(int32_t) * (size_t)MOE_PERMUTE_NOALLOC_MAX_COUNTS, stream);
+}
+
+extern "C" int mxfp8_quantize_grouped(const uint16_t* in, int R, int C, const int32_t* split_sizes, int E,
+                                      uint8_t* codes, uint8_t* atoms, void* stream) {
+  if (R < 0 || C < 0 || E < 1 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (C % 128) return MOE_ERR_UNSUPPORTED;
+  if (R == 0 || C == 0) return MOE_OK;
+  if (!in || !split_sizes || !codes || !atoms) return MOE_ERR_INVALID_ARG;
+  return quant_cols_grouped_launch(in, R, C, split_sizes, E, codes, atoms, as_stream(stream));
+}
+
+extern "C" size_t mxfp8_grouped_atoms_bytes(int E, int R, int C) {
+  if (E < 1 || R < 0 || C < 0) return 0;
+  return mma_atoms_bytes(E, R, C);
 }
 

@@ -438,7 +438,8 @@ __global__ void __launch_bounds__(256) scales_to_atoms_kernel(const uint8_t* __r
 // ------------------------------------------------------------ MXFP8 quantiser
 // axis 0: blocks of 32 along the columns of each row. 4 lanes per block.
 __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ in, long long nvec, int cols,
-                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+                                                         int mma_scales, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ scales) {
   // nvec = rows * cols / 8; vector v covers columns [8*(v % (cols/8)), +8) of row v / (cols/8)
   const long long stride = (long long)gridDim.x * blockDim.x;
   // the loop runs while the warp's first vector is in range, so all 32 lanes stay
@@ -449,7 +450,107 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     const uint2 q = mxfp8_quant8(live ? __ldg(in + v) : make_uint4(0, 0, 0, 0), &sc);
     if (live) {
       *reinterpret_cast<uint2*>(codes + v * 8) = q;
-      if ((threadIdx.x & 3) == 0) scales[v >> 2] = sc;
+      if ((threadIdx.x & 3) == 0) {
+        if (mma_scales) {
+          const long long row = v / (cols >> 3);
+          const int kb = (int)((v % (cols >> 3)) >> 2);
+          scales[mma_scale_offset((size_t)(row >> 7), (int)(row & 127), kb, cols / 128)] = sc;
+        } else {
+          scales[v >> 2] = sc;
+        }
+      }
+    }
+  }
+}
+
+// Blocks of 32 rows restarting at every expert's first row, per column, for the
+// weight-gradient GEMMs (contraction over the expert's rows). in/codes [R, C] (codes keep
+// the layout: MN-major operands); the last block of an expert covers its remaining rows
+// only (as if zero-padded). Scales go to MMA atoms numbered per expert: expert e owns
+// KG_e = ceil(n_e / 128) k-groups; atom (e, column group cg, k-group kg) sits at
+// (kgoff_e * C/128 + cg * KG_e + kg) * 512 with kgoff_e = sum of KG over earlier experts.
+// Scale bytes of k-blocks past an expert's end (up to the next multiple of 4) are zero.
+// One CUDA block = one 32-row block x 256 columns; blockIdx.x walks the 32-row blocks of
+// all experts (sum of ceil(n_e / 32) of them), blockIdx.y the column tiles.
+__global__ void __launch_bounds__(256) quant_cols_grouped_kernel(const __nv_bfloat16* __restrict__ in, int C,
+                                                                 const int32_t* __restrict__ split_sizes, int E,
+                                                                 uint8_t* __restrict__ codes,
+                                                                 uint8_t* __restrict__ atoms) {
+  extern __shared__ int32_t tabs[];   // [E+1] row offsets, [E+1] 32-row block offsets, [E+1] k-group offsets
+  int32_t* roff = tabs;
+  int32_t* boff = tabs + (E + 1);
+  int32_t* koff = tabs + 2 * (E + 1);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int cr = 0, cb = 0, ck = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? split_sizes[e] : 0;
+      const int nb = (n + 31) / 32, nk = (n + 127) / 128;
+      int ir = n, ib = nb, ik = nk;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yb = __shfl_up_sync(0xffffffffu, ib, o);
+        const int yk = __shfl_up_sync(0xffffffffu, ik, o);
+        if (lane >= o) {
+          ir += yr;
+          ib += yb;
+          ik += yk;
+        }
+      }
+      if (e < E) {
+        roff[e] = cr + ir - n;
+        boff[e] = cb + ib - nb;
+        koff[e] = ck + ik - nk;
+      }
+      cr += __shfl_sync(0xffffffffu, ir, 31);
+      cb += __shfl_sync(0xffffffffu, ib, 31);
+      ck += __shfl_sync(0xffffffffu, ik, 31);
+    }
+    if (lane == 0) {
+      roff[E] = cr;
+      boff[E] = cb;
+      koff[E] = ck;
+    }
+  }
+  __syncthreads();
+  const int CG = C / 128;
+  for (int blk = blockIdx.x; blk < boff[E]; blk += gridDim.x) {
+    int lo = 0, hi = E - 1;   // expert owning 32-row block `blk`
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (boff[mid] <= blk) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int j = blk - boff[e];                 // block index inside the expert
+    const int n = roff[e + 1] - roff[e];
+    const int r0 = roff[e] + 32 * j;
+    const int nrows = min(32, n - 32 * j);
+    const int KG = (n + 127) / 128;
+    const int c = blockIdx.y * 256 + threadIdx.x;
+    if (c >= C) continue;
+    float f[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      f[i] = (i < nrows) ? __bfloat162float(in[(size_t)(r0 + i) * C + c]) : 0.f;
+      amax = fmaxf(amax, fabsf(f[i]));
+    }
+    const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+    const int code = max(bexp - 8, 0);
+    const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const __nv_fp8x2_storage_t pq =
+          __nv_cvt_float2_to_fp8x2(make_float2(f[i] * inv, f[i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      if (i < nrows) codes[(size_t)(r0 + i) * C + c] = (uint8_t)(pq & 0xFF);
+      if (i + 1 < nrows) codes[(size_t)(r0 + i + 1) * C + c] = (uint8_t)(pq >> 8);
+    }
+    const size_t grp = (size_t)koff[e] * CG + (size_t)(c / 128) * KG;   // this column group's first atom
+    atoms[mma_scale_offset(grp, c % 128, j, 1) ] = (uint8_t)code;
+    if (32 * (j + 1) >= n) {   // the expert's last block: zero the unused bytes of its atom
+      for (int jj = j + 1; jj < ((j >> 2) + 1) * 4; ++jj) atoms[mma_scale_offset(grp, c % 128, jj, 1)] = 0;
     }
   }
 }

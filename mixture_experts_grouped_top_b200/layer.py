@@ -47,6 +47,7 @@ class MoEExpertLayer:
                       if training else None)
         self.w1 = self.w2 = None
         self.w1_scale = self.w2_scale = None
+        self.xp_bf16 = None
         self._bwd = None
 
     # --------------------------------------------------------------- weights
@@ -70,6 +71,11 @@ class MoEExpertLayer:
                         w2_scale=self.w2_scale, yp=self.yp, saved=self.saved, workspace=self.mlp_ws, F=self.F,
                         stream=stream)
         moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
+        if self.training and self.prec == MXFP8:
+            # the MXFP8 weight gradient re-quantises xp along its rows: keep a bf16 copy
+            if self.xp_bf16 is None:
+                self.xp_bf16 = torch.empty((self.R, self.H), dtype=torch.bfloat16, device=self.device)
+            moe_permute_rows(x, self.perm["row_map"], self.k, out=self.xp_bf16, stream=stream)
         return self.out
 
     # -------------------------------------------------------------- backward
@@ -96,7 +102,8 @@ class MoEExpertLayer:
             self._alloc_bwd()
         b = self._bwd
         moe_permute_rows(grad_out, self.perm["row_map"], self.k, out=b["dy_perm"], stream=stream)
-        grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], self.perm["xp"], self.w1, self.w2,
+        xp = self.perm["xp"] if self.prec == BF16 else self.xp_bf16
+        grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], xp, self.w1_master, self.w2_master,
                         self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"], dw1=b["dw1"],
                         dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream)
         moe_unpermute(b["dxp"], self.perm["row_map"], self.T, self.k, out=b["dx"], stream=stream)

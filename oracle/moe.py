@@ -317,3 +317,53 @@ def moe_forward_sampled(x, idx, prob, w1, w2, tokens, a_round="bf16") -> np.ndar
     for j in range(idx.shape[1]):
         out += terms[j]
     return out
+
+
+def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=None, a=None):
+    """Backward of the MXFP8 layer: every GEMM on operands quantised along its own
+    contraction axis, computed in float64.
+
+    fc2 dgrad: dy along H times w2 along H (transposed);  fc2 wgrad: a and dy along rows
+    (32-row blocks restarting at each expert);  fc1 dgrad: dh along 2F times w1 along 2F;
+    fc1 wgrad: xp and dh along rows. h = [g | u] is the forward's saved pre-activation.
+    The path stores dh and the recomputed a in bf16 before quantising them; the oracle
+    does the same unless ``dh`` / ``a`` (e.g. the values a GPU produced) are given.
+    Returns (dxp, dw1, dw2, dprobs_perm, dh_exact, a_exact).
+    """
+    dy = f64(dy_perm)
+    xp = f64(xp)
+    w1 = f64(w1)
+    w2 = f64(w2)
+    pp = f64(probs_perm)
+    h = f64(h)
+    split = np.asarray(split_sizes, dtype=np.int64)
+    E, F, H = w2.shape
+    w2q = mxfp8.dequantize(*mxfp8.quantize(w2, axis=0), axis=0)        # [E, F, H] along H
+    w1q = mxfp8.dequantize(*mxfp8.quantize(w1, axis=0), axis=0)        # [E, H, 2F] along 2F
+    dyq = mxfp8.dequantize(*mxfp8.quantize(dy, axis=0), axis=0)        # along H
+    da = np.zeros((dy.shape[0], F))
+    start = 0
+    for e, n in enumerate(split):
+        da[start:start + n] = dyq[start:start + n] @ w2q[e].T
+        start += n
+    g, u = h[:, :F], h[:, F:]
+    p = pp[:, None]
+    dh_exact = np.concatenate([da * p * u * silu_grad(g), da * p * silu(g)], axis=1)
+    dprob = np.sum(da * silu(g) * u, axis=1)
+    a_exact = silu(g) * u * p
+    dh_use = round_to_bf16(dh_exact) if dh is None else f64(dh)
+    a_use = round_to_bf16(a_exact) if a is None else f64(a)
+    deq_rows = lambda v: mxfp8.dequantize_grouped_rows(*mxfp8.quantize_grouped_rows(v, split), split)
+    aq, dyc, xc, dhc = deq_rows(a_use), deq_rows(dy), deq_rows(xp), deq_rows(dh_use)
+    dhq = mxfp8.dequantize(*mxfp8.quantize(dh_use, axis=0), axis=0)    # along 2F
+    dxp = np.zeros_like(xp)
+    dw1 = np.zeros_like(w1)
+    dw2 = np.zeros_like(w2)
+    start = 0
+    for e, n in enumerate(split):
+        rows = slice(start, start + n)
+        dw2[e] = aq[rows].T @ dyc[rows]
+        dxp[rows] = dhq[rows] @ w1q[e].T
+        dw1[e] = xc[rows].T @ dhc[rows]
+        start += n
+    return dxp, dw1, dw2, dprob, dh_exact, a_exact

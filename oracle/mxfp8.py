@@ -131,3 +131,38 @@ def dequantize(codes, scales, axis: int, transpose_out: bool = False) -> np.ndar
         return dequantize_blocks_last_axis(codes, scales)
     return np.swapaxes(dequantize_blocks_last_axis(np.swapaxes(codes, -1, -2),
                                                    np.swapaxes(scales, -1, -2)), -1, -2)
+
+
+def quantize_grouped_rows(v, split_sizes) -> tuple[np.ndarray, list]:
+    """Quantise expert-contiguous rows ``v[R, C]`` along the rows, per column, in blocks
+    of 32 rows that restart at every expert's first row; an expert's last block covers
+    its remaining rows, as if padded with zeros.
+
+    Returns codes [R, C] and, per expert, its scales [ceil(n_e/32), C].
+    """
+    v = np.asarray(v, dtype=np.float64)
+    codes = np.zeros(v.shape, dtype=np.uint8)
+    scales = []
+    start = 0
+    for n in np.asarray(split_sizes, dtype=np.int64):
+        nb = (n + BLOCK - 1) // BLOCK
+        padded = np.zeros((nb * BLOCK, v.shape[1]))
+        padded[:n] = v[start:start + n]
+        c, s = quantize(padded, axis=1)
+        codes[start:start + n] = c[:n]
+        scales.append(s)
+        start += n
+    return codes, scales
+
+
+def dequantize_grouped_rows(codes, scales, split_sizes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    out = np.zeros(codes.shape)
+    start = 0
+    for n, s in zip(np.asarray(split_sizes, dtype=np.int64), scales):
+        nb = (n + BLOCK - 1) // BLOCK
+        padded = np.zeros((nb * BLOCK, codes.shape[1]), dtype=np.uint8)
+        padded[:n] = codes[start:start + n]
+        out[start:start + n] = dequantize(padded, s, axis=1)[:n]
+        start += n
+    return out

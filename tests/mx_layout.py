@@ -31,3 +31,24 @@ def tile_atoms_to_plain(atoms, split_sizes, ks):
         out.append(padded[g * 128: g * 128 + n])
         g += (n + 127) // 128
     return np.concatenate(out) if out else np.zeros((0, ks), np.uint8), padded, groups
+
+
+def grouped_scales_to_atoms(scales_per_expert, split_sizes, C):
+    """Per-expert [ceil(n_e/32), C] scales (blocks along rows) -> the grouped atom layout:
+    expert e owns KG_e = ceil(n_e/128) k-groups; atom (cg, kg) of expert e at
+    (kgoff_e * C/128 + cg * KG_e + kg); unused block bytes are zero."""
+    CG = C // 128
+    atoms = []
+    for n, s in zip(split_sizes, scales_per_expert):
+        n = int(n)
+        kg = (n + 127) // 128
+        if kg == 0:
+            continue
+        blocks = np.zeros((kg * 4, C), dtype=np.uint8)
+        blocks[: s.shape[0]] = s
+        # [kg*4, C] -> per (cg, kg): atom[word(c%128), byte = block % 4]
+        b = blocks.reshape(kg, 4, CG, 128).transpose(2, 0, 3, 1)       # [cg, kg, c, byte]
+        out = np.empty((CG, kg, 128, 4), dtype=np.uint8)
+        out[:, :, _WORD, :] = b
+        atoms.append(out.reshape(-1))
+    return np.concatenate(atoms) if atoms else np.zeros(0, np.uint8)

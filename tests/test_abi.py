@@ -65,7 +65,11 @@ def test_other_entry_points_reject_bad_arguments():
     assert h.grouped_mlp_fwd(None, None, None, 0, 16, 128, 256, None, None, None, None, None, 0, None, None,
                              None, 0, None) == 1                                       # E = 0
     assert h.grouped_mlp_bwd(None, None, 4, 16, 128, 256, None, None, None, None, 1, None, None, None, None,
-                             None, None, 0, None) == 2                                 # MXFP8 backward
+                             None, None, 0, None) == 1                                 # null operands
+    assert h.grouped_mlp_bwd(None, None, 4, 16, 128, 256, None, None, None, None, 7, None, None, None, None,
+                             None, None, 0, None) == 1                                 # unknown precision
+    assert h.mxfp8_quantize_grouped(None, 64, 100, None, 4, None, None, None) == 2    # C % 128
+    assert h.grouped_mlp_bwd_workspace_offset(4, 64, 128, 256, 0, 1) == 2 ** 64 - 1  # no `a` part for BF16
     assert h.mxfp8_quantize(None, 1, 4, 33, 0, 0, 0, None, None, None) == 1            # null input
     assert h.mxfp8_quantize(None, 1, 4, 64, 0, 1, 0, None, None, None) == 1            # transpose with axis 0
     assert h.mxfp8_quantize(None, 1, 128, 128, 0, 0, 1, None, None, None) == 1         # MMA scales need axis 1

@@ -172,3 +172,23 @@ def test_sampled_forward_equals_per_token_definition():
     ref = moe.moe_forward_per_token(x, idx, prob, w1, w2, "bf16", tokens=toks)
     got = moe.moe_forward_sampled(x, idx, prob, w1, w2, toks, "bf16")
     assert np.max(np.abs(got - ref)) <= 1e-13 * np.max(np.abs(ref))
+
+
+def test_mxfp8_backward_close_to_exact_backward():
+    # the MXFP8 backward is the exact backward up to MXFP8 quantisation error (catches
+    # transposed operands, wrong terms or mixed-up axes, which give O(1) differences)
+    T, H, F, E, k = 40, 64, 64, 3, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=51)
+    row_map, split, _ = moe.permute_index(idx, E)
+    xp = moe.permute_rows(x, row_map, k)
+    pp = moe.permute_probs(prob, row_map)
+    _, h, _ = moe.grouped_mlp_fwd(xp, split, w1, w2, pp, a_round="f64")
+    dy = np.random.default_rng(3).normal(size=xp.shape)
+    ref = moe.grouped_mlp_bwd(dy, xp, split, w1, w2, pp, a_round="f64")
+    got = moe.grouped_mlp_bwd_mxfp8(dy, xp, split, w1, w2, pp, h)
+    for g, r in zip(got[:4], ref[:4]):
+        rel = np.max(np.abs(g - r)) / np.max(np.abs(r))
+        assert rel < 0.08, rel
+    # dh before quantisation is the exact SwiGLU backward of the quantised da
+    assert got[4].shape == (xp.shape[0], 2 * F)
+    assert np.allclose(got[5], moe.silu(h[:, :F]) * h[:, F:] * pp[:, None])

@@ -119,3 +119,26 @@ def test_axis_and_transpose_layouts():
     with pytest.raises(ValueError):
         mxfp8.quantize(rng.normal(size=(4, 33)), axis=0)
     assert math.isnan(mxfp8.e4m3_decode_code(0x7F))
+
+
+def test_grouped_rows_quantiser_pins():
+    rng = np.random.default_rng(21)
+    split = [64, 0, 45, 7, 96]
+    v = rng.normal(size=(sum(split), 40)) * np.exp(rng.uniform(-5, 5, (1, 40)))
+    codes, scales = mxfp8.quantize_grouped_rows(v, split)
+    # a group of whole blocks is the plain column quantiser on that group
+    c0, s0 = mxfp8.quantize(v[:64], axis=1)
+    assert np.array_equal(codes[:64], c0) and np.array_equal(scales[0], s0)
+    assert scales[1].shape == (0, 40)
+    # a partial block: the rows of the group padded with zeros (hand-built)
+    g = v[64:109]
+    pad = np.zeros((64, 40))
+    pad[:45] = g
+    c2, s2 = mxfp8.quantize(pad, axis=1)
+    assert np.array_equal(codes[64:109], c2[:45]) and np.array_equal(scales[2], s2)
+    # blocks never mix experts: quantising each group alone gives the same codes
+    c3, s3 = mxfp8.quantize_grouped_rows(v[109:116], [7])
+    assert np.array_equal(codes[109:116], c3) and np.array_equal(scales[3], s3[0])
+    # dequantised values are within the MXFP8 rounding bound of the input
+    d = mxfp8.dequantize_grouped_rows(codes, scales, split)
+    assert np.max(np.abs(d - v) / np.maximum(np.abs(v), 1e-300)) <= 0.126 or np.allclose(d, v, rtol=0.126)
