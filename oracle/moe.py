@@ -367,3 +367,130 @@ def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=No
         dw1[e] = xc[rows].T @ dhc[rows]
         start += n
     return dxp, dw1, dw2, dprob, dh_exact, a_exact
+
+
+def expert_rows(split_sizes, e) -> slice:
+    off = int(np.sum(np.asarray(split_sizes, dtype=np.int64)[:e]))
+    return slice(off, off + int(np.asarray(split_sizes)[e]))
+
+
+def bwd_sampled_bf16(dy_perm, xp, split_sizes, w1, w2, probs_perm, rows, experts, cols1, cols2):
+    """Sampled entries of the BF16 backward (the analytic gradient of
+    :func:`grouped_mlp_fwd` with `a` rounded to bf16), computed in float64:
+
+    dxp and dprobs_perm for the permuted ``rows``; for every expert in ``experts``,
+    dw2[e][:, cols2] and dw1[e][:, cols1] over all of that expert's rows.
+    """
+    split = np.asarray(split_sizes, dtype=np.int64)
+    offs = np.concatenate([[0], np.cumsum(split)])
+    F = w2.shape[1]
+
+    def swiglu_bwd(rsel, e):
+        x_r = f64(xp[rsel])
+        w1e = f64(w1[e])
+        w2e = f64(w2[e])
+        h = x_r @ w1e
+        g, u = h[:, :F], h[:, F:]
+        p = f64(probs_perm[rsel])[:, None] if not isinstance(rsel, slice) else f64(probs_perm)[rsel][:, None]
+        da = f64(dy_perm[rsel]) @ w2e.T
+        dh = np.concatenate([da * p * u * silu_grad(g), da * p * silu(g)], axis=1)
+        a = round_to_bf16(silu(g) * u * p)
+        dp = np.sum(da * silu(g) * u, axis=1)
+        return x_r, w1e, dh, a, dp
+
+    rows = np.asarray(rows, dtype=np.int64)
+    dxp = np.zeros((rows.size, xp.shape[1]))
+    dpp = np.zeros(rows.size)
+    for e in range(len(split)):
+        sel = np.nonzero((rows >= offs[e]) & (rows < offs[e + 1]))[0]
+        if sel.size == 0:
+            continue
+        _, w1e, dh, _, dp = swiglu_bwd(rows[sel], e)
+        dxp[sel] = dh @ w1e.T
+        dpp[sel] = dp
+    dw1, dw2 = {}, {}
+    for e in experts:
+        rs = slice(int(offs[e]), int(offs[e + 1]))
+        if rs.stop == rs.start:
+            dw1[e] = np.zeros((xp.shape[1], len(cols1)))
+            dw2[e] = np.zeros((F, len(cols2)))
+            continue
+        x_r, _, dh, a, _ = swiglu_bwd(rs, e)
+        dw2[e] = a.T @ f64(dy_perm[rs])[:, cols2]
+        dw1[e] = x_r.T @ dh[:, cols1]
+    return dxp, dpp, dw1, dw2
+
+
+def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_scales=None):
+    """MXFP8 forward of individual routed rows (x_rows[i] is the token's bf16 row routed
+    to expert expert_of_rows[i] with probability prob_rows[i]), float64 on quantised
+    operands. The oracle quantises x along H and each needed expert's weights along their
+    contraction axis itself. fc2 runs on the oracle's own `a` codes unless ``a_codes`` /
+    ``a_scales`` (rows x F, F/32) are given. Returns (yp, a_codes, a_scales)."""
+    xr = f64(x_rows)
+    prob_rows = f64(prob_rows)
+    experts = np.asarray(expert_of_rows, dtype=np.int64)
+    F = w2.shape[1]
+    xq = mxfp8.dequantize(*mxfp8.quantize(xr, axis=0), axis=0)
+    yp = np.zeros((xr.shape[0], w2.shape[2]))
+    own_c = np.zeros((xr.shape[0], F), dtype=np.uint8)
+    own_s = np.zeros((xr.shape[0], F // 32), dtype=np.uint8)
+    for e in np.unique(experts):
+        sel = np.nonzero(experts == e)[0]
+        w1q = mxfp8.dequantize(*mxfp8.quantize(f64(w1[e]), axis=1), axis=1)     # along H
+        w2q = mxfp8.dequantize(*mxfp8.quantize(f64(w2[e]), axis=1), axis=1)     # along F
+        hh = xq[sel] @ w1q
+        a = silu(hh[:, :F]) * hh[:, F:] * prob_rows[sel, None]
+        c, s = mxfp8.quantize(a, axis=0)
+        own_c[sel], own_s[sel] = c, s
+        if a_codes is None:
+            aq = mxfp8.dequantize(c, s, axis=0)
+        else:
+            aq = mxfp8.dequantize(np.asarray(a_codes)[sel], np.asarray(a_scales)[sel], axis=0)
+        yp[sel] = aq @ w2q
+    return yp, own_c, own_s
+
+
+def bwd_sampled_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh, a, rows, experts, cols):
+    """Sampled entries of :func:`grouped_mlp_bwd_mxfp8`, float64 on quantised operands.
+
+    For the permuted ``rows``: dh_exact (from dy along H and w2 along H), dprobs, and dxp
+    (from ``dh`` along 2F and w1 along 2F). For every expert in ``experts`` and the column
+    samples ``cols = (f_cols, h_cols, hh_cols, j_cols)``: dw2[e][f_cols][:, h_cols] (``a``
+    and dy along the expert's rows) and dw1[e][hh_cols][:, j_cols] (xp and ``dh`` along
+    rows). ``h`` is the forward's [g | u]; ``dh`` and ``a`` are the stored bf16 values.
+    """
+    split = np.asarray(split_sizes, dtype=np.int64)
+    offs = np.concatenate([[0], np.cumsum(split)])
+    F = w2.shape[1]
+    rows = np.asarray(rows, dtype=np.int64)
+    out = {"dh": np.zeros((rows.size, 2 * F)), "dp": np.zeros(rows.size), "dxp": np.zeros((rows.size, xp.shape[1]))}
+    for e in range(len(split)):
+        sel = np.nonzero((rows >= offs[e]) & (rows < offs[e + 1]))[0]
+        if sel.size == 0:
+            continue
+        r = rows[sel]
+        w2q = mxfp8.dequantize(*mxfp8.quantize(f64(w2[e]), axis=0), axis=0)      # [F, H] along H
+        w1q = mxfp8.dequantize(*mxfp8.quantize(f64(w1[e]), axis=0), axis=0)      # [H, 2F] along 2F
+        dyq = mxfp8.dequantize(*mxfp8.quantize(f64(dy_perm[r]), axis=0), axis=0)
+        da = dyq @ w2q.T
+        hh = f64(h[r])
+        g, u = hh[:, :F], hh[:, F:]
+        p = f64(probs_perm[r])[:, None]
+        out["dh"][sel] = np.concatenate([da * p * u * silu_grad(g), da * p * silu(g)], axis=1)
+        out["dp"][sel] = np.sum(da * silu(g) * u, axis=1)
+        dhq = mxfp8.dequantize(*mxfp8.quantize(f64(dh[r]), axis=0), axis=0)
+        out["dxp"][sel] = dhq @ w1q.T
+    f_cols, h_cols, hh_cols, j_cols = cols
+    out["dw2"], out["dw1"] = {}, {}
+    for e in experts:
+        rs = slice(int(offs[e]), int(offs[e + 1]))
+        n = rs.stop - rs.start
+        deq_rows = lambda v: mxfp8.dequantize_grouped_rows(*mxfp8.quantize_grouped_rows(v, [n]), [n])
+        if n == 0:
+            out["dw2"][e] = np.zeros((len(f_cols), len(h_cols)))
+            out["dw1"][e] = np.zeros((len(hh_cols), len(j_cols)))
+            continue
+        out["dw2"][e] = deq_rows(f64(a[rs][:, f_cols])).T @ deq_rows(f64(dy_perm[rs][:, h_cols]))
+        out["dw1"][e] = deq_rows(f64(xp[rs][:, hh_cols])).T @ deq_rows(f64(dh[rs][:, j_cols]))
+    return out

@@ -1,0 +1,144 @@
+"""Full-size parity of the benchmark workloads (same shapes and launch configuration as
+bench.py), checked on outputs the oracle can compute one by one: sampled tokens/rows and
+sampled weight-gradient entries (each depends only on its own column over one expert).
+
+Tolerances: BF16 outputs max|err| / max|ref| <= 1e-2 over the sampled set; MXFP8 outputs
+within 2e-3 * max|ref| plus their own bf16 storage rounding (2^-8 |ref|) against the
+oracle on the same quantised operands.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_grouped_top_b200 as mb
+from oracle import moe as om
+import workloads
+from tests.mx_layout import tile_atoms_to_plain
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def rel(got, ref):
+    g = got.float().cpu().numpy() if hasattr(got, "cpu") else np.asarray(got)
+    return float(np.max(np.abs(g - ref)) / np.max(np.abs(ref)))
+
+
+def within_mx(got, ref, name, tol=2e-3):
+    g = got.float().cpu().numpy() if hasattr(got, "cpu") else np.asarray(got)
+    bound = tol * np.max(np.abs(ref)) + 2.0 ** -8 * np.abs(ref)
+    assert np.all(np.abs(g - ref) <= bound), f"{name}: worst excess {np.max(np.abs(g - ref) - bound):.3e}"
+
+
+def sample_rows(split, n, seed):
+    """n seeded permuted rows plus the first and last row of the smallest non-empty and
+    of the largest expert."""
+    rng = np.random.default_rng(seed)
+    R = int(np.sum(split))
+    offs = np.concatenate([[0], np.cumsum(split)])
+    nz = [e for e in range(len(split)) if split[e] > 0]
+    small = min(nz, key=lambda e: split[e])
+    large = max(nz, key=lambda e: split[e])
+    extra = [offs[small], offs[small + 1] - 1, offs[large], offs[large + 1] - 1]
+    return np.unique(np.concatenate([rng.choice(R, size=n, replace=False), extra])).astype(np.int64), small, large
+
+
+def test_qwen3_full_size_fwd_bwd_bf16():
+    cfg = workloads.CONFIGS["qwen3_30b_a3b_bf16_fwdbwd"]
+    d = workloads.make_layer_inputs(cfg)
+    layer = mb.MoEExpertLayer(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, training=True)
+    layer.set_weights(d["w1"].to(DEV), d["w2"].to(DEV))
+    out = layer.forward(d["x"].to(DEV), d["logits"].to(DEV)).cpu()
+    dx, dw1, dw2, dprob = layer.backward(d["grad_out"].to(DEV))
+    assert mb.moe_device_status() == 0
+    split = layer.perm["split_sizes"].cpu().numpy()
+    assert split.sum() == cfg.R and np.all(split[-4:] == 0)          # the forced-empty experts
+    ridx, rprob = om.route(d["logits"], cfg.k)
+    assert np.array_equal(layer.idx.cpu().numpy(), ridx)
+    toks = workloads.sample_tokens(cfg.T, 256, seed=3)
+    ref = om.moe_forward_sampled(d["x"], ridx, rprob, d["w1"], d["w2"], toks, a_round="bf16")
+    assert rel(out[toks], ref) <= 1e-2
+    # backward on the GPU's own permuted inputs (bit-exact by the permutation tests)
+    b = layer._bwd
+    rows, small, large = sample_rows(split, 512, seed=4)
+    experts = [small, large, cfg.E - 1, 17, 60]
+    c1 = np.sort(np.random.default_rng(5).choice(2 * cfg.F, 16, replace=False))
+    c2 = np.sort(np.random.default_rng(6).choice(cfg.H, 16, replace=False))
+    xp, dyp, pp = layer.perm["xp"].cpu(), b["dy_perm"].cpu(), layer.perm["probs_perm"].cpu()
+    rdxp, rdpp, rdw1, rdw2 = om.bwd_sampled_bf16(dyp, xp, split, d["w1"], d["w2"], pp, rows, experts, c1, c2)
+    assert rel(b["dxp"].cpu()[rows], rdxp) <= 1e-2
+    assert rel(b["dprobs_perm"].cpu()[rows], rdpp) <= 1e-2
+    for e in experts:
+        g1, g2 = dw1[e][:, c1].cpu(), dw2[e][:, c2].cpu()
+        if split[e] == 0:
+            assert torch.count_nonzero(g1) == 0 and torch.count_nonzero(g2) == 0
+        else:
+            assert rel(g1, rdw1[e]) <= 1e-2 and rel(g2, rdw2[e]) <= 1e-2
+
+
+def test_mixtral_mxfp8_full_size_fwd():
+    cfg = workloads.CONFIGS["mixtral_mxfp8_fwd"]
+    d = workloads.make_layer_inputs(cfg)
+    layer = mb.MoEExpertLayer(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, "mxfp8", training=True)
+    layer.set_weights(d["w1"].to(DEV), d["w2"].to(DEV))
+    layer.forward(d["x"].to(DEV), d["logits"].to(DEV))
+    assert mb.moe_device_status() == 0
+    R, F = cfg.R, cfg.F
+    split = layer.perm["split_sizes"].cpu().numpy()
+    ridx, rprob = om.route(d["logits"], cfg.k)
+    row_map = layer.perm["row_map"].cpu().numpy()
+    assert np.array_equal(row_map, om.permute_index(ridx, cfg.E)[0])
+    # sampled routed rows of the smallest and the largest expert
+    rows_all, small, large = sample_rows(split, 4096, seed=7)
+    offs = np.concatenate([[0], np.cumsum(split)])
+    keep = ((rows_all >= offs[small]) & (rows_all < offs[small + 1])) | \
+           ((rows_all >= offs[large]) & (rows_all < offs[large + 1]))
+    rows = rows_all[keep]
+    slot_of_row = np.empty(R, dtype=np.int64)
+    slot_of_row[row_map] = np.arange(R)
+    slots = slot_of_row[rows]
+    toks, js = slots // cfg.k, slots % cfg.k
+    off_a = (R * 2 * F * 2 + 255) // 256 * 256
+    a_codes = layer.saved[off_a: off_a + R * F].view(R, F).cpu().numpy()
+    off_s = off_a + (R * F + 255) // 256 * 256
+    a_scales, _, _ = tile_atoms_to_plain(layer.saved[off_s:].cpu().numpy(), split, F // 32)
+    yp_ref, own_c, own_s = om.fwd_rows_mxfp8(d["x"][toks], rprob[toks, js], ridx[toks, js], d["w1"], d["w2"],
+                                             a_codes=a_codes[rows], a_scales=a_scales[rows])
+    assert np.mean(a_codes[rows] == own_c) >= 0.99 and np.mean(a_scales[rows] == own_s) >= 0.99
+    within_mx(layer.yp.cpu()[rows], yp_ref, "yp")
+
+
+def test_genomic_mxfp8_full_size_fwd_bwd():
+    cfg = workloads.CONFIGS["genomic_mixtral_mxfp8_fwdbwd"]
+    d = workloads.make_layer_inputs(cfg)
+    layer = mb.MoEExpertLayer(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, "mxfp8", training=True)
+    layer.set_weights(d["w1"].to(DEV), d["w2"].to(DEV))
+    layer.forward(d["x"].to(DEV), d["logits"].to(DEV))
+    dx, dw1, dw2, dprob = layer.backward(d["grad_out"].to(DEV))
+    assert mb.moe_device_status() == 0
+    R, H, F, E = cfg.R, cfg.H, cfg.F, cfg.E
+    split = layer.perm["split_sizes"].cpu().numpy()
+    assert split[0] > 0.4 * R                                            # expert 0 carries the skew
+    b = layer._bwd
+    off_dh = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 0)
+    off_a = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 1)
+    dh = b["ws"][off_dh: off_dh + R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
+    a = b["ws"][off_a: off_a + R * F * 2].view(torch.bfloat16).view(R, F).cpu()
+    h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
+    rows_all, small, large = sample_rows(split, 2048, seed=8)
+    offs = np.concatenate([[0], np.cumsum(split)])
+    keep = ((rows_all >= offs[small]) & (rows_all < offs[small + 1])) | \
+           ((rows_all >= offs[large]) & (rows_all < offs[large + 1]))
+    rows = rows_all[keep]
+    rng = np.random.default_rng(9)
+    cols = (np.sort(rng.choice(F, 16, replace=False)), np.sort(rng.choice(H, 16, replace=False)),
+            np.sort(rng.choice(H, 16, replace=False)), np.sort(rng.choice(2 * F, 16, replace=False)))
+    ref = om.bwd_sampled_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
+                               layer.perm["probs_perm"].cpu(), h, dh, a, rows, [small, large], cols)
+    within_mx(dh[rows], ref["dh"], "dh")
+    within_mx(b["dxp"].cpu()[rows], ref["dxp"], "dxp")
+    gp = b["dprobs_perm"].cpu().numpy()[rows]
+    assert np.max(np.abs(gp - ref["dp"])) <= 2e-3 * np.max(np.abs(ref["dp"]))
+    for e in (small, large):
+        within_mx(dw2[e].cpu()[np.ix_(cols[0], cols[1])], ref["dw2"][e], f"dw2[{e}]")
+        within_mx(dw1[e].cpu()[np.ix_(cols[2], cols[3])], ref["dw1"][e], f"dw1[{e}]")

@@ -192,3 +192,56 @@ def test_mxfp8_backward_close_to_exact_backward():
     # dh before quantisation is the exact SwiGLU backward of the quantised da
     assert got[4].shape == (xp.shape[0], 2 * F)
     assert np.allclose(got[5], moe.silu(h[:, :F]) * h[:, F:] * pp[:, None])
+
+
+def test_sampled_backward_equals_full_backward():
+    rng = np.random.default_rng(0)
+    T, H, F, E, k = 30, 16, 8, 3, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=61)
+    rm, split, _ = moe.permute_index(idx, E)
+    xp = moe.permute_rows(x, rm, k)
+    pp = moe.permute_probs(prob, rm)
+    dy = rng.normal(size=xp.shape)
+    ref = moe.grouped_mlp_bwd(dy, xp, split, w1, w2, pp, a_round="bf16")
+    rows, c1, c2 = np.array([0, 5, 17, 59]), [0, 3, 7], [1, 2]
+    dxp, dpp, dw1, dw2 = moe.bwd_sampled_bf16(dy, xp, split, w1, w2, pp, rows, [0, 2], c1, c2)
+    assert np.allclose(dxp, ref[0][rows], rtol=0, atol=1e-12) and np.allclose(dpp, ref[3][rows], atol=1e-12)
+    assert np.allclose(dw1[2], ref[1][2][:, c1], atol=1e-12) and np.allclose(dw2[0], ref[2][0][:, c2], atol=1e-12)
+
+
+def test_sampled_mxfp8_backward_equals_full_mxfp8_backward():
+    rng = np.random.default_rng(1)
+    T, H, F, E, k = 40, 64, 64, 3, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=71)
+    rm, split, _ = moe.permute_index(idx, E)
+    xp = moe.permute_rows(x, rm, k)
+    pp = moe.permute_probs(prob, rm)
+    _, h, _ = moe.grouped_mlp_fwd(xp, split, w1, w2, pp, a_round="f64")
+    dy = rng.normal(size=xp.shape)
+    full = moe.grouped_mlp_bwd_mxfp8(dy, xp, split, w1, w2, pp, h)
+    dh = moe.round_to_bf16(full[4])
+    a = moe.round_to_bf16(full[5])
+    rows = np.array([1, 7, 33, 79])
+    cols = ([3, 9], [0, 63], [5, 6], [2, 100])
+    s = moe.bwd_sampled_mxfp8(dy, xp, split, w1, w2, pp, h, dh, a, rows, [0, 1, 2], cols)
+    assert np.allclose(s["dxp"], full[0][rows], atol=1e-12) and np.allclose(s["dp"], full[3][rows], atol=1e-12)
+    assert np.allclose(s["dh"], full[4][rows], atol=1e-12)
+    for e in range(3):
+        assert np.allclose(s["dw2"][e], full[2][e][np.ix_(cols[0], cols[1])], atol=1e-12)
+        assert np.allclose(s["dw1"][e], full[1][e][np.ix_(cols[2], cols[3])], atol=1e-12)
+
+
+def test_mxfp8_forward_rows_equal_grouped_forward():
+    T, H, F, E, k = 24, 64, 64, 3, 2
+    x, idx, prob, w1, w2 = _layer(T, H, F, E, k, seed=81)
+    rm, split, _ = moe.permute_index(idx, E)
+    xc, xs = mxfp8.quantize(x, axis=0)
+    w1c, w1s = moe.quantize_weights_kmajor(w1, "rows")
+    w2c, w2s = moe.quantize_weights_kmajor(w2, "rows")
+    yp, ac, asc, _ = moe.grouped_mlp_fwd_mxfp8(moe.permute_rows(xc, rm, k), moe.permute_rows(xs, rm, k), split,
+                                               w1c, w1s, w2c, w2s, moe.permute_probs(prob, rm))
+    # rows of token t, slot j live at rm[t*k + j]
+    toks = np.repeat(np.arange(T), k)
+    rows = rm
+    ypr, c, s = moe.fwd_rows_mxfp8(x[toks], prob.reshape(-1), idx.reshape(-1), w1, w2)
+    assert np.allclose(ypr, yp[rows], atol=1e-12) and np.array_equal(c, ac[rows]) and np.array_equal(s, asc[rows])
