@@ -32,7 +32,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;                       // fp8: 128 bytes of K per row (one swizzle span)
 constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;                 // 4 control warps + 8 epilogue warps
 constexpr int kABytes = BM * BK;              // 16 KB
 constexpr int kBBytes = BN * BK;              // 32 KB
 constexpr int kSfaBytes = 512;                // 128 rows x 4 scale bytes
@@ -43,7 +43,7 @@ constexpr uint32_t kAcc1Col = 224;
 constexpr uint32_t kSfaCol = 480;
 constexpr uint32_t kSfbCol = 484;
 constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kStages * (kSfaBytes + kSfbBytes) + 1024 +
-                           3 * (kMaxE + 1) * 4;
+                           4 * (kMaxE + 1) * 4;
 }  // namespace mx
 
 enum MxEpiKind : int {
@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
   int32_t* kg_off = tile_off + (kMaxE + 1);   // K-grouped: k-groups (128 rows) of earlier experts
+  int32_t* order = kg_off + (kMaxE + 1);      // K-grouped: experts by decreasing row count
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -100,9 +101,9 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 256);
     }
-    mbar_init(tovl, 128);
+    mbar_init(tovl, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -152,8 +153,12 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (KGROUP) {
+    rank_experts_by_rows(row_off, E, order);
+    __syncthreads();
+  }
 
-  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K};
+  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K, order};
   // the walker's k-block count assumes 64-wide blocks; MXFP8 uses 128-wide ones
   auto kblocks = [&](const TileInfo& ti) { return KGROUP ? (ti.rows + BK - 1) / BK : p.K / BK; };
   const int total = walk.total();
@@ -297,7 +302,8 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp - 4;
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int half = (warp - 4) >> 2;     // half of the tile's columns this warp drains
     const int r_local = q * 32 + lane;
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
@@ -325,15 +331,18 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           ok_row = row_ok;
           orow = row * p.ldo;
         }
-        const int first = acc ? 0 : 7;   // the 32-column strip shared with the other accumulator
+        // the 32-column strip shared with the other accumulator: chunk 7 of acc0 (upper
+        // half), chunk 0 of acc1 (lower half); its owner drains it first, then signals
+        const bool owner = acc ? (half == 0) : (half == 1);
+        if (!owner) mbar_arrive(tovl);
 #pragma unroll 1
-        for (int it = 0; it < 8; ++it) {
-          const int c = (it == 0) ? first : (acc ? it : it - 1);
+        for (int it = 0; it < 4; ++it) {
+          const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
           uint32_t v0[16], v1[16];
           tmem_ld_32x32b_x16(t_row + c * 32, v0);
           tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
           tmem_wait_ld();
-          if (it == 0) {
+          if (owner && it == 0) {
             tc_fence_before();
             mbar_arrive(tovl);
           }
@@ -366,16 +375,17 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
         __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
         __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const int n0 = ti.n_blk * BN;
-        const int first = acc ? 0 : 7;
+        const bool owner = acc ? (half == 0) : (half == 1);
+        if (!owner) mbar_arrive(tovl);
         float dp = 0.f;
 #pragma unroll 1
-        for (int it = 0; it < 8; ++it) {
-          const int c = (it == 0) ? first : (acc ? it : it - 1);
+        for (int it = 0; it < 4; ++it) {
+          const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
           uint32_t v0[16], v1[16];
           tmem_ld_32x32b_x16(t_row + c * 32, v0);
           tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
           tmem_wait_ld();
-          if (it == 0) {
+          if (owner && it == 0) {
             tc_fence_before();
             mbar_arrive(tovl);
           }
@@ -425,24 +435,27 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
             }
           }
         }
-        if (row_ok) p.dprob_part[(long long)ti.n_blk * p.M + row] = dp;
+        if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
       } else {
         // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
         const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
         const int n0 = ti.n_blk * 128;
         uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
         __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
-        const int first = acc ? 0 : 3;
+        // output chunk 3 of acc0 (its up columns are the shared strip) belongs to the
+        // upper half, chunk 0 of acc1 (gate columns) to the lower half
+        const bool owner = acc ? (half == 0) : (half == 1);
+        if (!owner) mbar_arrive(tovl);
 #pragma unroll 1
-        for (int it = 0; it < 4; ++it) {
-          const int c = (it == 0) ? first : (acc ? it : it - 1);
+        for (int it = 0; it < 2; ++it) {
+          const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
           uint32_t g0[16], g1[16], u0[16], u1[16];
           tmem_ld_32x32b_x16(t_row + c * 32, g0);
           tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
           tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
           tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
           tmem_wait_ld();
-          if (it == 0) {
+          if (owner && it == 0) {
             tc_fence_before();
             mbar_arrive(tovl);
           }
@@ -490,10 +503,11 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
         }
       }
       if (EPI == MXEPI_SWIGLU_Q) {
-        // rows past the expert's end store zero scales
+        // this half's two scale bytes (chunks 2*half, 2*half+1); rows past the expert store 0
         const size_t g = (size_t)(tile_off[ti.e] / NT + ti.m_blk);
-        *reinterpret_cast<uint32_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk, p.N / 128)) =
-            sc_word;
+        *reinterpret_cast<uint16_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk + 2 * half,
+                                                                     p.N / 128)) =
+            (uint16_t)(sc_word >> (16 * half));
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

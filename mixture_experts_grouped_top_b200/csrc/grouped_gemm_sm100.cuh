@@ -6,7 +6,8 @@
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16 for
 //               bf16) into one of two tensor-memory accumulators (2 x 256 fp32 columns);
 //   warp 2      tensor-memory allocator;
-//   warps 4..7  epilogue: tcgen05.ld the accumulator (thread = row), apply the fused
+//   warps 4..11 epilogue: tcgen05.ld the accumulator (thread = row; two warps per
+//               32-lane quadrant, each taking half of the columns), apply the fused
 //               epilogue, store to global memory, release the accumulator.
 // Two grouping modes:
 //   M-grouped   rows of expert e are [off_e, off_e + n_e) of A and of the output; B is
@@ -31,7 +32,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;                                   // bf16: 128 bytes of K per row
 constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;                          // 4 control warps + 8 epilogue warps
 constexpr int kABytes = BM * BK * 2;                     // 16 KB
 constexpr int kBBytes = BN * BK * 2;                     // 32 KB
 constexpr int kChunkBytes = 64 * BK * 2;                 // one 64-wide MN chunk, 8 KB
@@ -39,7 +40,7 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;                           // two 256-column accumulators
 constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 1024 /*barriers*/ +
-                           2 * (kMaxE + 1) * 4 /*expert prefix tables*/;
+                           3 * (kMaxE + 1) * 4 /*expert prefix tables, expert order*/;
 constexpr uint64_t kTimeoutNs = 4000000000ull;           // 4 s per wait
 }  // namespace gg
 
@@ -64,7 +65,7 @@ struct GemmParams {
   const float* probs;          // [R] probability of each permuted row (nullable -> 1)
   const void* aux;             // DSwiGLU: saved h [R, 2F]
   long long ld_aux;
-  float* dprob_part;           // DSwiGLU: [ceil(N/256)][R] partial sums
+  float* dprob_part;           // DSwiGLU: [2 * ceil(N/256)][R] partial sums (one per N tile half)
   int F;                       // SwiGLU / DSwiGLU: width of the gate half
   int out_f32;                 // EPI_STORE: write fp32 instead of bf16
   uint64_t timeout_ns;
@@ -84,6 +85,7 @@ struct TileWalker {
   const int32_t* row_off;   // smem [E+1]
   const int32_t* tile_off;  // smem [E+1]
   int E, MT, NT, K;
+  const int32_t* order;     // K-grouped: experts by decreasing row count (longest tiles first)
   int cursor = 0;
 
   __device__ __forceinline__ int total() const { return tile_off[E]; }
@@ -92,8 +94,9 @@ struct TileWalker {
     TileInfo ti;
     if (KGROUP) {
       const int per = MT * NT;
-      ti.e = t / per;
-      const int local = t - ti.e * per;
+      const int rank = t / per;
+      ti.e = order[rank];
+      const int local = t - rank * per;
       ti.m_blk = local % MT;
       ti.n_blk = local / MT;
       ti.row0 = row_off[ti.e];
@@ -114,6 +117,21 @@ struct TileWalker {
     return ti;
   }
 };
+
+// Rank experts by decreasing row count (ties: lower index first) into order[0..E),
+// using every thread of the block; row_off must be complete. Static round-robin over
+// tiles in this order hands the longest contractions out first.
+__device__ __forceinline__ void rank_experts_by_rows(const int32_t* row_off, int E, int32_t* order) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int n = row_off[e + 1] - row_off[e];
+    int rank = 0;
+    for (int o = 0; o < E; ++o) {
+      const int m = row_off[o + 1] - row_off[o];
+      rank += (m > n) || (m == n && o < e);
+    }
+    order[rank] = e;
+  }
+}
 
 // Column of the B operand (output column space) of 64-wide chunk c of an N tile.
 template <int EPI>
@@ -143,6 +161,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
+  int32_t* order = tile_off + (kMaxE + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -158,7 +177,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 256);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -204,8 +223,12 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (KGROUP) {
+    rank_experts_by_rows(row_off, E, order);
+    __syncthreads();
+  }
 
-  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K};
+  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K, order};
   const int total = walk.total();
 
   if (warp == 0) {
@@ -331,7 +354,8 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------------- epilogue
-    const int q = warp - 4;                 // TMEM lane quadrant of this warp
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = (warp - 4) >> 2;       // which half of the tile's columns it drains
     const int r_local = q * 32 + lane;      // accumulator row owned by this thread
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
@@ -357,7 +381,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
         }
         const int n0 = ti.n_blk * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 16) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(t_row + c, v);
           tmem_wait_ld();
@@ -385,7 +409,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
         const int n0 = ti.n_blk * 128;
         __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 16) {
+        for (int c = half * 64; c < half * 64 + 64; c += 16) {
           uint32_t g[16], u[16];
           tmem_ld_32x32b_x16(t_row + c, g);
           tmem_ld_32x32b_x16(t_row + 128 + c, u);
@@ -430,7 +454,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
         const int n0 = ti.n_blk * BN;
         float dp = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 16) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(t_row + c, v);
           tmem_wait_ld();
@@ -469,7 +493,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
             du_dst[1] = ou[1];
           }
         }
-        if (row_ok) p.dprob_part[(long long)ti.n_blk * p.M + row] = dp;
+        if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

@@ -147,7 +147,8 @@ int quant_rows_launch(const void* in, long long rows, int cols, int mma, uint8_t
 int quant_cols_grouped_launch(const void* in, int R, int C, const int32_t* split_sizes, int E, uint8_t* codes,
                               uint8_t* atoms, cudaStream_t st) {
   const int blocks32 = R / 32 + E;   // upper bound of sum(ceil(n_e / 32))
-  dim3 grid(std::min(blocks32, device_props().sm_count * 32), (C + 255) / 256);
+  const int ytiles = (C + 1023) / 1024;
+  dim3 grid(std::min(blocks32, std::max(1, device_props().sm_count * 16 / ytiles)), ytiles);
   quant_cols_grouped_kernel<<<grid, 256, 3 * (E + 1) * sizeof(int32_t), st>>>(
       reinterpret_cast<const __nv_bfloat16*>(in), C, split_sizes, E, codes, atoms);
   count_launch();
@@ -520,7 +521,7 @@ size_t bwd_part_bytes(int part, int E, int R, int H, int F) {
   switch (part) {
     case 0: return align_up(r * 2 * f * 2, 256);
     case 1: return align_up(r * f * 2, 256);
-    case 2: return align_up((size_t)((F + gg::BN - 1) / gg::BN) * r * 4, 256);
+    case 2: return align_up((size_t)(2 * ((F + gg::BN - 1) / gg::BN)) * r * 4, 256);
     case 3: return align_up(e * f * h, 256) + align_up(e * f * h / 32, 256);
     case 4: return align_up(e * h * 2 * f, 256) + align_up(e * h * 2 * f / 32, 256);
     case 5: return align_up(r * h, 256) + align_up(r * h / 32, 256) + mma_atoms_bytes(E, R, H);
@@ -591,7 +592,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   uint8_t* xc = part(10);
   uint8_t* xc_a = xc + align_up((size_t)R * H, 256);
   const uint16_t* h_saved = reinterpret_cast<const uint16_t*>(saved);
-  const int nparts = (F + gg::BN - 1) / gg::BN;
+  const int nparts = 2 * ((F + gg::BN - 1) / gg::BN);   // one partial per N-tile half
   int rc;
   // weights along their other axis (the masters change every optimizer step)
   if ((rc = quant_rows_launch(w2, (long long)E * F, H, 1, w2q, w2a, st))) return rc;
@@ -705,7 +706,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
       reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256));
   uint16_t* dh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + bwd_part_offset(0, E, R, H, F, MOE_BF16));
   float* dpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + bwd_part_offset(2, E, R, H, F, MOE_BF16));
-  const int nparts = (F + gg::BN - 1) / gg::BN;
+  const int nparts = 2 * ((F + gg::BN - 1) / gg::BN);   // one partial per N-tile half
 
   CUtensorMap ta, tb;
   int rc;
