@@ -229,33 +229,30 @@ def run_ours(args, world, rank, local):
 
     # ------------------------------------------------ end to end through host buffers
     # every step: pinned host -> device copies of the step's inputs, the path, and a
-    # device -> host read of its result (the layer output; with backward also dx)
+    # device -> host read of its result (the layer output; with backward also dx), through
+    # the package's HostPipeline (transfers overlapped with the neighbouring steps' compute)
     x_h = d["x"].pin_memory()
     lg_h = d["logits"].pin_memory()
     g_h = d["grad_out"].pin_memory() if training else None
     out_h = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
     dx_h = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() if training else None
-    xd, lgd = torch.empty_like(x), torch.empty_like(logits)
-    gd = torch.empty_like(grad) if training else None
+    pipe = mb.HostPipeline(layer)
 
     def e2e_step():
-        xd.copy_(x_h, non_blocking=True)
-        lgd.copy_(lg_h, non_blocking=True)
-        out = layer.forward(xd, lgd)
-        out_h.copy_(out, non_blocking=True)
-        if training:
-            gd.copy_(g_h, non_blocking=True)
-            dx = layer.backward(gd)[0]
-            dx_h.copy_(dx, non_blocking=True)
+        if training and prec == "mxfp8":
+            layer.set_weights(w1, w2)
+        pipe.step(x_h, lg_h, out_h, g_h, dx_h)
 
     for _ in range(2):
         e2e_step()
+    pipe.flush()
     torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(K):
         e2e_step()
+    pipe.flush()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world)

@@ -278,4 +278,4 @@ def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precisi
     return dxp, dw1, dw2, dprobs_perm
 
 
-from .layer import MoEExpertLayer, moe_layer_forward  # noqa: E402,F401
+from .layer import HostPipeline, MoEExpertLayer, moe_layer_forward  # noqa: E402,F401

@@ -118,3 +118,67 @@ def moe_layer_forward(x, logits, w1, w2, k: int, precision="bf16", stream=None):
     layer = MoEExpertLayer(T, H, F2 // 2, E, k, precision, device=x.device)
     layer.set_weights(w1, w2, stream=stream)
     return layer.forward(x, logits, stream=stream), layer
+
+
+class HostPipeline:
+    """Run a layer on host (pinned) buffers with the transfers overlapped.
+
+    Each call to :meth:`step` uploads one batch (x, logits, and grad_out for a training
+    layer) on an upload stream, runs the layer on the compute stream, and downloads its
+    result (the output; with backward also dx) on a download stream. Device input and
+    output buffers are double-buffered, so step i's upload and step i-1's download run
+    while step i-1 / i compute. :meth:`flush` waits for everything issued.
+    """
+
+    def __init__(self, layer: MoEExpertLayer):
+        self.layer = layer
+        dev = layer.device
+        T, H, E = layer.T, layer.H, layer.E
+        bf = torch.bfloat16
+        self.compute = torch.cuda.current_stream(dev)
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.x = [torch.empty((T, H), dtype=bf, device=dev) for _ in range(2)]
+        self.lg = [torch.empty((T, E), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.g = [torch.empty((T, H), dtype=bf, device=dev) for _ in range(2)] if layer.training else None
+        self.out = [torch.empty((T, H), dtype=bf, device=dev) for _ in range(2)]
+        self.dx = [torch.empty((T, H), dtype=bf, device=dev) for _ in range(2)] if layer.training else None
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.inputs_free = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    def step(self, x_h, logits_h, out_h, grad_h=None, dx_h=None):
+        b = self.i & 1
+        # upload into buffer b once the step that last used it has consumed its inputs
+        self.up.wait_event(self.inputs_free[b])
+        with torch.cuda.stream(self.up):
+            self.x[b].copy_(x_h, non_blocking=True)
+            self.lg[b].copy_(logits_h, non_blocking=True)
+            if self.g is not None:
+                self.g[b].copy_(grad_h, non_blocking=True)
+            self.uploaded[b].record(self.up)
+        # compute once the inputs are there and the previous download of buffer b is done
+        self.compute.wait_event(self.uploaded[b])
+        self.compute.wait_event(self.downloaded[b])
+        with torch.cuda.stream(self.compute):
+            out = self.layer.forward(self.x[b], self.lg[b], stream=self.compute)
+            self.out[b].copy_(out, non_blocking=True)
+            if self.g is not None:
+                dx = self.layer.backward(self.g[b], stream=self.compute)[0]
+                self.dx[b].copy_(dx, non_blocking=True)
+            self.inputs_free[b].record(self.compute)
+            self.computed[b].record(self.compute)
+        # download the result
+        self.down.wait_event(self.computed[b])
+        with torch.cuda.stream(self.down):
+            out_h.copy_(self.out[b], non_blocking=True)
+            if self.dx is not None:
+                dx_h.copy_(self.dx[b], non_blocking=True)
+            self.downloaded[b].record(self.down)
+        self.i += 1
+
+    def flush(self):
+        self.compute.wait_stream(self.up)
+        self.compute.wait_stream(self.down)
