@@ -1,0 +1,238 @@
+// Grouped GEMM on a pair of SMs (tcgen05.mma.cta_group::2), BF16, M-grouped.
+//
+// A 2-CTA cluster computes 256 x 256 output tiles: each CTA loads its own 128 rows of A
+// and its own half (128 columns) of B into its shared memory, the pair leader issues
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16) that reads both CTAs' operands, and each
+// CTA receives the 128 x 256 fp32 accumulator of its rows in its own tensor memory. Per
+// SM, a 64-wide k-stage moves 32 KB through shared memory instead of 48 KB for a 1-SM
+// 128 x 256 tile, and 6 stages fit instead of 4.
+//
+// Synchronisation: both CTAs' TMA loads complete on the leader's `full` barrier (the
+// 2-SM TMA form); the leader's MMA commits arrive on the `empty` and `tfull` barriers of
+// both CTAs (multicast commit, no multicast loads); both CTAs' epilogue warps arrive on
+// the leader's `tempty` barrier. Waits are bounded like in the 1-SM kernel.
+//
+// For fc1 the leader's half of B is the gate columns [n0, n0+128) and the other CTA's
+// the up columns [F+n0, F+n0+128), so each CTA's accumulator holds [gate | up] for its
+// rows and the ScaledSwiGLU epilogue stays thread-local.
+#pragma once
+#include "grouped_gemm_sm100.cuh"
+
+namespace moe {
+
+namespace g2 {
+constexpr int BM = 256;                       // rows of a pair tile
+constexpr int BMC = 128;                      // rows per CTA
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kStages = 6;
+constexpr int kThreads = 384;
+constexpr int kABytes = BMC * BK * 2;         // 16 KB
+constexpr int kBBytes = (BN / 2) * BK * 2;    // 16 KB: this CTA's half of B
+constexpr int kChunkBytes = 64 * BK * 2;      // 8 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kMaxE = 1024;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024 + 2 * (kMaxE + 1) * 4;
+}  // namespace g2
+
+template <bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
+    grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                  const GemmParams p) {
+  using namespace g2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full = bars;                      // used in the leader
+  uint64_t* empty = bars + kStages;           // both CTAs
+  uint64_t* tfull = bars + 2 * kStages;       // both CTAs
+  uint64_t* tempty = bars + 2 * kStages + 2;  // used in the leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
+  int32_t* tile_off = row_off + (kMaxE + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int E = p.E;
+  const int NT = (EPI == EPI_SWIGLU) ? (p.N / 128) : (p.N + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);   // 8 epilogue warps in each CTA of the pair
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 3) {
+    int carry_r = 0, carry_t = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? p.split_sizes[e] : 0;
+      const int tiles = (e < E) ? ((n + BM - 1) / BM) * NT : 0;
+      int ir = n, it = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yt = __shfl_up_sync(0xffffffffu, it, o);
+        if (lane >= o) {
+          ir += yr;
+          it += yt;
+        }
+      }
+      if (e < E) {
+        row_off[e] = carry_r + ir - n;
+        tile_off[e] = carry_t + it - tiles;
+      }
+      carry_r += __shfl_sync(0xffffffffu, ir, 31);
+      carry_t += __shfl_sync(0xffffffffu, it, 31);
+    }
+    if (lane == 0) {
+      row_off[E] = carry_r;
+      tile_off[E] = carry_t;
+    }
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  TileWalker<false, BM> walk{row_off, tile_off, E, 0, NT, p.K, nullptr};
+  const int total = walk.total();
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileInfo ti = walk.decode(t);
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          const int k0 = kb * BK;
+          tma_load_3d_pair(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0 + BMC * rank, 0);
+          uint8_t* b_dst = sB + stage * kBBytes;
+          if (B_MN) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int col = (EPI == EPI_SWIGLU) ? (rank == 0 ? 0 : p.F) + ti.n_blk * 128 + 64 * c
+                                                  : ti.n_blk * BN + 128 * rank + 64 * c;
+              tma_load_3d_pair(b_dst + c * kChunkBytes, &tmB, &full[stage], col, k0, ti.e);
+            }
+          } else {
+            tma_load_3d_pair(b_dst, &tmB, &full[stage], k0, ti.n_blk * BN + 128 * rank, ti.e);
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let this CTA's copies land before it can exit (their bytes count on the leader)
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 100000000ull) {
+        }
+        (void)issued;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (pair leader)
+    if (leader) {
+      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+        const TileInfo ti = walk.decode(t);
+        const int acc = lt & 1;
+        if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+            const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t adesc = make_sdesc(a_addr + kk * 32, 16, 1024, 2);
+              const uint64_t bdesc = B_MN ? make_sdesc(b_addr + kk * 2048, kChunkBytes, 1024, 2)
+                                          : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
+              mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_pair(&empty[stage]);
+          }
+          __syncwarp();
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_pair(&tfull[acc]);
+        __syncwarp();
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r_local = q * 32 + lane;
+    const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
+    int lt = 0;
+    for (int t = pair; t < total; t += npairs, ++lt) {
+      const TileInfo ti = walk.decode(t);
+      const int acc = lt & 1;
+      if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
+      bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();   // neither CTA leaves while the other can still signal it
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -80,7 +80,7 @@ struct TileInfo {
   int num_kb;     // k-blocks
 };
 
-template <bool KGROUP>
+template <bool KGROUP, int TBM = gg::BM>
 struct TileWalker {
   const int32_t* row_off;   // smem [E+1]
   const int32_t* tile_off;  // smem [E+1]
@@ -106,12 +106,12 @@ struct TileWalker {
       while (tile_off[cursor + 1] <= t) ++cursor;
       ti.e = cursor;
       const int n_e = row_off[ti.e + 1] - row_off[ti.e];
-      const int mt = (n_e + gg::BM - 1) / gg::BM;
+      const int mt = (n_e + TBM - 1) / TBM;
       const int local = t - tile_off[ti.e];
       ti.m_blk = local % mt;
       ti.n_blk = local / mt;
-      ti.row0 = row_off[ti.e] + ti.m_blk * gg::BM;
-      ti.rows = min(gg::BM, n_e - ti.m_blk * gg::BM);
+      ti.row0 = row_off[ti.e] + ti.m_blk * TBM;
+      ti.rows = min(TBM, n_e - ti.m_blk * TBM);
       ti.num_kb = K / gg::BK;
     }
     return ti;
@@ -141,6 +141,143 @@ __device__ __forceinline__ int b_chunk_col(int n_blk, int c, int F) {
     return (c < 2) ? n0 + 64 * c : F + n0 + 64 * (c - 2);
   }
   return n_blk * gg::BN + 64 * c;
+}
+
+// Drain one BF16 accumulator tile: this thread owns row `tile_row` of the tile (its TMEM
+// lane is folded into t_row) and the columns of `half`; applies the fused epilogue EPI.
+template <int EPI>
+__device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const TileInfo& ti, uint32_t t_row, int half,
+                                                   int tile_row, int tile_bm) {
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+
+  if (EPI == EPI_STORE || EPI == EPI_WGRAD) {
+    const bool zero = (ti.num_kb == 0);
+    long long orow;
+    bool row_ok;
+    if (EPI == EPI_WGRAD) {
+      const int m = ti.m_blk * tile_bm + tile_row;
+      row_ok = m < p.M;
+      orow = (long long)ti.e * p.out_batch + (long long)m * p.ldo;
+    } else {
+      row_ok = tile_row < ti.rows;
+      orow = (long long)(ti.row0 + tile_row) * p.ldo;
+    }
+    const int n0 = ti.n_blk * gg::BN;
+#pragma unroll 1
+    for (int c = half * (gg::BN / 2); c < (half + 1) * (gg::BN / 2); c += 16) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(t_row + c, v);
+      tmem_wait_ld();
+      if (row_ok && n0 + c < p.N) {
+        if (EPI == EPI_STORE && p.out_f32) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+          uint4 o[2];
+          uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c);
+          dst[0] = o[0];
+          dst[1] = o[1];
+        }
+      }
+    }
+  } else if (EPI == EPI_SWIGLU) {
+    const bool row_ok = tile_row < ti.rows;
+    const long long row = ti.row0 + tile_row;
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const int n0 = ti.n_blk * 128;
+    __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
+#pragma unroll 1
+    for (int c = half * 64; c < half * 64 + 64; c += 16) {
+      uint32_t g[16], u[16];
+      tmem_ld_32x32b_x16(t_row + c, g);
+      tmem_ld_32x32b_x16(t_row + 128 + c, u);
+      tmem_wait_ld();
+      if (row_ok) {
+        uint4 o[2];
+        uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+          const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+          ow[i] = pack_bf16x2(silu_f(g0) * u0 * pr, silu_f(g1) * u1 * pr);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c);
+        dst[0] = o[0];
+        dst[1] = o[1];
+        if (hout) {
+          uint4 hg[2], hu[2];
+          uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
+          uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            hgw[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+            huw[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+          }
+          uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c);
+          hd[0] = hg[0];
+          hd[1] = hg[1];
+          uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c);
+          hd2[0] = hu[0];
+          hd2[1] = hu[1];
+        }
+      }
+    }
+  } else if (EPI == EPI_DSWIGLU) {
+    // acc = da for columns [n0, n0+256) of F; h = [g | u] saved by the forward
+    const bool row_ok = tile_row < ti.rows;
+    const long long row = ti.row0 + tile_row;
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
+    __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
+    const int n0 = ti.n_blk * gg::BN;
+    float dp = 0.f;
+#pragma unroll 1
+    for (int c = half * (gg::BN / 2); c < (half + 1) * (gg::BN / 2); c += 16) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(t_row + c, v);
+      tmem_wait_ld();
+      if (row_ok && n0 + c < p.N) {
+        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + n0 + c);
+        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + n0 + c);
+        uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
+        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
+        uint4 og[2], ou[2];
+        uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
+        uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 gg2 = __bfloat1622float2(g2[i]);
+          const float2 uu2 = __bfloat1622float2(u2[i]);
+          float dg[2], du[2];
+          const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float da = __uint_as_float(v[2 * i + j]);
+            const float sg = 1.0f / (1.0f + expf(-gs[j]));
+            const float sl = gs[j] * sg;
+            dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+            du[j] = da * pr * sl;
+            dp = fmaf(da, sl * us[j], dp);
+          }
+          ogw[i] = pack_bf16x2(dg[0], dg[1]);
+          ouw[i] = pack_bf16x2(du[0], du[1]);
+        }
+        uint4* dg_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + n0 + c);
+        dg_dst[0] = og[0];
+        dg_dst[1] = og[1];
+        uint4* du_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + n0 + c);
+        du_dst[0] = ou[0];
+        du_dst[1] = ou[1];
+      }
+    }
+    if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
+  }
 }
 
 template <bool A_MN, bool B_MN, bool KGROUP, int EPI>
@@ -365,136 +502,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-
-      if (EPI == EPI_STORE || EPI == EPI_WGRAD) {
-        const bool zero = (ti.num_kb == 0);
-        long long orow;
-        bool row_ok;
-        if (EPI == EPI_WGRAD) {
-          const int m = ti.m_blk * BM + r_local;
-          row_ok = m < p.M;
-          orow = (long long)ti.e * p.out_batch + (long long)m * p.ldo;
-        } else {
-          row_ok = r_local < ti.rows;
-          orow = (long long)(ti.row0 + r_local) * p.ldo;
-        }
-        const int n0 = ti.n_blk * BN;
-#pragma unroll 1
-        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + c, v);
-          tmem_wait_ld();
-          if (row_ok && n0 + c < p.N) {
-            if (EPI == EPI_STORE && p.out_f32) {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-              uint4 o[2];
-              uint32_t* ow = reinterpret_cast<uint32_t*>(o);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-              uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c);
-              dst[0] = o[0];
-              dst[1] = o[1];
-            }
-          }
-        }
-      } else if (EPI == EPI_SWIGLU) {
-        const bool row_ok = r_local < ti.rows;
-        const long long row = ti.row0 + r_local;
-        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-        const int n0 = ti.n_blk * 128;
-        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
-#pragma unroll 1
-        for (int c = half * 64; c < half * 64 + 64; c += 16) {
-          uint32_t g[16], u[16];
-          tmem_ld_32x32b_x16(t_row + c, g);
-          tmem_ld_32x32b_x16(t_row + 128 + c, u);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint4 o[2];
-            uint32_t* ow = reinterpret_cast<uint32_t*>(o);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              ow[i] = pack_bf16x2(silu_f(g0) * u0 * pr, silu_f(g1) * u1 * pr);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c);
-            dst[0] = o[0];
-            dst[1] = o[1];
-            if (hout) {
-              uint4 hg[2], hu[2];
-              uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
-              uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                hgw[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                huw[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
-              }
-              uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c);
-              hd[0] = hg[0];
-              hd[1] = hg[1];
-              uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c);
-              hd2[0] = hu[0];
-              hd2[1] = hu[1];
-            }
-          }
-        }
-      } else if (EPI == EPI_DSWIGLU) {
-        // acc = da for columns [n0, n0+256) of F; h = [g | u] saved by the forward
-        const bool row_ok = r_local < ti.rows;
-        const long long row = ti.row0 + r_local;
-        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
-        __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
-        const int n0 = ti.n_blk * BN;
-        float dp = 0.f;
-#pragma unroll 1
-        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + c, v);
-          tmem_wait_ld();
-          if (row_ok && n0 + c < p.N) {
-            const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + n0 + c);
-            const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + n0 + c);
-            uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
-            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
-            uint4 og[2], ou[2];
-            uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
-            uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 gg2 = __bfloat1622float2(g2[i]);
-              const float2 uu2 = __bfloat1622float2(u2[i]);
-              float dg[2], du[2];
-              const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const float da = __uint_as_float(v[2 * i + j]);
-                const float sg = 1.0f / (1.0f + expf(-gs[j]));
-                const float sl = gs[j] * sg;
-                dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
-                du[j] = da * pr * sl;
-                dp = fmaf(da, sl * us[j], dp);
-              }
-              ogw[i] = pack_bf16x2(dg[0], dg[1]);
-              ouw[i] = pack_bf16x2(du[0], du[1]);
-            }
-            uint4* dg_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + n0 + c);
-            dg_dst[0] = og[0];
-            dg_dst[1] = og[1];
-            uint4* du_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + n0 + c);
-            du_dst[0] = ou[0];
-            du_dst[1] = ou[1];
-          }
-        }
-        if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
-      }
+      bf16_epilogue_tile<EPI>(p, ti, t_row, half, r_local, BM);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

@@ -10,6 +10,7 @@
 
 #include "moe_grouped.h"
 #include "grouped_gemm_mxf8_sm100.cuh"
+#include "grouped_gemm_pair_sm100.cuh"
 #include "grouped_gemm_sm100.cuh"
 #include "token_kernels.cuh"
 
@@ -109,6 +110,34 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
   const int grid = device_props().sm_count;
   kern<<<grid, gg::kThreads, gg::kSmemBytes, st>>>(ta, tb, p);
+  count_launch();
+  return launch_status();
+}
+
+// CTA-pair kernels: launch as many 2-CTA clusters as can be resident at once (a
+// persistent grid larger than that would leave some pairs waiting for others to finish).
+template <bool B_MN, int EPI>
+int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+  auto kern = grouped_gemm_bf16_pair_kernel<B_MN, EPI>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int pairs = 0;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g2::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(device_props().sm_count, 1, 1);
+    cfg.blockDim = dim3(g2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = g2::kSmemBytes;
+    cfg.attrs = nullptr;   // the kernel declares its 2-CTA cluster at compile time
+    cfg.numAttrs = 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_props().sm_count / 2;
+    pairs = std::min(n, device_props().sm_count / 2);
+    cudaGetLastError();
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  kern<<<2 * pairs, g2::kThreads, g2::kSmemBytes, st>>>(ta, tb, p);
   count_launch();
   return launch_status();
 }
@@ -491,7 +520,7 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   p1.ldo2 = 2 * F;
   p1.probs = probs_perm;
   p1.F = F;
-  if ((rc = launch_gemm<false, true, false, EPI_SWIGLU>(ta, tb, p1, st))) return rc;
+  if ((rc = launch_gemm_pair<true, EPI_SWIGLU>(ta, tb, p1, st))) return rc;
   // fc2: A = a [R, F] (K-major), B = w2 [E, F, H] (MN-major)
   if ((rc = tmap_bf16_2d(&ta, a_buf, R, F, gg::BM))) return rc;
   if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, 64))) return rc;
@@ -502,7 +531,7 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   p2.out = yp;
   p2.ldo = H;
   p2.out_f32 = out_f32;
-  return launch_gemm<false, true, false, EPI_STORE>(ta, tb, p2, st);
+  return launch_gemm_pair<true, EPI_STORE>(ta, tb, p2, st);
 }
 
 }  // extern "C"
@@ -712,7 +741,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   int rc;
   // fc2 dgrad + SwiGLU backward: A = dy [R, H] (K-major), B = w2 [E, F, H] read as [E, N=F, K=H] (K-major)
   if ((rc = tmap_bf16_2d(&ta, dy_perm, R, H, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, gg::BN))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, g2::BN / 2))) return rc;
   GemmParams p = base_params(split_sizes, E);
   p.M = R;
   p.N = F;
@@ -724,7 +753,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.ld_aux = 2 * F;
   p.dprob_part = dpart;
   p.F = F;
-  if ((rc = launch_gemm<false, false, false, EPI_DSWIGLU>(ta, tb, p, st))) return rc;
+  if ((rc = launch_gemm_pair<false, EPI_DSWIGLU>(ta, tb, p, st))) return rc;
   if (dprobs_perm) {
     const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
     reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
@@ -743,14 +772,14 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   if ((rc = launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh [R, 2F] (K-major), B = w1 [E, H, 2F] read as [E, N=H, K=2F] (K-major)
   if ((rc = tmap_bf16_2d(&ta, dh, R, 2 * F, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, gg::BN))) return rc;
+  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, g2::BN / 2))) return rc;
   p = base_params(split_sizes, E);
   p.M = R;
   p.N = H;
   p.K = 2 * F;
   p.out = dxp;
   p.ldo = H;
-  if ((rc = launch_gemm<false, false, false, EPI_STORE>(ta, tb, p, st))) return rc;
+  if ((rc = launch_gemm_pair<false, EPI_STORE>(ta, tb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e. A = xp [R, H] (MN-major), B = dh [R, 2F] (MN-major)
   if ((rc = tmap_bf16_2d(&ta, xp, R, H, 64))) return rc;
   if ((rc = tmap_bf16_2d(&tb, dh, R, 2 * F, 64))) return rc;
