@@ -1,0 +1,329 @@
+// MXFP8 grouped GEMM on a pair of SMs (tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale),
+// M-grouped (ragged expert rows): fc1 + ScaledSwiGLU + MXFP8 quantisation, fc2, and the
+// two data-gradient GEMMs of the backward.
+//
+// Pages: "Efficient MoE training for biological foundation models" (news.bpdata.com
+// sections 2-3: MXFP8 operands with one scale per 32 K values consumed by the tensor
+// cores, the fused GroupedLinear -> ScaledSwiGLU -> GroupedLinear chain).
+//
+// A 2-CTA cluster computes 256 x 256 output tiles; the pair leader issues M=256, N=256,
+// K=32 MMAs that read each CTA's 128 rows of A and 128 rows (its half) of B.
+//
+// Feeding: issuing a TMA copy costs about the same whatever its size, so a copy per
+// 512-byte scale atom every 128-wide k-block starved the tensor pipe. Here
+//   * a k-stage is 256 wide: ONE copy per operand per stage brings two 128-byte k-chunks
+//     of 128 rows (a 4-D view of the codes, box {128, 128, 2, 1}): 64 KB per CTA, 3 stages;
+//   * scale atoms travel on their own two-slot ring, four k-blocks per copy (2 KB): per
+//     two stages, one copy for this CTA's A rows and two for the B tile's two 128-row
+//     groups (the block-scaled pair MMA reads every N column's scales from each CTA's own
+//     tensor memory, so both CTAs fetch both B groups). The leader copies a k-block's
+//     atoms into both CTAs' tensor memory (tcgen05.cp.cta_group::2) before its MMAs.
+//
+// Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [224, 480),
+// A scales at 480, B scales at 484..491; `tovl` and `tempty` live in the leader and count
+// one arrival per epilogue warp of both CTAs. Waits are bounded like in every other
+// kernel of this library.
+#pragma once
+#include "grouped_gemm_mxf8_sm100.cuh"
+
+namespace moe {
+
+namespace mx2 {
+constexpr int BM = 256;                       // rows of a pair tile
+constexpr int BMC = 128;                      // rows per CTA
+constexpr int BN = 256;
+constexpr int BK = 256;                       // k per stage: two 128-byte chunks
+constexpr int kStages = 3;
+constexpr int kThreads = 384;
+constexpr int kChunkBytes = 128 * 128;        // one k-chunk of 128 rows, 16 KB
+constexpr int kABytes = BMC * BK;             // 32 KB
+constexpr int kBBytes = (BN / 2) * BK;        // 32 KB: this CTA's half of B
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kSfKb = 4;                      // k-blocks (of 128) per scale copy
+constexpr int kSfGroupBytes = kSfKb * 512;    // 2 KB: one row group's atoms for kSfKb k-blocks
+constexpr int kSfSlotBytes = 3 * kSfGroupBytes;   // A group, B lower group, B upper group
+constexpr int kSfSlots = 2;
+
+constexpr int kMaxE = 1024;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBytes =
+    1024 + kStages * kStageBytes + kSfSlots * kSfSlotBytes + 1024 + 3 * (kMaxE + 1) * 4;
+}  // namespace mx2
+
+// tmA / tmB: E4M3 codes [rows, K] / [E][b_rows][K] as {128, rows, K/128 chunks, batch},
+// box {128, 128, 2, 1}. tmSa / tmSb: scale atoms as uint32 tensors {128 words, K/128
+// k-blocks, row groups} with a box of four atoms (no swizzle); A's row groups are the
+// experts' 128-row tiles in order, B's are e * (b_rows / 128) + row / 128.
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
+    grouped_gemm_mxf8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                  const __grid_constant__ CUtensorMap tmSa, const __grid_constant__ CUtensorMap tmSb,
+                                  const MxGemmParams mp) {
+  using namespace mx2;
+  const GemmParams& p = mp.g;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kStages * kABytes;
+  uint8_t* sSf = sB + kStages * kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSf + kSfSlots * kSfSlotBytes);
+  uint64_t* full = bars;                      // used in the leader
+  uint64_t* empty = bars + kStages;           // both CTAs
+  uint64_t* tfull = bars + 2 * kStages;       // both CTAs
+  uint64_t* tempty = bars + 2 * kStages + 2;  // used in the leader
+  uint64_t* tovl = bars + 2 * kStages + 4;    // used in the leader
+  uint64_t* sfull = bars + 2 * kStages + 5;   // scale ring: used in the leader
+  uint64_t* sempty = sfull + kSfSlots;        // scale ring: both CTAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSfSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
+  int32_t* tile_off = row_off + (kMaxE + 1);
+  int32_t* grp_off = tile_off + (kMaxE + 1);  // 128-row scale groups of earlier experts
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int E = p.E;
+  const int NT = (EPI == MXEPI_SWIGLU_Q) ? (p.N / 128) : (p.N + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);   // 8 epilogue warps in each CTA of the pair
+    }
+    mbar_init(tovl, 16);
+    for (int s2 = 0; s2 < kSfSlots; ++s2) {
+      mbar_init(&sfull[s2], 1);
+      mbar_init(&sempty[s2], 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSa);
+    tma_prefetch_desc(&tmSb);
+  }
+  if (warp == 3) {
+    int carry_r = 0, carry_t = 0, carry_g = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? p.split_sizes[e] : 0;
+      const int tiles = (e < E) ? ((n + BM - 1) / BM) * NT : 0;
+      const int grps = (n + BMC - 1) / BMC;
+      int ir = n, it = tiles, ig = grps;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yt = __shfl_up_sync(0xffffffffu, it, o);
+        const int yg = __shfl_up_sync(0xffffffffu, ig, o);
+        if (lane >= o) {
+          ir += yr;
+          it += yt;
+          ig += yg;
+        }
+      }
+      if (e < E) {
+        row_off[e] = carry_r + ir - n;
+        tile_off[e] = carry_t + it - tiles;
+        grp_off[e] = carry_g + ig - grps;
+      }
+      carry_r += __shfl_sync(0xffffffffu, ir, 31);
+      carry_t += __shfl_sync(0xffffffffu, it, 31);
+      carry_g += __shfl_sync(0xffffffffu, ig, 31);
+    }
+    if (lane == 0) {
+      row_off[E] = carry_r;
+      tile_off[E] = carry_t;
+      grp_off[E] = carry_g;
+    }
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  TileWalker<false, BM> walk{row_off, tile_off, E, 0, NT, p.K, nullptr};
+  const int total = walk.total();
+  const int kblocks = p.K / 128;                      // 128-wide k-blocks (K is a multiple of 128)
+  const int num_st = (kblocks + 1) / 2;               // stages; an odd last k-block reads zeros past K
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0, sslot = 0;
+      uint32_t phase = 0, sphase = 0;
+      bool ok = true;
+      const int bgroups = mp.b_rows / 128;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileInfo ti = walk.decode(t);
+        const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
+        // this CTA's A rows and their scale group (past the expert: unused rows; a group
+        // index past the atom tensor reads zeros)
+        const int a_row = ti.row0 + BMC * (int)rank;
+        const int ga = grp_off[ti.e] + 2 * ti.m_blk + (int)rank;
+        // this CTA's half of B, and the scale groups of both halves
+        const int b_row = (EPI == MXEPI_SWIGLU_Q) ? (rank ? p.F : 0) + n0 : n0 + 128 * (int)rank;
+        const int gb0 = ti.e * bgroups + n0 / 128;
+        int gb1 = (EPI == MXEPI_SWIGLU_Q) ? ti.e * bgroups + (p.F + n0) / 128 : gb0 + 1;
+        if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+        for (int st = 0; st < num_st; ++st) {
+          if ((st & 1) == 0) {
+            // scale atoms of k-blocks [2 st, 2 st + 4) (past K: zeros)
+            if (!mbar_wait_bounded(&sempty[sslot], sphase ^ 1, abort_flag, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&sfull[sslot], 2 * kSfSlotBytes);
+            uint8_t* sd = sSf + sslot * kSfSlotBytes;
+            tma_load_3d_pair(sd, &tmSa, &sfull[sslot], 0, 2 * st, ga);
+            tma_load_3d_pair(sd + kSfGroupBytes, &tmSb, &sfull[sslot], 0, 2 * st, gb0);
+            tma_load_3d_pair(sd + 2 * kSfGroupBytes, &tmSb, &sfull[sslot], 0, 2 * st, gb1);
+            if (++sslot == kSfSlots) {
+              sslot = 0;
+              sphase ^= 1;
+            }
+          }
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, 2 * st, 0);
+          tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b_row, 2 * st, ti.e);
+
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let this CTA's copies land before it can exit (their bytes count on the leader)
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (pair leader)
+    if (leader) {
+      int stage = 0, sslot = 0;
+      uint32_t phase = 0, sphase = 0;
+      int lt = 0;
+      bool ok = true;
+      const uint32_t sfa_t = tmem_base + mx::kSfaCol;
+      const uint32_t sfb_t = tmem_base + mx::kSfbCol;
+      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+        const int acc = lt & 1;
+        if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+        if (lt > 0 && !mbar_wait_bounded(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (acc ? mx::kAcc1Col : 0u);
+        for (int st = 0; st < num_st; ++st) {
+          if ((st & 1) == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sf_s = smem_u32(sSf + sslot * kSfSlotBytes);
+            const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+            const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int kb = 2 * st + c;
+              if (kb < kblocks) {
+                // this k-block's atoms: entry kb % 4 of each 2 KB group of the slot
+                const uint32_t q = (uint32_t)(kb & (kSfKb - 1)) * 512;
+                tmem_cp_32x128b_warpx4_pair(sfa_t, make_sdesc(sf_s + q, 0, 128, 0));
+                tmem_cp_32x128b_warpx4_pair(sfb_t, make_sdesc(sf_s + kSfGroupBytes + q, 0, 128, 0));
+                tmem_cp_32x128b_warpx4_pair(sfb_t + 4, make_sdesc(sf_s + 2 * kSfGroupBytes + q, 0, 128, 0));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t adesc = make_sdesc(a_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
+                  const uint64_t bdesc = make_sdesc(b_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
+                  const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk);
+                  mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30),
+                                sfb_t | ((uint32_t)kk << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+                }
+              }
+            }
+            mma_commit_pair(&empty[stage]);
+            // the slot's last stage: release it once these MMAs have read their scales
+            if ((st & 1) == 1 || st == num_st - 1) mma_commit_pair(&sempty[sslot]);
+          }
+          __syncwarp();
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if ((st & 1) == 1 || st == num_st - 1) {
+            if (++sslot == kSfSlots) {
+              sslot = 0;
+              sphase ^= 1;
+            }
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_pair(&tfull[acc]);
+        __syncwarp();
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r_local = q * 32 + lane;
+    const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
+    const uint32_t tovl_leader = map_to_rank(smem_u32(tovl), 0);
+    int lt = 0;
+    for (int t = pair; t < total; t += npairs, ++lt) {
+      const TileInfo ti = walk.decode(t);
+      const int acc = lt & 1;
+      if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (acc ? mx::kAcc1Col : 0u) + ((uint32_t)(q * 32) << 16);
+      const uint32_t sc_word = mxf8_epilogue_tile<EPI>(mp, ti, t_row, acc, half, BMC * (int)rank + r_local, BM, [&] {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tovl_leader);
+      });
+      if (EPI == MXEPI_SWIGLU_Q && BMC * (int)rank < ti.rows) {
+        // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`; rows
+        // past the expert in it store 0 (a CTA entirely past the expert writes nothing)
+        const size_t g = (size_t)(grp_off[ti.e] + 2 * ti.m_blk + (int)rank);
+        *reinterpret_cast<uint16_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk + 2 * half,
+                                                                     p.N / 128)) =
+            (uint16_t)(sc_word >> (16 * half));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // neither CTA leaves while the other can still signal it
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

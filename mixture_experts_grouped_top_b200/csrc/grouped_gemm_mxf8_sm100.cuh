@@ -64,6 +64,210 @@ struct MxGemmParams {
   uint8_t* out_atoms;         // MXEPI_SWIGLU_Q: scales of `a` as atoms for the next GEMM (K = F)
 };
 
+// Drains one 128-row x 256-column accumulator (this thread's row: lane quadrant of
+// `t_row`, row r_local of the output tile) and runs the epilogue EPI on it. The 32-column
+// strip that acc0 and acc1 share is drained first by its owning half, which then calls
+// `strip_done()`; the other half calls it before reading anything (warp-uniform calls, so
+// the callee may signal once per warp). Returns the SwiGLU_Q row's four scale bytes.
+template <int EPI, class StripDone>
+__device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, const TileInfo& ti, uint32_t t_row,
+                                                       int acc, int half, int r_local, int tile_bm,
+                                                       StripDone&& strip_done) {
+  using mx::BN;
+  const GemmParams& p = mp.g;
+  const bool row_ok = r_local < ti.rows;
+  const long long row = ti.row0 + r_local;
+  uint32_t sc_word = 0;   // SwiGLU: this row's four scale bytes (k-blocks 4*n_blk..+3 of the next GEMM)
+
+  if (EPI == MXEPI_STORE || EPI == MXEPI_WGRAD) {
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    const int n0 = ti.n_blk * BN;
+    long long orow;
+    bool ok_row;
+    bool zero = false;
+    if (EPI == MXEPI_WGRAD) {
+      const int m = ti.m_blk * tile_bm + r_local;
+      ok_row = m < p.M;
+      orow = (long long)ti.e * p.out_batch + (long long)m * p.ldo;
+      zero = ti.rows == 0;
+    } else {
+      ok_row = row_ok;
+      orow = row * p.ldo;
+    }
+    // the 32-column strip shared with the other accumulator: chunk 7 of acc0 (upper
+    // half), chunk 0 of acc1 (lower half); its owner drains it first, then signals
+    const bool owner = acc ? (half == 0) : (half == 1);
+    if (!owner) strip_done();
+#pragma unroll 1
+    for (int it = 0; it < 4; ++it) {
+      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      uint32_t v0[16], v1[16];
+      tmem_ld_32x32b_x16(t_row + c * 32, v0);
+      tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
+      tmem_wait_ld();
+      if (owner && it == 0) {
+        tc_fence_before();
+        strip_done();
+      }
+      if (ok_row && n0 + c * 32 < p.N && p.out_f32) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dst[i] = make_uint4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
+          dst[4 + i] = make_uint4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
+        }
+      } else if (ok_row && n0 + c * 32 < p.N) {
+        uint4 o[4];
+        uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+          ow[8 + i] = zero ? 0u : pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = o[i];
+      }
+    }
+  } else if (EPI == MXEPI_DSWIGLU) {
+    // acc = da for columns [n0, n0+256) of F. With h = [g | u] from the forward:
+    // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u; a = SiLU(g) u p is
+    // recomputed (bf16) for the fc2 weight gradient.
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
+    __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
+    __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    const int n0 = ti.n_blk * BN;
+    const bool owner = acc ? (half == 0) : (half == 1);
+    if (!owner) strip_done();
+    float dp = 0.f;
+#pragma unroll 1
+    for (int it = 0; it < 4; ++it) {
+      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      uint32_t v0[16], v1[16];
+      tmem_ld_32x32b_x16(t_row + c * 32, v0);
+      tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
+      tmem_wait_ld();
+      if (owner && it == 0) {
+        tc_fence_before();
+        strip_done();
+      }
+      const int col = n0 + c * 32;
+      if (row_ok && col < p.N) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int cc = col + 16 * hh;
+          const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + cc);
+          const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + cc);
+          uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
+          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
+          uint4 og[2], ou[2], oa[2];
+          uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
+          uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
+          uint32_t* oaw = reinterpret_cast<uint32_t*>(oa);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 gg2 = __bfloat1622float2(g2[i]);
+            const float2 uu2 = __bfloat1622float2(u2[i]);
+            const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
+            float dg[2], du[2], av[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float da = __uint_as_float(hh ? v1[2 * i + j] : v0[2 * i + j]);
+              const float sg = 1.0f / (1.0f + expf(-gs[j]));
+              const float sl = gs[j] * sg;
+              dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+              du[j] = da * pr * sl;
+              av[j] = sl * us[j] * pr;
+              dp = fmaf(da, sl * us[j], dp);
+            }
+            ogw[i] = pack_bf16x2(dg[0], dg[1]);
+            ouw[i] = pack_bf16x2(du[0], du[1]);
+            oaw[i] = pack_bf16x2(av[0], av[1]);
+          }
+          uint4* d0 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + cc);
+          uint4* d1 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + cc);
+          uint4* d2 = reinterpret_cast<uint4*>(a_out + row * p.ldo + cc);
+          d0[0] = og[0];
+          d0[1] = og[1];
+          d1[0] = ou[0];
+          d1[1] = ou[1];
+          d2[0] = oa[0];
+          d2[1] = oa[1];
+        }
+      }
+    }
+    if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
+  } else {
+    // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const int n0 = ti.n_blk * 128;
+    uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
+    __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
+    // output chunk 3 of acc0 (its up columns are the shared strip) belongs to the
+    // upper half, chunk 0 of acc1 (gate columns) to the lower half
+    const bool owner = acc ? (half == 0) : (half == 1);
+    if (!owner) strip_done();
+#pragma unroll 1
+    for (int it = 0; it < 2; ++it) {
+      const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
+      uint32_t g0[16], g1[16], u0[16], u1[16];
+      tmem_ld_32x32b_x16(t_row + c * 32, g0);
+      tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
+      tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
+      tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
+      tmem_wait_ld();
+      if (owner && it == 0) {
+        tc_fence_before();
+        strip_done();
+      }
+      if (row_ok) {
+        float a[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          a[i] = silu_f(__uint_as_float(g0[i])) * __uint_as_float(u0[i]) * pr;
+          a[16 + i] = silu_f(__uint_as_float(g1[i])) * __uint_as_float(u1[i]) * pr;
+          amax = fmaxf(amax, fmaxf(fabsf(a[i]), fabsf(a[16 + i])));
+        }
+        const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+        const int code = max(bexp - 8, 0);
+        const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] *= inv;
+        uint32_t w0[4], w1[4];
+        pack_e4m3x16(a, w0);
+        pack_e4m3x16(a + 16, w1);
+        uint4* dst = reinterpret_cast<uint4*>(a_codes + row * p.ldo + n0 + c * 32);
+        dst[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+        dst[1] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        sc_word |= (uint32_t)code << (8 * c);
+        if (hout) {
+          uint4 hg[4], hu[4];
+          uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
+          uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            hgw[i] = pack_bf16x2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1]));
+            hgw[8 + i] = pack_bf16x2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1]));
+            huw[i] = pack_bf16x2(__uint_as_float(u0[2 * i]), __uint_as_float(u0[2 * i + 1]));
+            huw[8 + i] = pack_bf16x2(__uint_as_float(u1[2 * i]), __uint_as_float(u1[2 * i + 1]));
+          }
+          uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c * 32);
+          uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            hd[i] = hg[i];
+            hd2[i] = hu[i];
+          }
+        }
+      }
+    }
+  }
+  return sc_word;
+}
+
 template <bool KGROUP, int EPI>
 __global__ void __launch_bounds__(mx::kThreads, 1)
     grouped_gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -312,196 +516,8 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (acc ? kAcc1Col : 0u) + ((uint32_t)(q * 32) << 16);
-      const bool row_ok = r_local < ti.rows;
-      const long long row = ti.row0 + r_local;
-      uint32_t sc_word = 0;   // SwiGLU: this row's four scale bytes (k-blocks 4*n_blk..+3 of the next GEMM)
-
-      if (EPI == MXEPI_STORE || EPI == MXEPI_WGRAD) {
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-        const int n0 = ti.n_blk * BN;
-        long long orow;
-        bool ok_row;
-        bool zero = false;
-        if (EPI == MXEPI_WGRAD) {
-          const int m = ti.m_blk * BM + r_local;
-          ok_row = m < p.M;
-          orow = (long long)ti.e * p.out_batch + (long long)m * p.ldo;
-          zero = ti.rows == 0;
-        } else {
-          ok_row = row_ok;
-          orow = row * p.ldo;
-        }
-        // the 32-column strip shared with the other accumulator: chunk 7 of acc0 (upper
-        // half), chunk 0 of acc1 (lower half); its owner drains it first, then signals
-        const bool owner = acc ? (half == 0) : (half == 1);
-        if (!owner) mbar_arrive(tovl);
-#pragma unroll 1
-        for (int it = 0; it < 4; ++it) {
-          const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
-          uint32_t v0[16], v1[16];
-          tmem_ld_32x32b_x16(t_row + c * 32, v0);
-          tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
-          tmem_wait_ld();
-          if (owner && it == 0) {
-            tc_fence_before();
-            mbar_arrive(tovl);
-          }
-          if (ok_row && n0 + c * 32 < p.N && p.out_f32) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dst[i] = make_uint4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
-              dst[4 + i] = make_uint4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
-            }
-          } else if (ok_row && n0 + c * 32 < p.N) {
-            uint4 o[4];
-            uint32_t* ow = reinterpret_cast<uint32_t*>(o);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
-              ow[8 + i] = zero ? 0u : pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
-            }
-            uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = o[i];
-          }
-        }
-      } else if (EPI == MXEPI_DSWIGLU) {
-        // acc = da for columns [n0, n0+256) of F. With h = [g | u] from the forward:
-        // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u; a = SiLU(g) u p is
-        // recomputed (bf16) for the fc2 weight gradient.
-        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
-        __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
-        __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
-        const int n0 = ti.n_blk * BN;
-        const bool owner = acc ? (half == 0) : (half == 1);
-        if (!owner) mbar_arrive(tovl);
-        float dp = 0.f;
-#pragma unroll 1
-        for (int it = 0; it < 4; ++it) {
-          const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
-          uint32_t v0[16], v1[16];
-          tmem_ld_32x32b_x16(t_row + c * 32, v0);
-          tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
-          tmem_wait_ld();
-          if (owner && it == 0) {
-            tc_fence_before();
-            mbar_arrive(tovl);
-          }
-          const int col = n0 + c * 32;
-          if (row_ok && col < p.N) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int cc = col + 16 * half;
-              const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + cc);
-              const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + cc);
-              uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
-              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
-              const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
-              uint4 og[2], ou[2], oa[2];
-              uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
-              uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
-              uint32_t* oaw = reinterpret_cast<uint32_t*>(oa);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float2 gg2 = __bfloat1622float2(g2[i]);
-                const float2 uu2 = __bfloat1622float2(u2[i]);
-                const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
-                float dg[2], du[2], av[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                  const float da = __uint_as_float(half ? v1[2 * i + j] : v0[2 * i + j]);
-                  const float sg = 1.0f / (1.0f + expf(-gs[j]));
-                  const float sl = gs[j] * sg;
-                  dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
-                  du[j] = da * pr * sl;
-                  av[j] = sl * us[j] * pr;
-                  dp = fmaf(da, sl * us[j], dp);
-                }
-                ogw[i] = pack_bf16x2(dg[0], dg[1]);
-                ouw[i] = pack_bf16x2(du[0], du[1]);
-                oaw[i] = pack_bf16x2(av[0], av[1]);
-              }
-              uint4* d0 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + cc);
-              uint4* d1 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + cc);
-              uint4* d2 = reinterpret_cast<uint4*>(a_out + row * p.ldo + cc);
-              d0[0] = og[0];
-              d0[1] = og[1];
-              d1[0] = ou[0];
-              d1[1] = ou[1];
-              d2[0] = oa[0];
-              d2[1] = oa[1];
-            }
-          }
-        }
-        if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
-      } else {
-        // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
-        const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-        const int n0 = ti.n_blk * 128;
-        uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
-        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
-        // output chunk 3 of acc0 (its up columns are the shared strip) belongs to the
-        // upper half, chunk 0 of acc1 (gate columns) to the lower half
-        const bool owner = acc ? (half == 0) : (half == 1);
-        if (!owner) mbar_arrive(tovl);
-#pragma unroll 1
-        for (int it = 0; it < 2; ++it) {
-          const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
-          uint32_t g0[16], g1[16], u0[16], u1[16];
-          tmem_ld_32x32b_x16(t_row + c * 32, g0);
-          tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
-          tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
-          tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
-          tmem_wait_ld();
-          if (owner && it == 0) {
-            tc_fence_before();
-            mbar_arrive(tovl);
-          }
-          if (row_ok) {
-            float a[32];
-            float amax = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              a[i] = silu_f(__uint_as_float(g0[i])) * __uint_as_float(u0[i]) * pr;
-              a[16 + i] = silu_f(__uint_as_float(g1[i])) * __uint_as_float(u1[i]) * pr;
-              amax = fmaxf(amax, fmaxf(fabsf(a[i]), fabsf(a[16 + i])));
-            }
-            const int bexp = (int)((__float_as_uint(amax) >> 23) & 0xFF);
-            const int code = max(bexp - 8, 0);
-            const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) a[i] *= inv;
-            uint32_t w0[4], w1[4];
-            pack_e4m3x16(a, w0);
-            pack_e4m3x16(a + 16, w1);
-            uint4* dst = reinterpret_cast<uint4*>(a_codes + row * p.ldo + n0 + c * 32);
-            dst[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-            dst[1] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-            sc_word |= (uint32_t)code << (8 * c);
-            if (hout) {
-              uint4 hg[4], hu[4];
-              uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
-              uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                hgw[i] = pack_bf16x2(__uint_as_float(g0[2 * i]), __uint_as_float(g0[2 * i + 1]));
-                hgw[8 + i] = pack_bf16x2(__uint_as_float(g1[2 * i]), __uint_as_float(g1[2 * i + 1]));
-                huw[i] = pack_bf16x2(__uint_as_float(u0[2 * i]), __uint_as_float(u0[2 * i + 1]));
-                huw[8 + i] = pack_bf16x2(__uint_as_float(u1[2 * i]), __uint_as_float(u1[2 * i + 1]));
-              }
-              uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c * 32);
-              uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c * 32);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                hd[i] = hg[i];
-                hd2[i] = hu[i];
-              }
-            }
-          }
-        }
-      }
+      const uint32_t sc_word =
+          mxf8_epilogue_tile<EPI>(mp, ti, t_row, acc, half, r_local, BM, [&] { mbar_arrive(tovl); });
       if (EPI == MXEPI_SWIGLU_Q) {
         // this half's two scale bytes (chunks 2*half, 2*half+1); rows past the expert store 0
         const size_t g = (size_t)(tile_off[ti.e] / NT + ti.m_blk);

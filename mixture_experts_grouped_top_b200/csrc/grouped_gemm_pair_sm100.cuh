@@ -3,9 +3,14 @@
 // A 2-CTA cluster computes 256 x 256 output tiles: each CTA loads its own 128 rows of A
 // and its own half (128 columns) of B into its shared memory, the pair leader issues
 // tcgen05.mma.cta_group::2 (M=256, N=256, K=16) that reads both CTAs' operands, and each
-// CTA receives the 128 x 256 fp32 accumulator of its rows in its own tensor memory. Per
-// SM, a 64-wide k-stage moves 32 KB through shared memory instead of 48 KB for a 1-SM
-// 128 x 256 tile, and 6 stages fit instead of 4.
+// CTA receives the 128 x 256 fp32 accumulator of its rows in its own tensor memory.
+//
+// A k-stage is 128 wide and each operand of a stage arrives with ONE TMA copy: the tensor
+// maps view a matrix as 64-element (128-byte) chunks, so a box of two chunks x 128 rows
+// lands as two canonical 128-byte-swizzled tiles back to back (K-major: [chunk][row];
+// MN-major: [column chunk][k row]). Issuing a copy costs the TMA unit about the same
+// whatever its size, so two 32 KB copies per 1024-cycle stage keep the tensor pipe fed
+// where six 8-16 KB copies per 512-cycle stage did not. 3 stages of 64 KB per CTA.
 //
 // Synchronisation: both CTAs' TMA loads complete on the leader's `full` barrier (the
 // 2-SM TMA form); the leader's MMA commits arrive on the `empty` and `tfull` barriers of
@@ -24,18 +29,20 @@ namespace g2 {
 constexpr int BM = 256;                       // rows of a pair tile
 constexpr int BMC = 128;                      // rows per CTA
 constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int kStages = 6;
+constexpr int BK = 128;                       // k per stage: two 64-element chunks
+constexpr int kStages = 3;
 constexpr int kThreads = 384;
-constexpr int kABytes = BMC * BK * 2;         // 16 KB
-constexpr int kBBytes = (BN / 2) * BK * 2;    // 16 KB: this CTA's half of B
-constexpr int kChunkBytes = 64 * BK * 2;      // 8 KB
+constexpr int kABytes = BMC * BK * 2;         // 32 KB
+constexpr int kBBytes = (BN / 2) * BK * 2;    // 32 KB: this CTA's half of B
+constexpr int kChunkBytes = 128 * 64 * 2;     // one 64-element chunk of 128 rows (or k rows), 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024 + 2 * (kMaxE + 1) * 4;
 }  // namespace g2
 
+// tmA: A [rows, K] as {64, rows, K/64 chunks, 1}; tmB: B_MN ? [E][K rows][N] as
+// {64, K, N/64 chunks, E} : [E][N rows][K] as {64, N, K/64 chunks, E}; boxes {64, 128, 2, 1}.
 template <bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -118,6 +125,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
 
   TileWalker<false, BM> walk{row_off, tile_off, E, 0, NT, p.K, nullptr};
   const int total = walk.total();
+  const int num_kb = (p.K + BK - 1) / BK;   // a partial last stage reads zeros past K
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (both CTAs)
@@ -128,25 +136,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
         const TileInfo ti = walk.decode(t);
-        for (int kb = 0; kb < ti.num_kb; ++kb) {
+        const int a_row = ti.row0 + BMC * (int)rank;
+        // this CTA's half of B: columns (MN-major) or rows (K-major) [b0, b0 + 128)
+        const int b0 =
+            (EPI == EPI_SWIGLU) ? (rank == 0 ? 0 : p.F) + ti.n_blk * 128 : ti.n_blk * BN + 128 * (int)rank;
+        for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
-          const int k0 = kb * BK;
-          tma_load_3d_pair(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0 + BMC * rank, 0);
-          uint8_t* b_dst = sB + stage * kBBytes;
-          if (B_MN) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const int col = (EPI == EPI_SWIGLU) ? (rank == 0 ? 0 : p.F) + ti.n_blk * 128 + 64 * c
-                                                  : ti.n_blk * BN + 128 * rank + 64 * c;
-              tma_load_3d_pair(b_dst + c * kChunkBytes, &tmB, &full[stage], col, k0, ti.e);
-            }
-          } else {
-            tma_load_3d_pair(b_dst, &tmB, &full[stage], k0, ti.n_blk * BN + 128 * rank, ti.e);
-          }
+          tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, 2 * kb, 0);
+          if (B_MN)
+            tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, kb * BK, b0 / 64, ti.e);
+          else
+            tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b0, 2 * kb, ti.e);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -176,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
         if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < ti.num_kb; ++kb) {
+        for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
@@ -187,9 +191,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
             const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t adesc = make_sdesc(a_addr + kk * 32, 16, 1024, 2);
+              // K-major: chunk kk/4, 32 bytes per 16 k; MN-major: 16 k rows = 2048 bytes,
+              // column chunks kChunkBytes apart
+              const uint32_t koff = (uint32_t)(kk >> 2) * kChunkBytes + (uint32_t)(kk & 3) * 32;
+              const uint64_t adesc = make_sdesc(a_addr + koff, 16, 1024, 2);
               const uint64_t bdesc = B_MN ? make_sdesc(b_addr + kk * 2048, kChunkBytes, 1024, 2)
-                                          : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
+                                          : make_sdesc(b_addr + koff, 16, 1024, 2);
               mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit_pair(&empty[stage]);

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "moe_grouped.h"
+#include "grouped_gemm_mxf8_pair_sm100.cuh"
 #include "grouped_gemm_mxf8_sm100.cuh"
 #include "grouped_gemm_pair_sm100.cuh"
 #include "grouped_gemm_sm100.cuh"
@@ -68,10 +69,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D tiled tensor map with 128-byte swizzle: dims {d0 (contiguous), d1, d2},
-// byte strides of d1 and d2, box {box0, box1, 1}.
+// 3-D tiled tensor map (128-byte swizzle unless told otherwise): dims {d0 (contiguous),
+// d1, d2}, byte strides of d1 and d2, box {box0, box1, 1}.
 int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
-              uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1) {
+              uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (stride1 & 15) || (stride2 & 15)) return MOE_ERR_INVALID_ARG;
@@ -80,10 +82,34 @@ int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t 
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     fprintf(stderr, "moe_grouped: cuTensorMapEncodeTiled failed (%d)\n", (int)r);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// Stacked matrices [batch, rows, cols] (row-major, elem-byte elements, cols * elem a
+// multiple of 128) viewed as 128-byte column chunks: dims {128 / elem, rows, chunks,
+// batch}, box {128 / elem, 128, 2, 1}. One box lands as two 128-byte-swizzled tiles of
+// 128 rows back to back ([chunk][row]), the operand layout of the CTA-pair kernels.
+int tmap_chunks(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols,
+                uint32_t elem) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  const uint64_t row_bytes = cols * elem;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (row_bytes % 128)) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[4] = {128 / elem, rows, row_bytes / 128, batch};
+  cuuint64_t strides[3] = {row_bytes, 128, rows * row_bytes};
+  cuuint32_t box[4] = {128 / elem, 128, 2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(m, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fprintf(stderr, "moe_grouped: cuTensorMapEncodeTiled (chunked) failed (%d)\n", (int)r);
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
@@ -145,6 +171,41 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
 // E4M3 codes [batch, rows, cols] as a TMA source with box {128 bytes of K, box_rows}.
 int tmap_u8_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, cols, rows, batch, cols, rows * cols, 128, box_rows);
+}
+
+// MMA scale atoms [groups, kb4 atoms of 512 bytes] as a TMA source: uint32 tensor
+// {128 words, kb4, groups}, boxes of mx2::kSfKb consecutive atoms of one group (unswizzled).
+int tmap_atoms(CUtensorMap* m, const void* atoms, uint64_t groups, uint64_t kb4) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, atoms, 128, kb4, groups, 512, kb4 * 512, 128, mx2::kSfKb,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// MXFP8 CTA-pair kernels: as many 2-CTA clusters as can be resident at once.
+template <int EPI>
+int launch_gemm_mx_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
+                        const MxGemmParams& p, cudaStream_t st) {
+  auto kern = grouped_gemm_mxf8_pair_kernel<EPI>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int pairs = 0;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mx2::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(device_props().sm_count, 1, 1);
+    cfg.blockDim = dim3(mx2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = mx2::kSmemBytes;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_props().sm_count / 2;
+    pairs = std::min(n, device_props().sm_count / 2);
+    cudaGetLastError();
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  kern<<<2 * pairs, mx2::kThreads, mx2::kSmemBytes, st>>>(ta, tb, tsa, tsb, p);
+  count_launch();
+  return launch_status();
 }
 
 template <bool KG, int EPI>
@@ -441,8 +502,8 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   int rc;
   if ((rc = scales_to_atoms_launch(xp_scale, split_sizes, E, R, H, xp_atoms, st))) return rc;
   // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
-  if ((rc = tmap_u8_3d(&ta, xp, 1, R, H, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, w1, E, 2 * F, H, 128))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xp, 1, R, H, 1))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1, E, 2 * F, H, 1))) return rc;
   MxGemmParams p1;
   p1.g = base_params(split_sizes, E);
   p1.g.M = R;
@@ -458,10 +519,13 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p1.b_atoms = w1_scale;
   p1.b_rows = 2 * F;
   p1.out_atoms = a_atoms;
-  if ((rc = launch_gemm_mx<false, MXEPI_SWIGLU_Q>(ta, tb, p1, st))) return rc;
+  CUtensorMap tsa, tsb;
+  if ((rc = tmap_atoms(&tsa, xp_atoms, (uint64_t)R / 128 + E, H / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, w1_scale, (uint64_t)E * 2 * F / 128, H / 128))) return rc;
+  if ((rc = launch_gemm_mx_pair<MXEPI_SWIGLU_Q>(ta, tb, tsa, tsb, p1, st))) return rc;
   // fc2: A = a codes [R, F], B = w2 codes [E, H, F]
-  if ((rc = tmap_u8_3d(&ta, a_codes, 1, R, F, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, w2, E, H, F, 128))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, 1, R, F, 1))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, E, H, F, 1))) return rc;
   MxGemmParams p2;
   p2.g = base_params(split_sizes, E);
   p2.g.M = R;
@@ -474,7 +538,9 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p2.b_atoms = w2_scale;
   p2.b_rows = H;
   p2.out_atoms = nullptr;
-  return launch_gemm_mx<false, MXEPI_STORE>(ta, tb, p2, st);
+  if ((rc = tmap_atoms(&tsa, a_atoms, (uint64_t)R / 128 + E, F / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, w2_scale, (uint64_t)E * H / 128, F / 128))) return rc;
+  return launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p2, st);
 }
 
 }  // namespace
@@ -508,8 +574,8 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   CUtensorMap ta, tb;
   int rc;
   // fc1: A = xp [R, H] (K-major), B = w1 [E, H, 2F] (N contiguous: MN-major)
-  if ((rc = tmap_bf16_2d(&ta, xp, R, H, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, 1, R, H, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w1, E, H, 2 * F, 2))) return rc;
   GemmParams p1 = base_params(split_sizes, E);
   p1.M = R;
   p1.N = F;
@@ -522,8 +588,8 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   p1.F = F;
   if ((rc = launch_gemm_pair<true, EPI_SWIGLU>(ta, tb, p1, st))) return rc;
   // fc2: A = a [R, F] (K-major), B = w2 [E, F, H] (MN-major)
-  if ((rc = tmap_bf16_2d(&ta, a_buf, R, F, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_buf, 1, R, F, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w2, E, F, H, 2))) return rc;
   GemmParams p2 = base_params(split_sizes, E);
   p2.M = R;
   p2.N = H;
@@ -632,8 +698,8 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((rc = quant_cols_grouped_launch(dy_perm, R, H, split_sizes, E, dyc, dyc_a, st))) return rc;
   CUtensorMap ta, tb;
   // fc2 dgrad + SwiGLU backward: A = dy codes [R, H], B = w2 codes [E, F, H] (N = F)
-  if ((rc = tmap_u8_3d(&ta, dyr, 1, R, H, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, w2q, E, F, H, 128))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyr, 1, R, H, 1))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2q, E, F, H, 1))) return rc;
   MxGemmParams p;
   p.g = base_params(split_sizes, E);
   p.g.M = R;
@@ -652,7 +718,10 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.b_atoms = w2a;
   p.b_rows = F;
   p.out_atoms = nullptr;
-  if ((rc = launch_gemm_mx<false, MXEPI_DSWIGLU>(ta, tb, p, st))) return rc;
+  CUtensorMap tsa, tsb;
+  if ((rc = tmap_atoms(&tsa, dyr_a, (uint64_t)R / 128 + E, H / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, w2a, (uint64_t)E * F / 128, H / 128))) return rc;
+  if ((rc = launch_gemm_mx_pair<MXEPI_DSWIGLU>(ta, tb, tsa, tsb, p, st))) return rc;
   if (dprobs_perm) {
     const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
     reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
@@ -679,8 +748,8 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.b_rows = H;
   if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh codes [R, 2F], B = w1 codes [E, H, 2F] (N = H)
-  if ((rc = tmap_u8_3d(&ta, dhr, 1, R, 2 * F, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, w1q, E, H, 2 * F, 128))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhr, 1, R, 2 * F, 1))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1))) return rc;
   p.g = base_params(split_sizes, E);
   p.g.M = R;
   p.g.N = H;
@@ -690,7 +759,9 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.a_atoms = dhr_a;
   p.b_atoms = w1a;
   p.b_rows = H;
-  if ((rc = launch_gemm_mx<false, MXEPI_STORE>(ta, tb, p, st))) return rc;
+  if ((rc = tmap_atoms(&tsa, dhr_a, (uint64_t)R / 128 + E, 2 * F / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, w1a, (uint64_t)E * H / 128, 2 * F / 128))) return rc;
+  if ((rc = launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e
   if ((rc = tmap_u8_3d(&ta, xc, 1, R, H, mx::BM))) return rc;
   if ((rc = tmap_u8_3d(&tb, dhc, 1, R, 2 * F, mx::BM))) return rc;
@@ -740,8 +811,8 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   CUtensorMap ta, tb;
   int rc;
   // fc2 dgrad + SwiGLU backward: A = dy [R, H] (K-major), B = w2 [E, F, H] read as [E, N=F, K=H] (K-major)
-  if ((rc = tmap_bf16_2d(&ta, dy_perm, R, H, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w2, E, F, H, g2::BN / 2))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy_perm, 1, R, H, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w2, E, F, H, 2))) return rc;
   GemmParams p = base_params(split_sizes, E);
   p.M = R;
   p.N = F;
@@ -771,8 +842,8 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.out_batch = (long long)F * H;
   if ((rc = launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh [R, 2F] (K-major), B = w1 [E, H, 2F] read as [E, N=H, K=2F] (K-major)
-  if ((rc = tmap_bf16_2d(&ta, dh, R, 2 * F, gg::BM))) return rc;
-  if ((rc = tmap_bf16_3d(&tb, w1, E, H, 2 * F, g2::BN / 2))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, 1, R, 2 * F, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w1, E, H, 2 * F, 2))) return rc;
   p = base_params(split_sizes, E);
   p.M = R;
   p.N = H;
