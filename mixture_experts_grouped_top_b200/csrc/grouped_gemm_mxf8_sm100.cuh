@@ -403,8 +403,8 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           if (KGROUP) {
             // MN-major codes: box {128 columns, 128 rows} at the expert's k-th row block
             tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], ti.m_blk * BM, ti.row0 + k0, 0);
-            tma_load_3d(b_dst, &tmB, &full[stage], n0, ti.row0 + k0, 0);
-            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], n0 + 128, ti.row0 + k0, 0);
+            // both 128-column chunks of B in one copy (chunked view, box {128, 128 k rows, 2, 1})
+            tma_load_4d(b_dst, &tmB, &full[stage], 0, ti.row0 + k0, n0 / 128, 0);
           } else {
             tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
             tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);

@@ -388,6 +388,9 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
           const int k0 = kb * BK;
           if (!A_MN) {
             tma_load_3d(a_dst, &tmA, &full[stage], k0, ti.row0, 0);
+          } else if (KGROUP) {
+            // both 64-column chunks in one copy (chunked view, box {64, 64 k rows, 2, 1})
+            tma_load_4d(a_dst, &tmA, &full[stage], 0, ti.row0 + k0, ti.m_blk * (BM / 64), 0);
           } else {
 #pragma unroll
             for (int c = 0; c < 2; ++c)
@@ -395,15 +398,13 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
           }
           if (!B_MN) {
             tma_load_3d(b_dst, &tmB, &full[stage], k0, ti.n_blk * BN, ti.e);
+          } else if (KGROUP) {
+            // all four 64-column chunks in one copy (box {64, 64 k rows, 4, 1})
+            tma_load_4d(b_dst, &tmB, &full[stage], 0, ti.row0 + k0, ti.n_blk * (BN / 64), 0);
           } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              if (KGROUP)
-                tma_load_3d(b_dst + c * kChunkBytes, &tmB, &full[stage], ti.n_blk * BN + 64 * c, ti.row0 + k0, 0);
-              else
-                tma_load_3d(b_dst + c * kChunkBytes, &tmB, &full[stage], b_chunk_col<EPI>(ti.n_blk, c, p.F), k0,
-                            ti.e);
-            }
+            for (int c = 0; c < 4; ++c)
+              tma_load_3d(b_dst + c * kChunkBytes, &tmB, &full[stage], b_chunk_col<EPI>(ti.n_blk, c, p.F), k0, ti.e);
           }
           ++issued;
           if (++stage == kStages) {

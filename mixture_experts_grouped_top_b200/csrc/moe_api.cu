@@ -93,17 +93,19 @@ int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t 
 
 // Stacked matrices [batch, rows, cols] (row-major, elem-byte elements, cols * elem a
 // multiple of 128) viewed as 128-byte column chunks: dims {128 / elem, rows, chunks,
-// batch}, box {128 / elem, 128, 2, 1}. One box lands as two 128-byte-swizzled tiles of
-// 128 rows back to back ([chunk][row]), the operand layout of the CTA-pair kernels.
+// batch}, box {128 / elem, box_rows, box_chunks, 1}. One box lands as box_chunks
+// 128-byte-swizzled tiles of box_rows rows back to back ([chunk][row]): the operand layout
+// of the CTA-pair kernels (128 rows x 2 chunks) and of the MN-major weight-gradient
+// operands (64 k rows x 2 or 4 column chunks).
 int tmap_chunks(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols,
-                uint32_t elem) {
+                uint32_t elem, uint32_t box_rows = 128, uint32_t box_chunks = 2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   const uint64_t row_bytes = cols * elem;
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (row_bytes % 128)) return MOE_ERR_INVALID_ARG;
   cuuint64_t dims[4] = {128 / elem, rows, row_bytes / 128, batch};
   cuuint64_t strides[3] = {row_bytes, 128, rows * row_bytes};
-  cuuint32_t box[4] = {128 / elem, 128, 2, 1};
+  cuuint32_t box[4] = {128 / elem, box_rows, box_chunks, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = fn(m, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -736,7 +738,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc, xc_a, st))) return rc;
   // fc2 wgrad: dw2[e] = a_e^T dy_e (MN-major codes, contraction over the expert's rows)
   if ((rc = tmap_u8_3d(&ta, ac, 1, R, F, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, dyc, 1, R, H, mx::BM))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyc, 1, R, H, 1, mx::BK, 2))) return rc;
   p.g = base_params(split_sizes, E);
   p.g.M = F;
   p.g.N = H;
@@ -764,7 +766,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((rc = launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e
   if ((rc = tmap_u8_3d(&ta, xc, 1, R, H, mx::BM))) return rc;
-  if ((rc = tmap_u8_3d(&tb, dhc, 1, R, 2 * F, mx::BM))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhc, 1, R, 2 * F, 1, mx::BK, 2))) return rc;
   p.g = base_params(split_sizes, E);
   p.g.M = H;
   p.g.N = 2 * F;
@@ -832,8 +834,8 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
     if ((rc = launch_status())) return rc;
   }
   // fc2 wgrad: dw2[e] = a_e^T dy_e. A = a [R, F] (rows = K, MN-major), B = dy [R, H] (MN-major)
-  if ((rc = tmap_bf16_2d(&ta, a_buf, R, F, 64))) return rc;
-  if ((rc = tmap_bf16_2d(&tb, dy_perm, R, H, 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_buf, 1, R, F, 2, gg::BK, gg::BM / 64))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy_perm, 1, R, H, 2, gg::BK, gg::BN / 64))) return rc;
   p = base_params(split_sizes, E);
   p.M = F;
   p.N = H;
@@ -852,8 +854,8 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.ldo = H;
   if ((rc = launch_gemm_pair<false, EPI_STORE>(ta, tb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e. A = xp [R, H] (MN-major), B = dh [R, 2F] (MN-major)
-  if ((rc = tmap_bf16_2d(&ta, xp, R, H, 64))) return rc;
-  if ((rc = tmap_bf16_2d(&tb, dh, R, 2 * F, 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, 1, R, H, 2, gg::BK, gg::BM / 64))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, 1, R, 2 * F, 2, gg::BK, gg::BN / 64))) return rc;
   p = base_params(split_sizes, E);
   p.M = H;
   p.N = 2 * F;
