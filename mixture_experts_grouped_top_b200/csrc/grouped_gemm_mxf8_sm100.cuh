@@ -455,16 +455,23 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           break;
         }
         tc_fence_after();
+        int ksteps = BK / 32;   // K=32 MMAs of this stage
         if (KGROUP && (kb + 1) * BK > ti.rows) {
-          // clip the contraction at the expert's last row: zero K-rows >= valid (128-byte lines)
+          // clip the contraction at the expert's last row: MMAs only over the expert's
+          // K-rows; inside the last, partial 32-row step zero the rows >= valid of the
+          // three operand blocks (A, two halves of B; 128-byte lines)
           const int valid = ti.rows - kb * BK;
-          const int per = (BK - valid) * 8;   // 16-byte vectors per 128-row operand block
-          for (int i = lane; i < 3 * per; i += 32) {
-            const int blk = i / per, r = i % per;
-            uint8_t* base = (blk == 0) ? sA + stage * kABytes : sB + stage * kBBytes + (blk - 1) * BM * BK;
-            *reinterpret_cast<uint4*>(base + valid * 128 + r * 16) = make_uint4(0, 0, 0, 0);
+          ksteps = (valid + 31) / 32;
+          const int zr = ksteps * 32 - valid;   // 0..31 rows
+          if (zr > 0) {
+            for (int i = lane; i < 3 * zr * 8; i += 32) {
+              const int v = i & 7, rb = i >> 3;
+              const int blk = rb / zr, r = rb - blk * zr;
+              uint8_t* base = (blk == 0) ? sA + stage * kABytes : sB + stage * kBBytes + (blk - 1) * BM * BK;
+              *reinterpret_cast<uint4*>(base + (valid + r) * 128 + v * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
@@ -477,6 +484,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
+            if (kk >= ksteps) break;
             // K-major: next 32 K values are 32 bytes further in each 128-byte row;
             // MN-major: 32 rows further (4 x 8-row swizzle atoms), halves of B 16 KB apart
             const uint64_t adesc = KGROUP ? make_sdesc(a_addr + kk * 4096, BM * BK, 1024, 2)

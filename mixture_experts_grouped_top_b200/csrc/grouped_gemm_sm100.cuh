@@ -163,22 +163,28 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
       orow = (long long)(ti.row0 + tile_row) * p.ldo;
     }
     const int n0 = ti.n_blk * gg::BN;
+    // 64 columns per round: four tensor-memory loads in flight, one wait
 #pragma unroll 1
-    for (int c = half * (gg::BN / 2); c < (half + 1) * (gg::BN / 2); c += 16) {
-      uint32_t v[16];
-      tmem_ld_32x32b_x16(t_row + c, v);
+    for (int c0 = half * (gg::BN / 2); c0 < (half + 1) * (gg::BN / 2); c0 += 64) {
+      uint32_t v[4][16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld_32x32b_x16(t_row + c0 + 16 * j, v[j]);
       tmem_wait_ld();
-      if (row_ok && n0 + c < p.N) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 16 * j;
+        if (!row_ok || n0 + c >= p.N) continue;
         if (EPI == EPI_STORE && p.out_f32) {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(v[j][4 * i], v[j][4 * i + 1], v[j][4 * i + 2], v[j][4 * i + 3]);
         } else {
           uint4 o[2];
           uint32_t* ow = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            ow[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v[j][2 * i]), __uint_as_float(v[j][2 * i + 1]));
           uint4* dst = reinterpret_cast<uint4*>(out + orow + n0 + c);
           dst[0] = o[0];
           dst[1] = o[1];
@@ -447,19 +453,25 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
           break;
         }
         tc_fence_after();
+        int ksteps = BK / 16;   // K=16 MMAs of this stage
         if (KGROUP && (kb + 1) * BK > ti.rows) {
-          // clip the contraction at the end of the expert's rows: zero K-rows >= valid
+          // clip the contraction at the end of the expert's rows: MMAs only over the
+          // expert's K-rows; inside the last, partial 16-row step zero the rows >= valid
+          // of all six 64-wide operand chunks (A 2, B 4; row r of a chunk at r * 128 bytes)
           const int valid = ti.rows - kb * BK;
-          const int zrows = BK - valid;
-          uint8_t* a_st = sA + stage * kABytes;
-          uint8_t* b_st = sB + stage * kBBytes;
-          const int per_chunk = zrows * 8;   // 16-byte vectors per chunk
-          for (int i = lane; i < 6 * per_chunk; i += 32) {
-            const int c = i / per_chunk, r = i % per_chunk;
-            uint8_t* base = (c < 2) ? a_st + c * kChunkBytes : b_st + (c - 2) * kChunkBytes;
-            *reinterpret_cast<uint4*>(base + valid * 128 + r * 16) = make_uint4(0, 0, 0, 0);
+          ksteps = (valid + 15) / 16;
+          const int zr = ksteps * 16 - valid;   // 0..15 rows
+          if (zr > 0) {
+            uint8_t* a_st = sA + stage * kABytes;
+            uint8_t* b_st = sB + stage * kBBytes;
+            for (int i = lane; i < 6 * zr * 8; i += 32) {
+              const int v = i & 7, rc = i >> 3;
+              const int c = rc / zr, r = rc - c * zr;
+              uint8_t* base = (c < 2) ? a_st + c * kChunkBytes : b_st + (c - 2) * kChunkBytes;
+              *reinterpret_cast<uint4*>(base + (valid + r) * 128 + v * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
@@ -467,6 +479,7 @@ __global__ void __launch_bounds__(gg::kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
+            if (kk >= ksteps) break;
             const uint64_t adesc = A_MN ? make_sdesc(a_addr + kk * 2048, kChunkBytes, 1024, 2)
                                         : make_sdesc(a_addr + kk * 32, 16, 1024, 2);
             const uint64_t bdesc = B_MN ? make_sdesc(b_addr + kk * 2048, kChunkBytes, 1024, 2)

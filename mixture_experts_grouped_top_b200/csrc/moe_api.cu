@@ -117,16 +117,6 @@ int tmap_chunks(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_
   return MOE_OK;
 }
 
-// bf16 matrix [rows, cols] (row-major) as a TMA source. K-major operand: box {64 cols, box_rows}.
-int tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, cols, rows, 1, cols * 2, rows * cols * 2, 64, box_rows);
-}
-// bf16 stacked matrices [batch, rows, cols] as a TMA source with box {64 cols, box_rows}.
-int tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, cols, rows, batch, cols * 2, rows * cols * 2, 64,
-                   box_rows);
-}
-
 template <bool A_MN, bool B_MN, bool KG, int EPI>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
   auto kern = grouped_gemm_bf16_kernel<A_MN, B_MN, KG, EPI>;
