@@ -144,6 +144,20 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
       const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      const int col = n0 + c * 32;
+      const bool cols_ok = row_ok && col < p.N;
+      // the saved h of these 32 columns is requested first, so its global latency overlaps
+      // the tensor-memory loads and their wait
+      uint4 gva[4], uva[4];
+      if (cols_ok) {
+        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + col);
+        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gva[i] = gp[i];
+          uva[i] = up[i];
+        }
+      }
       uint32_t v0[16], v1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
@@ -152,16 +166,12 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         tc_fence_before();
         strip_done();
       }
-      const int col = n0 + c * 32;
-      if (row_ok && col < p.N) {
+      if (cols_ok) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int cc = col + 16 * hh;
-          const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + cc);
-          const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + cc);
-          uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
-          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
-          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva + 2 * hh);
+          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva + 2 * hh);
           uint4 og[2], ou[2], oa[2];
           uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
           uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);

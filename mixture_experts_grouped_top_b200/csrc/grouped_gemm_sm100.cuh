@@ -198,38 +198,48 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
     const int n0 = ti.n_blk * 128;
     __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
 #pragma unroll 1
-    for (int c = half * 64; c < half * 64 + 64; c += 16) {
-      uint32_t g[16], u[16];
-      tmem_ld_32x32b_x16(t_row + c, g);
-      tmem_ld_32x32b_x16(t_row + 128 + c, u);
-      tmem_wait_ld();
-      if (row_ok) {
-        uint4 o[2];
-        uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+      // 32 columns per round: four tensor-memory loads in flight, one wait
+      uint32_t gg2[2][16], uu2[2][16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-          const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-          ow[i] = pack_bf16x2(silu_f(g0) * u0 * pr, silu_f(g1) * u1 * pr);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c);
-        dst[0] = o[0];
-        dst[1] = o[1];
-        if (hout) {
-          uint4 hg[2], hu[2];
-          uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
-          uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+      for (int j = 0; j < 2; ++j) {
+        tmem_ld_32x32b_x16(t_row + c0 + 16 * j, gg2[j]);
+        tmem_ld_32x32b_x16(t_row + 128 + c0 + 16 * j, uu2[j]);
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = c0 + 16 * j;
+        const uint32_t* g = gg2[j];
+        const uint32_t* u = uu2[j];
+        if (row_ok) {
+          uint4 o[2];
+          uint32_t* ow = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            hgw[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-            huw[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            ow[i] = pack_bf16x2(silu_f(g0) * u0 * pr, silu_f(g1) * u1 * pr);
           }
-          uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c);
-          hd[0] = hg[0];
-          hd[1] = hg[1];
-          uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c);
-          hd2[0] = hu[0];
-          hd2[1] = hu[1];
+          uint4* dst = reinterpret_cast<uint4*>(out + row * p.ldo + n0 + c);
+          dst[0] = o[0];
+          dst[1] = o[1];
+          if (hout) {
+            uint4 hg[2], hu[2];
+            uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
+            uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              hgw[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+              huw[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+            }
+            uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c);
+            hd[0] = hg[0];
+            hd[1] = hg[1];
+            uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c);
+            hd2[0] = hu[0];
+            hd2[1] = hu[1];
+          }
         }
       }
     }
@@ -243,43 +253,65 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
     const int n0 = ti.n_blk * gg::BN;
     float dp = 0.f;
 #pragma unroll 1
-    for (int c = half * (gg::BN / 2); c < (half + 1) * (gg::BN / 2); c += 16) {
-      uint32_t v[16];
-      tmem_ld_32x32b_x16(t_row + c, v);
-      tmem_wait_ld();
-      if (row_ok && n0 + c < p.N) {
-        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + n0 + c);
-        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + n0 + c);
-        uint4 gv[2] = {gp[0], gp[1]}, uv[2] = {up[0], up[1]};
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
-        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uv);
-        uint4 og[2], ou[2];
-        uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
-        uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 gg2 = __bfloat1622float2(g2[i]);
-          const float2 uu2 = __bfloat1622float2(u2[i]);
-          float dg[2], du[2];
-          const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const float da = __uint_as_float(v[2 * i + j]);
-            const float sg = 1.0f / (1.0f + expf(-gs[j]));
-            const float sl = gs[j] * sg;
-            dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
-            du[j] = da * pr * sl;
-            dp = fmaf(da, sl * us[j], dp);
-          }
-          ogw[i] = pack_bf16x2(dg[0], dg[1]);
-          ouw[i] = pack_bf16x2(du[0], du[1]);
+    for (int c0 = half * (gg::BN / 2); c0 < (half + 1) * (gg::BN / 2); c0 += 32) {
+      // 32 columns per round: the saved h of the round is requested first, so its global
+      // latency overlaps the two tensor-memory loads and their wait
+      uint4 gva[4], uva[4];
+      const bool cols_ok0 = row_ok && n0 + c0 < p.N;
+      const bool cols_ok1 = row_ok && n0 + c0 + 16 < p.N;
+      if (cols_ok0) {
+        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + n0 + c0);
+        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + n0 + c0);
+        gva[0] = gp[0];
+        gva[1] = gp[1];
+        uva[0] = up[0];
+        uva[1] = up[1];
+        if (cols_ok1) {
+          gva[2] = gp[2];
+          gva[3] = gp[3];
+          uva[2] = up[2];
+          uva[3] = up[3];
         }
-        uint4* dg_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + n0 + c);
-        dg_dst[0] = og[0];
-        dg_dst[1] = og[1];
-        uint4* du_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + n0 + c);
-        du_dst[0] = ou[0];
-        du_dst[1] = ou[1];
+      }
+      uint32_t vv[2][16];
+      tmem_ld_32x32b_x16(t_row + c0, vv[0]);
+      tmem_ld_32x32b_x16(t_row + c0 + 16, vv[1]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int c = c0 + 16 * jj;
+        const uint32_t* v = vv[jj];
+        if (jj == 0 ? cols_ok0 : cols_ok1) {
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva + 2 * jj);
+          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva + 2 * jj);
+          uint4 og[2], ou[2];
+          uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
+          uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 gg2 = __bfloat1622float2(g2[i]);
+            const float2 uu2 = __bfloat1622float2(u2[i]);
+            float dg[2], du[2];
+            const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float da = __uint_as_float(v[2 * i + j]);
+              const float sg = 1.0f / (1.0f + expf(-gs[j]));
+              const float sl = gs[j] * sg;
+              dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+              du[j] = da * pr * sl;
+              dp = fmaf(da, sl * us[j], dp);
+            }
+            ogw[i] = pack_bf16x2(dg[0], dg[1]);
+            ouw[i] = pack_bf16x2(du[0], du[1]);
+          }
+          uint4* dg_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + n0 + c);
+          dg_dst[0] = og[0];
+          dg_dst[1] = og[1];
+          uint4* du_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + n0 + c);
+          du_dst[0] = ou[0];
+          du_dst[1] = ou[1];
+        }
       }
     }
     if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
