@@ -229,8 +229,8 @@ int quant_rows_launch(const void* in, long long rows, int cols, int mma, uint8_t
 int quant_cols_grouped_launch(const void* in, int R, int C, const int32_t* split_sizes, int E, uint8_t* codes,
                               uint8_t* atoms, cudaStream_t st) {
   const int blocks32 = R / 32 + E;   // upper bound of sum(ceil(n_e / 32))
-  const int ytiles = (C + 1023) / 1024;
-  dim3 grid(std::min(blocks32, std::max(1, device_props().sm_count * 16 / ytiles)), ytiles);
+  const int ytiles = (C + 511) / 512;   // 256 threads x 2 columns
+  dim3 grid(std::min(blocks32, std::max(1, device_props().sm_count * 24 / ytiles)), ytiles);
   quant_cols_grouped_kernel<<<grid, 256, 3 * (E + 1) * sizeof(int32_t), st>>>(
       reinterpret_cast<const __nv_bfloat16*>(in), C, split_sizes, E, codes, atoms);
   count_launch();

@@ -470,10 +470,11 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
 // KG_e = ceil(n_e / 128) k-groups; atom (e, column group cg, k-group kg) sits at
 // (kgoff_e * C/128 + cg * KG_e + kg) * 512 with kgoff_e = sum of KG over earlier experts.
 // Scale bytes of k-blocks past an expert's end (up to the next multiple of 4) are zero.
-// A thread quantises 4 adjacent columns of one 32-row block (8-byte loads, 4-byte code
-// stores); blockIdx.x walks the 32-row blocks of all experts (sum of ceil(n_e / 32) of
-// them), blockIdx.y the 1024-column tiles of 256 threads.
-__global__ void __launch_bounds__(256) quant_cols_grouped_kernel(const __nv_bfloat16* __restrict__ in, int C,
+// A thread quantises 2 adjacent columns of one 32-row block (4-byte loads, 2-byte code
+// stores; the block's 32 x 2 inputs stay packed in 32 registers so three blocks of 256
+// threads fit per SM); blockIdx.x walks the 32-row blocks of all experts (sum of
+// ceil(n_e / 32) of them), blockIdx.y the 512-column tiles of 256 threads.
+__global__ void __launch_bounds__(256, 3) quant_cols_grouped_kernel(const __nv_bfloat16* __restrict__ in, int C,
                                                                  const int32_t* __restrict__ split_sizes, int E,
                                                                  uint8_t* __restrict__ codes,
                                                                  uint8_t* __restrict__ atoms) {
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(256) quant_cols_grouped_kernel(const __nv_bflo
   }
   __syncthreads();
   const int CG = C / 128;
-  const int c0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;   // this thread's 4 columns
+  const int c0 = (blockIdx.y * blockDim.x + threadIdx.x) * 2;   // this thread's 2 columns
   if (c0 >= C) return;
   for (int blk = blockIdx.x; blk < boff[E]; blk += gridDim.x) {
     int lo = 0, hi = E - 1;   // expert owning 32-row block `blk`
@@ -531,44 +532,38 @@ __global__ void __launch_bounds__(256) quant_cols_grouped_kernel(const __nv_bflo
     const int r0 = roff[e] + 32 * j;
     const int nrows = min(32, n - 32 * j);
     const int KG = (n + 127) / 128;
-    uint2 raw[32];
-    float amax[4] = {0.f, 0.f, 0.f, 0.f};
+    // 32 rows x 2 columns held as packed bf16 pairs (32 registers): three blocks fit per SM
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(in + (size_t)r0 * C + c0);
+    const size_t row_words = (size_t)C / 2;
+    uint32_t raw[32];
+    float amax[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      raw[i] = (i < nrows) ? __ldg(reinterpret_cast<const uint2*>(in + (size_t)(r0 + i) * C + c0))
-                           : make_uint2(0, 0);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[i]);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const float2 f = __bfloat1622float2(h[q]);
-        amax[2 * q] = fmaxf(amax[2 * q], fabsf(f.x));
-        amax[2 * q + 1] = fmaxf(amax[2 * q + 1], fabsf(f.y));
-      }
+      raw[i] = (i < nrows) ? __ldg(src + i * row_words) : 0u;
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i]));
+      amax[0] = fmaxf(amax[0], fabsf(f.x));
+      amax[1] = fmaxf(amax[1], fabsf(f.y));
     }
-    float inv[4];
-    int code[4];
+    float inv[2];
+    int code[2];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       code[q] = max((int)((__float_as_uint(amax[q]) >> 23) & 0xFF) - 8, 0);
       inv[q] = __uint_as_float((uint32_t)(254 - code[q]) << 23);
     }
+    uint16_t* dst = reinterpret_cast<uint16_t*>(codes + (size_t)r0 * C + c0);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       if (i < nrows) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[i]);
-        const float2 a = __bfloat1622float2(h[0]);
-        const float2 b = __bfloat1622float2(h[1]);
-        const __nv_fp8x2_storage_t lo2 =
-            __nv_cvt_float2_to_fp8x2(make_float2(a.x * inv[0], a.y * inv[1]), __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t hi2 =
-            __nv_cvt_float2_to_fp8x2(make_float2(b.x * inv[2], b.y * inv[3]), __NV_SATFINITE, __NV_E4M3);
-        *reinterpret_cast<uint32_t*>(codes + (size_t)(r0 + i) * C + c0) = (uint32_t)lo2 | ((uint32_t)hi2 << 16);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i]));
+        dst[i * row_words] =
+            (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(a.x * inv[0], a.y * inv[1]), __NV_SATFINITE, __NV_E4M3);
       }
     }
     const size_t grp = (size_t)koff[e] * CG + (size_t)(c0 / 128) * KG;   // this column group's first atom
     const bool last = 32 * (j + 1) >= n;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       const int c = c0 + q;
       atoms[mma_scale_offset(grp, c % 128, j, 1)] = (uint8_t)code[q];
       if (last)   // the expert's last block: zero the unused bytes of its atom
