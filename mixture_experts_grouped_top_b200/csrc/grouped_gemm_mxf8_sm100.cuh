@@ -9,10 +9,12 @@
 //
 // Same tile walk and warp roles as the BF16 kernel (grouped_gemm_sm100.cuh). What is
 // specific to block scaling:
-//   * scales travel with every 128-wide k-block as 512-byte atoms (128 rows x 4 scale
-//     bytes, row r of the group at word (r % 32) * 4 + r / 32, the layout tcgen05.cp
-//     expects), already arranged so in global memory (mma_scale_offset): the producer
-//     fetches one atom for A and two for B with bulk copies on the stage's barrier;
+//   * scales are 512-byte atoms per 128-wide k-block (128 rows x 4 scale bytes, row r of
+//     the group at word (r % 32) * 4 + r / 32, the layout tcgen05.cp expects), already
+//     arranged so in global memory (mma_scale_offset), a row group's atoms for
+//     consecutive k-blocks contiguous: they travel on a two-slot ring of their own, one
+//     bulk copy per row group (A, and B's two 128-row halves) per four k-blocks, since a
+//     copy costs the copy engine about the same whatever its size;
 //   * the MMA thread moves the atoms into tensor memory with tcgen05.cp (32 lanes x 16 B,
 //     replicated to the four sub-partitions), then issues the four K=32 MMAs of the
 //     stage, selecting scale byte kk of each word through the scale-factor ids;
@@ -37,12 +39,16 @@ constexpr int kABytes = BM * BK;              // 16 KB
 constexpr int kBBytes = BN * BK;              // 32 KB
 constexpr int kSfaBytes = 512;                // 128 rows x 4 scale bytes
 constexpr int kSfbBytes = 1024;               // 256 rows x 4 scale bytes
+constexpr int kSfKb = 4;                      // k-blocks per scale copy
+constexpr int kSfGroupBytes = kSfKb * 512;    // one row group's atoms for kSfKb k-blocks
+constexpr int kSfSlotBytes = 3 * kSfGroupBytes;   // A group, B lower group, B upper group
+constexpr int kSfSlots = 2;
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 224;
 constexpr uint32_t kSfaCol = 480;
 constexpr uint32_t kSfbCol = 484;
-constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kStages * (kSfaBytes + kSfbBytes) + 1024 +
+constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kSfSlots * kSfSlotBytes + 1024 +
                            4 * (kMaxE + 1) * 4;
 }  // namespace mx
 
@@ -288,15 +294,16 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + kStages * kABytes;
-  uint8_t* sSfa = sB + kStages * kBBytes;
-  uint8_t* sSfb = sSfa + kStages * kSfaBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSfb + kStages * kSfbBytes);
+  uint8_t* sSf = sB + kStages * kBBytes;     // scale ring: kSfSlots slots of three 2 KB groups
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSf + kSfSlots * kSfSlotBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* tfull = bars + 2 * kStages;
   uint64_t* tempty = bars + 2 * kStages + 2;
   uint64_t* tovl = bars + 2 * kStages + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* sfull = bars + 2 * kStages + 5;
+  uint64_t* sempty = sfull + kSfSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSfSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -318,6 +325,10 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       mbar_init(&tempty[a], 256);
     }
     mbar_init(tovl, 256);
+    for (int s2 = 0; s2 < kSfSlots; ++s2) {
+      mbar_init(&sfull[s2], 1);
+      mbar_init(&sempty[s2], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -380,9 +391,9 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
+      int stage = 0, sslot = 0;
+      uint32_t phase = 0, sphase = 0;
+      int issued = 0, sissued = 0;
       bool ok = true;
       const int KB4 = KGROUP ? 0 : p.K / 128;
       const int bgroups = mp.b_rows / 128;
@@ -403,12 +414,31 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
         }
         for (int kb = 0; kb < num_kb; ++kb) {
+          if ((kb & (kSfKb - 1)) == 0) {
+            // scale atoms of k-blocks [kb, kb + n): each row group's atoms for consecutive
+            // k-blocks are contiguous, so one copy per group (never past this tile's last atom)
+            if (!mbar_wait_bounded(&sempty[sslot], sphase ^ 1, abort_flag, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            const uint32_t n = (uint32_t)min(kSfKb, num_kb - kb) * 512;
+            uint8_t* sd = sSf + sslot * kSfSlotBytes;
+            mbar_arrive_expect_tx(&sfull[sslot], 3 * n);
+            bulk_load(sd, mp.a_atoms + (ga + kb) * 512, n, &sfull[sslot]);
+            bulk_load(sd + kSfGroupBytes, mp.b_atoms + (gb0 + kb) * 512, n, &sfull[sslot]);
+            bulk_load(sd + 2 * kSfGroupBytes, mp.b_atoms + (gb1 + kb) * 512, n, &sfull[sslot]);
+            ++sissued;
+            if (++sslot == kSfSlots) {
+              sslot = 0;
+              sphase ^= 1;
+            }
+          }
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }
           const int k0 = kb * BK;
-          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes + kSfaBytes + kSfbBytes);
+          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes);
           uint8_t* b_dst = sB + stage * kBBytes;
           if (KGROUP) {
             // MN-major codes: box {128 columns, 128 rows} at the expert's k-th row block
@@ -420,9 +450,6 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
             tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
             tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, EPI == MXEPI_SWIGLU_Q ? p.F + n0 : n0 + 128, ti.e);
           }
-          bulk_load(sSfa + stage * kSfaBytes, mp.a_atoms + (ga + kb) * 512, 512, &full[stage]);
-          bulk_load(sSfb + stage * kSfbBytes, mp.b_atoms + (gb0 + kb) * 512, 512, &full[stage]);
-          bulk_load(sSfb + stage * kSfbBytes + 512, mp.b_atoms + (gb1 + kb) * 512, 512, &full[stage]);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -441,12 +468,23 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           while (!mbar_try_wait(&full[st], ph) && global_timer_ns() - t0 < 100000000ull) {
           }
         }
+        // and the scale copies still in flight
+        int ss = sslot, sp = sphase;
+        for (int i = 0; i < min(sissued, kSfSlots); ++i) {
+          if (--ss < 0) {
+            ss = kSfSlots - 1;
+            sp ^= 1;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&sfull[ss], sp) && global_timer_ns() - t0 < 100000000ull) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, sslot = 0;
+    uint32_t phase = 0, sphase = 0;
     int lt = 0;
     bool ok = true;
     const uint32_t sfa_t = tmem_base + kSfaCol;
@@ -460,6 +498,10 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (acc ? kAcc1Col : 0u);
       for (int kb = 0; kb < num_kb; ++kb) {
+        if ((kb & (kSfKb - 1)) == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
           ok = false;
           break;
@@ -485,11 +527,11 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           __syncwarp();
         }
         if (lane == 0) {
-          const uint32_t sfa_s = smem_u32(sSfa + stage * kSfaBytes);
-          const uint32_t sfb_s = smem_u32(sSfb + stage * kSfbBytes);
-          tmem_cp_32x128b_warpx4(sfa_t, make_sdesc(sfa_s, 0, 128, 0));
-          tmem_cp_32x128b_warpx4(sfb_t, make_sdesc(sfb_s, 0, 128, 0));
-          tmem_cp_32x128b_warpx4(sfb_t + 4, make_sdesc(sfb_s + kSfaBytes, 0, 128, 0));
+          // this k-block's atoms: entry kb % kSfKb of each group of the current scale slot
+          const uint32_t sf_s = smem_u32(sSf + sslot * kSfSlotBytes) + (uint32_t)(kb & (kSfKb - 1)) * 512;
+          tmem_cp_32x128b_warpx4(sfa_t, make_sdesc(sf_s, 0, 128, 0));
+          tmem_cp_32x128b_warpx4(sfb_t, make_sdesc(sf_s + kSfGroupBytes, 0, 128, 0));
+          tmem_cp_32x128b_warpx4(sfb_t + 4, make_sdesc(sf_s + 2 * kSfGroupBytes, 0, 128, 0));
           const uint32_t a_addr = smem_u32(sA + stage * kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
@@ -506,11 +548,19 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
                         (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
+          // the slot's last k-block: release it once these MMAs have read their scales
+          if ((kb & (kSfKb - 1)) == kSfKb - 1 || kb == num_kb - 1) mma_commit(&sempty[sslot]);
         }
         __syncwarp();
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;
+        }
+        if ((kb & (kSfKb - 1)) == kSfKb - 1 || kb == num_kb - 1) {
+          if (++sslot == kSfSlots) {
+            sslot = 0;
+            sphase ^= 1;
+          }
         }
       }
       if (!ok) break;
