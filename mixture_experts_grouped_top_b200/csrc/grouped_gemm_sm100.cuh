@@ -13,9 +13,12 @@
 //   M-grouped   rows of expert e are [off_e, off_e + n_e) of A and of the output; B is
 //               the expert's own [K, N] (or [N, K]) slice. Tiles never straddle two
 //               experts in the output: rows past n_e are computed but not stored.
+//               (The library runs its M-grouped GEMMs on CTA pairs, in
+//               grouped_gemm_pair_sm100.cuh, which reuses the epilogues below.)
 //   K-grouped   (weight gradients) C_e = A_e^T B_e with the contraction over the
-//               expert's rows; the last k-block is clipped by zeroing the rows past
-//               n_e in shared memory before the MMAs read it.
+//               expert's rows; in the expert's last k-block only the MMA steps holding
+//               its rows are issued, and the rows past n_e inside the last partial step
+//               are zeroed in shared memory before the MMAs read them.
 //
 // Pages: "Efficient MoE training for biological foundation models" (sitech.ge section
 // "Grouped experts instead of a Python loop"; news.bpdata.com section 1): one grouped
