@@ -130,7 +130,8 @@ class ClockSampler:
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["ptx_sm100.cuh", "token_kernels.cuh", "grouped_gemm_sm100.cuh", "grouped_gemm_mxf8_sm100.cuh",
-                  "grouped_gemm_pair_sm100.cuh", "grouped_gemm_mxf8_pair_sm100.cuh", "moe_api.cu"]
+                  "grouped_gemm_pair_sm100.cuh", "grouped_gemm_mxf8_pair_sm100.cuh",
+                  "grouped_gemm_kgroup_pair_sm100.cuh", "moe_api.cu"]
 
 
 def kernel_sources_sha256() -> str:

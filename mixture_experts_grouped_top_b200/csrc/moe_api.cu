@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "moe_grouped.h"
+#include "grouped_gemm_kgroup_pair_sm100.cuh"
 #include "grouped_gemm_mxf8_pair_sm100.cuh"
 #include "grouped_gemm_mxf8_sm100.cuh"
 #include "grouped_gemm_pair_sm100.cuh"
@@ -156,6 +157,32 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
   kern<<<2 * pairs, g2::kThreads, g2::kSmemBytes, st>>>(ta, tb, p);
+  count_launch();
+  return launch_status();
+}
+
+// BF16 weight-gradient GEMMs on CTA pairs: as many 2-CTA clusters as can be resident.
+int launch_wgrad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+  auto kern = grouped_wgrad_bf16_pair_kernel;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int pairs = 0;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kp::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(device_props().sm_count, 1, 1);
+    cfg.blockDim = dim3(kp::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kp::kSmemBytes;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_props().sm_count / 2;
+    pairs = std::min(n, device_props().sm_count / 2);
+    cudaGetLastError();
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  kern<<<2 * pairs, kp::kThreads, kp::kSmemBytes, st>>>(ta, tb, p);
   count_launch();
   return launch_status();
 }
@@ -824,15 +851,15 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
     if ((rc = launch_status())) return rc;
   }
   // fc2 wgrad: dw2[e] = a_e^T dy_e. A = a [R, F] (rows = K, MN-major), B = dy [R, H] (MN-major)
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_buf, 1, R, F, 2, gg::BK, gg::BM / 64))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy_perm, 1, R, H, 2, gg::BK, gg::BN / 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_buf, 1, R, F, 2, kp::BK, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy_perm, 1, R, H, 2, kp::BK, 2))) return rc;
   p = base_params(split_sizes, E);
   p.M = F;
   p.N = H;
   p.out = dw2;
   p.ldo = H;
   p.out_batch = (long long)F * H;
-  if ((rc = launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st))) return rc;
+  if ((rc = launch_wgrad_pair(ta, tb, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh [R, 2F] (K-major), B = w1 [E, H, 2F] read as [E, N=H, K=2F] (K-major)
   if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, 1, R, 2 * F, 2))) return rc;
   if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w1, E, H, 2 * F, 2))) return rc;
@@ -844,15 +871,15 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.ldo = H;
   if ((rc = launch_gemm_pair<false, EPI_STORE>(ta, tb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e. A = xp [R, H] (MN-major), B = dh [R, 2F] (MN-major)
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, 1, R, H, 2, gg::BK, gg::BM / 64))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, 1, R, 2 * F, 2, gg::BK, gg::BN / 64))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, 1, R, H, 2, kp::BK, 2))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dh, 1, R, 2 * F, 2, kp::BK, 2))) return rc;
   p = base_params(split_sizes, E);
   p.M = H;
   p.N = 2 * F;
   p.out = dw1;
   p.ldo = 2 * F;
   p.out_batch = (long long)H * 2 * F;
-  return launch_gemm<true, true, true, EPI_WGRAD>(ta, tb, p, st);
+  return launch_wgrad_pair(ta, tb, p, st);
 }
 
 }  // extern "C"
