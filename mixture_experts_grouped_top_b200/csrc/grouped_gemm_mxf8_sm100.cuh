@@ -9,7 +9,7 @@
 //
 // The library runs its M-grouped MXFP8 GEMMs on CTA pairs (grouped_gemm_mxf8_pair_sm100.cuh,
 // which reuses the epilogues below) and this kernel for the K-grouped weight gradients.
-// Same tile walk and warp roles as the BF16 kernel (grouped_gemm_sm100.cuh). What is
+// Same tile walk and warp roles as the BF16 kernels (grouped_gemm_sm100.cuh). What is
 // specific to block scaling:
 //   * scales are 512-byte atoms per 128-wide k-block (128 rows x 4 scale bytes, row r of
 //     the group at word (r % 32) * 4 + r / 32, the layout tcgen05.cp expects), already

@@ -1,20 +1,19 @@
-// Persistent grouped GEMM for sm_100a on the 5th-generation tensor cores.
+// Shared pieces of the persistent grouped GEMMs on sm_100a (5th-generation tensor cores):
+// parameters, the tile walker over ragged expert groups, the longest-expert-first order,
+// and the fused BF16 epilogues that drain a tensor-memory accumulator (thread = row; two
+// warps per 32-lane quadrant, each taking half of the columns).
 //
-// One CTA per SM walks a static round-robin list of output tiles spread over ragged
-// expert groups. Inside a CTA the work is warp-specialised:
-//   warp 0      TMA producer: fills a ring of kStages shared-memory stages;
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16 for
-//               bf16) into one of two tensor-memory accumulators (2 x 256 fp32 columns);
-//   warp 2      tensor-memory allocator;
-//   warps 4..11 epilogue: tcgen05.ld the accumulator (thread = row; two warps per
-//               32-lane quadrant, each taking half of the columns), apply the fused
-//               epilogue, store to global memory, release the accumulator.
+// The kernels that use them (each CTA warp-specialised: warp 0 TMA producer, warp 1 MMA
+// issuer, warp 2 tensor-memory allocator, warps 4..11 epilogue; one CTA per SM or one
+// 2-CTA cluster per SM pair, walking a static round-robin list of output tiles):
+//   grouped_gemm_pair_sm100.cuh         BF16 M-grouped GEMMs on CTA pairs
+//   grouped_gemm_kgroup_pair_sm100.cuh  BF16 K-grouped (weight-gradient) GEMMs on pairs
+//   grouped_gemm_mxf8_pair_sm100.cuh    MXFP8 M-grouped GEMMs on CTA pairs
+//   grouped_gemm_mxf8_sm100.cuh         MXFP8 K-grouped GEMMs on one SM
 // Two grouping modes:
 //   M-grouped   rows of expert e are [off_e, off_e + n_e) of A and of the output; B is
 //               the expert's own [K, N] (or [N, K]) slice. Tiles never straddle two
 //               experts in the output: rows past n_e are computed but not stored.
-//               (The library runs its M-grouped GEMMs on CTA pairs, in
-//               grouped_gemm_pair_sm100.cuh, which reuses the epilogues below.)
 //   K-grouped   (weight gradients) C_e = A_e^T B_e with the contraction over the
 //               expert's rows; in the expert's last k-block only the MMA steps holding
 //               its rows are issued, and the rows past n_e inside the last partial step
@@ -31,19 +30,10 @@
 namespace moe {
 
 namespace gg {
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;                                   // bf16: 128 bytes of K per row
-constexpr int kStages = 4;
-constexpr int kThreads = 384;                          // 4 control warps + 8 epilogue warps
-constexpr int kABytes = BM * BK * 2;                     // 16 KB
-constexpr int kBBytes = BN * BK * 2;                     // 32 KB
-constexpr int kChunkBytes = 64 * BK * 2;                 // one 64-wide MN chunk, 8 KB
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kMaxE = 1024;
-constexpr int kTmemCols = 512;                           // two 256-column accumulators
-constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 1024 /*barriers*/ +
-                           3 * (kMaxE + 1) * 4 /*expert prefix tables, expert order*/;
+constexpr int BM = 128;                                  // M of a 1-SM tile (default tile walker rows)
+constexpr int BN = 256;                                  // N of an output tile (epilogue column span)
+constexpr int BK = 64;                                   // k-block of TileInfo::num_kb (128 bytes of bf16)
+constexpr int kMaxE = 1024;                              // experts the kernels' shared tables hold
 constexpr uint64_t kTimeoutNs = 4000000000ull;           // 4 s per wait
 }  // namespace gg
 
@@ -134,16 +124,6 @@ __device__ __forceinline__ void rank_experts_by_rows(const int32_t* row_off, int
     }
     order[rank] = e;
   }
-}
-
-// Column of the B operand (output column space) of 64-wide chunk c of an N tile.
-template <int EPI>
-__device__ __forceinline__ int b_chunk_col(int n_blk, int c, int F) {
-  if (EPI == EPI_SWIGLU) {
-    const int n0 = n_blk * 128;
-    return (c < 2) ? n0 + 64 * c : F + n0 + 64 * (c - 2);
-  }
-  return n_blk * gg::BN + 64 * c;
 }
 
 // Drain one BF16 accumulator tile: this thread owns row `tile_row` of the tile (its TMEM
@@ -318,250 +298,6 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
       }
     }
     if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
-  }
-}
-
-template <bool A_MN, bool B_MN, bool KGROUP, int EPI>
-__global__ void __launch_bounds__(gg::kThreads, 1)
-    grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmParams p) {
-  using namespace gg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = bars + 2 * kStages + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
-  int32_t* tile_off = row_off + (kMaxE + 1);
-  int32_t* order = tile_off + (kMaxE + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = p.E;
-
-  // output tiling
-  const int NT = (EPI == EPI_SWIGLU) ? (p.N / 128) : (p.N + BN - 1) / BN;
-  const int MT = KGROUP ? (p.M + BM - 1) / BM : 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  // expert prefix tables (warp 3): rows and tiles
-  if (warp == 3) {
-    int carry_r = 0, carry_t = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      const int n = (e < E) ? p.split_sizes[e] : 0;
-      const int tiles = (e < E) ? (KGROUP ? MT * NT : ((n + BM - 1) / BM) * NT) : 0;
-      int ir = n, it = tiles;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
-        const int yt = __shfl_up_sync(0xffffffffu, it, o);
-        if (lane >= o) {
-          ir += yr;
-          it += yt;
-        }
-      }
-      if (e < E) {
-        row_off[e] = carry_r + ir - n;
-        tile_off[e] = carry_t + it - tiles;
-      }
-      carry_r += __shfl_sync(0xffffffffu, ir, 31);
-      carry_t += __shfl_sync(0xffffffffu, it, 31);
-    }
-    if (lane == 0) {
-      row_off[E] = carry_r;
-      tile_off[E] = carry_t;
-    }
-  }
-  if (warp == 2) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  if (KGROUP) {
-    rank_experts_by_rows(row_off, E, order);
-    __syncthreads();
-  }
-
-  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K, order};
-  const int total = walk.total();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileInfo ti = walk.decode(t);
-        for (int kb = 0; kb < ti.num_kb; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          uint8_t* a_dst = sA + stage * kABytes;
-          uint8_t* b_dst = sB + stage * kBBytes;
-          const int k0 = kb * BK;
-          if (!A_MN) {
-            tma_load_3d(a_dst, &tmA, &full[stage], k0, ti.row0, 0);
-          } else if (KGROUP) {
-            // both 64-column chunks in one copy (chunked view, box {64, 64 k rows, 2, 1})
-            tma_load_4d(a_dst, &tmA, &full[stage], 0, ti.row0 + k0, ti.m_blk * (BM / 64), 0);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_3d(a_dst + c * kChunkBytes, &tmA, &full[stage], ti.m_blk * BM + 64 * c, ti.row0 + k0, 0);
-          }
-          if (!B_MN) {
-            tma_load_3d(b_dst, &tmB, &full[stage], k0, ti.n_blk * BN, ti.e);
-          } else if (KGROUP) {
-            // all four 64-column chunks in one copy (box {64, 64 k rows, 4, 1})
-            tma_load_4d(b_dst, &tmB, &full[stage], 0, ti.row0 + k0, ti.n_blk * (BN / 64), 0);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tma_load_3d(b_dst + c * kChunkBytes, &tmB, &full[stage], b_chunk_col<EPI>(ti.n_blk, c, p.F), k0, ti.e);
-          }
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      if (!ok) {
-        // drain: let the copies already issued land before the CTA can exit
-        int st = stage, ph = phase;
-        for (int i = 0; i < min(issued, kStages); ++i) {
-          if (--st < 0) {
-            st = kStages - 1;
-            ph ^= 1;
-          }
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[st], ph) && global_timer_ns() - t0 < 100000000ull) {
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = make_idesc_bf16(BM, BN, A_MN, B_MN);
-    int stage = 0;
-    uint32_t phase = 0;
-    int lt = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
-      const TileInfo ti = walk.decode(t);
-      const int acc = lt & 1;
-      const uint32_t acc_phase = (lt >> 1) & 1;
-      if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, p.timeout_ns)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kb = 0; kb < ti.num_kb; ++kb) {
-        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        int ksteps = BK / 16;   // K=16 MMAs of this stage
-        if (KGROUP && (kb + 1) * BK > ti.rows) {
-          // clip the contraction at the end of the expert's rows: MMAs only over the
-          // expert's K-rows; inside the last, partial 16-row step zero the rows >= valid
-          // of all six 64-wide operand chunks (A 2, B 4; row r of a chunk at r * 128 bytes)
-          const int valid = ti.rows - kb * BK;
-          ksteps = (valid + 15) / 16;
-          const int zr = ksteps * 16 - valid;   // 0..15 rows
-          if (zr > 0) {
-            uint8_t* a_st = sA + stage * kABytes;
-            uint8_t* b_st = sB + stage * kBBytes;
-            for (int i = lane; i < 6 * zr * 8; i += 32) {
-              const int v = i & 7, rc = i >> 3;
-              const int c = rc / zr, r = rc - c * zr;
-              uint8_t* base = (c < 2) ? a_st + c * kChunkBytes : b_st + (c - 2) * kChunkBytes;
-              *reinterpret_cast<uint4*>(base + (valid + r) * 128 + v * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-          }
-          __syncwarp();
-        }
-        if (lane == 0) {
-          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (kk >= ksteps) break;
-            const uint64_t adesc = A_MN ? make_sdesc(a_addr + kk * 2048, kChunkBytes, 1024, 2)
-                                        : make_sdesc(a_addr + kk * 32, 16, 1024, 2);
-            const uint64_t bdesc = B_MN ? make_sdesc(b_addr + kk * 2048, kChunkBytes, 1024, 2)
-                                        : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
-            mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&empty[stage]);
-        }
-        __syncwarp();
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (!ok) break;
-      if (lane == 0) {
-        if (ti.num_kb > 0)
-          mma_commit(&tfull[acc]);
-        else
-          mbar_arrive(&tfull[acc]);
-      }
-      __syncwarp();
-    }
-  } else if (warp >= 4) {
-    // ----------------------------------------------------------------- epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int half = (warp - 4) >> 2;       // which half of the tile's columns it drains
-    const int r_local = q * 32 + lane;      // accumulator row owned by this thread
-    int lt = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
-      const TileInfo ti = walk.decode(t);
-      const int acc = lt & 1;
-      const uint32_t acc_phase = (lt >> 1) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, p.timeout_ns)) break;
-      tc_fence_after();
-      const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      bf16_epilogue_tile<EPI>(p, ti, t_row, half, r_local, BM);
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 2) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

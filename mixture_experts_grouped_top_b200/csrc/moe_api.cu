@@ -118,21 +118,6 @@ int tmap_chunks(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_
   return MOE_OK;
 }
 
-template <bool A_MN, bool B_MN, bool KG, int EPI>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
-  auto kern = grouped_gemm_bf16_kernel<A_MN, B_MN, KG, EPI>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gg::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  const int grid = device_props().sm_count;
-  kern<<<grid, gg::kThreads, gg::kSmemBytes, st>>>(ta, tb, p);
-  count_launch();
-  return launch_status();
-}
-
 // CTA-pair kernels: launch as many 2-CTA clusters as can be resident at once (a
 // persistent grid larger than that would leave some pairs waiting for others to finish).
 template <bool B_MN, int EPI>
