@@ -234,8 +234,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = mb.moe_launch_count()
-    with ClockSampler(local, os.path.join(ROOT, "gpurun_out", "clocks.csv")
-                      if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None) as clocks:
+    with ClockSampler(local, args.clocks_csv) as clocks:
         wall0 = time.perf_counter()
         t0.record(stream)
         for i in range(K):
@@ -401,6 +400,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs on a smaller batch)")
     ap.add_argument("--cpu-baseline-tokens", type=int, default=256)
     ap.add_argument("--reference-tokens", type=int, default=64)
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region in this file")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
