@@ -421,12 +421,15 @@ def bwd_sampled_bf16(dy_perm, xp, split_sizes, w1, w2, probs_perm, rows, experts
     return dxp, dpp, dw1, dw2
 
 
-def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_scales=None):
+def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_scales=None, details=False):
     """MXFP8 forward of individual routed rows (x_rows[i] is the token's bf16 row routed
     to expert expert_of_rows[i] with probability prob_rows[i]), float64 on quantised
     operands. The oracle quantises x along H and each needed expert's weights along their
     contraction axis itself. fc2 runs on the oracle's own `a` codes unless ``a_codes`` /
-    ``a_scales`` (rows x F, F/32) are given. Returns (yp, a_codes, a_scales)."""
+    ``a_scales`` (rows x F, F/32) are given. Returns (yp, a_codes, a_scales); with
+    ``details`` also a dict with fc1's exact output ``h`` [rows, 2F] and ``sum_abs``, the
+    sum over H of |x_q * w1_q| per element of h (the magnitude an fp32 accumulation of
+    that dot product is rounded against)."""
     xr = f64(x_rows)
     prob_rows = f64(prob_rows)
     experts = np.asarray(expert_of_rows, dtype=np.int64)
@@ -435,11 +438,16 @@ def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_sc
     yp = np.zeros((xr.shape[0], w2.shape[2]))
     own_c = np.zeros((xr.shape[0], F), dtype=np.uint8)
     own_s = np.zeros((xr.shape[0], F // 32), dtype=np.uint8)
+    h_all = np.zeros((xr.shape[0], 2 * F)) if details else None
+    sabs = np.zeros((xr.shape[0], 2 * F)) if details else None
     for e in np.unique(experts):
         sel = np.nonzero(experts == e)[0]
         w1q = mxfp8.dequantize(*mxfp8.quantize(f64(w1[e]), axis=1), axis=1)     # along H
         w2q = mxfp8.dequantize(*mxfp8.quantize(f64(w2[e]), axis=1), axis=1)     # along F
         hh = xq[sel] @ w1q
+        if details:
+            h_all[sel] = hh
+            sabs[sel] = np.abs(xq[sel]) @ np.abs(w1q)
         a = silu(hh[:, :F]) * hh[:, F:] * prob_rows[sel, None]
         c, s = mxfp8.quantize(a, axis=0)
         own_c[sel], own_s[sel] = c, s
@@ -448,6 +456,8 @@ def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_sc
         else:
             aq = mxfp8.dequantize(np.asarray(a_codes)[sel], np.asarray(a_scales)[sel], axis=0)
         yp[sel] = aq @ w2q
+    if details:
+        return yp, own_c, own_s, {"h": h_all, "sum_abs": sabs}
     return yp, own_c, own_s
 
 

@@ -3,8 +3,9 @@
 fc2's output is compared with the oracle run on the same quantised operands (xp and
 weight codes, which are bit-exact by the quantiser tests, and the `a` codes the fc1
 epilogue emitted): max|err| / max|ref| <= 2e-3. fc1's quantised `a` is compared with the
-oracle's own quantisation of its fp64 `a`: codes may differ only where fp32 and fp64
-land on opposite sides of a rounding boundary, i.e. by one E4M3 step.
+oracle's own quantisation of its fp64 `a`: codes and scales may differ only where fp32
+and fp64 land on opposite sides of a rounding boundary (one E4M3 step, with the exact
+value within the fp32 error bound of the midpoint; see tests/mx_checks.py).
 """
 import numpy as np
 import pytest
@@ -14,6 +15,7 @@ import mixture_experts_grouped_top_b200 as mb
 from oracle import moe as om
 from oracle import mxfp8 as oq
 import workloads
+from tests.mx_checks import assert_boundary_flips, swiglu_fp32_error_bound
 from tests.mx_layout import plain_to_atoms, tile_atoms_to_plain
 
 pytestmark = pytest.mark.gpu
@@ -99,13 +101,20 @@ def test_grouped_mlp_fwd_mxfp8_parity(T, H, F, E, k, empty):
         cpu(o["xp"]), cpu(o["xp_scale"]), split, cpu(r["w1c"]), cpu(r["w1s"]), cpu(r["w2c"]), cpu(r["w2s"]),
         cpu(o["probs_perm"]))
     gc, gs = cpu(r["a_codes"]), cpu(r["a_scales"])
-    assert np.mean(gc == rac_own) >= 0.99
-    assert np.mean(gs == ras_own) >= 0.99
-    a_exact = om.silu(rh[:, :F]) * rh[:, F:] * cpu(o["probs_perm"])[:, None]
-    deq = oq.dequantize_blocks_last_axis(gc, gs)
-    x = oq.e8m0_value(ras_own).repeat(32, axis=1)
-    # within one E4M3 step of the exact value (3 mantissa bits) plus the subnormal spacing
-    assert np.all(np.abs(deq - a_exact) <= 0.126 * np.abs(a_exact) + 2.0 ** -9 * x * 2)
+    pp = cpu(o["probs_perm"]).astype(np.float64)[:, None]
+    a_exact = om.silu(rh[:, :F]) * rh[:, F:] * pp
+    # codes and scales may differ from the oracle's only by rounding-boundary flips of the
+    # fp32 arithmetic, bounded per element from the magnitudes of fc1's products
+    xq = np.abs(oq.dequantize_blocks_last_axis(cpu(o["xp"]), cpu(o["xp_scale"])))
+    w1q = np.abs(oq.dequantize_blocks_last_axis(cpu(r["w1c"]), cpu(r["w1s"])))       # [E, 2F, H]
+    sabs = np.zeros((xq.shape[0], 2 * F))
+    s0 = 0
+    for e, n in enumerate(split):
+        sabs[s0:s0 + n] = xq[s0:s0 + n] @ w1q[e].T
+        s0 += n
+    err = swiglu_fp32_error_bound(rh[:, :F], rh[:, F:], pp, sabs[:, :F], sabs[:, F:], H)
+    rep = assert_boundary_flips(gc, gs, a_exact, "a", err=err)
+    assert rep["code_flips"] <= 0.01 * gc.size
 
 
 def test_mxfp8_layer_end_to_end_against_fully_oracle_chain():
