@@ -72,11 +72,14 @@ class MoEExpertLayer:
                         stream=stream)
         moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
         if self.training and self.prec == MXFP8:
-            # the MXFP8 weight gradient re-quantises xp along its rows: keep a bf16 copy
-            if self.xp_bf16 is None:
-                self.xp_bf16 = torch.empty((self.R, self.H), dtype=torch.bfloat16, device=self.device)
-            moe_permute_rows(x, self.perm["row_map"], self.k, out=self.xp_bf16, stream=stream)
+            self.permute_for_backward(x, stream=stream)
         return self.out
+
+    def permute_for_backward(self, x: torch.Tensor, stream=None):
+        """The MXFP8 weight gradient re-quantises xp along its rows: keep a bf16 copy."""
+        if self.xp_bf16 is None:
+            self.xp_bf16 = torch.empty((self.R, self.H), dtype=torch.bfloat16, device=self.device)
+        moe_permute_rows(x, self.perm["row_map"], self.k, out=self.xp_bf16, stream=stream)
 
     # -------------------------------------------------------------- backward
     def _alloc_bwd(self):
