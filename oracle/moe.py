@@ -84,6 +84,39 @@ def route(logits, k: int, renorm: bool = True):
     return order.astype(np.int32), prob
 
 
+def route_bwd(logits, idx, dprob, renorm: bool = True) -> np.ndarray:
+    """Gradient of the router's probabilities with respect to its logits.
+
+    The forward's steps, in order (``route``): s = softmax(l) over all E experts; the
+    selected probabilities q_j = s[idx_j]; with ``renorm`` p_j = q_j / Z, Z = sum_j q_j
+    (else p_j = q_j). Given dL/dp_j (``dprob`` [T, k]) and the forward's ``idx``, the
+    chain rule runs those steps backwards:
+        renorm:  dq_j = (dprob_j - sum_m dprob_m p_m) / Z      else  dq_j = dprob_j
+        gather:  ds_b = sum_j [idx_j == b] dq_j
+        softmax: dl_b = s_b * (ds_b - sum_c ds_c s_c)
+    Returns dlogits float64 [T, E]. The routing weights are what trains the router: each
+    token's expert outputs are weighted by them (sitech.ge, introduction).
+    """
+    lg = f64(logits)
+    idx = np.asarray(idx, dtype=np.int64)
+    dp = f64(dprob)
+    T, E = lg.shape
+    m = lg.max(axis=1, keepdims=True)
+    ex = np.exp(lg - m)
+    soft = ex / ex.sum(axis=1, keepdims=True)
+    q = np.take_along_axis(soft, idx, axis=1)
+    if renorm:
+        Z = q.sum(axis=1, keepdims=True)
+        p = q / Z
+        dq = (dp - np.sum(dp * p, axis=1, keepdims=True)) / Z
+    else:
+        dq = dp
+    ds = np.zeros((T, E))
+    for j in range(idx.shape[1]):
+        ds[np.arange(T), idx[:, j]] += dq[:, j]
+    return soft * (ds - np.sum(ds * soft, axis=1, keepdims=True))
+
+
 # ------------------------------------------------------------------------- permutation
 def permute_index(idx, E: int):
     """Stable counting sort of the flat slots by expert.

@@ -111,3 +111,75 @@ def test_unpermute_of_permute_is_identity(k):
 def test_permute_rejects_out_of_range():
     with pytest.raises(ValueError):
         moe.permute_index(np.array([[0, 3]]), 3)
+
+
+# ------------------------------------------------------------------ router backward
+def _torch_route_grad(lg, idx, dprob, renorm):
+    """dL/dlogits by torch fp64 autograd of softmax -> gather -> renormalise."""
+    import torch
+    lt = torch.tensor(lg, dtype=torch.float64, requires_grad=True)
+    q = torch.gather(torch.softmax(lt, dim=1), 1, torch.tensor(idx, dtype=torch.int64))
+    p = q / q.sum(dim=1, keepdim=True) if renorm else q
+    (p * torch.tensor(dprob)).sum().backward()
+    return lt.grad.numpy()
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+@pytest.mark.parametrize("E,k", [(4, 1), (8, 2), (16, 5), (7, 7), (128, 8)])
+def test_route_bwd_matches_torch_autograd(E, k, renorm):
+    rng = np.random.default_rng(E + 100 * k)
+    lg = rng.normal(size=(50, E)) * 2.0
+    idx, _ = moe.route(lg, k, renorm)
+    dprob = rng.normal(size=(50, k))
+    got = moe.route_bwd(lg, idx, dprob, renorm)
+    ref = _torch_route_grad(lg, idx, dprob, renorm)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_route_bwd_matches_finite_differences(renorm):
+    # logits with gaps of at least 0.5 between sorted values: the selection does not
+    # change under the perturbation, so the probabilities are smooth there
+    rng = np.random.default_rng(7)
+    T, E, k = 6, 9, 3
+    lg = np.stack([rng.permutation(E) * 0.5 + rng.uniform(0, 0.1) for _ in range(T)])
+    idx, _ = moe.route(lg, k, renorm)
+    dprob = rng.normal(size=(T, k))
+    got = moe.route_bwd(lg, idx, dprob, renorm)
+    eps = 1e-6
+    for t, b in [(0, 0), (1, 4), (3, 8), (5, 2), (2, 6)]:
+        lp, lm = lg.copy(), lg.copy()
+        lp[t, b] += eps
+        lm[t, b] -= eps
+        ip, pp = moe.route(lp, k, renorm)
+        im, pm = moe.route(lm, k, renorm)
+        assert np.array_equal(ip, idx) and np.array_equal(im, idx)
+        fd = (np.sum(pp * dprob) - np.sum(pm * dprob)) / (2 * eps)
+        assert abs(fd - got[t, b]) <= 1e-8 * max(1.0, abs(fd))
+
+
+def test_route_bwd_invariants_and_special_cases():
+    rng = np.random.default_rng(11)
+    T, E, k = 40, 12, 4
+    lg = rng.normal(size=(T, E))
+    idx, prob = moe.route(lg, k, True)
+    dprob = rng.normal(size=(T, k))
+    # shifting every logit of a token leaves the probabilities unchanged: rows sum to 0
+    for renorm in (True, False):
+        g = moe.route_bwd(lg, idx, dprob, renorm)
+        assert np.max(np.abs(g.sum(axis=1))) <= 1e-14
+    # with renormalisation the probabilities are the softmax over the selected logits
+    # only: no gradient reaches the others (zero up to fp64 rounding of <ds, s> = 0)
+    g = moe.route_bwd(lg, idx, dprob, True)
+    mask = np.ones((T, E), dtype=bool)
+    mask[np.arange(T)[:, None], idx] = False
+    assert np.max(np.abs(g[mask])) <= 1e-15
+    # constant upstream gradient with renormalisation: sum_j p_j = 1, so dlogits = 0
+    assert np.max(np.abs(moe.route_bwd(lg, idx, np.ones((T, k)), True))) <= 1e-15
+    # k = E with renorm is the plain softmax: the textbook Jacobian p * (d - <d, p>)
+    idx_all, p_all = moe.route(lg, E, True)
+    d = rng.normal(size=(T, E))
+    g = moe.route_bwd(lg, idx_all, d, True)
+    ref = np.zeros((T, E))
+    np.put_along_axis(ref, idx_all, p_all * (d - np.sum(d * p_all, axis=1, keepdims=True)), axis=1)
+    np.testing.assert_allclose(g, ref, rtol=1e-12, atol=1e-15)
