@@ -4,8 +4,9 @@
 The headline step is one forward + backward pass of the whole path on one batch of the
 genomic long-sequence Mixtral-shaped MXFP8 layer (T=32768 tokens, H=4096, F=14336,
 8 experts, top-2, expert 0 favoured): weight quantisation of the bf16 masters ->
-moe_route -> moe_permute -> grouped_mlp_fwd (fc1 + ScaledSwiGLU, fc2) -> moe_unpermute
--> moe_permute_rows(grad) -> grouped_mlp_bwd -> moe_unpermute(dxp) + moe_gather_slots.
+moe_route_permute (router + permutation) -> grouped_mlp_fwd (fc1 + ScaledSwiGLU, fc2) ->
+moe_unpermute -> moe_permute_rows(grad) -> grouped_mlp_bwd -> moe_unpermute(dxp) +
+moe_gather_slots -> moe_route_bwd (router logits' gradient).
 The same line reports, under ``workloads``, the other single-GPU layers (Mixtral BF16
 and MXFP8 forward, Qwen3-30B-A3B BF16 forward + backward) with their own roofline
 fractions, and the bandwidth of the permute and combine kernels.
@@ -42,6 +43,7 @@ import workloads  # noqa: E402
 
 DEFAULT_WORKLOAD = "genomic_mixtral_mxfp8_fwdbwd"
 SECONDARY_WORKLOADS = ["mixtral_bf16_fwd", "mixtral_mxfp8_fwd", "qwen3_30b_a3b_bf16_fwdbwd"]
+FUSED_COMBINE_WORKLOADS = ["mixtral_bf16_fwd", "qwen3_30b_a3b_bf16_fwdbwd"]
 METRIC = "grouped-MLP TFLOP/s & tokens/s (fwd, fwd+bwd) on 1 B200; % of tensor-core peak"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 MXFP8_PEAK_FILE = os.path.join(ROOT, "profiles", "mxfp8_peak.json")
@@ -271,8 +273,9 @@ def ev():
     return torch.cuda.Event(enable_timing=True)
 
 
-def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
-    """Time `steps` passes of the whole path on one workload. Returns the JSON fields."""
+def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fused_combine=False):
+    """Time `steps` passes of the whole path on one workload. Returns the JSON fields.
+    fused_combine: the combine runs inside fc2's epilogue (grouped_mlp_fwd_combine)."""
     import mixture_experts_grouped_top_b200 as mb
 
     dev = torch.device("cuda", local)
@@ -280,7 +283,8 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
     training = cfg.passes == "fwd+bwd"
     prec = cfg.precision
     d = workloads.make_layer_inputs(cfg, seed=rank_seed(cfg.seed, rank), with_grad=training)
-    layer = mb.MoEExpertLayer(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, prec, training=training, device=dev)
+    layer = mb.MoEExpertLayer(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, prec, training=training, device=dev,
+                              fused_combine=fused_combine)
     w1, w2 = d["w1"].to(dev), d["w2"].to(dev)
     layer.set_weights(w1, w2)
     x, logits = d["x"].to(dev), d["logits"].to(dev)
@@ -297,15 +301,23 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
         if training and prec == "mxfp8":
             layer.set_weights(w1, w2)   # a training step re-quantises the bf16 masters
         mark(1)
-        mb.moe_route(logits, cfg.k, True, idx=layer.idx, prob=layer.prob)
-        mb.moe_permute(x, layer.idx, layer.prob, cfg.E, prec, out=layer.perm, workspace=layer.perm_ws)
+        layer.perm["idx"], layer.perm["prob"] = layer.idx, layer.prob
+        mb.moe_route_permute(logits, x, cfg.k, True, prec, out=layer.perm, workspace=layer.perm_ws)
         mark(2)
-        mb.grouped_mlp_fwd(layer.perm["xp"], layer.perm["split_sizes"], layer.w1, layer.w2,
-                           layer.perm["probs_perm"], prec, xp_scale=layer.perm.get("xp_scale"),
-                           w1_scale=layer.w1_scale, w2_scale=layer.w2_scale, yp=layer.yp, saved=layer.saved,
-                           workspace=layer.mlp_ws, F=cfg.F)
-        mark(3)
-        mb.moe_unpermute(layer.yp, layer.perm["row_map"], cfg.T, cfg.k, out=layer.out)
+        if fused_combine:
+            mb.grouped_mlp_fwd_combine(layer.perm["xp"], layer.perm["split_sizes"], layer.w1, layer.w2,
+                                       layer.perm["probs_perm"], layer.perm["row_map"], cfg.T, cfg.k, prec,
+                                       xp_scale=layer.perm.get("xp_scale"), w1_scale=layer.w1_scale,
+                                       w2_scale=layer.w2_scale, out=layer.out, saved=layer.saved,
+                                       workspace=layer.mlp_ws, F=cfg.F)
+            mark(3)
+        else:
+            mb.grouped_mlp_fwd(layer.perm["xp"], layer.perm["split_sizes"], layer.w1, layer.w2,
+                               layer.perm["probs_perm"], prec, xp_scale=layer.perm.get("xp_scale"),
+                               w1_scale=layer.w1_scale, w2_scale=layer.w2_scale, yp=layer.yp, saved=layer.saved,
+                               workspace=layer.mlp_ws, F=cfg.F)
+            mark(3)
+            mb.moe_unpermute(layer.yp, layer.perm["row_map"], cfg.T, cfg.k, out=layer.out)
         mark(4)
         if training:
             if layer._bwd is None:
@@ -322,6 +334,7 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
             mark(6)
             mb.moe_unpermute(b["dxp"], layer.perm["row_map"], cfg.T, cfg.k, out=b["dx"])
             mb.moe_gather_slots(b["dprobs_perm"], layer.perm["row_map"], out=b["dprob"].view(-1))
+            mb.moe_route_bwd(None, layer.idx, layer.prob, b["dprob"], True, dlogits=b["dlogits"])
 
     for _ in range(warmup):
         step()
@@ -354,7 +367,7 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
         return statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
 
     mlp_ms = mean_ms(2, 3) + (mean_ms(5, 6) if training else 0.0)
-    perm_ms, unperm_ms = mean_ms(1, 2), mean_ms(3, 4)
+    perm_ms, unperm_ms = mean_ms(1, 2), (mean_ms(3, 4) if not fused_combine else 0.0)
     quant_ms = mean_ms(0, 1) if training and prec == "mxfp8" else 0.0
 
     flops = cfg.gemm_flops()
@@ -392,9 +405,10 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True):
                      "traffic": measured_traffic(cfg.name), "avg_launch_ms": round(mlp_ms, 4)},
         "bandwidth": {
             "permute": {"GB/s": round(perm_bytes / (perm_ms * 1e-3) / 1e9, 1), "ms": round(perm_ms, 4),
-                        "bytes": perm_bytes, "note": "moe_route + moe_permute call (index kernels included)"},
-            "unpermute": {"GB/s": round(unperm_bytes / (unperm_ms * 1e-3) / 1e9, 1), "ms": round(unperm_ms, 4),
-                          "bytes": unperm_bytes},
+                        "bytes": perm_bytes, "note": "moe_route_permute call (routing and index kernels included)"},
+            "unpermute": ({"GB/s": round(unperm_bytes / (unperm_ms * 1e-3) / 1e9, 1), "ms": round(unperm_ms, 4),
+                           "bytes": unperm_bytes} if not fused_combine else
+                          {"note": "fused into fc2's epilogue (timed inside grouped_mlp_fwd_combine)"}),
             "hbm_peak_gbs": hbm, "hbm_peak_source": f"{psrc} copy", "spec_gbs": SPEC_HBM_GBS},
         "clocks": clocks.summary(),
     }
@@ -561,6 +575,15 @@ def run_ours(args, world, rank, local):
             torch.cuda.empty_cache()
             res.pop("config", None)
             line["workloads"][name] = res
+            if name in FUSED_COMBINE_WORKLOADS:
+                # the same layer with the combine fused into fc2's epilogue
+                fres, d = run_workload(workloads.CONFIGS[name], args, world, rank, local, args.workload_steps,
+                                       args.warmup, with_e2e=False, fused_combine=True)
+                del d
+                gc.collect()
+                torch.cuda.empty_cache()
+                res["fused_combine"] = {k: fres[k] for k in ("value", "ms_per_step", "tokens_per_s", "clocks")}
+                res["fused_combine"]["roofline_frac"] = fres["roofline"]["frac"]
         line["gpu_launches"] = head["gpu_launches"]
     return line
 

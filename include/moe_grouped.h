@@ -68,6 +68,20 @@ MOE_API int moe_device_status(void* stream);
 MOE_API uint64_t moe_launch_count(void);
 
 /*
+ * moe_test_stall_gemm — test hook for the timeout path; the pages have no counterpart.
+ * Arms a one-shot stall: the grouped GEMM launches of this process (from grouped_mlp_fwd
+ * and grouped_mlp_bwd, in launch order) let `skip` launches through, and in the next one
+ * the TMA producers issue no copies and every wait gets a budget of timeout_ns
+ * (1e5 .. 1e10 ns) instead of 4 s. The first wait for data then runs out: the kernel sets
+ * MOE_ERR_TIMEOUT in the device error word, its other roles see the abort or run out in
+ * turn, every CTA frees its tensor memory and the launch returns; the context stays
+ * usable and later calls run normally. The stalled call's outputs are undefined.
+ * Launch order: grouped_mlp_fwd = fc1, fc2; grouped_mlp_bwd = fc2 dgrad, fc2 wgrad,
+ * fc1 dgrad, fc1 wgrad.
+ */
+MOE_API int moe_test_stall_gemm(int skip, uint64_t timeout_ns);
+
+/*
  * moe_route — top-k router softmax.
  * Pages: sitech.ge introduction and news.bpdata.com "dense vs MoE": every token is sent
  * to a few experts whose outputs are weighted by routing weights.
@@ -79,8 +93,46 @@ MOE_API uint64_t moe_launch_count(void);
  */
 MOE_API int moe_route(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* prob, void* stream);
 
-/* Bytes of device scratch moe_permute needs (per-block expert histograms). */
+/*
+ * moe_route_bwd — gradient of the router's probabilities with respect to its logits.
+ * Pages: sitech.ge introduction (each token's expert outputs are weighted by its routing
+ * weights, so the router learns through those weights).
+ * The forward (moe_route) is s = softmax(logits) over all E experts, q_j = s[idx_j], and
+ * p_j = q_j / sum_m q_m with renorm (else p_j = q_j). Given dprob = dL/dp, writes
+ * dlogits = dL/dlogits by the chain rule through those steps:
+ *   renorm != 0: dlogits[b] = sum over slots j with idx_j == b of p_j (dprob_j - D),
+ *                D = sum_m dprob_m p_m; experts that no slot chose get 0 (logits unused);
+ *   renorm == 0: dlogits[b] = s_b (ds_b - sum_c ds_c s_c), ds_b = sum of dprob_j over the
+ *                slots j with idx_j == b; s recomputed from logits in fp32.
+ *   logits [T, E] fp32 (input; may be NULL with renorm); idx [T, k] int32 and
+ *   prob [T, k] fp32 (the forward's outputs); dprob [T, k] fp32 (input);
+ *   dlogits [T, E] fp32 (output, every entry written).
+ * An index outside [0, E) sets MOE_ERR_DEVICE_CHECK in the device error word and that
+ * slot contributes nothing.
+ */
+MOE_API int moe_route_bwd(const float* logits, const int32_t* idx, const float* prob, const float* dprob, int T,
+                          int E, int k, int renorm, float* dlogits, void* stream);
+
+/* Bytes of device scratch moe_permute and moe_route_permute need (per-block expert
+ * histograms, and a counter for the fused call). */
 MOE_API size_t moe_permute_workspace_size(int T, int k, int E);
+
+/*
+ * moe_route_permute — moe_route followed by moe_permute, with the routing, the per-block
+ * expert histogram and its scan in one kernel launch (three launches instead of five).
+ * Same pages as the two calls. Same arguments and outputs, bit for bit, as
+ *   moe_route(logits, T, E, k, renorm, idx, prob) then
+ *   moe_permute(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm,
+ *               split_sizes, offsets, workspace, workspace_bytes);
+ * here idx and prob are outputs and both are required. The fused launch covers k that
+ * divides 1024 and E <= 256; other shapes run the two calls' kernels. workspace: at least
+ * moe_permute_workspace_size(T, k, E) bytes (its last 256 bytes hold a counter that the
+ * call zeroes itself). Calls that share a workspace must not overlap on the GPU.
+ */
+MOE_API int moe_route_permute(const float* logits, const uint16_t* x, int T, int H, int E, int k, int renorm,
+                              int precision, int32_t* idx, float* prob, void* xp, uint8_t* xp_scale,
+                              int32_t* row_map, float* probs_perm, int32_t* split_sizes, int32_t* offsets,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * moe_permute — stable permutation of the T*k routed slots into expert-contiguous rows.
@@ -129,7 +181,9 @@ MOE_API int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob
  * device current); make that first call before any stream capture. All calls share the
  * one table and it keeps the last call's contents (every entry a call reads is written
  * by the same call first), so calls whose GPU work overlaps — on two streams, or from
- * two host threads — race on it and must be serialised by the caller.
+ * two host threads — race on it and must be serialised by the caller. The looked-up
+ * address is kept for the life of the process: do not call this after cudaDeviceReset on
+ * that device (the table would be at a new address in the new context).
  */
 MOE_API int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
                                 int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
@@ -223,13 +277,46 @@ MOE_API int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32
                     const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
                     void* stream);
 
-/* Bytes of scratch grouped_mlp_bwd needs: dh [R, 2F] bf16 and dprob partial sums; for
- * MOE_MXFP8 also the recomputed a [R, F] bf16 and every quantised GEMM operand. */
+/* Bytes of scratch grouped_mlp_fwd_combine needs: grouped_mlp_fwd's workspace, then an
+ * fp32 [T, H] accumulator and the token of every row. */
+MOE_API size_t grouped_mlp_fwd_combine_workspace_size(int E, int R, int H, int F, int precision, int training,
+                                                      int T);
+
+/*
+ * grouped_mlp_fwd_combine — grouped_mlp_fwd with the unpermute/combine fused into fc2's
+ * epilogue (a variant: the routing weights are already applied inside the MLP, sitech.ge
+ * "Grouped experts instead of a Python loop", so the combine is a plain sum).
+ * out[t] = sum_j yp[row_map[t*k + j]] without writing yp: each fc2 output row is added,
+ * from its fp32 accumulator, into an fp32 [T, H] accumulator of its token with 16-byte
+ * vector atomics; one pass then rounds that to bf16 out [T, H]. Same arguments as
+ * grouped_mlp_fwd (no yp, precision without MOE_OUT_F32) plus row_map [R] (moe_permute's)
+ * and T, k with R = T*k. Every row is added in fp32 once, so out is the fp32 sum of the
+ * k accumulators rounded once: for k = 2 the result does not depend on the order of the
+ * adds; for k > 2 it may differ between runs in the last fp32 bits before rounding.
+ * workspace: grouped_mlp_fwd_combine_workspace_size(...) bytes.
+ */
+MOE_API int grouped_mlp_fwd_combine(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R,
+                                   int H, int F, const void* w1, const uint8_t* w1_scale, const void* w2,
+                                   const uint8_t* w2_scale, const float* probs_perm, int precision,
+                                   const int32_t* row_map, int T, int k, uint16_t* out, void* saved, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Bytes of scratch grouped_mlp_bwd needs: MOE_BF16: dh [R, 2F] bf16 and dprob partial
+ * sums; MOE_MXFP8: the dprob partial sums and every quantised GEMM operand. */
 MOE_API size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision);
 
-/* Byte offset, inside grouped_mlp_bwd's workspace, of part 0 (dh = [dg | du] [R, 2F]
- * bf16) or part 1 (MOE_MXFP8 only: the recomputed a [R, F] bf16); (size_t)-1 otherwise.
- * The parts hold the last call's values after it completes. */
+/* Byte offset, inside grouped_mlp_bwd's workspace, of one intermediate of the last call
+ * (valid after it completes; (size_t)-1 for a part the precision does not have):
+ *   MOE_BF16  part 0: dh = [dg | du] [R, 2F] bf16;
+ *   MOE_MXFP8 part 7: the recomputed a quantised along the expert's rows: codes [R, F],
+ *             then (256-byte aligned) its scale atoms in the layout of
+ *             mxfp8_quantize_grouped;
+ *             part 8: dh quantised along its 2F columns: codes [R, 2F], then scale atoms
+ *             grouped per 128-row expert tile (row group sum_{e'<e} ceil(n_e'/128) + m
+ *             for rows [off_e + 128 m, +128); atom j of a group = k-blocks 4j..4j+3,
+ *             row r at 32-bit word (r % 32) * 4 + r / 32; rows past the expert: zeros);
+ *             part 9: dh quantised along the expert's rows: codes [R, 2F], then atoms as
+ *             part 7. */
 MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part);
 
 /*
@@ -249,7 +336,9 @@ MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int 
  * axis (blocks of 32): dy and dh along columns for the data gradients, and dy, a
  * (recomputed from h), dh and xp along rows — in 32-row blocks restarting at every
  * expert's first row — for the weight gradients; the weights are re-quantised along
- * their other axis. Requires H % 128 == 0 for MOE_MXFP8.
+ * their other axis. dh and a are quantised (both ways) by the fc2-dgrad kernel that
+ * computes them, from fp32; they never exist at 16 bits. Requires H % 128 == 0 for
+ * MOE_MXFP8.
  */
 MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
                             const void* xp, const void* w1, const void* w2, const float* probs_perm, int precision,

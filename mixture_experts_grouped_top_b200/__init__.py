@@ -66,6 +66,13 @@ def moe_launch_count() -> int:
     return int(lib().moe_launch_count())
 
 
+def moe_test_stall_gemm(skip: int, timeout_ns: int) -> None:
+    """Test hook: after `skip` grouped GEMM launches, the next one issues no loads and its
+    waits run out after timeout_ns (it then reports MOE_ERR_TIMEOUT through
+    moe_device_status)."""
+    _check("moe_test_stall_gemm", lib().moe_test_stall_gemm(int(skip), int(timeout_ns)))
+
+
 def moe_status_string(status: int) -> str:
     return lib().moe_status_string(status).decode()
 
@@ -78,6 +85,59 @@ def moe_route(logits, k: int, renorm: bool = True, idx=None, prob=None, stream=N
     prob = torch.empty((T, k), dtype=torch.float32, device=logits.device) if prob is None else prob
     _check("moe_route", lib().moe_route(_p(logits), T, E, k, int(bool(renorm)), _p(idx), _p(prob), _stream(stream)))
     return idx, prob
+
+
+def moe_route_bwd(logits, idx, prob, dprob, renorm: bool = True, dlogits=None, stream=None):
+    """dL/dlogits [T, E] fp32 from dL/dprob [T, k] and the forward's idx / prob (logits
+    may be None with renorm)."""
+    _need(idx, torch.int32, "idx")
+    _need(prob, torch.float32, "prob")
+    _need(dprob, torch.float32, "dprob")
+    T, k = idx.shape
+    if logits is not None:
+        _need(logits, torch.float32, "logits")
+        E = logits.shape[1]
+    elif dlogits is not None:
+        E = dlogits.shape[1]
+    else:
+        raise ValueError("pass logits or dlogits (to give E)")
+    dlogits = torch.empty((T, E), dtype=torch.float32, device=idx.device) if dlogits is None else dlogits
+    _check("moe_route_bwd", lib().moe_route_bwd(_p(logits), _p(idx), _p(prob), _p(dprob), T, E, k,
+                                                int(bool(renorm)), _p(dlogits), _stream(stream)))
+    return dlogits
+
+
+def moe_route_permute(logits, x, k: int, renorm: bool = True, precision="bf16", out=None, workspace=None,
+                      stream=None):
+    """moe_route + moe_permute with the routing and index build fused. Returns the
+    moe_permute dict plus idx and prob."""
+    _need(logits, torch.float32, "logits")
+    _need(x, torch.bfloat16, "x")
+    prec = _PREC[precision]
+    T, E = logits.shape
+    H = x.shape[1]
+    R = T * k
+    dev = x.device
+    o = dict(out or {})
+    o.setdefault("idx", torch.empty((T, k), dtype=torch.int32, device=dev))
+    o.setdefault("prob", torch.empty((T, k), dtype=torch.float32, device=dev))
+    if "xp" not in o:
+        o["xp"] = torch.empty((R, H), dtype=torch.bfloat16 if prec == BF16 else torch.uint8, device=dev)
+    if prec == MXFP8 and "xp_scale" not in o:
+        o["xp_scale"] = torch.empty((R, H // 32), dtype=torch.uint8, device=dev)
+    o.setdefault("row_map", torch.empty(R, dtype=torch.int32, device=dev))
+    o.setdefault("probs_perm", torch.empty(R, dtype=torch.float32, device=dev))
+    o.setdefault("split_sizes", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = torch.empty(moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=dev)
+    rc = lib().moe_route_permute(_p(logits), _p(x), T, H, E, k, int(bool(renorm)), prec, _p(o["idx"]), _p(o["prob"]),
+                                 _p(o["xp"]), _p(o.get("xp_scale")), _p(o["row_map"]), _p(o["probs_perm"]),
+                                 _p(o["split_sizes"]), _p(o["offsets"]), _p(workspace), workspace.numel(),
+                                 _stream(stream))
+    _check("moe_route_permute", rc)
+    o.setdefault("xp_scale", None)
+    return o
 
 
 def moe_permute_workspace_size(T: int, k: int, E: int) -> int:
@@ -244,6 +304,31 @@ def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm=None, precision="bf16", 
                                workspace.numel(), _stream(stream))
     _check("grouped_mlp_fwd", rc)
     return yp, saved
+
+
+def grouped_mlp_fwd_combine_workspace_size(E, R, H, F, precision="bf16", training=False, T=0) -> int:
+    return int(lib().grouped_mlp_fwd_combine_workspace_size(E, R, H, F, _PREC[precision], int(bool(training)), T))
+
+
+def grouped_mlp_fwd_combine(xp, split_sizes, w1, w2, probs_perm, row_map, T, k, precision="bf16", xp_scale=None,
+                            w1_scale=None, w2_scale=None, out=None, saved=None, workspace=None, F=None, stream=None):
+    """grouped_mlp_fwd + moe_unpermute with the combine fused into fc2's epilogue: returns
+    out [T, H] bf16 (and writes `saved` when given)."""
+    prec = _PREC[precision]
+    R, H = xp.shape
+    E = split_sizes.numel()
+    if F is None:
+        F = w2.shape[1] if prec == BF16 else w2.shape[2]
+    dev = xp.device
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    ws_bytes = grouped_mlp_fwd_combine_workspace_size(E, R, H, F, precision, saved is not None, T)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    rc = lib().grouped_mlp_fwd_combine(_p(xp), _p(xp_scale), _p(split_sizes), E, R, H, F, _p(w1), _p(w1_scale),
+                                       _p(w2), _p(w2_scale), _p(probs_perm), prec, _p(row_map), T, k, _p(out),
+                                       _p(saved), _p(workspace), workspace.numel(), _stream(stream))
+    _check("grouped_mlp_fwd_combine", rc)
+    return out
 
 
 def grouped_mlp_bwd_workspace_size(E, R, H, F, precision="bf16") -> int:

@@ -16,7 +16,11 @@ SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_device_status": (_i, [_vp]),
     "moe_launch_count": (ctypes.c_uint64, []),
+    "moe_test_stall_gemm": (_i, [_i, ctypes.c_uint64]),
     "moe_route": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_route_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
+    "moe_route_permute": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                               _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -26,6 +30,9 @@ SIGNATURES = {
     "grouped_mlp_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "grouped_mlp_saved_size": (_sz, [_i, _i, _i, _i, _i]),
     "grouped_mlp_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "grouped_mlp_fwd_combine_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "grouped_mlp_fwd_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _vp, _vp,
+                                     _vp, _sz, _vp]),
     "grouped_mlp_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "grouped_mlp_bwd": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                              _vp]),

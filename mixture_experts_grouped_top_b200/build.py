@@ -49,7 +49,10 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
     if not force and up_to_date():
         return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"),
+    # MOE_NVCC_FLAGS: extra nvcc flags for experiments with the kernels' compile-time
+    # shapes (e.g. "-DMOE_MX2_STAGES=6 -DMOE_MX2_CHUNKS=1")
+    env_flags = os.environ.get("MOE_NVCC_FLAGS", "").split()
+    cmd = [_nvcc(), *NVCC_FLAGS, *env_flags, *(extra_flags or []), "-I", os.path.join(ROOT, "include"),
            "-o", LIB + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd), flush=True)

@@ -74,7 +74,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
   uint64_t* rready = bars + 3 * kStages;       // leader: the second CTA has zeroed its ragged stage
   uint64_t* tfull = bars + 4 * kStages;        // both CTAs
   uint64_t* tempty = bars + 4 * kStages + 2;   // leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * kStages + 4);
+  uint64_t* drained = bars + 4 * kStages + 4;  // second CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -98,6 +99,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 16);   // 8 epilogue warps in each CTA of the pair
     }
+    mbar_init(drained, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -154,8 +156,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      ArmedRing ring, pring;   // leader: full; second CTA: its own ragged-stage barriers pfull
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
+      for (int t = pair; t < total && ok && !p.stall_loads; t += npairs) {
         const TileInfo ti = walk.decode(t);
         const int nk = stages_of(ti);
         // this CTA's 128 columns of A and of B, as 64-column chunk indices
@@ -168,7 +171,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
           }
           const int k0 = ti.row0 + kb * BK;
           if (kb < nk - 1 || (ti.rows % BK) == 0) {
-            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+            if (leader) {
+              mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+              ring.arm(stage, phase);
+            }
             tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, k0, ca, 0);
             tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, k0, cb, 0);
           } else {
@@ -176,6 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
             // zero its rows past the expert before the MMAs read them
             uint64_t* bar = leader ? &full[stage] : &pfull[stage];
             mbar_arrive_expect_tx(bar, kStageBytes);
+            (leader ? ring : pring).arm(stage, phase);
             tma_load_4d(sA + stage * kABytes, &tmA, bar, 0, k0, ca, 0);
             tma_load_4d(sB + stage * kBBytes, &tmB, bar, 0, k0, cb, 0);
           }
@@ -185,12 +192,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // let this CTA's copies land before it can exit
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 100000000ull) {
-        }
-      }
+      // no copy may still be landing when either CTA leaves: the second CTA's own
+      // ragged-stage copies complete on its pfull barriers, the rest on the leader's
+      if (!leader && !ok) pring.drain(pfull, kStages, p.timeout_ns);
+      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kStages, ring);
     }
   } else if (warp == 1 && !leader) {
     // -------------------- second CTA: zero its rows of each ragged stage, tell the leader
@@ -226,7 +231,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
       const TileInfo ti = walk.decode(t);
       const int nk = stages_of(ti);
       const int acc = lt & 1;
-      if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+      if (!mbar_wait_bounded<true>(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = 0; kb < nk; ++kb) {
@@ -242,7 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
           const int valid = ti.rows - kb * BK;
           ksteps = (valid + 15) / 16;
           kp_zero_rows(sA + stage * kABytes, sB + stage * kBBytes, valid, ksteps * 16, lane);
-          if (!mbar_wait_bounded(&rready[stage], (rmask >> stage) & 1u, abort_flag, p.timeout_ns)) {
+          if (!mbar_wait_bounded<true>(&rready[stage], (rmask >> stage) & 1u, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }

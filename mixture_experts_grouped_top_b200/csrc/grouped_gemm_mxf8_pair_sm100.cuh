@@ -32,17 +32,26 @@ namespace mx2 {
 constexpr int BM = 256;                       // rows of a pair tile
 constexpr int BMC = 128;                      // rows per CTA
 constexpr int BN = 256;
-constexpr int BK = 256;                       // k per stage: two 128-byte chunks
-constexpr int kStages = 3;
+#ifndef MOE_MX2_CHUNKS
+#define MOE_MX2_CHUNKS 2
+#endif
+#ifndef MOE_MX2_STAGES
+#define MOE_MX2_STAGES 3
+#endif
+constexpr int kChunks = MOE_MX2_CHUNKS;       // 128-byte k-chunks per stage (1 or 2)
+constexpr int BK = 128 * kChunks;             // k per stage
+constexpr int kStages = MOE_MX2_STAGES;
 constexpr int kThreads = 384;
 constexpr int kChunkBytes = 128 * 128;        // one k-chunk of 128 rows, 16 KB
-constexpr int kABytes = BMC * BK;             // 32 KB
-constexpr int kBBytes = (BN / 2) * BK;        // 32 KB: this CTA's half of B
+constexpr int kABytes = BMC * BK;             // 16 KB per chunk
+constexpr int kBBytes = (BN / 2) * BK;        // 16 KB per chunk: this CTA's half of B
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kSfKb = 4;                      // k-blocks (of 128) per scale copy
 constexpr int kSfGroupBytes = kSfKb * 512;    // 2 KB: one row group's atoms for kSfKb k-blocks
 constexpr int kSfSlotBytes = 3 * kSfGroupBytes;   // A group, B lower group, B upper group
 constexpr int kSfSlots = 2;
+constexpr int kStPerSf = kSfKb / kChunks;     // stages per scale slot
+static_assert(kChunks == 1 || kChunks == 2, "one or two k-chunks per stage");
 
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
@@ -74,7 +83,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   uint64_t* tovl = bars + 2 * kStages + 4;    // used in the leader
   uint64_t* sfull = bars + 2 * kStages + 5;   // scale ring: used in the leader
   uint64_t* sempty = sfull + kSfSlots;        // scale ring: both CTAs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSfSlots);
+  uint64_t* drained = sempty + kSfSlots;      // used in the second CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -101,6 +111,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
       mbar_init(&sfull[s2], 1);
       mbar_init(&sempty[s2], 1);
     }
+    mbar_init(drained, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -157,16 +168,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   TileWalker<false, BM> walk{row_off, tile_off, E, 0, NT, p.K, nullptr};
   const int total = walk.total();
   const int kblocks = p.K / 128;                      // 128-wide k-blocks (K is a multiple of 128)
-  const int num_st = (kblocks + 1) / 2;               // stages; an odd last k-block reads zeros past K
+  const int num_st = (kblocks + kChunks - 1) / kChunks;   // stages; a partial last stage reads zeros past K
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0, sslot = 0;
       uint32_t phase = 0, sphase = 0;
+      ArmedRing ring, sring;
       bool ok = true;
       const int bgroups = mp.b_rows / 128;
-      for (int t = pair; t < total && ok; t += npairs) {
+      for (int t = pair; t < total && ok && !p.stall_loads; t += npairs) {
         const TileInfo ti = walk.decode(t);
         const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
         // this CTA's A rows and their scale group (past the expert: unused rows; a group
@@ -179,17 +191,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
         int gb1 = (EPI == MXEPI_SWIGLU_Q) ? ti.e * bgroups + (p.F + n0) / 128 : gb0 + 1;
         if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
         for (int st = 0; st < num_st; ++st) {
-          if ((st & 1) == 0) {
-            // scale atoms of k-blocks [2 st, 2 st + 4) (past K: zeros)
+          if (st % kStPerSf == 0) {
+            // scale atoms of k-blocks [kChunks st, kChunks st + 4) (past K: zeros)
             if (!mbar_wait_bounded(&sempty[sslot], sphase ^ 1, abort_flag, p.timeout_ns)) {
               ok = false;
               break;
             }
-            if (leader) mbar_arrive_expect_tx(&sfull[sslot], 2 * kSfSlotBytes);
+            if (leader) {
+              mbar_arrive_expect_tx(&sfull[sslot], 2 * kSfSlotBytes);
+              sring.arm(sslot, sphase);
+            }
             uint8_t* sd = sSf + sslot * kSfSlotBytes;
-            tma_load_3d_pair(sd, &tmSa, &sfull[sslot], 0, 2 * st, ga);
-            tma_load_3d_pair(sd + kSfGroupBytes, &tmSb, &sfull[sslot], 0, 2 * st, gb0);
-            tma_load_3d_pair(sd + 2 * kSfGroupBytes, &tmSb, &sfull[sslot], 0, 2 * st, gb1);
+            tma_load_3d_pair(sd, &tmSa, &sfull[sslot], 0, kChunks * st, ga);
+            tma_load_3d_pair(sd + kSfGroupBytes, &tmSb, &sfull[sslot], 0, kChunks * st, gb0);
+            tma_load_3d_pair(sd + 2 * kSfGroupBytes, &tmSb, &sfull[sslot], 0, kChunks * st, gb1);
             if (++sslot == kSfSlots) {
               sslot = 0;
               sphase ^= 1;
@@ -199,9 +214,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
-          tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, 2 * st, 0);
-          tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b_row, 2 * st, ti.e);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+            ring.arm(stage, phase);
+          }
+          tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, kChunks * st, 0);
+          tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b_row, kChunks * st, ti.e);
 
           if (++stage == kStages) {
             stage = 0;
@@ -209,12 +227,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // let this CTA's copies land before it can exit (their bytes count on the leader)
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 100000000ull) {
-        }
-      }
+      // no copy may still be landing when either CTA leaves
+      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kStages, ring, sfull, kSfSlots, &sring);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
@@ -227,12 +241,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
       const uint32_t sfb_t = tmem_base + mx::kSfbCol;
       for (int t = pair; t < total && ok; t += npairs, ++lt) {
         const int acc = lt & 1;
-        if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
-        if (lt > 0 && !mbar_wait_bounded(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
+        if (!mbar_wait_bounded<true>(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+        if (lt > 0 && !mbar_wait_bounded<true>(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc ? mx::kAcc1Col : 0u);
         for (int st = 0; st < num_st; ++st) {
-          if ((st & 1) == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
+          if (st % kStPerSf == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -246,8 +260,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             const uint32_t a_addr = smem_u32(sA + stage * kABytes);
             const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const int kb = 2 * st + c;
+            for (int c = 0; c < kChunks; ++c) {
+              const int kb = kChunks * st + c;
               if (kb < kblocks) {
                 // this k-block's atoms: entry kb % 4 of each 2 KB group of the slot
                 const uint32_t q = (uint32_t)(kb & (kSfKb - 1)) * 512;
@@ -266,14 +280,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             }
             mma_commit_pair(&empty[stage]);
             // the slot's last stage: release it once these MMAs have read their scales
-            if ((st & 1) == 1 || st == num_st - 1) mma_commit_pair(&sempty[sslot]);
+            if (st % kStPerSf == kStPerSf - 1 || st == num_st - 1) mma_commit_pair(&sempty[sslot]);
           }
           __syncwarp();
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
-          if ((st & 1) == 1 || st == num_st - 1) {
+          if (st % kStPerSf == kStPerSf - 1 || st == num_st - 1) {
             if (++sslot == kSfSlots) {
               sslot = 0;
               sphase ^= 1;
@@ -299,10 +313,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (acc ? mx::kAcc1Col : 0u) + ((uint32_t)(q * 32) << 16);
-      const uint32_t sc_word = mxf8_epilogue_tile<EPI>(mp, ti, t_row, acc, half, BMC * (int)rank + r_local, BM, [&] {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tovl_leader);
-      });
+      const uint32_t sc_word = mxf8_epilogue_tile<EPI>(
+          mp, ti, t_row, acc, half, BMC * (int)rank + r_local, BM,
+          [&] {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tovl_leader);
+          },
+          grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e]);
       if (EPI == MXEPI_SWIGLU_Q && BMC * (int)rank < ti.rows) {
         // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`; rows
         // past the expert in it store 0 (a CTA entirely past the expert writes nothing)

@@ -70,17 +70,69 @@ struct MxGemmParams {
   const uint8_t* b_atoms;
   int b_rows;                 // rows of each expert's B (2F for fc1, H for fc2)
   uint8_t* out_atoms;         // MXEPI_SWIGLU_Q: scales of `a` as atoms for the next GEMM (K = F)
+  // MXEPI_DSWIGLU: the MXFP8 operands of the backward's remaining GEMMs, quantised in the
+  // epilogue: dh = [dg | du] along its columns (codes [R, 2F], tile atoms, K = 2F), dh and
+  // the recomputed a along each expert's rows (codes [R, 2F] / [R, F], grouped atoms)
+  uint8_t* dh_rows;
+  uint8_t* dh_rows_atoms;
+  uint8_t* dh_cols;
+  uint8_t* dh_cols_atoms;
+  uint8_t* a_cols;
+  uint8_t* a_cols_atoms;
 };
+
+// E4M3 codes of 32 fp32 values (one lane's row) quantised along the 32 LANES of the warp:
+// for each column j the block maximum is the warp-wide max of |v[j]| (one redux: the bits
+// of a non-negative float order like the float), E8M0 code max(exp(amax) - 8, 0), element
+// scaled by 2^(127 - code) exactly and rounded to nearest even with saturation. Lanes
+// that hold no row pass zeros. Every lane of the warp must call this together. Returns
+// the codes in `w` (byte j = column j) and, in lane j, the scale code of column j.
+__device__ __forceinline__ uint32_t quant_cols_warp32(const float (&v)[32], uint32_t (&w)[8], int lane) {
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
+    const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + 1])));
+    const int c0 = max((int)(m0 >> 23) - 8, 0), c1 = max((int)(m1 >> 23) - 8, 0);
+    const float i0 = __uint_as_float((uint32_t)(254 - c0) << 23), i1 = __uint_as_float((uint32_t)(254 - c1) << 23);
+    const uint32_t pair =
+        (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v[j] * i0, v[j + 1] * i1), __NV_SATFINITE, __NV_E4M3);
+    if ((j & 2) == 0)
+      w[j >> 2] = pair;
+    else
+      w[j >> 2] |= pair << 16;
+    if (lane == j) mine = (uint32_t)c0;
+    if (lane == j + 1) mine = (uint32_t)c1;
+  }
+  return mine;
+}
+
+// E4M3 codes of 32 fp32 values of one row quantised as one block along the row; returns
+// the block's scale code.
+__device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
+  const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= inv;
+  pack_e4m3x16(v, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
+  pack_e4m3x16(v + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
+  return (uint32_t)code;
+}
 
 // Drains one 128-row x 256-column accumulator (this thread's row: lane quadrant of
 // `t_row`, row r_local of the output tile) and runs the epilogue EPI on it. The 32-column
 // strip that acc0 and acc1 share is drained first by its owning half, which then calls
 // `strip_done()`; the other half calls it before reading anything (warp-uniform calls, so
 // the callee may signal once per warp). Returns the SwiGLU_Q row's four scale bytes.
+// DSWIGLU also takes the expert's first 128-row group (grp0: groups of earlier experts)
+// and its row count n_e, which place its scale atoms.
 template <int EPI, class StripDone>
 __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, const TileInfo& ti, uint32_t t_row,
                                                        int acc, int half, int r_local, int tile_bm,
-                                                       StripDone&& strip_done) {
+                                                       StripDone&& strip_done, int grp0 = 0, int n_e = 0) {
   using mx::BN;
   const GemmParams& p = mp.g;
   const bool row_ok = r_local < ti.rows;
@@ -117,7 +169,11 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         tc_fence_before();
         strip_done();
       }
-      if (ok_row && n0 + c * 32 < p.N && p.out_f32) {
+      if (EPI == MXEPI_STORE && ok_row && n0 + c * 32 < p.N && p.row_token) {
+        float* d = p.out32 + (long long)p.row_token[row] * p.ldo + n0 + c * 32;
+        combine_add16(d, v0);
+        combine_add16(d + 16, v1);
+      } else if (ok_row && n0 + c * 32 < p.N && p.out_f32) {
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c * 32);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -139,32 +195,45 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     }
   } else if (EPI == MXEPI_DSWIGLU) {
     // acc = da for columns [n0, n0+256) of F. With h = [g | u] from the forward:
-    // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u; a = SiLU(g) u p is
-    // recomputed (bf16) for the fc2 weight gradient.
+    // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u, and a = SiLU(g) u p
+    // recomputed. All three are quantised here from fp32 into the operands of the GEMMs
+    // that follow (see MxGemmParams): dh along its columns (this row's 32-column blocks),
+    // dh and a along the expert's rows (32-row blocks = this warp's lanes: a pair tile
+    // starts at a multiple of 256 rows of its expert, so the blocks restart at every
+    // expert; lanes past the expert's end count as zeros).
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
     const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
-    __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
-    __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
     const int n0 = ti.n_blk * BN;
+    const int F = p.F, F2 = 2 * p.F;
+    const int lane = threadIdx.x & 31;
+    const int cta = r_local >> 7;                              // which 128-row group of the tile
+    const bool grp_ok = 128 * cta < ti.rows;                   // it holds rows of this expert
+    const bool half_ok = n0 + 128 * half < p.N;                // F % 128 == 0: halves are whole
+    const int KG = (n_e + 127) / 128;                          // the expert's 128-row groups
+    const int jb = 8 * ti.m_blk + (r_local >> 5);              // this warp's 32-row block of the expert
     const bool owner = acc ? (half == 0) : (half == 1);
     if (!owner) strip_done();
     float dp = 0.f;
+    uint32_t sg_word = 0, su_word = 0;   // this row's scale codes of its four dg / du blocks
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
       const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
       const int col = n0 + c * 32;
-      const bool cols_ok = row_ok && col < p.N;
+      const bool live = grp_ok && half_ok;                     // warp-uniform
       // the saved h of these 32 columns is requested first, so its global latency overlaps
       // the tensor-memory loads and their wait
       uint4 gva[4], uva[4];
-      if (cols_ok) {
+      if (live && row_ok) {
         const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + col);
-        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + col);
+        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + F + col);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           gva[i] = gp[i];
           uva[i] = up[i];
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) gva[i] = uva[i] = make_uint4(0, 0, 0, 0);
       }
       uint32_t v0[16], v1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
@@ -174,47 +243,76 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         tc_fence_before();
         strip_done();
       }
-      if (cols_ok) {
+      if (!live) continue;
+      float dg[32], du[32], av[32];
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva);
+      const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int cc = col + 16 * hh;
-          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva + 2 * hh);
-          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva + 2 * hh);
-          uint4 og[2], ou[2], oa[2];
-          uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
-          uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
-          uint32_t* oaw = reinterpret_cast<uint32_t*>(oa);
+      for (int i = 0; i < 16; ++i) {
+        const float2 gg2 = __bfloat1622float2(g2[i]);
+        const float2 uu2 = __bfloat1622float2(u2[i]);
+        const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 gg2 = __bfloat1622float2(g2[i]);
-            const float2 uu2 = __bfloat1622float2(u2[i]);
-            const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
-            float dg[2], du[2], av[2];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const float da = __uint_as_float(hh ? v1[2 * i + j] : v0[2 * i + j]);
-              const float sg = 1.0f / (1.0f + expf(-gs[j]));
-              const float sl = gs[j] * sg;
-              dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
-              du[j] = da * pr * sl;
-              av[j] = sl * us[j] * pr;
-              dp = fmaf(da, sl * us[j], dp);
-            }
-            ogw[i] = pack_bf16x2(dg[0], dg[1]);
-            ouw[i] = pack_bf16x2(du[0], du[1]);
-            oaw[i] = pack_bf16x2(av[0], av[1]);
-          }
-          uint4* d0 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + cc);
-          uint4* d1 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + cc);
-          uint4* d2 = reinterpret_cast<uint4*>(a_out + row * p.ldo + cc);
-          d0[0] = og[0];
-          d0[1] = og[1];
-          d1[0] = ou[0];
-          d1[1] = ou[1];
-          d2[0] = oa[0];
-          d2[1] = oa[1];
+        for (int j = 0; j < 2; ++j) {
+          const int k = 2 * i + j;
+          const float da = row_ok ? __uint_as_float(k < 16 ? v0[k] : v1[k - 16]) : 0.f;
+          const float sg = 1.0f / (1.0f + expf(-gs[j]));
+          const float sl = gs[j] * sg;
+          dg[k] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+          du[k] = da * pr * sl;
+          av[k] = sl * us[j] * pr;   // zero for lanes without a row (h was zero-filled)
+          dp = fmaf(da, sl * us[j], dp);
         }
       }
+      // along the expert's rows (warp-wide blocks): dh for fc1 wgrad, a for fc2 wgrad
+      uint32_t w[8];
+      const size_t gcol_dh = (size_t)grp0 * (F2 / 128) + (size_t)KG * (col / 128);
+      const size_t gcol_du = (size_t)grp0 * (F2 / 128) + (size_t)KG * ((F + col) / 128);
+      const size_t gcol_a = (size_t)grp0 * (F / 128) + (size_t)KG * (col / 128);
+      uint32_t sc = quant_cols_warp32(dg, w, lane);
+      mp.dh_cols_atoms[mma_scale_offset(gcol_dh, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(mp.dh_cols + row * F2 + col);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      sc = quant_cols_warp32(du, w, lane);
+      mp.dh_cols_atoms[mma_scale_offset(gcol_du, (F + col + lane) % 128, jb, 1)] = (uint8_t)sc;
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(mp.dh_cols + row * F2 + F + col);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      sc = quant_cols_warp32(av, w, lane);
+      mp.a_cols_atoms[mma_scale_offset(gcol_a, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(mp.a_cols + row * F + col);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      // along this row's columns: dh for fc1 dgrad (K = 2F)
+      sg_word |= quant_row32(dg, w) << (8 * (c & 3));
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(mp.dh_rows + row * F2 + col);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      su_word |= quant_row32(du, w) << (8 * (c & 3));
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(mp.dh_rows + row * F2 + F + col);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+    if (grp_ok && half_ok) {
+      // this CTA's 128 rows are row group grp0 + 2 m_blk + cta of dh's tile atoms; rows
+      // past the expert store zero scales (their codes are never read)
+      const size_t g = (size_t)grp0 + 2 * ti.m_blk + cta;
+      const int kb_g = (n0 + 128 * half) / 32, kb_u = (F + n0 + 128 * half) / 32;
+      *reinterpret_cast<uint32_t*>(mp.dh_rows_atoms + mma_scale_offset(g, r_local & 127, kb_g, F2 / 128)) =
+          row_ok ? sg_word : 0u;
+      *reinterpret_cast<uint32_t*>(mp.dh_rows_atoms + mma_scale_offset(g, r_local & 127, kb_u, F2 / 128)) =
+          row_ok ? su_word : 0u;
     }
     if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
   } else {
@@ -399,7 +497,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       bool ok = true;
       const int KB4 = KGROUP ? 0 : p.K / 128;
       const int bgroups = mp.b_rows / 128;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = blockIdx.x; t < total && ok && !p.stall_loads; t += gridDim.x) {
         const TileInfo ti = walk.decode(t);
         const int num_kb = kblocks(ti);
         const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
@@ -466,9 +564,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
             st = kStages - 1;
             ph ^= 1;
           }
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[st], ph) && global_timer_ns() - t0 < 100000000ull) {
-          }
+          mbar_wait_drain(&full[st], ph, p.timeout_ns);
         }
         // and the scale copies still in flight
         int ss = sslot, sp = sphase;
@@ -477,9 +573,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
             ss = kSfSlots - 1;
             sp ^= 1;
           }
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&sfull[ss], sp) && global_timer_ns() - t0 < 100000000ull) {
-          }
+          mbar_wait_drain(&sfull[ss], sp, p.timeout_ns);
         }
       }
     }

@@ -57,7 +57,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
   uint64_t* empty = bars + kStages;           // both CTAs
   uint64_t* tfull = bars + 2 * kStages;       // both CTAs
   uint64_t* tempty = bars + 2 * kStages + 2;  // used in the leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  uint64_t* drained = bars + 2 * kStages + 4; // used in the second CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -78,6 +79,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 16);   // 8 epilogue warps in each CTA of the pair
     }
+    mbar_init(drained, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -132,9 +134,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int issued = 0;
+      ArmedRing ring;
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
+      for (int t = pair; t < total && ok && !p.stall_loads; t += npairs) {
         const TileInfo ti = walk.decode(t);
         const int a_row = ti.row0 + BMC * (int)rank;
         // this CTA's half of B: columns (MN-major) or rows (K-major) [b0, b0 + 128)
@@ -145,26 +147,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+            ring.arm(stage, phase);
+          }
           tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, 2 * kb, 0);
           if (B_MN)
             tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, kb * BK, b0 / 64, ti.e);
           else
             tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b0, 2 * kb, ti.e);
-          ++issued;
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      if (!ok) {
-        // let this CTA's copies land before it can exit (their bytes count on the leader)
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 100000000ull) {
-        }
-        (void)issued;
-      }
+      // no copy may still be landing when either CTA leaves
+      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kStages, ring);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
@@ -177,7 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       for (int t = pair; t < total && ok; t += npairs, ++lt) {
         const TileInfo ti = walk.decode(t);
         const int acc = lt & 1;
-        if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
+        if (!mbar_wait_bounded<true>(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < num_kb; ++kb) {

@@ -61,8 +61,24 @@ struct GemmParams {
   float* dprob_part;           // DSwiGLU: [2 * ceil(N/256)][R] partial sums (one per N tile half)
   int F;                       // SwiGLU / DSwiGLU: width of the gate half
   int out_f32;                 // EPI_STORE: write fp32 instead of bf16
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;         // budget of every wait
+  int stall_loads;             // test hook: the producers issue no copies, so the first wait runs out
+  // EPI_STORE with the combine fused: row r is added (fp32 vector atomics) into
+  // out32[row_token[r]] instead of being stored (out32 [T, ldo] fp32, zeroed beforehand)
+  const int32_t* row_token;
+  float* out32;
 };
+
+// Adds 16 fp32 accumulator values (raw bits) to out32[0..16) with four 16-byte vector
+// atomics (sm_90+); the adds into one token's row commute for two terms, so a top-2
+// combine is exact and reproducible.
+__device__ __forceinline__ void combine_add16(float* out32, const uint32_t* v) {
+  float4* d = reinterpret_cast<float4*>(out32);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    atomicAdd(d + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
+}
 
 // Tile decoding shared by the three roles; every role walks the same tile sequence.
 struct TileInfo {
@@ -75,6 +91,10 @@ struct TileInfo {
 
 template <bool KGROUP, int TBM = gg::BM>
 struct TileWalker {
+#ifndef MOE_GROUP_M
+#define MOE_GROUP_M 8
+#endif
+  static constexpr int kGroupM = MOE_GROUP_M;   // M-grouped: m-blocks per band of the tile order
   const int32_t* row_off;   // smem [E+1]
   const int32_t* tile_off;  // smem [E+1]
   int E, MT, NT, K;
@@ -101,8 +121,15 @@ struct TileWalker {
       const int n_e = row_off[ti.e + 1] - row_off[ti.e];
       const int mt = (n_e + TBM - 1) / TBM;
       const int local = t - tile_off[ti.e];
-      ti.m_blk = local % mt;
-      ti.n_blk = local / mt;
+      // grouped order: bands of kGroupM m-blocks; inside a band every n-block in turn,
+      // the band's m-blocks fastest. The tiles in flight at once (one per CTA or pair)
+      // then share a few A row blocks and a few B column blocks, which stay in L2, where
+      // an m-fastest walk over a large expert streams all of its A rows once per n-block.
+      const int band = local / (kGroupM * NT);
+      const int gm = min(kGroupM, mt - band * kGroupM);
+      const int r = local - band * kGroupM * NT;
+      ti.m_blk = band * kGroupM + r % gm;
+      ti.n_blk = r / gm;
       ti.row0 = row_off[ti.e] + ti.m_blk * TBM;
       ti.rows = min(TBM, n_e - ti.m_blk * TBM);
       ti.num_kb = K / gg::BK;
@@ -110,6 +137,25 @@ struct TileWalker {
     return ti;
   }
 };
+
+// Producer exit of a CTA-pair kernel. Both CTAs' 2-SM copies complete on the leader's
+// barriers, so the leader waits (bounded) until the last phase it armed on every ring
+// slot has completed — every copy of both CTAs for those stages has landed — and then
+// arrives on the second CTA's `drained` barrier. A second CTA whose producer gave up
+// waits (bounded) for that arrival before it may leave; on a run without errors the
+// leader's waits end as soon as the last stages land.
+__device__ __forceinline__ void pair_producer_drain(bool leader, bool ok, uint64_t* drained, uint64_t budget_ns,
+                                                    uint64_t* full, int nfull, const ArmedRing& ring,
+                                                    uint64_t* full2 = nullptr, int nfull2 = 0,
+                                                    const ArmedRing* ring2 = nullptr) {
+  if (leader) {
+    ring.drain(full, nfull, budget_ns);
+    if (ring2) ring2->drain(full2, nfull2, budget_ns);
+    mbar_arrive_cluster(map_to_rank(smem_u32(drained), 1));
+  } else if (!ok) {
+    mbar_wait_drain<true>(drained, 0, budget_ns);
+  }
+}
 
 // Rank experts by decreasing row count (ties: lower index first) into order[0..E),
 // using every thread of the block; row_off must be complete. Static round-robin over
@@ -157,7 +203,9 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
       for (int j = 0; j < 4; ++j) {
         const int c = c0 + 16 * j;
         if (!row_ok || n0 + c >= p.N) continue;
-        if (EPI == EPI_STORE && p.out_f32) {
+        if (EPI == EPI_STORE && p.row_token) {
+          combine_add16(p.out32 + (long long)p.row_token[ti.row0 + tile_row] * p.ldo + n0 + c, v[j]);
+        } else if (EPI == EPI_STORE && p.out_f32) {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.out) + orow + n0 + c);
 #pragma unroll
           for (int i = 0; i < 4; ++i)

@@ -273,12 +273,23 @@ int quant_cols_grouped_launch(const void* in, int R, int C, const int32_t* split
 int scales_to_atoms_launch(const uint8_t* plain, const int32_t* split_sizes, int E, int R, int K, uint8_t* atoms,
                            cudaStream_t st);
 
+// One-shot stall armed by moe_test_stall_gemm: the wait budget of the stalled launch (0 =
+// none armed) and how many grouped GEMM launches to let through before it.
+std::atomic<uint64_t> g_stall_ns{0};
+std::atomic<int> g_stall_skip{0};
+
 GemmParams base_params(const int32_t* split_sizes, int E) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.E = E;
   p.split_sizes = split_sizes;
   p.timeout_ns = gg::kTimeoutNs;
+  const uint64_t stall = g_stall_ns.load();
+  if (stall && g_stall_skip.fetch_sub(1) == 0) {
+    g_stall_ns.store(0);
+    p.timeout_ns = stall;
+    p.stall_loads = 1;
+  }
   return p;
 }
 
@@ -299,6 +310,13 @@ const char* moe_status_string(int s) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_test_stall_gemm(int skip, uint64_t timeout_ns) {
+  if (skip < 0 || timeout_ns < 100000ull || timeout_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  g_stall_skip.store(skip);
+  g_stall_ns.store(timeout_ns);
+  return MOE_OK;
+}
 
 int moe_device_status(void* stream) {
   cudaStream_t st = as_stream(stream);
@@ -337,11 +355,43 @@ int moe_route(const float* logits, int T, int E, int k, int renorm, int32_t* idx
   return launch_status();
 }
 
-size_t moe_permute_workspace_size(int T, int k, int E) {
-  if (T < 0 || k < 1 || E < 1) return 0;
-  const size_t R = (size_t)T * k;
+int moe_route_bwd(const float* logits, const int32_t* idx, const float* prob, const float* dprob, int T, int E,
+                  int k, int renorm, float* dlogits, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!idx || !prob || !dprob || !dlogits || (!renorm && !logits)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int threads = 256, wpb = threads / 32;
+  const int grid = std::min((T + wpb - 1) / wpb, device_props().sm_count * 16);
+  const int vpl = (E + 31) / 32;
+#define MOE_ROUTE_BWD_CASE(V)                                                                              \
+  case V:                                                                                                  \
+    route_bwd_kernel<V><<<grid, threads, 0, st>>>(logits, idx, prob, dprob, T, E, k, renorm, dlogits); \
+    break;
+  switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : vpl <= 8 ? 8 : vpl <= 16 ? 16 : 32) {
+    MOE_ROUTE_BWD_CASE(1)
+    MOE_ROUTE_BWD_CASE(2)
+    MOE_ROUTE_BWD_CASE(4)
+    MOE_ROUTE_BWD_CASE(8)
+    MOE_ROUTE_BWD_CASE(16)
+    MOE_ROUTE_BWD_CASE(32)
+  }
+#undef MOE_ROUTE_BWD_CASE
+  count_launch();
+  return launch_status();
+}
+
+namespace {
+// counts table of the index build, then (256-byte aligned) the fused path's counter
+size_t permute_counts_bytes(size_t R, int E) {
   const size_t nblk = (R + kPermuteChunk - 1) / kPermuteChunk;
   return align_up(std::max<size_t>(nblk, 1) * E * sizeof(int32_t), 256);
+}
+}  // namespace
+
+size_t moe_permute_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return permute_counts_bytes((size_t)T * k, E) + 256;
 }
 
 int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, int k, uint16_t* dst, void* stream) {
@@ -357,6 +407,12 @@ int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, 
   return launch_status();
 }
 
+namespace {
+int permute_rows_from_counts(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
+                             int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                             const int32_t* counts, cudaStream_t st);
+}  // namespace
+
 int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k, int precision,
                 void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm, int32_t* split_sizes,
                 int32_t* offsets, void* workspace, size_t workspace_bytes, void* stream) {
@@ -371,7 +427,7 @@ int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T,
   if (R > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if (T > 0 && (!x || !idx || !xp || !row_map || !workspace)) return MOE_ERR_INVALID_ARG;
   if (precision == MOE_MXFP8 && T > 0 && !xp_scale) return MOE_ERR_INVALID_ARG;
-  if (workspace_bytes < moe_permute_workspace_size(T, k, E)) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < permute_counts_bytes((size_t)R, E)) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 15) return MOE_ERR_INVALID_ARG;
   if (R == 0) {
     // no rows: every expert is empty
@@ -386,6 +442,19 @@ int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T,
   const int P = std::max(1, 1024 / E);
   permute_scan_kernel<<<1, 1024, (size_t)(P * E + E) * sizeof(int32_t), st>>>(counts, nblk, E, (int)R, split_sizes,
                                                                                 offsets);
+  count_launch(2);
+  return permute_rows_from_counts(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, counts,
+                                  st);
+}
+
+namespace {
+// Passes 3 and 4 of the permutation: stable ranks (row_map, probs_perm) from the scanned
+// counts, then the data movement (with the MXFP8 row quantisation).
+int permute_rows_from_counts(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
+                             int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                             const int32_t* counts, cudaStream_t st) {
+  const long long R = (long long)T * k;
+  const int nblk = (int)((R + kPermuteChunk - 1) / kPermuteChunk);
   static std::once_flag once;
   std::call_once(once, []() {
     cudaFuncSetAttribute(permute_rowmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * kMaxExperts * 4);
@@ -400,8 +469,61 @@ int moe_permute(const uint16_t* x, const int32_t* idx, const float* prob, int T,
     permute_rows_mxfp8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), T, H, k, row_map,
                                                     reinterpret_cast<uint8_t*>(xp), xp_scale);
   }
-  count_launch(4);
+  count_launch(2);
   return launch_status();
+}
+}  // namespace
+
+int moe_route_permute(const float* logits, const uint16_t* x, int T, int H, int E, int k, int renorm, int precision,
+                      int32_t* idx, float* prob, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                      int32_t* split_sizes, int32_t* offsets, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32 || H < 8) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_BF16 && (H % 8)) return MOE_ERR_UNSUPPORTED;
+  if (precision == MOE_MXFP8 && (H % 32)) return MOE_ERR_UNSUPPORTED;
+  if (!split_sizes || !offsets) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k;
+  if (R > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (!logits || !x || !idx || !prob || !xp || !row_map || !workspace)) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_MXFP8 && T > 0 && !xp_scale) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe_permute_workspace_size(T, k, E)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 15) return MOE_ERR_INVALID_ARG;
+  if (T == 0)
+    return moe_permute(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, split_sizes, offsets,
+                       workspace, workspace_bytes, stream);
+  const int vpl = (E + 31) / 32;
+  if ((kPermuteChunk % k) != 0 || vpl > 8) {
+    // outside the fused kernel's shapes: the two calls it stands for
+    const int rc = moe_route(logits, T, E, k, renorm, idx, prob, stream);
+    if (rc != MOE_OK) return rc;
+    return moe_permute(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, split_sizes, offsets,
+                       workspace, workspace_bytes, stream);
+  }
+  cudaStream_t st = as_stream(stream);
+  const int nblk = (int)((R + kPermuteChunk - 1) / kPermuteChunk);
+  int32_t* counts = reinterpret_cast<int32_t*>(workspace);
+  unsigned int* done =
+      reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(workspace) + permute_counts_bytes((size_t)R, E));
+  if (cudaMemsetAsync(done, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const int P = std::max(1, 1024 / E);
+  const size_t smem = (size_t)std::max(E, (P + 1) * E) * sizeof(int32_t);
+#define MOE_ROUTE_INDEX_CASE(V)                                                                             \
+  case V:                                                                                                   \
+    route_index_kernel<V><<<nblk, 1024, smem, st>>>(logits, T, E, k, renorm, idx, prob, counts, nblk, split_sizes, \
+                                                    offsets, done);                                         \
+    break;
+  switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : 8) {
+    MOE_ROUTE_INDEX_CASE(1)
+    MOE_ROUTE_INDEX_CASE(2)
+    MOE_ROUTE_INDEX_CASE(4)
+    MOE_ROUTE_INDEX_CASE(8)
+  }
+#undef MOE_ROUTE_INDEX_CASE
+  count_launch();
+  const int rc = launch_status();
+  if (rc != MOE_OK) return rc;
+  return permute_rows_from_counts(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, counts, st);
 }
 
 int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const float* prob, int T, int H, int k, uint16_t* out,
@@ -490,7 +612,8 @@ namespace {
 
 int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H,
                           int F, const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
-                          const float* probs_perm, void* yp, int out_f32, void* saved, void* ws, cudaStream_t st) {
+                          const float* probs_perm, void* yp, int out_f32, void* saved, void* ws, cudaStream_t st,
+                          const int32_t* row_token, float* out32) {
   if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
   if (!xp_scale || !w1_scale || !w2_scale) return MOE_ERR_INVALID_ARG;
   // workspace: xp scale atoms [, a codes, a scale atoms]; training keeps a in `saved`
@@ -506,9 +629,9 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   int rc;
   if ((rc = scales_to_atoms_launch(xp_scale, split_sizes, E, R, H, xp_atoms, st))) return rc;
   // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xp, 1, R, H, 1))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1, E, 2 * F, H, 1))) return rc;
-  MxGemmParams p1;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xp, 1, R, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1, E, 2 * F, H, 1, 128, mx2::kChunks))) return rc;
+  MxGemmParams p1{};
   p1.g = base_params(split_sizes, E);
   p1.g.M = R;
   p1.g.N = F;
@@ -528,9 +651,9 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   if ((rc = tmap_atoms(&tsb, w1_scale, (uint64_t)E * 2 * F / 128, H / 128))) return rc;
   if ((rc = launch_gemm_mx_pair<MXEPI_SWIGLU_Q>(ta, tb, tsa, tsb, p1, st))) return rc;
   // fc2: A = a codes [R, F], B = w2 codes [E, H, F]
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, 1, R, F, 1))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, E, H, F, 1))) return rc;
-  MxGemmParams p2;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, 1, R, F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, E, H, F, 1, 128, mx2::kChunks))) return rc;
+  MxGemmParams p2{};
   p2.g = base_params(split_sizes, E);
   p2.g.M = R;
   p2.g.N = H;
@@ -544,30 +667,29 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p2.out_atoms = nullptr;
   if ((rc = tmap_atoms(&tsa, a_atoms, (uint64_t)R / 128 + E, F / 128))) return rc;
   if ((rc = tmap_atoms(&tsb, w2_scale, (uint64_t)E * H / 128, F / 128))) return rc;
+  p2.g.row_token = row_token;
+  p2.g.out32 = out32;
   return launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p2, st);
 }
 
-}  // namespace
-
-extern "C" {
-
-int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
-                    const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
-                    const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
-                    void* stream) {
+// The forward; with row_token, fc2's rows are added into out32[row_token[r]] (fused
+// combine) instead of being stored to yp.
+int grouped_mlp_fwd_impl(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H,
+                         int F, const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                         const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
+                         cudaStream_t st, const int32_t* row_token, float* out32) {
   const int out_f32 = (precision & MOE_OUT_F32) ? 1 : 0;
   precision &= ~MOE_OUT_F32;
   if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
   if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
   if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
   if (R == 0) return MOE_OK;
-  if (!xp || !split_sizes || !w1 || !w2 || !yp || !ws) return MOE_ERR_INVALID_ARG;
+  if (!xp || !split_sizes || !w1 || !w2 || (!yp && !row_token) || !ws) return MOE_ERR_INVALID_ARG;
   const int training = saved != nullptr;
   if (ws_bytes < grouped_mlp_workspace_size(E, R, H, F, precision, training)) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = as_stream(stream);
   if (precision == MOE_MXFP8)
     return grouped_mlp_fwd_mxfp8(xp, xp_scale, split_sizes, E, R, H, F, w1, w1_scale, w2, w2_scale, probs_perm, yp,
-                                 out_f32, saved, ws, st);
+                                 out_f32, saved, ws, st, row_token, out32);
 
   uint16_t* h_buf = nullptr;
   uint16_t* a_buf = reinterpret_cast<uint16_t*>(ws);
@@ -601,7 +723,58 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
   p2.out = yp;
   p2.ldo = H;
   p2.out_f32 = out_f32;
+  p2.row_token = row_token;
+  p2.out32 = out32;
   return launch_gemm_pair<true, EPI_STORE>(ta, tb, p2, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
+                    const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                    const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
+                    void* stream) {
+  return grouped_mlp_fwd_impl(xp, xp_scale, split_sizes, E, R, H, F, w1, w1_scale, w2, w2_scale, probs_perm,
+                              precision, yp, saved, ws, ws_bytes, as_stream(stream), nullptr, nullptr);
+}
+
+size_t grouped_mlp_fwd_combine_workspace_size(int E, int R, int H, int F, int precision, int training, int T) {
+  if (R < 0 || F < 0 || T < 0) return 0;
+  return grouped_mlp_workspace_size(E, R, H, F, precision, training) + align_up((size_t)T * H * 4, 256) +
+         align_up((size_t)R * 4, 256);
+}
+
+int grouped_mlp_fwd_combine(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H,
+                            int F, const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
+                            const float* probs_perm, int precision, const int32_t* row_map, int T, int k,
+                            uint16_t* out, void* saved, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || k < 1 || k > 32 || (long long)T * k != R || (precision & MOE_OUT_F32)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!row_map || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (H % 8)) return MOE_ERR_INVALID_ARG;
+  const int training = saved != nullptr;
+  if (ws_bytes < grouped_mlp_fwd_combine_workspace_size(E, R, H, F, precision, training, T))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const size_t base = grouped_mlp_workspace_size(E, R, H, F, precision, training);
+  float* out32 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + base);
+  int32_t* row_token =
+      reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(out32) + align_up((size_t)T * H * 4, 256));
+  if (cudaMemsetAsync(out32, 0, (size_t)T * H * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  row_token_kernel<<<std::min((R + 255) / 256, device_props().sm_count * 8), 256, 0, st>>>(row_map, R, k, row_token);
+  count_launch();
+  int rc = launch_status();
+  if (rc) return rc;
+  rc = grouped_mlp_fwd_impl(xp, xp_scale, split_sizes, E, R, H, F, w1, w1_scale, w2, w2_scale, probs_perm, precision,
+                            nullptr, saved, ws, base, st, row_token, out32);
+  if (rc) return rc;
+  const long long n8 = (long long)T * H / 8;
+  f32_to_bf16_kernel<<<(int)std::min<long long>((n8 + 255) / 256, (long long)device_props().sm_count * 8), 256, 0,
+                       st>>>(reinterpret_cast<const float4*>(out32), n8, reinterpret_cast<uint4*>(out));
+  count_launch();
+  return launch_status();
 }
 
 }  // extern "C"
@@ -609,36 +782,34 @@ int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32_t* spli
 namespace {
 
 // Backward workspace parts (each 256-byte aligned, in this order):
-//   0 dh bf16 [R, 2F];  1 a bf16 [R, F] (MXFP8 only: recomputed for the fc2 weight gradient);
-//   2 dprob partial sums [ceil(F/256)][R] fp32;  MXFP8 only, quantised operands:
+//   0 dh bf16 [R, 2F] (BF16 only);  2 dprob partial sums [ceil(F/256)][R] fp32;
+//   MXFP8 only, quantised operands:
 //   3 w2 codes [E, F, H] + scale atoms;  4 w1 codes [E, H, 2F] + atoms;
 //   5 dy codes [R, H] + plain scales + atoms (along H);  6 dy codes + atoms (along rows);
-//   7 a codes [R, F] + atoms (rows);  8 dh codes [R, 2F] + plain scales + atoms (along 2F);
+//   7 a codes [R, F] + atoms (rows);  8 dh codes [R, 2F] + atoms (along 2F);
 //   9 dh codes + atoms (rows);  10 xp codes [R, H] + atoms (rows).
-size_t bwd_part_bytes(int part, int E, int R, int H, int F) {
+// (Part 1 is no longer used: the MXFP8 fc2-dgrad epilogue quantises a and dh itself.)
+size_t bwd_part_bytes(int part, int E, int R, int H, int F, int precision) {
   const size_t r = (size_t)R, e = (size_t)E, h = (size_t)H, f = (size_t)F;
+  const bool mx = precision == MOE_MXFP8;
   switch (part) {
-    case 0: return align_up(r * 2 * f * 2, 256);
-    case 1: return align_up(r * f * 2, 256);
+    case 0: return mx ? 0 : align_up(r * 2 * f * 2, 256);
     case 2: return align_up((size_t)(2 * ((F + gg::BN - 1) / gg::BN)) * r * 4, 256);
-    case 3: return align_up(e * f * h, 256) + align_up(e * f * h / 32, 256);
-    case 4: return align_up(e * h * 2 * f, 256) + align_up(e * h * 2 * f / 32, 256);
-    case 5: return align_up(r * h, 256) + align_up(r * h / 32, 256) + mma_atoms_bytes(E, R, H);
-    case 6: return align_up(r * h, 256) + mma_atoms_bytes(E, R, H);
-    case 7: return align_up(r * f, 256) + mma_atoms_bytes(E, R, F);
-    case 8: return align_up(r * 2 * f, 256) + align_up(r * 2 * f / 32, 256) + mma_atoms_bytes(E, R, 2 * F);
-    case 9: return align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F);
-    case 10: return align_up(r * h, 256) + mma_atoms_bytes(E, R, H);
+    case 3: return mx ? align_up(e * f * h, 256) + align_up(e * f * h / 32, 256) : 0;
+    case 4: return mx ? align_up(e * h * 2 * f, 256) + align_up(e * h * 2 * f / 32, 256) : 0;
+    case 5: return mx ? align_up(r * h, 256) + align_up(r * h / 32, 256) + mma_atoms_bytes(E, R, H) : 0;
+    case 6: return mx ? align_up(r * h, 256) + mma_atoms_bytes(E, R, H) : 0;
+    case 7: return mx ? align_up(r * f, 256) + mma_atoms_bytes(E, R, F) : 0;
+    case 8: return mx ? align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F) : 0;
+    case 9: return mx ? align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F) : 0;
+    case 10: return mx ? align_up(r * h, 256) + mma_atoms_bytes(E, R, H) : 0;
     default: return 0;
   }
 }
 
 size_t bwd_part_offset(int part, int E, int R, int H, int F, int precision) {
   size_t off = 0;
-  for (int i = 0; i < part; ++i) {
-    if (precision != MOE_MXFP8 && i == 1) continue;
-    off += bwd_part_bytes(i, E, R, H, F);
-  }
+  for (int i = 0; i < part; ++i) off += bwd_part_bytes(i, E, R, H, F, precision);
   return off;
 }
 
@@ -648,13 +819,13 @@ extern "C" {
 
 size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision) {
   if (R < 0 || F < 0 || E < 1) return 0;
-  return bwd_part_offset(precision == MOE_MXFP8 ? 11 : 3, E, R, H, F, precision) + 256;
+  return bwd_part_offset(11, E, R, H, F, precision) + 256;
 }
 
 size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part) {
-  if (R < 0 || F < 0 || E < 1 || part < 0 || part > 1) return (size_t)-1;
-  if (part == 1 && precision != MOE_MXFP8) return (size_t)-1;
-  return bwd_part_offset(part, E, R, H, F, precision);
+  if (R < 0 || F < 0 || E < 1) return (size_t)-1;
+  const bool ok = precision == MOE_MXFP8 ? (part >= 7 && part <= 9) : part == 0;
+  return ok ? bwd_part_offset(part, E, R, H, F, precision) : (size_t)-1;
 }
 
 }  // extern "C"
@@ -668,8 +839,6 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   auto part = [&](int i) { return base + bwd_part_offset(i, E, R, H, F, MOE_MXFP8); };
-  uint16_t* dh = reinterpret_cast<uint16_t*>(part(0));
-  uint16_t* a_bf = reinterpret_cast<uint16_t*>(part(1));
   float* dpart = reinterpret_cast<float*>(part(2));
   const size_t efh = (size_t)E * F * H;
   uint8_t* w2q = part(3);
@@ -684,8 +853,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   uint8_t* ac = part(7);
   uint8_t* ac_a = ac + align_up((size_t)R * F, 256);
   uint8_t* dhr = part(8);
-  uint8_t* dhr_s = dhr + align_up((size_t)R * 2 * F, 256);
-  uint8_t* dhr_a = dhr_s + align_up((size_t)R * 2 * F / 32, 256);
+  uint8_t* dhr_a = dhr + align_up((size_t)R * 2 * F, 256);
   uint8_t* dhc = part(9);
   uint8_t* dhc_a = dhc + align_up((size_t)R * 2 * F, 256);
   uint8_t* xc = part(10);
@@ -702,17 +870,13 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((rc = quant_cols_grouped_launch(dy_perm, R, H, split_sizes, E, dyc, dyc_a, st))) return rc;
   CUtensorMap ta, tb;
   // fc2 dgrad + SwiGLU backward: A = dy codes [R, H], B = w2 codes [E, F, H] (N = F)
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyr, 1, R, H, 1))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2q, E, F, H, 1))) return rc;
-  MxGemmParams p;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyr, 1, R, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2q, E, F, H, 1, 128, mx2::kChunks))) return rc;
+  MxGemmParams p{};
   p.g = base_params(split_sizes, E);
   p.g.M = R;
   p.g.N = F;
   p.g.K = H;
-  p.g.out = a_bf;
-  p.g.ldo = F;
-  p.g.out2 = dh;
-  p.g.ldo2 = 2 * F;
   p.g.aux = h_saved;
   p.g.ld_aux = 2 * F;
   p.g.probs = probs_perm;
@@ -722,6 +886,13 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.b_atoms = w2a;
   p.b_rows = F;
   p.out_atoms = nullptr;
+  // the epilogue quantises dh and the recomputed a for the three GEMMs that follow
+  p.dh_rows = dhr;
+  p.dh_rows_atoms = dhr_a;
+  p.dh_cols = dhc;
+  p.dh_cols_atoms = dhc_a;
+  p.a_cols = ac;
+  p.a_cols_atoms = ac_a;
   CUtensorMap tsa, tsb;
   if ((rc = tmap_atoms(&tsa, dyr_a, (uint64_t)R / 128 + E, H / 128))) return rc;
   if ((rc = tmap_atoms(&tsb, w2a, (uint64_t)E * F / 128, H / 128))) return rc;
@@ -732,11 +903,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
     count_launch();
     if ((rc = launch_status())) return rc;
   }
-  // operands of the remaining GEMMs
-  if ((rc = quant_cols_grouped_launch(a_bf, R, F, split_sizes, E, ac, ac_a, st))) return rc;
-  if ((rc = quant_rows_launch(dh, R, 2 * F, 0, dhr, dhr_s, st))) return rc;
-  if ((rc = scales_to_atoms_launch(dhr_s, split_sizes, E, R, 2 * F, dhr_a, st))) return rc;
-  if ((rc = quant_cols_grouped_launch(dh, R, 2 * F, split_sizes, E, dhc, dhc_a, st))) return rc;
+  // xp along its rows for the fc1 weight gradient
   if ((rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc, xc_a, st))) return rc;
   // fc2 wgrad: dw2[e] = a_e^T dy_e (MN-major codes, contraction over the expert's rows)
   if ((rc = tmap_u8_3d(&ta, ac, 1, R, F, mx::BM))) return rc;
@@ -752,8 +919,8 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.b_rows = H;
   if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh codes [R, 2F], B = w1 codes [E, H, 2F] (N = H)
-  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhr, 1, R, 2 * F, 1))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1))) return rc;
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhr, 1, R, 2 * F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1, 128, mx2::kChunks))) return rc;
   p.g = base_params(split_sizes, E);
   p.g.M = R;
   p.g.N = H;
@@ -898,7 +1065,7 @@ extern "C" int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const 
                                    int k, int precision, void* xp, uint8_t* xp_scale, int32_t* row_map,
                                    float* probs_perm, int32_t* split_sizes, int32_t* offsets, void* stream) {
   if (T < 0 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_permute_workspace_size(T, k, E);
+  const size_t need = permute_counts_bytes((size_t)T * k, E);
   if (need > sizeof(int32_t) * (size_t)MOE_PERMUTE_NOALLOC_MAX_COUNTS) {
     fprintf(stderr,
             "moe_permute_noalloc: T*k=%lld with E=%d needs %zu bytes of scratch; the static table holds %zu "

@@ -78,15 +78,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test with cluster-scope acquire semantics: for barriers that other CTAs of the
+// cluster arrive on (with release.cluster), so that their writes before the arrive are
+// visible to this thread after the wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Gives up after `budget_ns`
 // nanoseconds (or when *abort becomes non-zero), flags DEVERR_TIMEOUT and returns false.
+// CLUSTER: acquire at cluster scope (the barrier receives arrivals from other CTAs).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   uint64_t budget_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     if ((++spins & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > budget_ns) {
@@ -97,6 +115,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
   }
 }
+
+// On the way out of a kernel that gave up: wait (at most budget_ns, whatever the abort
+// flag says, flagging nothing more) until the phase with the given parity has completed,
+// i.e. until the copies counted on it have landed. Returns false if the budget ran out.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!(CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)))
+    if (global_timer_ns() - t0 > budget_ns) return false;
+  return true;
+}
+
+// Ring bookkeeping of a TMA producer for the exit drain: which slots it armed at least
+// once and the phase parity of each slot's last arming.
+struct ArmedRing {
+  uint32_t armed = 0, parity = 0;
+  __device__ __forceinline__ void arm(int slot, uint32_t phase) {
+    armed |= 1u << slot;
+    parity = (parity & ~(1u << slot)) | ((phase & 1u) << slot);
+  }
+  // wait (bounded) for the last armed phase of every slot of `bars`
+  __device__ __forceinline__ void drain(uint64_t* bars, int nslots, uint64_t budget_ns) const {
+    for (int s = 0; s < nslots; ++s)
+      if ((armed >> s) & 1u) mbar_wait_drain(&bars[s], (parity >> s) & 1u, budget_ns);
+  }
+};
 
 // --------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

@@ -18,69 +18,169 @@ constexpr int kPermuteThreads = 256;  // 8 warps, 128 consecutive slots per warp
 constexpr int kMaxExperts = 1024;
 
 // ------------------------------------------------------------------------ routing
-// One warp per token. Softmax over all E logits in fp32, then the k largest logits
-// (ties -> lower expert index) in descending order; with renorm the k probabilities
-// are divided by their sum.
+// One warp routes one token: softmax over all E logits in fp32, then the k largest
+// logits (ties -> lower expert index) in descending order; with renorm the k
+// probabilities are divided by their sum. Lane j (< k) returns choice j.
 template <int VPL>  // logits held per lane: ceil(E / 32)
+__device__ __forceinline__ void route_one_token(const float* __restrict__ row, int E, int k, int renorm, int lane,
+                                                int& e_out, float& p_out) {
+  float v[VPL];
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? row[e] : -INFINITY;
+    m = fmaxf(m, v[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if (lane + 32 * i < E) s += expf(v[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+
+  uint32_t taken = 0;
+  float psum = 0.f;
+  float pk = 0.f;   // lane j (< k) keeps probability j
+  int ek = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    const float p = expf(bv - m) / s;
+    psum += p;
+    if (lane == j) {
+      pk = p;
+      ek = be;
+    }
+  }
+  e_out = ek;
+  p_out = renorm ? pk / psum : pk;
+}
+
+template <int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int renorm, int32_t* __restrict__ idx,
                                                          float* __restrict__ prob) {
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
-    const float* row = logits + (size_t)t * E;
-    float v[VPL];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = (e < E) ? row[e] : -INFINITY;
-      m = fmaxf(m, v[i]);
+    int e;
+    float p;
+    route_one_token<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, p);
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = e;
+      prob[(size_t)t * k + lane] = p;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i)
-      if (lane + 32 * i < E) s += expf(v[i] - m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  }
+}
 
-    uint32_t taken = 0;
-    float psum = 0.f;
-    float pk = 0.f;   // lane j (< k) keeps probability j
-    int ek = 0;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+// Router backward, one warp per token: dlogits [T, E] from dL/dprob [T, k] and the
+// forward's idx / prob. The forward is s = softmax(l), q_j = s[idx_j], p_j = q_j / Z with
+// Z = sum_j q_j (renorm) or p_j = q_j. By the chain rule dl_b = s_b (ds_b - <ds, s>) with
+// ds_b the sum of dq_j over the slots that chose b.
+//  * renorm: dq_j = (dprob_j - D) / Z with D = sum_m dprob_m p_m; then <ds, s> = 0 and
+//    s_b ds_b = p_j (dprob_j - D), so dl_b = sum over slots j choosing b of p_j (dprob_j - D)
+//    and 0 for experts nobody chose; the logits are not needed.
+//  * no renorm: dq_j = dprob_j and s is recomputed from the logits in fp32.
+template <int VPL>
+__global__ void __launch_bounds__(256) route_bwd_kernel(const float* __restrict__ logits,
+                                                        const int32_t* __restrict__ idx,
+                                                        const float* __restrict__ prob,
+                                                        const float* __restrict__ dprob, int T, int E, int k,
+                                                        int renorm, float* __restrict__ dlogits) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int ej = -1;
+    float pj = 0.f, dj = 0.f;
+    if (lane < k) {
+      ej = idx[(size_t)t * k + lane];
+      pj = prob[(size_t)t * k + lane];
+      dj = dprob[(size_t)t * k + lane];
+      if (ej < 0 || ej >= E) {
+        flag_error(DEVERR_BAD_INDEX);
+        ej = -1;
+      }
+    }
+    float acc[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+    float* out = dlogits + (size_t)t * E;
+    if (renorm) {
+      float D = dj * pj;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
+      const float gj = pj * (dj - D);
+      for (int j = 0; j < k; ++j) {
+        const int eb = __shfl_sync(0xffffffffu, ej, j);
+        const float gb = __shfl_sync(0xffffffffu, gj, j);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (lane + 32 * i == eb) acc[i] += gb;
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (lane + 32 * i < E) out[lane + 32 * i] = acc[i];
+    } else {
+      // ds_b: sum of dprob_j over the slots that chose b
+      for (int j = 0; j < k; ++j) {
+        const int eb = __shfl_sync(0xffffffffu, ej, j);
+        const float db = __shfl_sync(0xffffffffu, dj, j);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (lane + 32 * i == eb) acc[i] += db;
+      }
+      const float* row = logits + (size_t)t * E;
+      float v[VPL];
+      float m = -INFINITY;
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
-          bv = v[i];
-          be = e;
-        }
+        v[i] = (e < E) ? row[e] : -INFINITY;
+        m = fmaxf(m, v[i]);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        v[i] = (lane + 32 * i < E) ? expf(v[i] - m) : 0.f;
+        z += v[i];
       }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      const float p = expf(bv - m) / s;
-      psum += p;
-      if (lane == j) {
-        pk = p;
-        ek = be;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      const float inv = 1.0f / z;
+      float dot = 0.f;   // <ds, s>
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        v[i] *= inv;
+        dot = fmaf(acc[i], v[i], dot);
       }
-    }
-    if (lane < k) {
-      idx[(size_t)t * k + lane] = ek;
-      prob[(size_t)t * k + lane] = renorm ? pk / psum : pk;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (lane + 32 * i < E) out[lane + 32 * i] = v[i] * (acc[i] - dot);
     }
   }
 }
@@ -109,12 +209,11 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_hist_kernel(const int
 
 // Pass 2 (one block of 1024 threads, E <= 1024): split_sizes, offsets, and the first
 // row of every (block, expert) pair, written over the counts. Threads form a [P][E]
-// grid (P = 1024 / E) that splits the blocks into P contiguous ranges.
-__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ counts, int nblk, int E, int R,
-                                                            int32_t* __restrict__ split_sizes,
-                                                            int32_t* __restrict__ offsets) {
-  extern __shared__ int32_t sm[];
-  __shared__ int32_t wsum[32];
+// grid (P = 1024 / E) that splits the blocks into P contiguous ranges. `sm` holds
+// (P + 1) * E int32. The counts are read past L1 (they may come from other SMs).
+__device__ __forceinline__ void scan_block_counts(int32_t* __restrict__ counts, int nblk, int E, int R,
+                                                  int32_t* __restrict__ split_sizes, int32_t* __restrict__ offsets,
+                                                  int32_t* sm, int32_t* wsum) {
   const int P = max(1, (int)blockDim.x / E);
   int32_t* part = sm;          // [P][E] partial sums, then their exclusive prefix over p
   int32_t* off = sm + P * E;   // [E] first row of each expert
@@ -122,7 +221,7 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
   for (int tid = threadIdx.x; tid < E * P; tid += blockDim.x) {
     const int p = tid / E, e = tid % E;
     int acc = 0;
-    for (int b = p * per; b < min(nblk, (p + 1) * per); ++b) acc += counts[(size_t)b * E + e];
+    for (int b = p * per; b < min(nblk, (p + 1) * per); ++b) acc += __ldcg(counts + (size_t)b * E + e);
     part[p * E + e] = acc;
   }
   __syncthreads();
@@ -170,11 +269,61 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
     const int p = tid / E, ee = tid % E;
     int base = off[ee] + part[p * E + ee];
     for (int b = p * per; b < min(nblk, (p + 1) * per); ++b) {
-      const int c = counts[(size_t)b * E + ee];
+      const int c = __ldcg(counts + (size_t)b * E + ee);
       counts[(size_t)b * E + ee] = base;
       base += c;
     }
   }
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ counts, int nblk, int E, int R,
+                                                            int32_t* __restrict__ split_sizes,
+                                                            int32_t* __restrict__ offsets) {
+  extern __shared__ int32_t sm[];
+  __shared__ int32_t wsum[32];
+  scan_block_counts(counts, nblk, E, R, split_sizes, offsets, sm, wsum);
+}
+
+// Route + index build in one launch (1024 threads per block, k divides kPermuteChunk):
+// block b routes tokens [b * 1024/k, (b+1) * 1024/k) — exactly the slots of histogram
+// chunk b — and writes that chunk's expert histogram; the last block to finish (a
+// device-wide counter, zeroed before the launch and reset by that block) then runs the
+// scan of pass 2. Replaces the route, histogram and scan launches of the unfused path.
+template <int VPL>
+__global__ void __launch_bounds__(1024, 1) route_index_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                              int renorm, int32_t* __restrict__ idx,
+                                                              float* __restrict__ prob, int32_t* __restrict__ counts,
+                                                              int nblk, int32_t* __restrict__ split_sizes,
+                                                              int32_t* __restrict__ offsets,
+                                                              unsigned int* __restrict__ done) {
+  extern __shared__ int32_t sm[];       // hist [E], then the scan's (P + 1) * E
+  __shared__ int32_t wsum[32];
+  __shared__ int is_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tpb = kPermuteChunk / k;
+  const int t0 = blockIdx.x * tpb, t1 = min(T, t0 + tpb);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sm[e] = 0;
+  __syncthreads();
+  for (int t = t0 + warp; t < t1; t += (int)(blockDim.x >> 5)) {
+    int e;
+    float p;
+    route_one_token<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, p);
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = e;
+      prob[(size_t)t * k + lane] = p;
+      atomicAdd(&sm[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = sm[e];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == (unsigned)(nblk - 1));
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  scan_block_counts(counts, nblk, E, T * k, split_sizes, offsets, sm, wsum);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 // Pass 3: stable ranks inside the block. Warp w owns slots [w*128, w*128+128) of the
@@ -317,6 +466,27 @@ __global__ void __launch_bounds__(256) permute_rows_mxfp8_kernel(const uint4* __
 }
 
 // ------------------------------------------------------------- unpermute/combine
+// row_token[row_map[s]] = s / k: the token of every permuted row (for the fused combine).
+__global__ void __launch_bounds__(256) row_token_kernel(const int32_t* __restrict__ row_map, int R, int k,
+                                                        int32_t* __restrict__ row_token) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < R; s += gridDim.x * blockDim.x) {
+    const int r = row_map[s];
+    if (r >= 0 && r < R)
+      row_token[r] = s / k;
+    else
+      flag_error(DEVERR_BAD_INDEX);
+  }
+}
+
+// out[i] = bf16(in[i]) for n8 groups of 8 fp32 values (the fused combine's last step).
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ in, long long n8,
+                                                          uint4* __restrict__ out) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = in[2 * i], b = in[2 * i + 1];
+    out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
 // out[t] = sum_j w_tj * yp[row_map[t*k+j]] (w = 1 without prob), fp32 accumulation in
 // slot order, rounded once to bf16.
 __global__ void __launch_bounds__(256) unpermute_bf16_kernel(const uint4* __restrict__ yp,

@@ -1,7 +1,8 @@
 """One MoE expert-MLP layer on preallocated device buffers, sequencing the C-ABI calls.
 
-forward:  moe_route -> moe_permute -> grouped_mlp_fwd -> moe_unpermute
+forward:  moe_route_permute (route + permutation) -> grouped_mlp_fwd -> moe_unpermute
 backward: moe_permute_rows(grad_out) -> grouped_mlp_bwd -> moe_unpermute(dxp) -> moe_gather_slots
+          -> moe_route_bwd (dlogits)
 
 All arithmetic runs in libmoe_grouped.so; this module only owns buffers and call order.
 """
@@ -10,19 +11,21 @@ from __future__ import annotations
 import torch
 
 from . import (BF16, MXFP8, _PREC, grouped_mlp_bwd, grouped_mlp_bwd_workspace_size, grouped_mlp_fwd,
-               grouped_mlp_saved_size, grouped_mlp_workspace_size, moe_gather_slots, moe_permute,
-               moe_permute_rows, moe_permute_workspace_size, moe_route, moe_unpermute, mxfp8_quantize)
+               grouped_mlp_fwd_combine, grouped_mlp_fwd_combine_workspace_size, grouped_mlp_saved_size, grouped_mlp_workspace_size, moe_gather_slots, moe_permute_rows,
+               moe_permute_workspace_size, moe_route_bwd, moe_route_permute, moe_unpermute, mxfp8_quantize)
 
 
 class MoEExpertLayer:
     def __init__(self, T: int, H: int, F: int, E: int, k: int, precision="bf16", training: bool = False,
-                 renorm: bool = True, device="cuda"):
+                 renorm: bool = True, device="cuda", fused_combine: bool = False):
         self.T, self.H, self.F, self.E, self.k = T, H, F, E, k
         self.R = T * k
         self.prec = _PREC[precision]
         self.precision = "bf16" if self.prec == BF16 else "mxfp8"
         self.training = training
         self.renorm = renorm
+        # fused_combine: fc2's epilogue adds its rows into the token outputs (no yp)
+        self.fused_combine = fused_combine
         dev = torch.device(device)
         self.device = dev
         R = self.R
@@ -39,10 +42,11 @@ class MoEExpertLayer:
         if self.prec == MXFP8:
             self.perm["xp_scale"] = torch.empty((R, H // 32), dtype=u8, device=dev)
         self.perm_ws = torch.empty(max(moe_permute_workspace_size(T, k, E), 1), dtype=u8, device=dev)
-        self.yp = torch.empty((R, H), dtype=bf, device=dev)
+        self.yp = None if fused_combine else torch.empty((R, H), dtype=bf, device=dev)
         self.out = torch.empty((T, H), dtype=bf, device=dev)
-        self.mlp_ws = torch.empty(grouped_mlp_workspace_size(E, R, H, F, self.precision, training), dtype=u8,
-                                  device=dev)
+        ws_bytes = (grouped_mlp_fwd_combine_workspace_size(E, R, H, F, self.precision, training, T) if fused_combine
+                    else grouped_mlp_workspace_size(E, R, H, F, self.precision, training))
+        self.mlp_ws = torch.empty(ws_bytes, dtype=u8, device=dev)
         self.saved = (torch.empty(grouped_mlp_saved_size(E, R, H, F, self.precision), dtype=u8, device=dev)
                       if training else None)
         self.w1 = self.w2 = None
@@ -63,14 +67,22 @@ class MoEExpertLayer:
 
     # --------------------------------------------------------------- forward
     def forward(self, x: torch.Tensor, logits: torch.Tensor, stream=None) -> torch.Tensor:
-        moe_route(logits, self.k, self.renorm, idx=self.idx, prob=self.prob, stream=stream)
-        moe_permute(x, self.idx, self.prob, self.E, self.precision, out=self.perm, workspace=self.perm_ws,
-                    stream=stream)
-        grouped_mlp_fwd(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2, self.perm["probs_perm"],
-                        self.precision, xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
-                        w2_scale=self.w2_scale, yp=self.yp, saved=self.saved, workspace=self.mlp_ws, F=self.F,
-                        stream=stream)
-        moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
+        self.perm["idx"], self.perm["prob"] = self.idx, self.prob
+        moe_route_permute(logits, x, self.k, self.renorm, self.precision, out=self.perm, workspace=self.perm_ws,
+                          stream=stream)
+        self.logits = logits
+        if self.fused_combine:
+            grouped_mlp_fwd_combine(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2,
+                                    self.perm["probs_perm"], self.perm["row_map"], self.T, self.k, self.precision,
+                                    xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
+                                    w2_scale=self.w2_scale, out=self.out, saved=self.saved, workspace=self.mlp_ws,
+                                    F=self.F, stream=stream)
+        else:
+            grouped_mlp_fwd(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2, self.perm["probs_perm"],
+                            self.precision, xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
+                            w2_scale=self.w2_scale, yp=self.yp, saved=self.saved, workspace=self.mlp_ws, F=self.F,
+                            stream=stream)
+            moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
         if self.training and self.prec == MXFP8:
             self.permute_for_backward(x, stream=stream)
         return self.out
@@ -93,12 +105,14 @@ class MoEExpertLayer:
             "dprobs_perm": torch.empty(R, dtype=torch.float32, device=dev),
             "dx": torch.empty((T, H), dtype=bf, device=dev),
             "dprob": torch.empty((T, self.k), dtype=torch.float32, device=dev),
+            "dlogits": torch.empty((T, E), dtype=torch.float32, device=dev),
             "ws": torch.empty(grouped_mlp_bwd_workspace_size(E, R, H, F, self.precision), dtype=torch.uint8,
                               device=dev),
         }
 
-    def backward(self, grad_out: torch.Tensor, stream=None):
-        """Gradients of the last forward: returns (dx [T,H], dw1, dw2, dprob [T,k])."""
+    def backward(self, grad_out: torch.Tensor, stream=None, router: bool = True):
+        """Gradients of the last forward: returns (dx [T,H], dw1, dw2, dprob [T,k]); with
+        ``router`` the router's dlogits [T,E] are in ``self.dlogits`` too."""
         if not self.training:
             raise RuntimeError("layer was built without training=True")
         if self._bwd is None:
@@ -111,6 +125,10 @@ class MoEExpertLayer:
                         dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream)
         moe_unpermute(b["dxp"], self.perm["row_map"], self.T, self.k, out=b["dx"], stream=stream)
         moe_gather_slots(b["dprobs_perm"], self.perm["row_map"], out=b["dprob"].view(-1), stream=stream)
+        if router:
+            moe_route_bwd(None if self.renorm else self.logits, self.idx, self.prob, b["dprob"], self.renorm,
+                          dlogits=b["dlogits"], stream=stream)
+        self.dlogits = b["dlogits"] if router else None
         return b["dx"], b["dw1"], b["dw2"], b["dprob"]
 
 

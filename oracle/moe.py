@@ -352,15 +352,18 @@ def moe_forward_sampled(x, idx, prob, w1, w2, tokens, a_round="bf16") -> np.ndar
     return out
 
 
-def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=None, a=None):
+def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=None, a=None, dh_wgrad=None):
     """Backward of the MXFP8 layer: every GEMM on operands quantised along its own
     contraction axis, computed in float64.
 
     fc2 dgrad: dy along H times w2 along H (transposed);  fc2 wgrad: a and dy along rows
     (32-row blocks restarting at each expert);  fc1 dgrad: dh along 2F times w1 along 2F;
     fc1 wgrad: xp and dh along rows. h = [g | u] is the forward's saved pre-activation.
-    The path stores dh and the recomputed a in bf16 before quantising them; the oracle
-    does the same unless ``dh`` / ``a`` (e.g. the values a GPU produced) are given.
+    dh and the recomputed a are quantised from their exact values (the fused backward
+    quantises them in the kernel that computes them; they are never stored at a lower
+    precision first). ``dh`` / ``a`` replace those values (e.g. by the dequantised codes a
+    GPU produced, which quantise to themselves along their own axis); ``dh_wgrad``
+    replaces dh for the fc1 weight gradient only (default: ``dh``).
     Returns (dxp, dw1, dw2, dprobs_perm, dh_exact, a_exact).
     """
     dy = f64(dy_perm)
@@ -384,10 +387,11 @@ def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=No
     dh_exact = np.concatenate([da * p * u * silu_grad(g), da * p * silu(g)], axis=1)
     dprob = np.sum(da * silu(g) * u, axis=1)
     a_exact = silu(g) * u * p
-    dh_use = round_to_bf16(dh_exact) if dh is None else f64(dh)
-    a_use = round_to_bf16(a_exact) if a is None else f64(a)
+    dh_use = dh_exact if dh is None else f64(dh)
+    a_use = a_exact if a is None else f64(a)
+    dh_w = dh_use if dh_wgrad is None else f64(dh_wgrad)
     deq_rows = lambda v: mxfp8.dequantize_grouped_rows(*mxfp8.quantize_grouped_rows(v, split), split)
-    aq, dyc, xc, dhc = deq_rows(a_use), deq_rows(dy), deq_rows(xp), deq_rows(dh_use)
+    aq, dyc, xc, dhc = deq_rows(a_use), deq_rows(dy), deq_rows(xp), deq_rows(dh_w)
     dhq = mxfp8.dequantize(*mxfp8.quantize(dh_use, axis=0), axis=0)    # along 2F
     dxp = np.zeros_like(xp)
     dw1 = np.zeros_like(w1)
@@ -494,14 +498,16 @@ def fwd_rows_mxfp8(x_rows, prob_rows, expert_of_rows, w1, w2, a_codes=None, a_sc
     return yp, own_c, own_s
 
 
-def bwd_sampled_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh, a, rows, experts, cols):
+def bwd_sampled_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh, a, rows, experts, cols, dh_wgrad=None):
     """Sampled entries of :func:`grouped_mlp_bwd_mxfp8`, float64 on quantised operands.
 
     For the permuted ``rows``: dh_exact (from dy along H and w2 along H), dprobs, and dxp
     (from ``dh`` along 2F and w1 along 2F). For every expert in ``experts`` and the column
     samples ``cols = (f_cols, h_cols, hh_cols, j_cols)``: dw2[e][f_cols][:, h_cols] (``a``
-    and dy along the expert's rows) and dw1[e][hh_cols][:, j_cols] (xp and ``dh`` along
-    rows). ``h`` is the forward's [g | u]; ``dh`` and ``a`` are the stored bf16 values.
+    and dy along the expert's rows) and dw1[e][hh_cols][:, j_cols] (xp and ``dh_wgrad``,
+    default ``dh``, along rows). ``h`` is the forward's [g | u]; ``dh`` and ``a`` are the
+    values the GEMMs consume (e.g. dequantised GPU codes), indexed as ``dh[rows]`` and
+    ``a[rows_slice, cols]`` / ``dh_wgrad[rows_slice, cols]`` only.
     """
     split = np.asarray(split_sizes, dtype=np.int64)
     offs = np.concatenate([[0], np.cumsum(split)])
@@ -534,6 +540,7 @@ def bwd_sampled_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh, a, ro
             out["dw2"][e] = np.zeros((len(f_cols), len(h_cols)))
             out["dw1"][e] = np.zeros((len(hh_cols), len(j_cols)))
             continue
-        out["dw2"][e] = deq_rows(f64(a[rs][:, f_cols])).T @ deq_rows(f64(dy_perm[rs][:, h_cols]))
-        out["dw1"][e] = deq_rows(f64(xp[rs][:, hh_cols])).T @ deq_rows(f64(dh[rs][:, j_cols]))
+        out["dw2"][e] = deq_rows(f64(a[rs, f_cols])).T @ deq_rows(f64(dy_perm[rs][:, h_cols]))
+        dhw = dh if dh_wgrad is None else dh_wgrad
+        out["dw1"][e] = deq_rows(f64(xp[rs][:, hh_cols])).T @ deq_rows(f64(dhw[rs, j_cols]))
     return out

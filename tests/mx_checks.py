@@ -44,6 +44,48 @@ def swiglu_fp32_error_bound(g, u, p, sum_abs_g, sum_abs_u, K: int):
     return np.abs(dsilu * u * p) * eps_g + np.abs(silu * p) * eps_u + 16.0 * U * np.abs(silu * u * p)
 
 
+def dswiglu_fp32_error_bounds(g, u, p, sum_abs_da, K: int):
+    """Bounds on |x_fp32 - x| for the SwiGLU backward's dg, du and the recomputed a, when
+    da is a K-term dot product accumulated in fp32 by the tensor cores (the bound of
+    swiglu_fp32_error_bound on da) and g, u, p are exact inputs; the epilogue's own fp32
+    work adds a few ulps of each value (|da| is at most sum |dy w|)."""
+    U = 2.0 ** -24
+    eps_da = 4.0 * (K // 32 + 1) * U * np.asarray(sum_abs_da, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-g))
+    silu = g * s
+    dsilu = s * (1.0 + g * (1.0 - s))
+    return (np.abs(p * u * dsilu) * eps_da + 16.0 * U * np.abs(p * u * dsilu) * np.abs(sum_abs_da),
+            np.abs(p * silu) * eps_da + 16.0 * U * np.abs(p * silu) * np.abs(sum_abs_da),
+            16.0 * U * np.abs(silu * u * p))
+
+
+def boundary_flips_grouped_rows(codes, scales, exact, split, err=None, **tol):
+    """The same check for codes quantised along each expert's rows (32-row blocks that
+    restart at every expert): codes / exact / err [R, C], scales a per-expert list of
+    [ceil(n_e/32), C]. Each expert's rows are padded to whole blocks with zeros and
+    transposed, so that the blocks run along the last axis."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    exact = np.asarray(exact, dtype=np.float64)
+    err = np.zeros(exact.shape) if err is None else np.asarray(err, dtype=np.float64)
+    total = {"scale_flips": 0, "code_flips": 0, "bad_scales": 0, "bad_codes": 0, "worst_mid_dist": 0.0}
+    ok_all, r0 = True, 0
+    for n, sc in zip(split, scales):
+        n = int(n)
+        if n == 0:
+            continue
+        npad = (n + 31) // 32 * 32
+        pad = lambda a, dt: np.concatenate([a[r0:r0 + n], np.zeros((npad - n, a.shape[1]), dtype=dt)])
+        ok, rep = boundary_flips(pad(codes, np.uint8).T, np.asarray(sc).T, pad(exact, np.float64).T,
+                                 pad(err, np.float64).T, **tol)
+        ok_all &= ok
+        for k in total:
+            total[k] = max(total[k], rep[k]) if k == "worst_mid_dist" else total[k] + rep[k]
+        r0 += n
+    return ok_all, total
+
+
 def boundary_flips(codes, scales, exact, err=None, step_tol=1e-3, amax_tol=1e-4):
     """Return (ok, report) for kernel codes [n, C] / scales [n, C/32] against exact [n, C];
     ``err`` [n, C] bounds how far fp32 arithmetic can move each exact value."""

@@ -52,3 +52,21 @@ def grouped_scales_to_atoms(scales_per_expert, split_sizes, C):
         out[:, :, _WORD, :] = b
         atoms.append(out.reshape(-1))
     return np.concatenate(atoms) if atoms else np.zeros(0, np.uint8)
+
+
+def grouped_atoms_to_scales(atoms, split_sizes, C):
+    """Inverse of grouped_scales_to_atoms: per-expert [ceil(n_e/32), C] scales."""
+    CG = C // 128
+    a = np.asarray(atoms, dtype=np.uint8)
+    out, base = [], 0
+    for n in split_sizes:
+        n = int(n)
+        kg = (n + 127) // 128
+        if kg == 0:
+            out.append(np.zeros((0, C), dtype=np.uint8))
+            continue
+        blk = a[base * 512: (base + CG * kg) * 512].reshape(CG, kg, 128, 4)[:, :, _WORD, :]   # [cg, kg, c, byte]
+        scales = blk.transpose(1, 3, 0, 2).reshape(kg * 4, C)
+        out.append(scales[: (n + 31) // 32])
+        base += CG * kg
+    return out

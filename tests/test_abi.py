@@ -36,7 +36,9 @@ def test_status_strings():
 
 
 def test_workspace_sizes():
-    assert moe_b200.moe_permute_workspace_size(8192, 2, 8) == 16 * 8 * 4 + (256 - 16 * 8 * 4 % 256) % 256
+    # the 16 blocks' expert histograms (256-byte aligned) plus 256 bytes for the fused
+    # route + permutation call's counter
+    assert moe_b200.moe_permute_workspace_size(8192, 2, 8) == 16 * 8 * 4 + (256 - 16 * 8 * 4 % 256) % 256 + 256
     assert moe_b200.grouped_mlp_workspace_size(8, 16384, 4096, 14336) >= 16384 * 14336 * 2
     assert moe_b200.grouped_mlp_saved_size(8, 100, 256, 128) >= 100 * 3 * 128 * 2
     assert moe_b200.grouped_mlp_bwd_workspace_size(8, 100, 256, 128) >= 100 * 256 * 2
@@ -53,6 +55,17 @@ def test_route_rejects_bad_arguments(args):
     p, T, E, k, renorm = args
     rc = h.moe_route(ctypes.c_void_p(p), T, E, k, renorm, None, None, None)
     assert rc == 1
+
+
+def test_router_backward_and_fused_route_reject_bad_arguments():
+    h = moe_b200.lib()
+    # k > E, no logits without renorm, workspace too small: refused before any launch
+    assert h.moe_route_bwd(None, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 2, 3, 1,
+                           ctypes.c_void_p(16), None) == 1
+    assert h.moe_route_bwd(None, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8, 2, 0,
+                           ctypes.c_void_p(16), None) == 1
+    p = ctypes.c_void_p(256)
+    assert h.moe_route_permute(p, p, 16, 64, 8, 2, 1, 0, p, p, p, None, p, p, p, p, p, 16, None) == 1
 
 
 def test_other_entry_points_reject_bad_arguments():

@@ -13,8 +13,9 @@ import torch
 import mixture_experts_grouped_top_b200 as mb
 from oracle import moe as om
 import workloads
-from tests.mx_checks import assert_boundary_flips, swiglu_fp32_error_bound
-from tests.mx_layout import tile_atoms_to_plain
+from oracle import mxfp8 as oq
+from tests.mx_checks import assert_boundary_flips, dswiglu_fp32_error_bounds, swiglu_fp32_error_bound
+from tests.mx_layout import grouped_atoms_to_scales, tile_atoms_to_plain
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -128,13 +129,42 @@ def test_genomic_mxfp8_full_size_fwd_bwd():
     split = layer.perm["split_sizes"].cpu().numpy()
     assert split[0] > 0.4 * R                                            # expert 0 carries the skew
     b = layer._bwd
-    off_dh = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 0)
-    off_a = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 1)
-    dh = b["ws"][off_dh: off_dh + R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
-    a = b["ws"][off_a: off_a + R * F * 2].view(torch.bfloat16).view(R, F).cpu()
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
-    rows_all, small, large = sample_rows(split, 2048, seed=8)
+    ws = b["ws"]
+
+    def part(i, ncols):
+        off = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", i)
+        codes = ws[off: off + R * ncols].view(R, ncols)                      # stays on the device
+        atoms = ws[off + (R * ncols + 255) // 256 * 256:].cpu().numpy()
+        return codes, atoms
+
+    dhr, dhr_at = part(8, 2 * F)
+    dhr_s, _, _ = tile_atoms_to_plain(dhr_at, split, 2 * F // 32)
+    dhc, dhc_at = part(9, 2 * F)
+    dhc_s = grouped_atoms_to_scales(dhc_at, split, 2 * F)
+    ac, ac_at = part(7, F)
+    ac_s = grouped_atoms_to_scales(ac_at, split, F)
     offs = np.concatenate([[0], np.cumsum(split)])
+
+    class RowsDeq:
+        """dh along 2F, dequantised on demand for the rows asked for."""
+        def __getitem__(self, rows):
+            return oq.dequantize_blocks_last_axis(dhr[torch.as_tensor(rows, device=DEV)].cpu().numpy(),
+                                                  dhr_s[rows])
+
+    class ColsDeq:
+        """codes along each expert's rows, dequantised on demand for one expert's rows and
+        the columns asked for."""
+        def __init__(self, codes, scales):
+            self.codes, self.scales = codes, scales
+
+        def __getitem__(self, key):
+            rs, cols = key
+            e = int(np.searchsorted(offs, rs.start, side="right") - 1)
+            c = self.codes[rs][:, torch.as_tensor(cols, device=DEV)].cpu().numpy()
+            return oq.dequantize_grouped_rows(c, [self.scales[e][:, cols]], [rs.stop - rs.start])
+
+    rows_all, small, large = sample_rows(split, 2048, seed=8)
     keep = ((rows_all >= offs[small]) & (rows_all < offs[small + 1])) | \
            ((rows_all >= offs[large]) & (rows_all < offs[large + 1]))
     rows = rows_all[keep]
@@ -142,8 +172,22 @@ def test_genomic_mxfp8_full_size_fwd_bwd():
     cols = (np.sort(rng.choice(F, 16, replace=False)), np.sort(rng.choice(H, 16, replace=False)),
             np.sort(rng.choice(H, 16, replace=False)), np.sort(rng.choice(2 * F, 16, replace=False)))
     ref = om.bwd_sampled_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
-                               layer.perm["probs_perm"].cpu(), h, dh, a, rows, [small, large], cols)
-    within_mx(dh[rows], ref["dh"], "dh")
+                               layer.perm["probs_perm"].cpu(), h, RowsDeq(), ColsDeq(ac, ac_s), rows,
+                               [small, large], cols, dh_wgrad=ColsDeq(dhc, dhc_s))
+    # dh along 2F at the sampled rows: only rounding-boundary flips against the exact dh;
+    # the fp32 error bound takes |da| magnitudes from the oracle's fc2-dgrad operands
+    sabs = np.zeros((rows.size, F))
+    dyq = np.abs(oq.dequantize(*oq.quantize(om.f64(b["dy_perm"][torch.as_tensor(rows, device=DEV)].cpu()), axis=0),
+                               axis=0))
+    for e in (small, large):
+        sel = (rows >= offs[e]) & (rows < offs[e + 1])
+        w2q = np.abs(oq.dequantize(*oq.quantize(om.f64(d["w2"][e]), axis=0), axis=0))
+        sabs[sel] = dyq[sel] @ w2q.T
+    hh = om.f64(h[torch.as_tensor(rows)])
+    pp = om.f64(layer.perm["probs_perm"].cpu()[torch.as_tensor(rows)])[:, None]
+    e_dg, e_du, _ = dswiglu_fp32_error_bounds(hh[:, :F], hh[:, F:], pp, sabs, H)
+    assert_boundary_flips(dhr[torch.as_tensor(rows, device=DEV)].cpu().numpy(), dhr_s[rows], ref["dh"], "dh",
+                          err=np.concatenate([e_dg, e_du], axis=1))
     within_mx(b["dxp"].cpu()[rows], ref["dxp"], "dxp")
     gp = b["dprobs_perm"].cpu().numpy()[rows]
     assert np.max(np.abs(gp - ref["dp"])) <= 2e-3 * np.max(np.abs(ref["dp"]))

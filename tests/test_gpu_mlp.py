@@ -37,6 +37,11 @@ FWD_CASES = [
     (300, 512, 256, 3, 1, ()),
     (100, 192, 128, 8, 4, (0, 7)),
     (1000, 320, 512, 16, 2, (2, 5, 11)),
+    # degenerate routings: one expert (E=1, k=1, p=1); every row on one expert (k=1);
+    # every token on the same two experts (k=2), each of them holding all T rows
+    (300, 256, 256, 1, 1, ()),
+    (257, 128, 256, 5, 1, (0, 1, 2, 4)),
+    (300, 128, 256, 4, 2, (0, 2)),
 ]
 
 
@@ -101,6 +106,9 @@ BWD_CASES = [
     (256, 128, 256, 4, 2, ()),
     (600, 256, 384, 5, 2, (3,)),
     (300, 192, 256, 8, 4, (1, 6)),
+    (300, 256, 256, 1, 1, ()),
+    (257, 128, 256, 5, 1, (0, 1, 2, 4)),
+    (300, 128, 256, 4, 2, (0, 2)),
 ]
 
 

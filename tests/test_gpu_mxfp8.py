@@ -74,6 +74,9 @@ MX_CASES = [
     (300, 256, 256, 4, 2, ()),
     (600, 512, 384, 5, 2, (3,)),
     (1000, 384, 640, 16, 2, (2, 5, 11)),
+    (300, 256, 256, 1, 1, ()),              # one expert
+    (257, 256, 256, 5, 1, (0, 1, 2, 4)),    # every row on one expert
+    (300, 256, 256, 4, 2, (0, 2)),          # every token on the same two experts
 ]
 
 

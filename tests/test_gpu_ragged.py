@@ -67,6 +67,29 @@ def test_bf16_backward_ragged_expert_sizes():
     assert np.max(np.abs(got - rdxp)) <= 1e-2 * np.max(np.abs(rdxp))
 
 
+# experts that span more than the weight-gradient ring's three 128-row stages and end
+# ragged, and sizes around one and two stages; H = F = 384 puts a ragged 128-column tail
+# in the second CTA of each pair's last output tile
+SPLIT_BF16_DEEP = [4 * 128 + 5, 3 * 128 + 17, 255, 256, 257, 0, 1]
+
+
+def test_bf16_backward_ragged_deep_experts():
+    H, F = 384, 384
+    d, E, T = routed_inputs(SPLIT_BF16_DEEP, H, F, seed=23)
+    layer, (dx, dw1, dw2, dprob) = run_layer(d, T, H, F, E, "bf16")
+    split = layer.perm["split_sizes"].cpu().numpy()
+    assert list(split) == SPLIT_BF16_DEEP
+    b = layer._bwd
+    rdxp, rdw1, rdw2, rdpp, _ = om.grouped_mlp_bwd(b["dy_perm"].cpu(), layer.perm["xp"].cpu(), split, d["w1"],
+                                                    d["w2"], layer.perm["probs_perm"].cpu(), a_round="bf16")
+    for e, n in enumerate(SPLIT_BF16_DEEP):
+        if n == 0:
+            assert torch.count_nonzero(dw1[e]) == 0 and torch.count_nonzero(dw2[e]) == 0
+            continue
+        assert per_expert_rel(dw1, rdw1, e) <= 1e-2, (e, n)
+        assert per_expert_rel(dw2, rdw2, e) <= 1e-2, (e, n)
+
+
 def within_expert(got, ref, e, name, tol=2e-3):
     g = got[e].float().cpu().numpy()
     r = ref[e]
@@ -75,6 +98,8 @@ def within_expert(got, ref, e, name, tol=2e-3):
 
 
 def test_mxfp8_backward_ragged_expert_sizes():
+    from tests.test_gpu_mxfp8_bwd import fused_operands
+    from oracle import mxfp8 as oq
     H, F = 256, 128
     d, E, T = routed_inputs(SPLIT_MX, H, F, seed=22)
     layer, (dx, dw1, dw2, dprob) = run_layer(d, T, H, F, E, "mxfp8")
@@ -82,14 +107,13 @@ def test_mxfp8_backward_ragged_expert_sizes():
     assert list(split) == SPLIT_MX
     R = T
     b = layer._bwd
-    ws = b["ws"]
-    off_dh = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 0)
-    off_a = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 1)
-    dh = ws[off_dh: off_dh + R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
-    a = ws[off_a: off_a + R * F * 2].view(torch.bfloat16).view(R, F).cpu()
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
+    (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(b["ws"], E, R, H, F, split)
     ref = om.grouped_mlp_bwd_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
-                                   layer.perm["probs_perm"].cpu(), h, dh=dh, a=a)
+                                   layer.perm["probs_perm"].cpu(), h,
+                                   dh=oq.dequantize_blocks_last_axis(dhr, dhr_s),
+                                   a=oq.dequantize_grouped_rows(ac, ac_s, split),
+                                   dh_wgrad=oq.dequantize_grouped_rows(dhc, dhc_s, split))
     _, rdw1, rdw2, _, _, _ = ref
     for e, n in enumerate(SPLIT_MX):
         if n == 0:

@@ -219,8 +219,7 @@ def test_sampled_mxfp8_backward_equals_full_mxfp8_backward():
     _, h, _ = moe.grouped_mlp_fwd(xp, split, w1, w2, pp, a_round="f64")
     dy = rng.normal(size=xp.shape)
     full = moe.grouped_mlp_bwd_mxfp8(dy, xp, split, w1, w2, pp, h)
-    dh = moe.round_to_bf16(full[4])
-    a = moe.round_to_bf16(full[5])
+    dh, a = full[4], full[5]
     rows = np.array([1, 7, 33, 79])
     cols = ([3, 9], [0, 63], [5, 6], [2, 100])
     s = moe.bwd_sampled_mxfp8(dy, xp, split, w1, w2, pp, h, dh, a, rows, [0, 1, 2], cols)
