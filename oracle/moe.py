@@ -34,7 +34,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import mxfp8
+from . import fp8, mxfp8
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -158,6 +158,44 @@ def unpermute(yp, row_map, T: int, k: int, prob=None) -> np.ndarray:
     for j in range(k):
         w = 1.0 if prob is None else f64(prob)[:, j][:, None]
         out += w * yp[rm[:, j]]
+    return out
+
+
+# ------------------------------------------------------------- capacity-padded dispatch
+def capacity_keep(idx, E: int, C: int) -> np.ndarray:
+    """Capacity-padded dispatch: every expert takes at most C of the slots routed to it,
+    the first ones in flat slot order s = t*k + j; later slots are dropped (the padded
+    ``batched_mm`` expert back-end of Transformers v5 named on the "NeMo AutoModel" page,
+    section on Transformers v5 features, runs one batched GEMM over [E, C] rows).
+    Returns keep, bool [T, k]."""
+    flat = np.asarray(idx, dtype=np.int64).reshape(-1)
+    keep = np.zeros(flat.size, dtype=bool)
+    taken = np.zeros(E, dtype=np.int64)
+    for s, e in enumerate(flat):
+        if taken[e] < C:
+            keep[s] = True
+            taken[e] += 1
+    return keep.reshape(np.asarray(idx).shape)
+
+
+def moe_forward_capacity(x, idx, prob, w1, w2, C: int, a_round="bf16") -> np.ndarray:
+    """The layer with expert capacity C: out[t] = sum over the token's KEPT slots j of
+    (SiLU(x_t W1g_e) * (x_t W1u_e) * p_tj) W2_e; a dropped slot contributes nothing."""
+    x = f64(x)
+    idx = np.asarray(idx, dtype=np.int64)
+    prob = f64(prob)
+    w1 = f64(w1)
+    w2 = f64(w2)
+    F = w2.shape[1]
+    keep = capacity_keep(idx, w1.shape[0], C)
+    out = np.zeros((x.shape[0], x.shape[1]))
+    for t in range(x.shape[0]):
+        for j in range(idx.shape[1]):
+            if not keep[t, j]:
+                continue
+            e = idx[t, j]
+            h = x[t] @ w1[e]
+            out[t] += _round_a(silu(h[:F]) * h[F:] * prob[t, j], a_round) @ w2[e]
     return out
 
 
@@ -544,3 +582,79 @@ def bwd_sampled_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh, a, ro
         dhw = dh if dh_wgrad is None else dh_wgrad
         out["dw1"][e] = deq_rows(f64(xp[rs][:, hh_cols])).T @ deq_rows(f64(dhw[rs, j_cols]))
     return out
+
+
+# ------------------------------------------------------------ per-tensor FP8 expert MLP
+def grouped_mlp_fwd_fp8(xp, split_sizes, w1, w2, probs_perm, a_codes=None, a_scale=None):
+    """The layer with per-tensor FP8 (current scaling, E4M3), float64 on quantised
+    operands: xp one scale over all rows, each expert's w1[e] / w2[e] its own scale; the
+    fc1 output a = SiLU(g) * u * p is stored in bf16 (its amax is only known once all of it
+    exists) and quantised with one scale over [R, F], unless ``a_codes`` / ``a_scale`` (a
+    GPU's) are given. Returns (yp, a_codes, a_scale, h)."""
+    xq = fp8.qdq(f64(xp), "e4m3")
+    w1 = f64(w1)
+    w2 = f64(w2)
+    pp = f64(probs_perm)
+    E, F, H = w2.shape[0], w2.shape[1], w2.shape[2]
+    w1q = np.stack([fp8.qdq(w1[e], "e4m3") for e in range(E)])
+    w2q = np.stack([fp8.qdq(w2[e], "e4m3") for e in range(E)])
+    R = xq.shape[0]
+    h_all = np.zeros((R, 2 * F))
+    a_all = np.zeros((R, F))
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        h = xq[rows] @ w1q[e]
+        h_all[rows] = h
+        a_all[rows] = silu(h[:, :F]) * h[:, F:] * pp[rows, None]
+        start += n
+    if a_codes is None:
+        a_codes, a_scale = fp8.quantize_tensor(round_to_bf16(a_all), "e4m3")
+    aq = fp8.dequantize_tensor(a_codes, a_scale, "e4m3")
+    yp = np.zeros((R, H))
+    start = 0
+    for e, n in enumerate(np.asarray(split_sizes, dtype=np.int64)):
+        rows = slice(start, start + n)
+        yp[rows] = aq[rows] @ w2q[e]
+        start += n
+    return yp, a_codes, a_scale, h_all
+
+
+def grouped_mlp_bwd_fp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, a_codes, a_scale, dh=None):
+    """Backward of :func:`grouped_mlp_fwd_fp8`: gradients in E5M2 with one scale per
+    tensor (dy over [R, H], dh over [R, 2F]), forward operands in E4M3 as in the forward
+    (per-tensor scales have no axis, so the forward's codes of xp, a and the weights serve
+    the backward's GEMMs too). dh is stored in bf16 before its quantisation unless ``dh``
+    (e.g. a GPU's values) is given. Returns (dxp, dw1, dw2, dprobs_perm, dh_exact)."""
+    dyq = fp8.qdq(f64(dy_perm), "e5m2")
+    xq = fp8.qdq(f64(xp), "e4m3")
+    aq = fp8.dequantize_tensor(a_codes, a_scale, "e4m3")
+    w1 = f64(w1)
+    w2 = f64(w2)
+    pp = f64(probs_perm)
+    h = f64(h)
+    E, F = w2.shape[0], w2.shape[1]
+    w1q = np.stack([fp8.qdq(w1[e], "e4m3") for e in range(E)])
+    w2q = np.stack([fp8.qdq(w2[e], "e4m3") for e in range(E)])
+    split = np.asarray(split_sizes, dtype=np.int64)
+    da = np.zeros((dyq.shape[0], F))
+    start = 0
+    for e, n in enumerate(split):
+        da[start:start + n] = dyq[start:start + n] @ w2q[e].T
+        start += n
+    g, u = h[:, :F], h[:, F:]
+    p = pp[:, None]
+    dh_exact = np.concatenate([da * p * u * silu_grad(g), da * p * silu(g)], axis=1)
+    dprob = np.sum(da * silu(g) * u, axis=1)
+    dhq = fp8.qdq(round_to_bf16(dh_exact) if dh is None else f64(dh), "e5m2")
+    dxp = np.zeros_like(xq)
+    dw1 = np.zeros_like(w1)
+    dw2 = np.zeros_like(w2)
+    start = 0
+    for e, n in enumerate(split):
+        rows = slice(start, start + n)
+        dw2[e] = aq[rows].T @ dyq[rows]
+        dxp[rows] = dhq[rows] @ w1q[e].T
+        dw1[e] = xq[rows].T @ dhq[rows]
+        start += n
+    return dxp, dw1, dw2, dprob, dh_exact

@@ -244,3 +244,33 @@ def test_mxfp8_forward_rows_equal_grouped_forward():
     rows = rm
     ypr, c, s = moe.fwd_rows_mxfp8(x[toks], prob.reshape(-1), idx.reshape(-1), w1, w2)
     assert np.allclose(ypr, yp[rows], atol=1e-12) and np.array_equal(c, ac[rows]) and np.array_equal(s, asc[rows])
+
+
+# ------------------------------------------------------------ capacity-padded dispatch
+def test_capacity_keep_is_first_C_slots_per_expert():
+    rng = np.random.default_rng(12)
+    T, E, k = 50, 5, 2
+    idx, _ = moe.route(rng.normal(size=(T, E)) + np.array([2.0, 1.0, 0, 0, -3.0]), k)
+    for C in (0, 1, 7, 20, 100):
+        keep = moe.capacity_keep(idx, E, C)
+        flat, kf = idx.reshape(-1), keep.reshape(-1)
+        for e in range(E):
+            slots = np.nonzero(flat == e)[0]               # ascending slot order
+            assert np.array_equal(np.nonzero(kf & (flat == e))[0], slots[:C])
+        assert kf.sum() == sum(min(int((flat == e).sum()), C) for e in range(E))
+
+
+def test_capacity_forward_special_cases():
+    x, idx, prob, w1, w2 = _layer(24, 8, 6, 4, 2, seed=13)
+    ref = moe.moe_forward_per_token(x, idx, prob, w1, w2, "f64")
+    # a capacity that holds every slot is the dropless layer
+    big = moe.moe_forward_capacity(x, idx, prob, w1, w2, C=24 * 2, a_round="f64")
+    np.testing.assert_allclose(big, ref, rtol=1e-13, atol=1e-13)
+    # no capacity: nothing is computed
+    assert np.all(moe.moe_forward_capacity(x, idx, prob, w1, w2, C=0, a_round="f64") == 0)
+    # a dropped slot is the same as a zero routing probability (p scales a inside ScaledSwiGLU)
+    keep = moe.capacity_keep(idx, 4, 5)
+    assert not keep.all()
+    got = moe.moe_forward_capacity(x, idx, prob, w1, w2, C=5, a_round="f64")
+    np.testing.assert_allclose(got, moe.moe_forward_per_token(x, idx, np.where(keep, prob, 0.0), w1, w2, "f64"),
+                               rtol=1e-13, atol=1e-13)
