@@ -44,6 +44,7 @@ import workloads  # noqa: E402
 DEFAULT_WORKLOAD = "genomic_mixtral_mxfp8_fwdbwd"
 SECONDARY_WORKLOADS = ["mixtral_bf16_fwd", "mixtral_mxfp8_fwd", "qwen3_30b_a3b_bf16_fwdbwd"]
 FUSED_COMBINE_WORKLOADS = ["mixtral_bf16_fwd", "qwen3_30b_a3b_bf16_fwdbwd"]
+CAPACITY_WORKLOADS = ["mixtral_bf16_fwd"]
 METRIC = "grouped-MLP TFLOP/s & tokens/s (fwd, fwd+bwd) on 1 B200; % of tensor-core peak"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 MXFP8_PEAK_FILE = os.path.join(ROOT, "profiles", "mxfp8_peak.json")
@@ -332,6 +333,9 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
                                layer.perm["probs_perm"], layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"], dw2=b["dw2"],
                                dprobs_perm=b["dprobs_perm"], workspace=b["ws"])
             mark(6)
+            if world > 1:
+                # data-parallel replicas: the weight gradients are summed over the ranks
+                mb.allreduce_grads([b["dw1"], b["dw2"]])
             mb.moe_unpermute(b["dxp"], layer.perm["row_map"], cfg.T, cfg.k, out=b["dx"])
             mb.moe_gather_slots(b["dprobs_perm"], layer.perm["row_map"], out=b["dprob"].view(-1))
             mb.moe_route_bwd(None, layer.idx, layer.prob, b["dprob"], True, dlogits=b["dlogits"])
@@ -395,7 +399,8 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
                    "gemm_flop_per_step_per_gpu": flops,
                    "l2": "inputs larger than L2: the expert weights (%.2f GB bf16) are re-read every step"
                          % ((d["w1"].numel() + d["w2"].numel()) * 2 / 1e9),
-                   "parallelism": f"dp{world} replicas" if world > 1 else "single GPU"},
+                   "parallelism": (f"dp{world} replicas" + (", dw1/dw2 all-reduced (NCCL) every step" if training
+                                                              else "")) if world > 1 else "single GPU"},
         "roofline": {"kernel": ("grouped_mlp_fwd + grouped_mlp_bwd (the six tcgen05 grouped GEMMs and the "
                                 "backward's quantisation passes)" if training else
                                 "grouped_mlp_fwd (fc1 gate|up + ScaledSwiGLU, fc2: two tcgen05 grouped GEMMs)"),
@@ -456,6 +461,52 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
         del pipe
     del layer
     return res, d
+
+
+def run_capacity(cfg, args, local, factor: float, steps: int, warmup: int):
+    """The capacity-padded dispatch (the padded batched_mm back-end) on a forward
+    workload, as a comparison point: route, moe_permute_capacity (C = ceil(factor T k /
+    E) rows per expert, overflow dropped), the grouped GEMMs over E*C rows, unpermute."""
+    import math
+    import mixture_experts_grouped_top_b200 as mb
+    dev = torch.device("cuda", local)
+    d = workloads.make_layer_inputs(cfg, with_grad=False)
+    C = int(math.ceil(factor * cfg.T * cfg.k / cfg.E))
+    x, logits = d["x"].to(dev), d["logits"].to(dev)
+    w1, w2 = d["w1"].to(dev), d["w2"].to(dev)
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+    prob = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    o = mb.moe_permute_capacity(x, *mb.moe_route(logits, cfg.k, True, idx=idx, prob=prob), cfg.E, C)
+    ws = torch.empty(mb.moe_permute_capacity_workspace_size(cfg.T, cfg.k, cfg.E), dtype=torch.uint8, device=dev)
+    mlp_ws = torch.empty(mb.grouped_mlp_workspace_size(cfg.E, cfg.E * C, cfg.H, cfg.F), dtype=torch.uint8, device=dev)
+    yp = torch.empty((cfg.E * C, cfg.H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mb.moe_route(logits, cfg.k, True, idx=idx, prob=prob)
+        mb.moe_permute_capacity(x, idx, prob, cfg.E, C, out=o, workspace=ws)
+        mb.grouped_mlp_fwd(o["xp"], o["split_sizes"], w1, w2, o["probs_perm"], yp=yp, workspace=mlp_ws)
+        mb.moe_unpermute(yp, o["row_map"], cfg.T, cfg.k, out=out)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    t0, t1 = ev(), ev()
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if mb.moe_device_status() != 0:
+        raise RuntimeError("device error in the capacity-padded run")
+    ms = t0.elapsed_time(t1) / steps
+    kept = int(o["kept"].sum().item())
+    return {"capacity_factor": factor, "C": C, "ms_per_step": round(ms, 4),
+            "value": round(cfg.gemm_flops() / (ms * 1e-3) / 1e12, 3),
+            "padded_gemm_tflop": round(6.0 * cfg.H * cfg.F * cfg.E * C / 1e12, 3),
+            "dropped_slot_frac": round(1.0 - kept / cfg.R, 5),
+            "note": "value = the dropless layer's algorithmic FLOPs / time (padding computed, overflow dropped)"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
@@ -584,6 +635,11 @@ def run_ours(args, world, rank, local):
                 torch.cuda.empty_cache()
                 res["fused_combine"] = {k: fres[k] for k in ("value", "ms_per_step", "tokens_per_s", "clocks")}
                 res["fused_combine"]["roofline_frac"] = fres["roofline"]["frac"]
+            if name in CAPACITY_WORKLOADS:
+                res["capacity_padded"] = [run_capacity(workloads.CONFIGS[name], args, local, f, args.workload_steps,
+                                                       args.warmup) for f in (1.0, 1.25)]
+                gc.collect()
+                torch.cuda.empty_cache()
         line["gpu_launches"] = head["gpu_launches"]
     return line
 

@@ -51,7 +51,7 @@ typedef enum {
   MOE_ERR_TIMEOUT = 5        /* a kernel wait exceeded its time budget */
 } moe_status_t;
 
-typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_precision_t;
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_FP8 = 2 } moe_precision_t;
 
 /* Flag OR-ed into grouped_mlp_fwd's `precision`: write yp as fp32 [R, H] instead of bf16
  * (the fc2 accumulator without the bf16 storage rounding). */
@@ -189,6 +189,29 @@ MOE_API int moe_permute_noalloc(const uint16_t* x, const int32_t* idx, const flo
                                 int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
                                 int32_t* split_sizes, int32_t* offsets, void* stream);
 
+/* Bytes of device scratch moe_permute_capacity needs. */
+MOE_API size_t moe_permute_capacity_workspace_size(int T, int k, int E);
+
+/*
+ * moe_permute_capacity — the capacity-padded dispatch of the padded "batched_mm" expert
+ * back-end (NeMo AutoModel page, Transformers v5 features: experts_implementation in
+ * {eager, batched_mm, grouped_mm}), as a comparison point for the dropless grouped path.
+ * Every expert gets exactly C rows: the first min(n_e, C) of its slots in slot order
+ * s = t*k + j (the stable order of moe_permute) fill rows [e*C, e*C + n_e), the rest of
+ * its C rows are zeros, and its slots past C are dropped (row_map[s] = -1; moe_unpermute
+ * and moe_gather_slots skip them, so a dropped slot contributes nothing).
+ *   x, idx, prob as moe_permute; C >= 0 the capacity (e.g. ceil(factor * T*k / E));
+ *   xp [E*C, H] bf16 (MOE_BF16) or E4M3 codes with xp_scale [E*C, H/32] (MOE_MXFP8);
+ *   row_map [R] int32 (slot -> padded row or -1); probs_perm [E*C] fp32 or NULL (zero on
+ *   padded rows); split_sizes [E] (= C each) and offsets [E+1] (= e*C) for
+ *   grouped_mlp_fwd on the padded rows; kept [E] int32 or NULL: min(n_e, C).
+ *   workspace: moe_permute_capacity_workspace_size(T, k, E) bytes.
+ */
+MOE_API int moe_permute_capacity(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
+                                 int C, int precision, void* xp, uint8_t* xp_scale, int32_t* row_map,
+                                 float* probs_perm, int32_t* split_sizes, int32_t* offsets, int32_t* kept,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * moe_permute_rows — the data movement of moe_permute alone, for a tensor that follows
  * an existing row_map (e.g. the gradient of the layer output in the backward pass):
@@ -265,6 +288,12 @@ MOE_API size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision)
  *   the fc1 epilogue quantises a along F (blocks of 32) and keeps its scales as MMA
  *   atoms whose row groups are the 128-row tiles of each expert (sum over earlier
  *   experts of ceil(n_e/128), then the tile index); requires H % 128 == 0.
+ * MOE_FP8 (per-tensor, see fp8_quantize): xp [R, H] E4M3 codes with xp_scale pointing
+ *   to ONE fp32 scale (passed as uint8_t*); w1 [E, 2F, H] and w2 [E, H, F] E4M3 codes
+ *   (fp8_quantize with transpose_out) with w1_scale / w2_scale pointing to E fp32 scales
+ *   (one per expert); the fc1 epilogue stores a in bf16 and keeps max |a|, then a is
+ *   quantised with one E4M3 scale for all rows and fc2 runs on those codes; the
+ *   products are rescaled by 1 / (s_A s_B) in the epilogues; requires H % 128 == 0.
  * split_sizes [E] int32 on the device (no host synchronisation happens); R = sum.
  * yp [R, H] bf16 output (fp32 when MOE_OUT_F32 is OR-ed into precision).
  * saved: NULL for inference, else a buffer of
@@ -276,6 +305,24 @@ MOE_API int grouped_mlp_fwd(const void* xp, const uint8_t* xp_scale, const int32
                     const void* w1, const uint8_t* w1_scale, const void* w2, const uint8_t* w2_scale,
                     const float* probs_perm, int precision, void* yp, void* saved, void* ws, size_t ws_bytes,
                     void* stream);
+
+/* Bytes of scratch fp8_quantize needs (one max per tensor). */
+MOE_API size_t fp8_quantize_workspace_size(int batch);
+
+/*
+ * fp8_quantize — per-tensor FP8 with current scaling (news.bpdata.com section 2, "FP8
+ * and MXFP8": FP8 keeps one scale per tensor; E4M3 for forward operands, E5M2 for
+ * gradients). For each of `batch` tensors in [batch, rows, cols] bf16: s = fmt_max /
+ * max |x| in fp32 (448 for E4M3, 57344 for E5M2; s = 1 for an all-zero tensor), and
+ * codes = the fp32 product x * s rounded to the format (nearest even, saturating); a
+ * code c stands for decode(c) / s.
+ *   fmt: 0 = E4M3, 1 = E5M2; transpose_out: codes [batch, cols, rows] (rows, cols
+ *   multiples of 32) instead of [batch, rows, cols] (rows * cols a multiple of 8);
+ *   codes uint8 (output); scales [batch] fp32 (output);
+ *   workspace: fp8_quantize_workspace_size(batch) bytes.
+ */
+MOE_API int fp8_quantize(const uint16_t* in, int batch, int rows, int cols, int fmt, int transpose_out, uint8_t* codes,
+                         float* scales, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of scratch grouped_mlp_fwd_combine needs: grouped_mlp_fwd's workspace, then an
  * fp32 [T, H] accumulator and the token of every row. */
@@ -332,6 +379,9 @@ MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int 
  * saved: the buffer filled by grouped_mlp_fwd in training mode (same precision).
  * Outputs: dxp [R, H] bf16, dw1 [E, H, 2F] bf16, dw2 [E, F, H] bf16 (experts with no rows
  * get zeros), dprobs_perm [R] fp32 (may be NULL).
+ * MOE_FP8: the gradients dy and dh are quantised to E5M2 with one scale each, the forward
+ * operands (xp, the saved a codes, the weights, one scale per expert) are E4M3; dh is
+ * stored in bf16 by the fc2-dgrad epilogue (with its max) before its quantisation.
  * MOE_MXFP8: all four GEMMs run on MXFP8 operands quantised along their own contraction
  * axis (blocks of 32): dy and dh along columns for the data gradients, and dy, a
  * (recomputed from h), dh and xp along rows — in 32-row blocks restarting at every

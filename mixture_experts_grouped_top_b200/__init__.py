@@ -16,8 +16,10 @@ from . import _lib
 
 BF16 = 0
 MXFP8 = 1
+FP8 = 2
 OUT_F32 = 0x100
-_PREC = {"bf16": BF16, "mxfp8": MXFP8, BF16: BF16, MXFP8: MXFP8}
+_PREC = {"bf16": BF16, "mxfp8": MXFP8, "fp8": FP8, BF16: BF16, MXFP8: MXFP8, FP8: FP8}
+_FP8_FMT = {"e4m3": 0, "e5m2": 1}
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
           4: "MOE_ERR_DEVICE_CHECK", 5: "MOE_ERR_TIMEOUT"}
@@ -192,6 +194,43 @@ def moe_permute_noalloc(x, idx, prob, E: int, precision="bf16", out=None, stream
     return o
 
 
+def moe_permute_capacity_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_permute_capacity_workspace_size(T, k, E))
+
+
+def moe_permute_capacity(x, idx, prob, E: int, C: int, precision="bf16", out=None, workspace=None, stream=None):
+    """Capacity-padded dispatch into [E*C] rows (slots past an expert's capacity dropped).
+    Returns a dict with xp, xp_scale (MXFP8), row_map, probs_perm, split_sizes, offsets, kept."""
+    _need(x, torch.bfloat16, "x")
+    _need(idx, torch.int32, "idx")
+    prec = _PREC[precision]
+    T, H = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    o = dict(out or {})
+    RC = E * C
+    if "xp" not in o:
+        o["xp"] = torch.empty((RC, H), dtype=torch.bfloat16 if prec == BF16 else torch.uint8, device=dev)
+    if prec == MXFP8 and "xp_scale" not in o:
+        o["xp_scale"] = torch.empty((RC, H // 32), dtype=torch.uint8, device=dev)
+    o.setdefault("row_map", torch.empty(T * k, dtype=torch.int32, device=dev))
+    if prob is not None:
+        o.setdefault("probs_perm", torch.empty(RC, dtype=torch.float32, device=dev))
+    o.setdefault("split_sizes", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    o.setdefault("kept", torch.empty(E, dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = torch.empty(max(moe_permute_capacity_workspace_size(T, k, E), 1), dtype=torch.uint8, device=dev)
+    rc = lib().moe_permute_capacity(_p(x), _p(idx), _p(prob), T, H, E, k, C, prec, _p(o["xp"]),
+                                    _p(o.get("xp_scale")), _p(o["row_map"]), _p(o.get("probs_perm")),
+                                    _p(o["split_sizes"]), _p(o["offsets"]), _p(o["kept"]), _p(workspace),
+                                    workspace.numel(), _stream(stream))
+    _check("moe_permute_capacity", rc)
+    o.setdefault("xp_scale", None)
+    o.setdefault("probs_perm", None)
+    return o
+
+
 def moe_permute_rows(src, row_map, k: int, out=None, stream=None):
     _need(src, torch.bfloat16, "src")
     T, H = src.shape
@@ -251,6 +290,23 @@ def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, sc
     if squeeze:
         return codes.reshape(cshape[1:]), (scales if mma_scales else scales.reshape(sshape[1:]))
     return codes, scales
+
+
+def fp8_quantize(x, fmt="e4m3", transpose_out=False, codes=None, scales=None, stream=None):
+    """Per-tensor FP8 (current scaling) of bf16 [batch, rows, cols] (or [rows, cols]): one
+    fp32 scale per batch matrix. Returns (codes uint8, scales fp32 [batch])."""
+    _need(x, torch.bfloat16, "x")
+    squeeze = x.dim() == 2
+    x3 = x.unsqueeze(0) if squeeze else x
+    B, rows, cols = x3.shape
+    cshape = (B, cols, rows) if transpose_out else (B, rows, cols)
+    codes = torch.empty(cshape, dtype=torch.uint8, device=x.device) if codes is None else codes
+    scales = torch.empty(B, dtype=torch.float32, device=x.device) if scales is None else scales
+    ws = torch.empty(max(int(lib().fp8_quantize_workspace_size(B)), 1), dtype=torch.uint8, device=x.device)
+    rc = lib().fp8_quantize(_p(x3), B, rows, cols, _FP8_FMT[fmt], int(bool(transpose_out)), _p(codes), _p(scales),
+                            _p(ws), ws.numel(), _stream(stream))
+    _check("fp8_quantize", rc)
+    return (codes.reshape(cshape[1:]) if squeeze else codes), scales
 
 
 def mxfp8_quantize_grouped(x, split_sizes, codes=None, atoms=None, stream=None):
@@ -363,4 +419,4 @@ def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precisi
     return dxp, dw1, dw2, dprobs_perm
 
 
-from .layer import HostPipeline, MoEExpertLayer, moe_layer_forward  # noqa: E402,F401
+from .layer import HostPipeline, MoEExpertLayer, allreduce_grads, moe_layer_forward  # noqa: E402,F401

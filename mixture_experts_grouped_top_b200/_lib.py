@@ -24,9 +24,14 @@ SIGNATURES = {
     "moe_permute_workspace_size": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_permute_capacity_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_permute_capacity": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                  _vp]),
     "moe_permute_rows": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_unpermute": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "mxfp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "fp8_quantize_workspace_size": (_sz, [_i]),
+    "fp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "grouped_mlp_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "grouped_mlp_saved_size": (_sz, [_i, _i, _i, _i, _i]),
     "grouped_mlp_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),

@@ -95,7 +95,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int E = p.E;
-  const int NT = (EPI == MXEPI_SWIGLU_Q) ? (p.N / 128) : (p.N + BN - 1) / BN;
+  const int NT = mx_swiglu(EPI) ? (p.N / 128) : (p.N + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -180,16 +180,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
       const int bgroups = mp.b_rows / 128;
       for (int t = pair; t < total && ok && !p.stall_loads; t += npairs) {
         const TileInfo ti = walk.decode(t);
-        const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
+        const int n0 = mx_swiglu(EPI) ? ti.n_blk * 128 : ti.n_blk * BN;
         // this CTA's A rows and their scale group (past the expert: unused rows; a group
         // index past the atom tensor reads zeros)
         const int a_row = ti.row0 + BMC * (int)rank;
         const int ga = grp_off[ti.e] + 2 * ti.m_blk + (int)rank;
         // this CTA's half of B, and the scale groups of both halves
-        const int b_row = (EPI == MXEPI_SWIGLU_Q) ? (rank ? p.F : 0) + n0 : n0 + 128 * (int)rank;
+        const int b_row = mx_swiglu(EPI) ? (rank ? p.F : 0) + n0 : n0 + 128 * (int)rank;
         const int gb0 = ti.e * bgroups + n0 / 128;
-        int gb1 = (EPI == MXEPI_SWIGLU_Q) ? ti.e * bgroups + (p.F + n0) / 128 : gb0 + 1;
-        if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+        int gb1 = mx_swiglu(EPI) ? ti.e * bgroups + (p.F + n0) / 128 : gb0 + 1;
+        if (!mx_swiglu(EPI) && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
         for (int st = 0; st < num_st; ++st) {
           if (st % kStPerSf == 0) {
             // scale atoms of k-blocks [kChunks st, kChunks st + 4) (past K: zeros)
@@ -272,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
                 for (int kk = 0; kk < 4; ++kk) {
                   const uint64_t adesc = make_sdesc(a_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
                   const uint64_t bdesc = make_sdesc(b_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
-                  const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk);
+                  const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk) | mp.ab_fmt;
                   mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30),
                                 sfb_t | ((uint32_t)kk << 30), (kb > 0 || kk > 0) ? 1u : 0u);
                 }

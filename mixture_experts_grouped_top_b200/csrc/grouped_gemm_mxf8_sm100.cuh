@@ -59,7 +59,12 @@ enum MxEpiKind : int {
   MXEPI_SWIGLU_Q = 1,   // a = SiLU(g) * u * p quantised to MXFP8 along the columns (+ bf16 h)
   MXEPI_DSWIGLU = 2,    // SwiGLU backward from da = acc and the saved h: dh, recomputed a (bf16), dprob partials
   MXEPI_WGRAD = 3,      // K-grouped: out[e, m, n] = bf16(acc), zeros for an expert without rows
+  MXEPI_SWIGLU_F8 = 4,  // per-tensor FP8 fc1: a = SiLU(g) * u * p stored bf16 (+ bf16 h), max |a| kept
+  MXEPI_DSWIGLU_F8 = 5, // per-tensor FP8 fc2 dgrad: dh stored bf16, max |dh| kept, dprob partials
 };
+
+// fc1 epilogues (N tiles pair gate columns with their up columns)
+__host__ __device__ constexpr bool mx_swiglu(int epi) { return epi == MXEPI_SWIGLU_Q || epi == MXEPI_SWIGLU_F8; }
 
 struct MxGemmParams {
   GemmParams g;               // E, M (rows R), N (output cols), K, split_sizes, out, ldo, out2/ldo2 (h), probs, F
@@ -79,7 +84,28 @@ struct MxGemmParams {
   uint8_t* dh_cols_atoms;
   uint8_t* a_cols;
   uint8_t* a_cols_atoms;
+  // Per-tensor FP8 (the operands are E4M3 / E5M2 codes with one scale per tensor; their
+  // block scales are all 2^0): ab_fmt is OR-ed into every instruction descriptor (A's
+  // format at bit 7, B's at bit 10: 0 = E4M3, 1 = E5M2); with deq_a set, the epilogue
+  // multiplies the accumulator by 1 / (deq_a[0] * deq_b[e]) (M-grouped: B's scale per
+  // expert; K-grouped: deq_b[0]); amax_out collects max |x| of the bf16 output (fp32 bits).
+  uint32_t ab_fmt;
+  const float* deq_a;
+  const float* deq_b;
+  unsigned int* amax_out;
 };
+
+// 1 / (s_a s_b) of a per-tensor FP8 GEMM, 1 otherwise.
+__device__ __forceinline__ float mx_deq_factor(const MxGemmParams& mp, int e) {
+  return mp.deq_a ? 1.0f / (mp.deq_a[0] * mp.deq_b[e]) : 1.0f;
+}
+
+// max over the warp of a non-negative float, folded into *out (fp32 bits, atomicMax):
+// every lane of the warp must call this together.
+__device__ __forceinline__ void warp_amax_to(unsigned int* out, float v) {
+  const unsigned int m = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(out, m);
+}
 
 // E4M3 codes of 32 fp32 values (one lane's row) quantised along the 32 LANES of the warp:
 // for each column j the block maximum is the warp-wide max of |v[j]| (one redux: the bits
@@ -158,6 +184,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     // half), chunk 0 of acc1 (lower half); its owner drains it first, then signals
     const bool owner = acc ? (half == 0) : (half == 1);
     if (!owner) strip_done();
+    const float deq = mx_deq_factor(mp, EPI == MXEPI_WGRAD ? 0 : ti.e);
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
       const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
@@ -168,6 +195,13 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
       if (owner && it == 0) {
         tc_fence_before();
         strip_done();
+      }
+      if (mp.deq_a) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v0[i] = __float_as_uint(__uint_as_float(v0[i]) * deq);
+          v1[i] = __float_as_uint(__uint_as_float(v1[i]) * deq);
+        }
       }
       if (EPI == MXEPI_STORE && ok_row && n0 + c * 32 < p.N && p.row_token) {
         float* d = p.out32 + (long long)p.row_token[row] * p.ldo + n0 + c * 32;
@@ -315,6 +349,143 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
           row_ok ? su_word : 0u;
     }
     if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
+  } else if (EPI == MXEPI_DSWIGLU_F8) {
+    // per-tensor FP8 fc2 dgrad: da = acc / (s_dy s_w2[e]); dg = da p u SiLU'(g),
+    // du = da p SiLU(g), dp += da SiLU(g) u; dh stored in bf16 (its per-tensor scale needs
+    // the max over the whole tensor, kept in amax_out)
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
+    __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
+    const int n0 = ti.n_blk * BN;
+    const float deq = mx_deq_factor(mp, ti.e);
+    const bool owner = acc ? (half == 0) : (half == 1);
+    if (!owner) strip_done();
+    float dp = 0.f, amax = 0.f;
+#pragma unroll 1
+    for (int it = 0; it < 4; ++it) {
+      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      const int col = n0 + c * 32;
+      const bool cols_ok = row_ok && col < p.N;
+      uint4 gva[4], uva[4];
+      if (cols_ok) {
+        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + col);
+        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gva[i] = gp[i];
+          uva[i] = up[i];
+        }
+      }
+      uint32_t v0[16], v1[16];
+      tmem_ld_32x32b_x16(t_row + c * 32, v0);
+      tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
+      tmem_wait_ld();
+      if (owner && it == 0) {
+        tc_fence_before();
+        strip_done();
+      }
+      if (cols_ok) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int cc = col + 16 * hh;
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva + 2 * hh);
+          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva + 2 * hh);
+          uint4 og[2], ou[2];
+          uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
+          uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 gg2 = __bfloat1622float2(g2[i]);
+            const float2 uu2 = __bfloat1622float2(u2[i]);
+            const float gs[2] = {gg2.x, gg2.y}, us[2] = {uu2.x, uu2.y};
+            float dg[2], du[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float da = __uint_as_float(hh ? v1[2 * i + j] : v0[2 * i + j]) * deq;
+              const float sg = 1.0f / (1.0f + expf(-gs[j]));
+              const float sl = gs[j] * sg;
+              dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
+              du[j] = da * pr * sl;
+              dp = fmaf(da, sl * us[j], dp);
+            }
+            ogw[i] = pack_bf16x2(dg[0], dg[1]);
+            ouw[i] = pack_bf16x2(du[0], du[1]);
+            // the amax of what is stored (the bf16 values the quantiser will read)
+            const float2 rg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ogw[i]));
+            const float2 ru = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ouw[i]));
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(rg.x), fabsf(rg.y)), fmaxf(fabsf(ru.x), fabsf(ru.y))));
+          }
+          uint4* d0 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + cc);
+          uint4* d1 = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + cc);
+          d0[0] = og[0];
+          d0[1] = og[1];
+          d1[0] = ou[0];
+          d1[1] = ou[1];
+        }
+      }
+    }
+    warp_amax_to(mp.amax_out, amax);
+    if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
+  } else if (EPI == MXEPI_SWIGLU_F8) {
+    // per-tensor FP8 fc1: h = acc / (s_x s_w1[e]); a = SiLU(g) * u * p stored in bf16
+    // (its per-tensor scale needs the max over all of a, kept in amax_out), h in bf16
+    const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
+    const int n0 = ti.n_blk * 128;
+    const float deq = mx_deq_factor(mp, ti.e);
+    __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
+    const bool owner = acc ? (half == 0) : (half == 1);
+    if (!owner) strip_done();
+    float amax = 0.f;
+#pragma unroll 1
+    for (int it = 0; it < 2; ++it) {
+      const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
+      uint32_t g0[16], g1[16], u0[16], u1[16];
+      tmem_ld_32x32b_x16(t_row + c * 32, g0);
+      tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
+      tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
+      tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
+      tmem_wait_ld();
+      if (owner && it == 0) {
+        tc_fence_before();
+        strip_done();
+      }
+      if (row_ok) {
+        float g[32], u[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          g[i] = __uint_as_float(g0[i]) * deq;
+          g[16 + i] = __uint_as_float(g1[i]) * deq;
+          u[i] = __uint_as_float(u0[i]) * deq;
+          u[16 + i] = __uint_as_float(u1[i]) * deq;
+        }
+        uint4 oa[4], hg[4], hu[4];
+        uint32_t* oaw = reinterpret_cast<uint32_t*>(oa);
+        uint32_t* hgw = reinterpret_cast<uint32_t*>(hg);
+        uint32_t* huw = reinterpret_cast<uint32_t*>(hu);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          oaw[i] = pack_bf16x2(silu_f(g[2 * i]) * u[2 * i] * pr, silu_f(g[2 * i + 1]) * u[2 * i + 1] * pr);
+          const float2 ra = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&oaw[i]));
+          amax = fmaxf(amax, fmaxf(fabsf(ra.x), fabsf(ra.y)));
+          hgw[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+          huw[i] = pack_bf16x2(u[2 * i], u[2 * i + 1]);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(a_out + row * p.ldo + n0 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = oa[i];
+        if (hout) {
+          uint4* hd = reinterpret_cast<uint4*>(hout + row * p.ldo2 + n0 + c * 32);
+          uint4* hd2 = reinterpret_cast<uint4*>(hout + row * p.ldo2 + p.F + n0 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            hd[i] = hg[i];
+            hd2[i] = hu[i];
+          }
+        }
+      }
+    }
+    warp_amax_to(mp.amax_out, amax);
   } else {
     // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
@@ -412,7 +583,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
-  const int NT = (EPI == MXEPI_SWIGLU_Q) ? (p.N / 128) : (p.N + BN - 1) / BN;
+  const int NT = mx_swiglu(EPI) ? (p.N / 128) : (p.N + BN - 1) / BN;
   const int MT = KGROUP ? (p.M + BM - 1) / BM : 0;
 
   if (threadIdx.x == 0) {
@@ -500,7 +671,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
       for (int t = blockIdx.x; t < total && ok && !p.stall_loads; t += gridDim.x) {
         const TileInfo ti = walk.decode(t);
         const int num_kb = kblocks(ti);
-        const int n0 = (EPI == MXEPI_SWIGLU_Q) ? ti.n_blk * 128 : ti.n_blk * BN;
+        const int n0 = mx_swiglu(EPI) ? ti.n_blk * 128 : ti.n_blk * BN;
         size_t ga, gb0, gb1;   // first atom of A's and of B's two 128-row halves (k-group 0)
         if (KGROUP) {
           const size_t kg = (size_t)(ti.rows + BK - 1) / BK;
@@ -510,8 +681,8 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
         } else {
           ga = (size_t)(tile_off[ti.e] / NT + ti.m_blk) * KB4;          // A row group (expert tile)
           gb0 = ((size_t)ti.e * bgroups + n0 / 128) * KB4;
-          gb1 = ((size_t)ti.e * bgroups + (EPI == MXEPI_SWIGLU_Q ? (p.F + n0) / 128 : n0 / 128 + 1)) * KB4;
-          if (EPI != MXEPI_SWIGLU_Q && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
+          gb1 = ((size_t)ti.e * bgroups + (mx_swiglu(EPI) ? (p.F + n0) / 128 : n0 / 128 + 1)) * KB4;
+          if (!mx_swiglu(EPI) && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
         }
         for (int kb = 0; kb < num_kb; ++kb) {
           if ((kb & (kSfKb - 1)) == 0) {
@@ -548,7 +719,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
           } else {
             tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
             tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
-            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, EPI == MXEPI_SWIGLU_Q ? p.F + n0 : n0 + 128, ti.e);
+            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, mx_swiglu(EPI) ? p.F + n0 : n0 + 128, ti.e);
           }
           ++issued;
           if (++stage == kStages) {
@@ -639,7 +810,7 @@ __global__ void __launch_bounds__(mx::kThreads, 1)
                                           : make_sdesc(a_addr + kk * 32, 16, 1024, 2);
             const uint64_t bdesc = KGROUP ? make_sdesc(b_addr + kk * 4096, BM * BK, 1024, 2)
                                           : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
-            const uint32_t idesc = make_idesc_mxf8(BM, BN, KGROUP, KGROUP, kk, kk);
+            const uint32_t idesc = make_idesc_mxf8(BM, BN, KGROUP, KGROUP, kk, kk) | mp.ab_fmt;
             mma_mxf8_ss(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30),
                         (kb > 0 || kk > 0) ? 1u : 0u);
           }

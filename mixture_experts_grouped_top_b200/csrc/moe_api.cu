@@ -293,9 +293,79 @@ GemmParams base_params(const int32_t* split_sizes, int E) {
   return p;
 }
 
+// ---------------------------------------------------------------- per-tensor FP8
+int fp8_amax_launch(const void* in, int batch, long long n, unsigned int* amax, cudaStream_t st) {
+  if (cudaMemsetAsync(amax, 0, (size_t)batch * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const long long n8 = n / 8;
+  if (n8 == 0) return MOE_OK;
+  const int gx = (int)std::max<long long>(1, std::min<long long>((n8 + 255) / 256,
+                                                                 (long long)device_props().sm_count * 8 / batch + 1));
+  amax_bf16_kernel<<<dim3(gx, batch), 256, 0, st>>>(reinterpret_cast<const uint4*>(in), n8, amax);
+  count_launch();
+  return launch_status();
+}
+
+int fp8_scale_launch(const unsigned int* amax, int batch, int e5m2, float* scale, cudaStream_t st) {
+  fp8_scale_kernel<<<(batch + 255) / 256, 256, 0, st>>>(amax, batch, e5m2, scale);
+  count_launch();
+  return launch_status();
+}
+
+int fp8_cast_launch(const void* in, int batch, long long n, const float* scale, int e5m2, uint8_t* codes,
+                    cudaStream_t st) {
+  const long long n8 = n / 8;
+  if (n8 == 0) return MOE_OK;
+  const int gx = (int)std::max<long long>(1, std::min<long long>((n8 + 255) / 256,
+                                                                 (long long)device_props().sm_count * 8 / batch + 1));
+  fp8_cast_kernel<<<dim3(gx, batch), 256, 0, st>>>(reinterpret_cast<const uint4*>(in), n8, scale, e5m2,
+                                                    reinterpret_cast<uint2*>(codes));
+  count_launch();
+  return launch_status();
+}
+
+// amax, scale and codes of `batch` tensors of n bf16 each (codes in the input's layout)
+int fp8_quantize_launch(const void* in, int batch, long long n, int e5m2, uint8_t* codes, float* scale,
+                        unsigned int* amax, cudaStream_t st) {
+  int rc;
+  if ((rc = fp8_amax_launch(in, batch, n, amax, st))) return rc;
+  if ((rc = fp8_scale_launch(amax, batch, e5m2, scale, st))) return rc;
+  return fp8_cast_launch(in, batch, n, scale, e5m2, codes, st);
+}
+
+// Block-scale atoms of per-tensor FP8 operands: every scale byte 127 (2^0), enough for
+// every A and B operand of the layer's grouped GEMMs.
+size_t fp8_unit_atoms_bytes(int E, int R, int H, int F) {
+  const size_t a = ((size_t)R / 128 + (size_t)E) * (size_t)(std::max(H, 2 * F) / 128);
+  const size_t b = (size_t)E * (size_t)(2 * F / 128) * (size_t)(H / 128);
+  return align_up(std::max(a, b) * 512, 256);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t fp8_quantize_workspace_size(int batch) { return batch < 1 ? 0 : align_up((size_t)batch * 4, 256); }
+
+int fp8_quantize(const uint16_t* in, int batch, int rows, int cols, int fmt, int transpose_out, uint8_t* codes,
+                 float* scales, void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 1 || rows < 0 || cols < 0 || (fmt != 0 && fmt != 1)) return MOE_ERR_INVALID_ARG;
+  const long long n = (long long)rows * cols;
+  if (n == 0) return MOE_OK;
+  if (!in || !codes || !scales || !workspace) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < fp8_quantize_workspace_size(batch)) return MOE_ERR_INVALID_ARG;
+  if (transpose_out ? ((rows % 32) || (cols % 32)) : (n % 8)) return MOE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(in) & 15) || (reinterpret_cast<uintptr_t>(codes) & 7)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(workspace);
+  int rc;
+  if ((rc = fp8_amax_launch(in, batch, n, amax, st))) return rc;
+  if ((rc = fp8_scale_launch(amax, batch, fmt, scales, st))) return rc;
+  if (!transpose_out) return fp8_cast_launch(in, batch, n, scales, fmt, codes, st);
+  fp8_cast_transpose_kernel<<<dim3(cols / 32, rows / 32, batch), 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(in), rows, cols, scales, fmt, codes);
+  count_launch();
+  return launch_status();
+}
 
 const char* moe_status_string(int s) {
   switch (s) {
@@ -526,6 +596,78 @@ int moe_route_permute(const float* logits, const uint16_t* x, int T, int H, int 
   return permute_rows_from_counts(x, idx, prob, T, H, E, k, precision, xp, xp_scale, row_map, probs_perm, counts, st);
 }
 
+size_t moe_permute_capacity_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  const size_t R = (size_t)T * k;
+  return permute_counts_bytes(R, E) + align_up(R * 4, 256) + 2 * align_up(((size_t)E + 1) * 4, 256);
+}
+
+int moe_permute_capacity(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k, int C,
+                         int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
+                         int32_t* split_sizes, int32_t* offsets, int32_t* kept, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32 || H < 8 || C < 0) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_BF16 && (H % 8)) return MOE_ERR_UNSUPPORTED;
+  if (precision == MOE_MXFP8 && (H % 32)) return MOE_ERR_UNSUPPORTED;
+  if (probs_perm && !prob) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k, RC = (long long)E * C;
+  if (R > 0x7fffffffLL || RC > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (!split_sizes || !offsets || (T > 0 && (!x || !idx || !xp || !row_map || !workspace))) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_MXFP8 && T > 0 && !xp_scale) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe_permute_capacity_workspace_size(T, k, E)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 15) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  // the padded rows of every expert hold zeros (their outputs are never combined, and a
+  // backward through them contributes nothing to the weight gradients)
+  const size_t elem = precision == MOE_BF16 ? 2 : 1;
+  if (RC > 0 && cudaMemsetAsync(xp, 0, (size_t)RC * H * elem, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (RC > 0 && precision == MOE_MXFP8 && cudaMemsetAsync(xp_scale, 0, (size_t)RC * (H / 32), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (RC > 0 && probs_perm && cudaMemsetAsync(probs_perm, 0, (size_t)RC * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint8_t* w = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* counts = reinterpret_cast<int32_t*>(w);
+  int32_t* row_full = reinterpret_cast<int32_t*>(w + permute_counts_bytes((size_t)R, E));
+  int32_t* split_full = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(row_full) + align_up((size_t)R * 4, 256));
+  int32_t* off_full =
+      reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(split_full) + align_up(((size_t)E + 1) * 4, 256));
+  if (R == 0) {
+    if (cudaMemsetAsync(split_full, 0, E * sizeof(int32_t), st) != cudaSuccess ||
+        cudaMemsetAsync(off_full, 0, (E + 1) * sizeof(int32_t), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  } else {
+    // the dropless stable permutation's index (rows only: no data, no probabilities)
+    const int nblk = (int)((R + kPermuteChunk - 1) / kPermuteChunk);
+    permute_hist_kernel<<<nblk, kPermuteThreads, E * sizeof(int32_t), st>>>(idx, (int)R, E, counts);
+    const int P = std::max(1, 1024 / E);
+    permute_scan_kernel<<<1, 1024, (size_t)(P * E + E) * sizeof(int32_t), st>>>(counts, nblk, E, (int)R, split_full,
+                                                                                  off_full);
+    static std::once_flag once;
+    std::call_once(once, []() {
+      cudaFuncSetAttribute(permute_rowmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * kMaxExperts * 4);
+    });
+    permute_rowmap_kernel<<<nblk, kPermuteThreads, (size_t)(kPermuteThreads / 32) * E * sizeof(int32_t), st>>>(
+        idx, nullptr, (int)R, E, counts, row_full, nullptr);
+    count_launch(3);
+  }
+  const long long work = std::max<long long>(R, E);
+  const int cgrid = (int)std::min<long long>((work + 255) / 256, (long long)device_props().sm_count * 8);
+  capacity_rows_kernel<<<cgrid, 256, 0, st>>>(idx, row_full, split_full, off_full, prob, (int)R, E, C, row_map,
+                                              probs_perm, split_sizes, offsets, kept);
+  count_launch();
+  if (R > 0) {
+    const int grid = std::min((T + 7) / 8, device_props().sm_count * 8);
+    if (precision == MOE_BF16)
+      permute_rows_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), T, H / 8, k, row_map,
+                                                     reinterpret_cast<uint4*>(xp));
+    else
+      permute_rows_mxfp8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), T, H, k, row_map,
+                                                      reinterpret_cast<uint8_t*>(xp), xp_scale);
+    count_launch();
+  }
+  return launch_status();
+}
+
 int moe_unpermute(const uint16_t* yp, const int32_t* row_map, const float* prob, int T, int H, int k, uint16_t* out,
                   void* stream) {
   if (T < 0 || H < 8 || (H % 8) || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
@@ -587,6 +729,12 @@ size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int
   (void)E;
   (void)H;
   if (R < 0 || F < 0) return 0;
+  if (precision == MOE_FP8) {
+    // unit block scales, the max word, a in bf16; a's codes and scale unless in `saved`
+    size_t b = fp8_unit_atoms_bytes(E, R, H, F) + 256 + align_up((size_t)R * F * 2, 256);
+    if (!training) b += align_up((size_t)R * F, 256) + 256;
+    return b + 256;
+  }
   if (training && precision != MOE_MXFP8) return 256;  // `a` lives in the saved buffer
   if (precision == MOE_MXFP8) {
     // xp scale atoms, plus `a` codes and scale atoms unless they live in the saved buffer
@@ -601,6 +749,8 @@ size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision) {
   (void)E;
   (void)H;
   if (R < 0 || F < 0) return 0;
+  if (precision == MOE_FP8)   // h bf16, a's E4M3 codes, a's scale
+    return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F, 256) + 256;
   if (precision == MOE_MXFP8)
     return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F);
   return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
@@ -672,6 +822,79 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   return launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p2, st);
 }
 
+// Per-tensor FP8 forward: fc1 on E4M3 codes with unit block scales, the epilogue
+// rescales by 1 / (s_x s_w1[e]), stores a in bf16 and keeps max |a|; a is quantised with
+// one scale; fc2 on its codes, rescaled by 1 / (s_a s_w2[e]).
+int grouped_mlp_fwd_fp8(const void* xp, const float* xp_scale, const int32_t* split_sizes, int E, int R, int H, int F,
+                        const void* w1, const float* w1_scale, const void* w2, const float* w2_scale,
+                        const float* probs_perm, void* yp, int out_f32, void* saved, void* ws, cudaStream_t st,
+                        const int32_t* row_token, float* out32) {
+  if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  if (!xp_scale || !w1_scale || !w2_scale) return MOE_ERR_INVALID_ARG;
+  uint8_t* unit = reinterpret_cast<uint8_t*>(ws);
+  const size_t ub = fp8_unit_atoms_bytes(E, R, H, F);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(unit + ub);
+  uint16_t* a_bf = reinterpret_cast<uint16_t*>(unit + ub + 256);
+  uint8_t* a_codes = reinterpret_cast<uint8_t*>(a_bf) + align_up((size_t)R * F * 2, 256);
+  uint16_t* h_buf = nullptr;
+  if (saved) {
+    h_buf = reinterpret_cast<uint16_t*>(saved);
+    a_codes = reinterpret_cast<uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256);
+  }
+  float* a_scale = reinterpret_cast<float*>(a_codes + align_up((size_t)R * F, 256));
+  if (cudaMemsetAsync(unit, 127, ub, st) != cudaSuccess || cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  CUtensorMap ta, tb, tsa, tsb;
+  int rc;
+  // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xp, 1, R, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1, E, 2 * F, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_atoms(&tsa, unit, (uint64_t)R / 128 + E, H / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, unit, (uint64_t)E * 2 * F / 128, H / 128))) return rc;
+  MxGemmParams p1{};
+  p1.g = base_params(split_sizes, E);
+  p1.g.M = R;
+  p1.g.N = F;
+  p1.g.K = H;
+  p1.g.out = a_bf;
+  p1.g.ldo = F;
+  p1.g.out2 = h_buf;
+  p1.g.ldo2 = 2 * F;
+  p1.g.probs = probs_perm;
+  p1.g.F = F;
+  p1.a_atoms = unit;
+  p1.b_atoms = unit;
+  p1.b_rows = 2 * F;
+  p1.deq_a = xp_scale;
+  p1.deq_b = w1_scale;
+  p1.amax_out = amax;
+  if ((rc = launch_gemm_mx_pair<MXEPI_SWIGLU_F8>(ta, tb, tsa, tsb, p1, st))) return rc;
+  // a: one E4M3 scale over all rows
+  if ((rc = fp8_scale_launch(amax, 1, 0, a_scale, st))) return rc;
+  if ((rc = fp8_cast_launch(a_bf, 1, (long long)R * F, a_scale, 0, a_codes, st))) return rc;
+  // fc2: A = a codes [R, F], B = w2 codes [E, H, F]
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, 1, R, F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, E, H, F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_atoms(&tsa, unit, (uint64_t)R / 128 + E, F / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, unit, (uint64_t)E * H / 128, F / 128))) return rc;
+  MxGemmParams p2{};
+  p2.g = base_params(split_sizes, E);
+  p2.g.M = R;
+  p2.g.N = H;
+  p2.g.K = F;
+  p2.g.out = yp;
+  p2.g.ldo = H;
+  p2.g.out_f32 = out_f32;
+  p2.g.row_token = row_token;
+  p2.g.out32 = out32;
+  p2.a_atoms = unit;
+  p2.b_atoms = unit;
+  p2.b_rows = H;
+  p2.deq_a = a_scale;
+  p2.deq_b = w2_scale;
+  return launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p2, st);
+}
+
 // The forward; with row_token, fc2's rows are added into out32[row_token[r]] (fused
 // combine) instead of being stored to yp.
 int grouped_mlp_fwd_impl(const void* xp, const uint8_t* xp_scale, const int32_t* split_sizes, int E, int R, int H,
@@ -681,12 +904,16 @@ int grouped_mlp_fwd_impl(const void* xp, const uint8_t* xp_scale, const int32_t*
   const int out_f32 = (precision & MOE_OUT_F32) ? 1 : 0;
   precision &= ~MOE_OUT_F32;
   if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
-  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8 && precision != MOE_FP8) return MOE_ERR_INVALID_ARG;
   if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
   if (R == 0) return MOE_OK;
   if (!xp || !split_sizes || !w1 || !w2 || (!yp && !row_token) || !ws) return MOE_ERR_INVALID_ARG;
   const int training = saved != nullptr;
   if (ws_bytes < grouped_mlp_workspace_size(E, R, H, F, precision, training)) return MOE_ERR_INVALID_ARG;
+  if (precision == MOE_FP8)
+    return grouped_mlp_fwd_fp8(xp, reinterpret_cast<const float*>(xp_scale), split_sizes, E, R, H, F, w1,
+                               reinterpret_cast<const float*>(w1_scale), w2, reinterpret_cast<const float*>(w2_scale),
+                               probs_perm, yp, out_f32, saved, ws, st, row_token, out32);
   if (precision == MOE_MXFP8)
     return grouped_mlp_fwd_mxfp8(xp, xp_scale, split_sizes, E, R, H, F, w1, w1_scale, w2, w2_scale, probs_perm, yp,
                                  out_f32, saved, ws, st, row_token, out32);
@@ -791,6 +1018,22 @@ namespace {
 // (Part 1 is no longer used: the MXFP8 fc2-dgrad epilogue quantises a and dh itself.)
 size_t bwd_part_bytes(int part, int E, int R, int H, int F, int precision) {
   const size_t r = (size_t)R, e = (size_t)E, h = (size_t)H, f = (size_t)F;
+  if (precision == MOE_FP8) {
+    // 0 dh bf16; 2 dprob partials; 3 w2 codes [E, F, H] + E scales; 4 w1 codes
+    // [E, H, 2F] + E scales; 5 dy codes [R, H] + scale; 8 dh codes [R, 2F] + scale;
+    // 10 xp codes [R, H] + scale; 11 max words + unit block scales
+    switch (part) {
+      case 0: return align_up(r * 2 * f * 2, 256);
+      case 2: return align_up((size_t)(2 * ((F + gg::BN - 1) / gg::BN)) * r * 4, 256);
+      case 3: return align_up(e * f * h, 256) + align_up(e * 4, 256);
+      case 4: return align_up(e * h * 2 * f, 256) + align_up(e * 4, 256);
+      case 5: return align_up(r * h, 256) + 256;
+      case 8: return align_up(r * 2 * f, 256) + 256;
+      case 10: return align_up(r * h, 256) + 256;
+      case 11: return align_up(e * 4 + 16, 256) + fp8_unit_atoms_bytes(E, R, H, F);
+      default: return 0;
+    }
+  }
   const bool mx = precision == MOE_MXFP8;
   switch (part) {
     case 0: return mx ? 0 : align_up(r * 2 * f * 2, 256);
@@ -819,18 +1062,148 @@ extern "C" {
 
 size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision) {
   if (R < 0 || F < 0 || E < 1) return 0;
-  return bwd_part_offset(11, E, R, H, F, precision) + 256;
+  return bwd_part_offset(12, E, R, H, F, precision) + 256;
 }
 
 size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part) {
   if (R < 0 || F < 0 || E < 1) return (size_t)-1;
-  const bool ok = precision == MOE_MXFP8 ? (part >= 7 && part <= 9) : part == 0;
+  const bool ok = precision == MOE_MXFP8 ? (part >= 7 && part <= 9)
+                  : precision == MOE_FP8 ? (part == 0 || part == 8)
+                                         : part == 0;
   return ok ? bwd_part_offset(part, E, R, H, F, precision) : (size_t)-1;
 }
 
 }  // extern "C"
 
 namespace {
+
+// Per-tensor FP8 backward: dy and dh in E5M2 (one scale each), xp, the saved a and the
+// weights (one scale per expert) in E4M3; per-tensor codes serve both orientations, so
+// the weight-gradient GEMMs read the same code arrays MN-major.
+int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
+                        const void* w1, const void* w2, const float* probs_perm, const void* saved, uint16_t* dxp,
+                        uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws, cudaStream_t st) {
+  if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  auto part = [&](int i) { return base + bwd_part_offset(i, E, R, H, F, MOE_FP8); };
+  uint16_t* dh = reinterpret_cast<uint16_t*>(part(0));
+  float* dpart = reinterpret_cast<float*>(part(2));
+  const size_t efh = (size_t)E * F * H;
+  uint8_t* w2q = part(3);
+  float* s_w2 = reinterpret_cast<float*>(w2q + align_up(efh, 256));
+  uint8_t* w1q = part(4);
+  float* s_w1 = reinterpret_cast<float*>(w1q + align_up(efh * 2, 256));
+  uint8_t* dyq = part(5);
+  float* s_dy = reinterpret_cast<float*>(dyq + align_up((size_t)R * H, 256));
+  uint8_t* dhq = part(8);
+  float* s_dh = reinterpret_cast<float*>(dhq + align_up((size_t)R * 2 * F, 256));
+  uint8_t* xq = part(10);
+  float* s_x = reinterpret_cast<float*>(xq + align_up((size_t)R * H, 256));
+  unsigned int* amax = reinterpret_cast<unsigned int*>(part(11));           // [E] (+ one for dh)
+  uint8_t* unit = part(11) + align_up((size_t)E * 4 + 16, 256);
+  const uint8_t* a_codes = reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256);
+  const float* a_scale = reinterpret_cast<const float*>(a_codes + align_up((size_t)R * F, 256));
+  const uint16_t* h_saved = reinterpret_cast<const uint16_t*>(saved);
+  const int nparts = 2 * ((F + gg::BN - 1) / gg::BN);
+  const uint32_t A_E5M2 = 1u << 7, B_E5M2 = 1u << 10;
+  int rc;
+  if (cudaMemsetAsync(unit, 127, fp8_unit_atoms_bytes(E, R, H, F), st) != cudaSuccess) return MOE_ERR_CUDA;
+  // operands: weights per expert (their own layout: K-major for the data gradients),
+  // dy and xp over all rows
+  if ((rc = fp8_quantize_launch(w2, E, (long long)F * H, 0, w2q, s_w2, amax, st))) return rc;
+  if ((rc = fp8_quantize_launch(w1, E, (long long)H * 2 * F, 0, w1q, s_w1, amax, st))) return rc;
+  if ((rc = fp8_quantize_launch(dy_perm, 1, (long long)R * H, 1, dyq, s_dy, amax, st))) return rc;
+  if ((rc = fp8_quantize_launch(xp, 1, (long long)R * H, 0, xq, s_x, amax, st))) return rc;
+  CUtensorMap ta, tb, tsa, tsb;
+  // fc2 dgrad + SwiGLU backward: A = dy (E5M2) [R, H], B = w2 (E4M3) [E, F, H]; dh bf16
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyq, 1, R, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2q, E, F, H, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_atoms(&tsa, unit, (uint64_t)R / 128 + E, H / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, unit, (uint64_t)E * F / 128, H / 128))) return rc;
+  if (cudaMemsetAsync(amax, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  MxGemmParams p{};
+  p.g = base_params(split_sizes, E);
+  p.g.M = R;
+  p.g.N = F;
+  p.g.K = H;
+  p.g.out2 = dh;
+  p.g.ldo2 = 2 * F;
+  p.g.aux = h_saved;
+  p.g.ld_aux = 2 * F;
+  p.g.probs = probs_perm;
+  p.g.dprob_part = dpart;
+  p.g.F = F;
+  p.a_atoms = unit;
+  p.b_atoms = unit;
+  p.b_rows = F;
+  p.ab_fmt = A_E5M2;
+  p.deq_a = s_dy;
+  p.deq_b = s_w2;
+  p.amax_out = amax;
+  if ((rc = launch_gemm_mx_pair<MXEPI_DSWIGLU_F8>(ta, tb, tsa, tsb, p, st))) return rc;
+  if (dprobs_perm) {
+    const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
+    reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
+    count_launch();
+    if ((rc = launch_status())) return rc;
+  }
+  // dh: one E5M2 scale
+  if ((rc = fp8_scale_launch(amax, 1, 1, s_dh, st))) return rc;
+  if ((rc = fp8_cast_launch(dh, 1, (long long)R * 2 * F, s_dh, 1, dhq, st))) return rc;
+  // fc2 wgrad: dw2[e] = a_e^T dy_e, A = a codes (E4M3) [R, F], B = dy codes (E5M2) [R, H]
+  if ((rc = tmap_u8_3d(&ta, a_codes, 1, R, F, mx::BM))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyq, 1, R, H, 1, mx::BK, 2))) return rc;
+  p = MxGemmParams{};
+  p.g = base_params(split_sizes, E);
+  p.g.M = F;
+  p.g.N = H;
+  p.g.out = dw2;
+  p.g.ldo = H;
+  p.g.out_batch = (long long)F * H;
+  p.a_atoms = unit;
+  p.b_atoms = unit;
+  p.b_rows = H;
+  p.ab_fmt = B_E5M2;
+  p.deq_a = a_scale;
+  p.deq_b = s_dy;
+  if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
+  // fc1 dgrad: dxp = dh w1[e]^T, A = dh codes (E5M2) [R, 2F], B = w1 codes [E, H, 2F]
+  if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhq, 1, R, 2 * F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1, 128, mx2::kChunks))) return rc;
+  if ((rc = tmap_atoms(&tsa, unit, (uint64_t)R / 128 + E, 2 * F / 128))) return rc;
+  if ((rc = tmap_atoms(&tsb, unit, (uint64_t)E * H / 128, 2 * F / 128))) return rc;
+  p = MxGemmParams{};
+  p.g = base_params(split_sizes, E);
+  p.g.M = R;
+  p.g.N = H;
+  p.g.K = 2 * F;
+  p.g.out = dxp;
+  p.g.ldo = H;
+  p.a_atoms = unit;
+  p.b_atoms = unit;
+  p.b_rows = H;
+  p.ab_fmt = A_E5M2;
+  p.deq_a = s_dh;
+  p.deq_b = s_w1;
+  if ((rc = launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p, st))) return rc;
+  // fc1 wgrad: dw1[e] = xp_e^T dh_e, A = xp codes (E4M3) [R, H], B = dh codes (E5M2)
+  if ((rc = tmap_u8_3d(&ta, xq, 1, R, H, mx::BM))) return rc;
+  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhq, 1, R, 2 * F, 1, mx::BK, 2))) return rc;
+  p = MxGemmParams{};
+  p.g = base_params(split_sizes, E);
+  p.g.M = H;
+  p.g.N = 2 * F;
+  p.g.out = dw1;
+  p.g.ldo = 2 * F;
+  p.g.out_batch = (long long)H * 2 * F;
+  p.a_atoms = unit;
+  p.b_atoms = unit;
+  p.b_rows = 2 * F;
+  p.ab_fmt = B_E5M2;
+  p.deq_a = s_x;
+  p.deq_b = s_dh;
+  return launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st);
+}
 
 int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
                           const void* xp, const void* w1, const void* w2, const float* probs_perm, const void* saved,
@@ -958,7 +1331,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
                     void* stream) {
   if (E < 1 || E > gg::kMaxE || R < 0 || H < 64 || F < 128) return MOE_ERR_INVALID_ARG;
   if ((H % 64) || (F % 128)) return MOE_ERR_UNSUPPORTED;
-  if (precision != MOE_BF16 && precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (precision != MOE_BF16 && precision != MOE_MXFP8 && precision != MOE_FP8) return MOE_ERR_INVALID_ARG;
   if (!split_sizes || !w1 || !w2 || !dw1 || !dw2) return MOE_ERR_INVALID_ARG;
   if (R > 0 && (!dy_perm || !xp || !saved || !dxp || !ws)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < grouped_mlp_bwd_workspace_size(E, R, H, F, precision)) return MOE_ERR_INVALID_ARG;
@@ -972,6 +1345,9 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   if (precision == MOE_MXFP8)
     return grouped_mlp_bwd_mxfp8(dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
                                  dprobs_perm, ws, st);
+  if (precision == MOE_FP8)
+    return grouped_mlp_bwd_fp8(dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
+                               dprobs_perm, ws, st);
   const uint16_t* h_buf = reinterpret_cast<const uint16_t*>(saved);
   const uint16_t* a_buf =
       reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256));

@@ -379,6 +379,129 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_rowmap_kernel(const i
   }
 }
 
+// Capacity-padded dispatch: slot s of expert e, ranked `rank` among that expert's slots in
+// slot order (the stable permutation's row minus the expert's offset), goes to row
+// e * C + rank of the padded [E * C] layout if rank < C, else it is dropped (row -1).
+// Threads e < E also write the padded layout's split sizes (all C), offsets and the
+// number of slots each expert kept.
+__global__ void __launch_bounds__(256) capacity_rows_kernel(const int32_t* __restrict__ idx,
+                                                            const int32_t* __restrict__ row_map_full,
+                                                            const int32_t* __restrict__ split_full,
+                                                            const int32_t* __restrict__ offsets_full,
+                                                            const float* __restrict__ prob, int R, int E, int C,
+                                                            int32_t* __restrict__ row_map, float* __restrict__ probs_perm,
+                                                            int32_t* __restrict__ split_sizes,
+                                                            int32_t* __restrict__ offsets, int32_t* __restrict__ kept) {
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int s = tid; s < R; s += gridDim.x * blockDim.x) {
+    const int e = idx[s];
+    const int r = row_map_full[s];
+    if (e < 0 || e >= E || r < 0) {
+      row_map[s] = -1;
+      continue;
+    }
+    const int rank = r - offsets_full[e];
+    if (rank < C) {
+      const int row = e * C + rank;
+      row_map[s] = row;
+      if (probs_perm) probs_perm[row] = prob[s];
+    } else {
+      row_map[s] = -1;
+    }
+  }
+  if (tid < E) {
+    split_sizes[tid] = C;
+    offsets[tid] = tid * C;
+    if (kept) kept[tid] = min(split_full[tid], C);
+    if (tid == E - 1) offsets[E] = E * C;
+  }
+}
+
+// ------------------------------------------------------------- per-tensor FP8
+// Current scaling: one scale per tensor (a batch of tensors: one per blockIdx.y), s =
+// fmt_max / max |x| in fp32 (1 for an all-zero tensor), codes = the fp32 product x * s
+// rounded to E4M3 or E5M2 (nearest even, saturating).
+__device__ __forceinline__ float fp8_max(int e5m2) { return e5m2 ? 57344.0f : 448.0f; }
+
+// max |x| of each tensor (n8 groups of 8 bf16 per tensor) into amax_bits[b] (fp32 bits;
+// zero before the launch).
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict__ in, long long n8,
+                                                        unsigned int* __restrict__ amax_bits) {
+  const uint4* src = in + (long long)blockIdx.y * n8;
+  float m = 0.f;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(src + i);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  const unsigned int r = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0 && r) atomicMax(amax_bits + blockIdx.y, r);
+}
+
+// scale[b] = fmt_max / amax[b] in fp32 (1 when amax is 0).
+__global__ void fp8_scale_kernel(const unsigned int* __restrict__ amax_bits, int batch, int e5m2,
+                                 float* __restrict__ scale) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+    const float a = __uint_as_float(amax_bits[b]);
+    scale[b] = a > 0.f ? fp8_max(e5m2) / a : 1.0f;
+  }
+}
+
+__device__ __forceinline__ uint32_t fp8_pack4(float a, float b, float c, float d, int e5m2) {
+  const __nv_fp8_interpretation_t f = e5m2 ? __NV_E5M2 : __NV_E4M3;
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, f) |
+         ((uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, f) << 16);
+}
+
+// codes of each tensor (n8 groups of 8 per tensor, blockIdx.y = tensor) with its scale.
+__global__ void __launch_bounds__(256) fp8_cast_kernel(const uint4* __restrict__ in, long long n8,
+                                                       const float* __restrict__ scale, int e5m2,
+                                                       uint2* __restrict__ codes) {
+  const uint4* src = in + (long long)blockIdx.y * n8;
+  uint2* dst = codes + (long long)blockIdx.y * n8;
+  const float s = scale[blockIdx.y];
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(src + i);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 p = __bfloat1622float2(h[j]);
+      f[2 * j] = p.x * s;
+      f[2 * j + 1] = p.y * s;
+    }
+    dst[i] = make_uint2(fp8_pack4(f[0], f[1], f[2], f[3], e5m2), fp8_pack4(f[4], f[5], f[6], f[7], e5m2));
+  }
+}
+
+// The same with the output transposed: in [b][rows][cols] -> codes [b][cols][rows]
+// (rows, cols multiples of 32). A block moves a 32 x 32 tile through shared memory.
+__global__ void __launch_bounds__(256) fp8_cast_transpose_kernel(const __nv_bfloat16* __restrict__ in, int rows,
+                                                                 int cols, const float* __restrict__ scale, int e5m2,
+                                                                 uint8_t* __restrict__ codes) {
+  __shared__ float tile[32][33];
+  const int b = blockIdx.z;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const float s = scale[b];
+  const __nv_bfloat16* src = in + (size_t)b * rows * cols;
+  uint8_t* dst = codes + (size_t)b * rows * cols;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty + 8 * i;
+    tile[r][tx] = __bfloat162float(src[(size_t)(r0 + r) * cols + c0 + tx]) * s;
+  }
+  __syncthreads();
+  // thread (ty, tx/4...): each of the 256 threads writes 4 consecutive codes of one output row
+  const int orow = threadIdx.x >> 3, oc = (threadIdx.x & 7) * 4;   // output row = input column
+  const uint32_t w = fp8_pack4(tile[oc][orow], tile[oc + 1][orow], tile[oc + 2][orow], tile[oc + 3][orow], e5m2);
+  *reinterpret_cast<uint32_t*>(dst + (size_t)(c0 + orow) * rows + r0 + oc) = w;
+}
+
 // ------------------------------------------------------------ permutation data
 // xp[row_map[t*k + j]] = x[t] for j < k. One warp per token, 16-byte vectors.
 __global__ void __launch_bounds__(256) permute_rows_bf16_kernel(const uint4* __restrict__ x, int T, int H8, int k,

@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (BF16, MXFP8, _PREC, grouped_mlp_bwd, grouped_mlp_bwd_workspace_size, grouped_mlp_fwd,
+from . import (BF16, FP8, MXFP8, _PREC, fp8_quantize, grouped_mlp_bwd, grouped_mlp_bwd_workspace_size, grouped_mlp_fwd,
                grouped_mlp_fwd_combine, grouped_mlp_fwd_combine_workspace_size, grouped_mlp_saved_size, grouped_mlp_workspace_size, moe_gather_slots, moe_permute_rows,
                moe_permute_workspace_size, moe_route_bwd, moe_route_permute, moe_unpermute, mxfp8_quantize)
 
@@ -21,7 +21,9 @@ class MoEExpertLayer:
         self.T, self.H, self.F, self.E, self.k = T, H, F, E, k
         self.R = T * k
         self.prec = _PREC[precision]
-        self.precision = "bf16" if self.prec == BF16 else "mxfp8"
+        self.precision = {BF16: "bf16", MXFP8: "mxfp8", FP8: "fp8"}[self.prec]
+        # the permutation moves bf16 rows except for MXFP8, whose permute quantises them
+        self.perm_precision = "mxfp8" if self.prec == MXFP8 else "bf16"
         self.training = training
         self.renorm = renorm
         # fused_combine: fc2's epilogue adds its rows into the token outputs (no yp)
@@ -33,7 +35,7 @@ class MoEExpertLayer:
         self.idx = torch.empty((T, k), dtype=i32, device=dev)
         self.prob = torch.empty((T, k), dtype=f32, device=dev)
         self.perm = {
-            "xp": torch.empty((R, H), dtype=bf if self.prec == BF16 else u8, device=dev),
+            "xp": torch.empty((R, H), dtype=u8 if self.prec == MXFP8 else bf, device=dev),
             "row_map": torch.empty(R, dtype=i32, device=dev),
             "probs_perm": torch.empty(R, dtype=f32, device=dev),
             "split_sizes": torch.empty(E, dtype=i32, device=dev),
@@ -41,6 +43,10 @@ class MoEExpertLayer:
         }
         if self.prec == MXFP8:
             self.perm["xp_scale"] = torch.empty((R, H // 32), dtype=u8, device=dev)
+        if self.prec == FP8:
+            # per-tensor E4M3 codes of the permuted rows and their scale
+            self.xq = torch.empty((R, H), dtype=u8, device=dev)
+            self.xq_scale = torch.empty(1, dtype=f32, device=dev)
         self.perm_ws = torch.empty(max(moe_permute_workspace_size(T, k, E), 1), dtype=u8, device=dev)
         self.yp = None if fused_combine else torch.empty((R, H), dtype=bf, device=dev)
         self.out = torch.empty((T, H), dtype=bf, device=dev)
@@ -61,6 +67,10 @@ class MoEExpertLayer:
         self.w1_master, self.w2_master = w1, w2
         if self.prec == BF16:
             self.w1, self.w2 = w1, w2
+        elif self.prec == FP8:
+            # one E4M3 scale per expert, codes K-major for the forward GEMMs
+            self.w1, self.w1_scale = fp8_quantize(w1, "e4m3", transpose_out=True, stream=stream)
+            self.w2, self.w2_scale = fp8_quantize(w2, "e4m3", transpose_out=True, stream=stream)
         else:
             self.w1, self.w1_scale = mxfp8_quantize(w1, axis=1, transpose_out=True, mma_scales=True, stream=stream)
             self.w2, self.w2_scale = mxfp8_quantize(w2, axis=1, transpose_out=True, mma_scales=True, stream=stream)
@@ -68,18 +78,22 @@ class MoEExpertLayer:
     # --------------------------------------------------------------- forward
     def forward(self, x: torch.Tensor, logits: torch.Tensor, stream=None) -> torch.Tensor:
         self.perm["idx"], self.perm["prob"] = self.idx, self.prob
-        moe_route_permute(logits, x, self.k, self.renorm, self.precision, out=self.perm, workspace=self.perm_ws,
-                          stream=stream)
+        moe_route_permute(logits, x, self.k, self.renorm, self.perm_precision, out=self.perm,
+                          workspace=self.perm_ws, stream=stream)
         self.logits = logits
+        xp, xp_scale = self.perm["xp"], self.perm.get("xp_scale")
+        if self.prec == FP8:
+            fp8_quantize(self.perm["xp"], "e4m3", codes=self.xq, scales=self.xq_scale, stream=stream)
+            xp, xp_scale = self.xq, self.xq_scale
         if self.fused_combine:
-            grouped_mlp_fwd_combine(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2,
+            grouped_mlp_fwd_combine(xp, self.perm["split_sizes"], self.w1, self.w2,
                                     self.perm["probs_perm"], self.perm["row_map"], self.T, self.k, self.precision,
-                                    xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
+                                    xp_scale=xp_scale, w1_scale=self.w1_scale,
                                     w2_scale=self.w2_scale, out=self.out, saved=self.saved, workspace=self.mlp_ws,
                                     F=self.F, stream=stream)
         else:
-            grouped_mlp_fwd(self.perm["xp"], self.perm["split_sizes"], self.w1, self.w2, self.perm["probs_perm"],
-                            self.precision, xp_scale=self.perm.get("xp_scale"), w1_scale=self.w1_scale,
+            grouped_mlp_fwd(xp, self.perm["split_sizes"], self.w1, self.w2, self.perm["probs_perm"],
+                            self.precision, xp_scale=xp_scale, w1_scale=self.w1_scale,
                             w2_scale=self.w2_scale, yp=self.yp, saved=self.saved, workspace=self.mlp_ws, F=self.F,
                             stream=stream)
             moe_unpermute(self.yp, self.perm["row_map"], self.T, self.k, out=self.out, stream=stream)
@@ -119,7 +133,7 @@ class MoEExpertLayer:
             self._alloc_bwd()
         b = self._bwd
         moe_permute_rows(grad_out, self.perm["row_map"], self.k, out=b["dy_perm"], stream=stream)
-        xp = self.perm["xp"] if self.prec == BF16 else self.xp_bf16
+        xp = self.xp_bf16 if self.prec == MXFP8 else self.perm["xp"]
         grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], xp, self.w1_master, self.w2_master,
                         self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"], dw1=b["dw1"],
                         dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream)
@@ -130,6 +144,23 @@ class MoEExpertLayer:
                           dlogits=b["dlogits"], stream=stream)
         self.dlogits = b["dlogits"] if router else None
         return b["dx"], b["dw1"], b["dw2"], b["dprob"]
+
+    def allreduce_weight_grads(self, group=None, average: bool = False):
+        """Sum (or average) dw1 and dw2 of the last backward over the data-parallel group."""
+        return allreduce_grads([self._bwd["dw1"], self._bwd["dw2"]], group=group, average=average)
+
+
+def allreduce_grads(tensors, group=None, average: bool = False):
+    """The data-parallel backward's one exchange: sum (or average) gradients over the
+    replicas of `group` in place with torch.distributed (NCCL over NVLink on GPUs, gloo on
+    CPU), one all-reduce per tensor, enqueued on the current stream."""
+    import torch.distributed as dist
+    n = dist.get_world_size(group)
+    for t in tensors:
+        dist.all_reduce(t, group=group)
+        if average and n > 1:
+            t.div_(n)
+    return tensors
 
 
 def moe_layer_forward(x, logits, w1, w2, k: int, precision="bf16", stream=None):
