@@ -598,6 +598,8 @@ def run_ours(args, world, rank, local):
     cfg = workloads.CONFIGS[args.workload]
     if args.tokens:
         cfg = dataclasses.replace(cfg, name=f"{cfg.name}_T{args.tokens}", T=args.tokens)
+    if args.ffn:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_F{args.ffn}", F=args.ffn)
     head, d = run_workload(cfg, args, world, rank, local, args.steps, args.warmup, with_e2e=True)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -614,7 +616,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": head["gpu_launches"], "roofline": head["roofline"], "bandwidth": head["bandwidth"],
         "clocks": head["clocks"], "cpu_baseline": cpu,
     }
-    if not args.no_workloads and not args.tokens:
+    if not args.no_workloads and not args.tokens and not args.ffn:
         line["workloads"] = {}
         for name in SECONDARY_WORKLOADS:
             if name == cfg.name:
@@ -655,6 +657,7 @@ def main(argv=None):
     ap.add_argument("--workload-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs on a smaller batch)")
+    ap.add_argument("--ffn", type=int, default=0, help="override F (profiling runs on smaller experts)")
     ap.add_argument("--cpu-baseline-tokens", type=int, default=48)
     ap.add_argument("--reference-tokens", type=int, default=32)
     ap.add_argument("--clocks-csv", default=None,

@@ -324,6 +324,14 @@ MOE_API size_t fp8_quantize_workspace_size(int batch);
 MOE_API int fp8_quantize(const uint16_t* in, int batch, int rows, int cols, int fmt, int transpose_out, uint8_t* codes,
                          float* scales, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Byte offset inside grouped_mlp_fwd's `saved` buffer of one of its parts ((size_t)-1
+ * for a part the precision does not have): part 0 = h [R, 2F] bf16 (all precisions);
+ * MOE_BF16 part 1 = a [R, F] bf16; MOE_MXFP8 part 1 = a codes along F [R, F], 2 = their
+ * scale atoms (row groups = the experts' 128-row tiles), 3 = a codes along the expert's
+ * rows [R, F] (the fc2 weight-gradient operand), 4 = their atoms (the layout of
+ * mxfp8_quantize_grouped); MOE_FP8 part 1 = a E4M3 codes [R, F], 2 = a's fp32 scale. */
+MOE_API size_t grouped_mlp_saved_offset(int E, int R, int H, int F, int precision, int part);
+
 /* Bytes of scratch grouped_mlp_fwd_combine needs: grouped_mlp_fwd's workspace, then an
  * fp32 [T, H] accumulator and the token of every row. */
 MOE_API size_t grouped_mlp_fwd_combine_workspace_size(int E, int R, int H, int F, int precision, int training,
@@ -355,15 +363,13 @@ MOE_API size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int pr
 /* Byte offset, inside grouped_mlp_bwd's workspace, of one intermediate of the last call
  * (valid after it completes; (size_t)-1 for a part the precision does not have):
  *   MOE_BF16  part 0: dh = [dg | du] [R, 2F] bf16;
- *   MOE_MXFP8 part 7: the recomputed a quantised along the expert's rows: codes [R, F],
- *             then (256-byte aligned) its scale atoms in the layout of
- *             mxfp8_quantize_grouped;
- *             part 8: dh quantised along its 2F columns: codes [R, 2F], then scale atoms
+ *   MOE_MXFP8 part 8: dh quantised along its 2F columns: codes [R, 2F], then scale atoms
  *             grouped per 128-row expert tile (row group sum_{e'<e} ceil(n_e'/128) + m
  *             for rows [off_e + 128 m, +128); atom j of a group = k-blocks 4j..4j+3,
  *             row r at 32-bit word (r % 32) * 4 + r / 32; rows past the expert: zeros);
- *             part 9: dh quantised along the expert's rows: codes [R, 2F], then atoms as
- *             part 7. */
+ *             part 9: dh quantised along the expert's rows: codes [R, 2F], then atoms in
+ *             the layout of mxfp8_quantize_grouped;
+ *   MOE_FP8   part 8: dh E5M2 codes [R, 2F], then (256-byte aligned) its fp32 scale. */
 MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part);
 
 /*
@@ -386,9 +392,9 @@ MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int 
  * axis (blocks of 32): dy and dh along columns for the data gradients, and dy, a
  * (recomputed from h), dh and xp along rows — in 32-row blocks restarting at every
  * expert's first row — for the weight gradients; the weights are re-quantised along
- * their other axis. dh and a are quantised (both ways) by the fc2-dgrad kernel that
- * computes them, from fp32; they never exist at 16 bits. Requires H % 128 == 0 for
- * MOE_MXFP8.
+ * their other axis. dh is quantised (both ways) by the fc2-dgrad kernel that computes
+ * it, from fp32, and never exists at 16 bits; a along rows comes from the forward (its
+ * fc1 epilogue quantises a both ways in training). Requires H % 128 == 0 for MOE_MXFP8.
  */
 MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
                             const void* xp, const void* w1, const void* w2, const float* probs_perm, int precision,

@@ -332,6 +332,10 @@ def grouped_mlp_saved_size(E, R, H, F, precision="bf16") -> int:
     return int(lib().grouped_mlp_saved_size(E, R, H, F, _PREC[precision]))
 
 
+def grouped_mlp_saved_offset(E, R, H, F, precision, part) -> int:
+    return int(lib().grouped_mlp_saved_offset(E, R, H, F, _PREC[precision], part))
+
+
 def grouped_mlp_fwd(xp, split_sizes, w1, w2, probs_perm=None, precision="bf16", xp_scale=None, w1_scale=None,
                     w2_scale=None, yp=None, saved=None, training=False, workspace=None, F=None, out_f32=False,
                     stream=None):

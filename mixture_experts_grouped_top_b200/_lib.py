@@ -34,6 +34,7 @@ SIGNATURES = {
     "fp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "grouped_mlp_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "grouped_mlp_saved_size": (_sz, [_i, _i, _i, _i, _i]),
+    "grouped_mlp_saved_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
     "grouped_mlp_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "grouped_mlp_fwd_combine_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "grouped_mlp_fwd_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _vp, _vp,

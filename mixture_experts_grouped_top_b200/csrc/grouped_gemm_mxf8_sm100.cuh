@@ -229,12 +229,13 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     }
   } else if (EPI == MXEPI_DSWIGLU) {
     // acc = da for columns [n0, n0+256) of F. With h = [g | u] from the forward:
-    // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u, and a = SiLU(g) u p
-    // recomputed. All three are quantised here from fp32 into the operands of the GEMMs
-    // that follow (see MxGemmParams): dh along its columns (this row's 32-column blocks),
-    // dh and a along the expert's rows (32-row blocks = this warp's lanes: a pair tile
-    // starts at a multiple of 256 rows of its expert, so the blocks restart at every
-    // expert; lanes past the expert's end count as zeros).
+    // dg = da p u SiLU'(g), du = da p SiLU(g), dp += da SiLU(g) u. dh = [dg | du] is
+    // quantised here from fp32 into the operands of the GEMMs that follow (see
+    // MxGemmParams): along its columns (this row's 32-column blocks) and along the
+    // expert's rows (32-row blocks = this warp's lanes: a pair tile starts at a multiple
+    // of 256 rows of its expert, so the blocks restart at every expert; lanes past the
+    // expert's end count as zeros). With a_cols set, a = SiLU(g) u p is recomputed and
+    // quantised along rows too (the layer's forward normally does that itself).
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
     const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
     const int n0 = ti.n_blk * BN;
@@ -290,7 +291,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         for (int j = 0; j < 2; ++j) {
           const int k = 2 * i + j;
           const float da = row_ok ? __uint_as_float(k < 16 ? v0[k] : v1[k - 16]) : 0.f;
-          const float sg = 1.0f / (1.0f + expf(-gs[j]));
+          const float sg = __frcp_rn(1.0f + expf(-gs[j]));   // the correctly rounded 1 / x
           const float sl = gs[j] * sg;
           dg[k] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
           du[k] = da * pr * sl;
@@ -317,12 +318,14 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
-      sc = quant_cols_warp32(av, w, lane);
-      mp.a_cols_atoms[mma_scale_offset(gcol_a, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
-      if (row_ok) {
-        uint4* d = reinterpret_cast<uint4*>(mp.a_cols + row * F + col);
-        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      if (mp.a_cols) {
+        sc = quant_cols_warp32(av, w, lane);
+        mp.a_cols_atoms[mma_scale_offset(gcol_a, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
+        if (row_ok) {
+          uint4* d = reinterpret_cast<uint4*>(mp.a_cols + row * F + col);
+          d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
       // along this row's columns: dh for fc1 dgrad (K = 2F)
       sg_word |= quant_row32(dg, w) << (8 * (c & 3));
@@ -402,7 +405,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const float da = __uint_as_float(hh ? v1[2 * i + j] : v0[2 * i + j]) * deq;
-              const float sg = 1.0f / (1.0f + expf(-gs[j]));
+              const float sg = __frcp_rn(1.0f + expf(-gs[j]));
               const float sl = gs[j] * sg;
               dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
               du[j] = da * pr * sl;
@@ -490,6 +493,9 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     // ScaledSwiGLU, then MXFP8 along the output columns (one 32-column block per chunk)
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
     const int n0 = ti.n_blk * 128;
+    const bool grp_ok = 128 * (r_local >> 7) < ti.rows;      // this CTA's rows hold some of the expert
+    const int KG = (n_e + 127) / 128;                        // the expert's 128-row groups
+    const int jb = 8 * ti.m_blk + (r_local >> 5);            // this warp's 32-row block of the expert
     uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
     __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
     // output chunk 3 of acc0 (its up columns are the shared strip) belongs to the
@@ -508,6 +514,26 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
       if (owner && it == 0) {
         tc_fence_before();
         strip_done();
+      }
+      if (mp.a_cols && grp_ok) {
+        // training: a along the expert's rows as well, for the fc2 weight gradient (the
+        // 32 lanes are 32 consecutive rows of one expert; rows past its end count as 0)
+        float a[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          a[i] = row_ok ? silu_f(__uint_as_float(g0[i])) * __uint_as_float(u0[i]) * pr : 0.f;
+          a[16 + i] = row_ok ? silu_f(__uint_as_float(g1[i])) * __uint_as_float(u1[i]) * pr : 0.f;
+        }
+        uint32_t w[8];
+        const int col = n0 + c * 32;
+        const uint32_t sc = quant_cols_warp32(a, w, threadIdx.x & 31);
+        mp.a_cols_atoms[mma_scale_offset((size_t)grp0 * (p.N / 128) + (size_t)KG * (col / 128),
+                                         (col + (threadIdx.x & 31)) % 128, jb, 1)] = (uint8_t)sc;
+        if (row_ok) {
+          uint4* d = reinterpret_cast<uint4*>(mp.a_cols + row * p.N + col);
+          d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
       if (row_ok) {
         float a[32];

@@ -745,14 +745,36 @@ size_t grouped_mlp_workspace_size(int E, int R, int H, int F, int precision, int
   return align_up((size_t)R * F * 2, 256) + 256;
 }
 
+size_t grouped_mlp_saved_offset(int E, int R, int H, int F, int precision, int part) {
+  if (R < 0 || F < 0 || E < 1 || part < 0) return (size_t)-1;
+  const size_t h = align_up((size_t)R * 2 * F * 2, 256), a = align_up((size_t)R * F, 256);
+  if (part == 0) return 0;
+  if (precision == MOE_MXFP8) {
+    const size_t at = mma_atoms_bytes(E, R, F);
+    switch (part) {
+      case 1: return h;                  // a codes along F (fc2's A)
+      case 2: return h + a;              // their scale atoms (tile groups)
+      case 3: return h + a + at;         // a codes along the expert's rows (fc2 wgrad's A)
+      case 4: return h + 2 * a + at;     // their atoms (grouped)
+      default: return (size_t)-1;
+    }
+  }
+  if (precision == MOE_FP8) {
+    if (part == 1) return h;             // a E4M3 codes
+    if (part == 2) return h + a;         // a's fp32 scale
+    return (size_t)-1;
+  }
+  return part == 1 ? h : (size_t)-1;     // BF16: a bf16
+}
+
 size_t grouped_mlp_saved_size(int E, int R, int H, int F, int precision) {
   (void)E;
   (void)H;
   if (R < 0 || F < 0) return 0;
   if (precision == MOE_FP8)   // h bf16, a's E4M3 codes, a's scale
     return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F, 256) + 256;
-  if (precision == MOE_MXFP8)
-    return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F);
+  if (precision == MOE_MXFP8)   // h; a along F (fc2) and along the expert's rows (fc2 wgrad)
+    return align_up((size_t)R * 2 * F * 2, 256) + 2 * (align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F));
   return align_up((size_t)R * 2 * F * 2, 256) + align_up((size_t)R * F * 2, 256);
 }
 
@@ -778,6 +800,9 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   CUtensorMap ta, tb;
   int rc;
   if ((rc = scales_to_atoms_launch(xp_scale, split_sizes, E, R, H, xp_atoms, st))) return rc;
+  // training: the fc1 epilogue also quantises a along the expert's rows (fc2 wgrad operand)
+  uint8_t* a_cols = saved ? a_atoms + mma_atoms_bytes(E, R, F) : nullptr;
+  uint8_t* a_cols_atoms = saved ? a_cols + align_up((size_t)R * F, 256) : nullptr;
   // fc1: A = xp codes [R, H], B = w1 codes [E, 2F, H] (both K-major)
   if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xp, 1, R, H, 1, 128, mx2::kChunks))) return rc;
   if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1, E, 2 * F, H, 1, 128, mx2::kChunks))) return rc;
@@ -796,6 +821,8 @@ int grouped_mlp_fwd_mxfp8(const void* xp, const uint8_t* xp_scale, const int32_t
   p1.b_atoms = w1_scale;
   p1.b_rows = 2 * F;
   p1.out_atoms = a_atoms;
+  p1.a_cols = a_cols;
+  p1.a_cols_atoms = a_cols_atoms;
   CUtensorMap tsa, tsb;
   if ((rc = tmap_atoms(&tsa, xp_atoms, (uint64_t)R / 128 + E, H / 128))) return rc;
   if ((rc = tmap_atoms(&tsb, w1_scale, (uint64_t)E * 2 * F / 128, H / 128))) return rc;
@@ -1042,7 +1069,7 @@ size_t bwd_part_bytes(int part, int E, int R, int H, int F, int precision) {
     case 4: return mx ? align_up(e * h * 2 * f, 256) + align_up(e * h * 2 * f / 32, 256) : 0;
     case 5: return mx ? align_up(r * h, 256) + align_up(r * h / 32, 256) + mma_atoms_bytes(E, R, H) : 0;
     case 6: return mx ? align_up(r * h, 256) + mma_atoms_bytes(E, R, H) : 0;
-    case 7: return mx ? align_up(r * f, 256) + mma_atoms_bytes(E, R, F) : 0;
+    case 7: return 0;   // (a along rows now comes from the forward's saved buffer)
     case 8: return mx ? align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F) : 0;
     case 9: return mx ? align_up(r * 2 * f, 256) + mma_atoms_bytes(E, R, 2 * F) : 0;
     case 10: return mx ? align_up(r * h, 256) + mma_atoms_bytes(E, R, H) : 0;
@@ -1067,7 +1094,7 @@ size_t grouped_mlp_bwd_workspace_size(int E, int R, int H, int F, int precision)
 
 size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int precision, int part) {
   if (R < 0 || F < 0 || E < 1) return (size_t)-1;
-  const bool ok = precision == MOE_MXFP8 ? (part >= 7 && part <= 9)
+  const bool ok = precision == MOE_MXFP8 ? (part == 8 || part == 9)
                   : precision == MOE_FP8 ? (part == 0 || part == 8)
                                          : part == 0;
   return ok ? bwd_part_offset(part, E, R, H, F, precision) : (size_t)-1;
@@ -1223,8 +1250,10 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   uint8_t* dyr_a = dyr_s + align_up((size_t)R * H / 32, 256);
   uint8_t* dyc = part(6);
   uint8_t* dyc_a = dyc + align_up((size_t)R * H, 256);
-  uint8_t* ac = part(7);
-  uint8_t* ac_a = ac + align_up((size_t)R * F, 256);
+  // a along the expert's rows: quantised by the forward's fc1 epilogue into `saved`
+  const uint8_t* ac = reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256) +
+                      align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F);
+  const uint8_t* ac_a = ac + align_up((size_t)R * F, 256);
   uint8_t* dhr = part(8);
   uint8_t* dhr_a = dhr + align_up((size_t)R * 2 * F, 256);
   uint8_t* dhc = part(9);
@@ -1259,13 +1288,11 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.b_atoms = w2a;
   p.b_rows = F;
   p.out_atoms = nullptr;
-  // the epilogue quantises dh and the recomputed a for the three GEMMs that follow
+  // the epilogue quantises dh for the two GEMMs of fc1 that follow
   p.dh_rows = dhr;
   p.dh_rows_atoms = dhr_a;
   p.dh_cols = dhc;
   p.dh_cols_atoms = dhc_a;
-  p.a_cols = ac;
-  p.a_cols_atoms = ac_a;
   CUtensorMap tsa, tsb;
   if ((rc = tmap_atoms(&tsa, dyr_a, (uint64_t)R / 128 + E, H / 128))) return rc;
   if ((rc = tmap_atoms(&tsb, w2a, (uint64_t)E * F / 128, H / 128))) return rc;

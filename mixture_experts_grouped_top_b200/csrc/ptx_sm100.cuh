@@ -378,7 +378,7 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
 }
 
 // --------------------------------------------------------------- small numerics
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + expf(-g)); }
 
 // 16 fp32 values -> 16 E4M3 codes (round to nearest even, saturating), packed in 4 words.
 __device__ __forceinline__ void pack_e4m3x16(const float* v, uint32_t (&w)[4]) {

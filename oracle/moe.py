@@ -399,9 +399,11 @@ def grouped_mlp_bwd_mxfp8(dy_perm, xp, split_sizes, w1, w2, probs_perm, h, dh=No
     fc1 wgrad: xp and dh along rows. h = [g | u] is the forward's saved pre-activation.
     dh and the recomputed a are quantised from their exact values (the fused backward
     quantises them in the kernel that computes them; they are never stored at a lower
-    precision first). ``dh`` / ``a`` replace those values (e.g. by the dequantised codes a
-    GPU produced, which quantise to themselves along their own axis); ``dh_wgrad``
-    replaces dh for the fc1 weight gradient only (default: ``dh``).
+    precision first). ``a`` is the forward's fc1 output (a fused forward quantises it
+    along rows for this GEMM in its own epilogue); by default it is recomputed from h.
+    ``dh`` / ``a`` replace those values (e.g. by the dequantised codes a GPU produced,
+    which quantise to themselves along their own axis); ``dh_wgrad`` replaces dh for the
+    fc1 weight gradient only (default: ``dh``).
     Returns (dxp, dw1, dw2, dprobs_perm, dh_exact, a_exact).
     """
     dy = f64(dy_perm)

@@ -142,8 +142,10 @@ def test_genomic_mxfp8_full_size_fwd_bwd():
     dhr_s, _, _ = tile_atoms_to_plain(dhr_at, split, 2 * F // 32)
     dhc, dhc_at = part(9, 2 * F)
     dhc_s = grouped_atoms_to_scales(dhc_at, split, 2 * F)
-    ac, ac_at = part(7, F)
-    ac_s = grouped_atoms_to_scales(ac_at, split, F)
+    off3 = mb.grouped_mlp_saved_offset(E, R, H, F, "mxfp8", 3)
+    ac = layer.saved[off3: off3 + R * F].view(R, F)                            # stays on the device
+    ac_s = grouped_atoms_to_scales(layer.saved[mb.grouped_mlp_saved_offset(E, R, H, F, "mxfp8", 4):].cpu().numpy(),
+                                   split, F)
     offs = np.concatenate([[0], np.cumsum(split)])
 
     class RowsDeq:

@@ -1,10 +1,10 @@
 """GPU parity of the MXFP8 backward: the grouped (row-wise, per-expert) quantiser bit for
 bit, and each backward GEMM against the fp64 oracle on the same quantised operands.
 
-The fc2-dgrad epilogue quantises dh = [dg | du] (along 2F and along the expert's rows)
-and the recomputed a (along rows) itself, from fp32: their codes and scales may differ
-from the oracle's quantisation of the exact values only by rounding-boundary flips within
-the fp32 error bound (tests/mx_checks.py). The other GEMMs are checked on the GPU's own
+The fc2-dgrad epilogue quantises dh = [dg | du] (along 2F and along the expert's rows),
+and the forward's fc1 epilogue a along the expert's rows, from fp32: their codes and
+scales may differ from the oracle's quantisation of the exact values only by
+rounding-boundary flips within the fp32 error bound (tests/mx_checks.py). The other GEMMs are checked on the GPU's own
 codes: dxp, dw1, dw2 (bf16) within 2e-3 * max|ref| plus their own bf16 storage rounding
 (half an ulp, at most 2^-8 |ref|); dprobs (fp32) within 2e-3 * max|ref|.
 """
@@ -16,7 +16,8 @@ import mixture_experts_grouped_top_b200 as mb
 from oracle import moe as om
 from oracle import mxfp8 as oq
 import workloads
-from tests.mx_checks import assert_boundary_flips, boundary_flips_grouped_rows, dswiglu_fp32_error_bounds
+from tests.mx_checks import (assert_boundary_flips, boundary_flips_grouped_rows, dswiglu_fp32_error_bounds,
+                             swiglu_fp32_error_bound)
 from tests.mx_layout import grouped_atoms_to_scales, grouped_scales_to_atoms, tile_atoms_to_plain
 
 pytestmark = pytest.mark.gpu
@@ -56,20 +57,43 @@ BWD_CASES = [
 ]
 
 
-def fused_operands(ws, E, R, H, F, split):
-    """The fc2-dgrad epilogue's MXFP8 outputs from the backward workspace: dh along 2F
-    (codes, plain scales), dh along rows and a along rows (codes, per-expert scales)."""
-    def part(i, ncols):
-        off = mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", i)
-        codes = ws[off: off + R * ncols].view(R, ncols).cpu().numpy()
-        atoms = ws[off + (R * ncols + 255) // 256 * 256:].cpu().numpy()
-        return codes, atoms
-    dhr, dhr_at = part(8, 2 * F)
+def fused_operands(layer, E, R, H, F, split):
+    """The MXFP8 operands quantised inside the GEMM epilogues: dh along 2F (codes, plain
+    scales) and dh along rows (codes, per-expert scales) from the fc2-dgrad epilogue (the
+    backward workspace), a along rows from the fc1 epilogue (the forward's saved buffer)."""
+    ws, saved = layer._bwd["ws"], layer.saved
+
+    def part(buf, off, ncols, atoms_off=None):
+        codes = buf[off: off + R * ncols].view(R, ncols).cpu().numpy()
+        a0 = off + (R * ncols + 255) // 256 * 256 if atoms_off is None else atoms_off
+        return codes, buf[a0:].cpu().numpy()
+
+    dhr, dhr_at = part(ws, mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 8), 2 * F)
     dhr_s, _, _ = tile_atoms_to_plain(dhr_at, split, 2 * F // 32)
-    dhc, dhc_at = part(9, 2 * F)
-    ac, ac_at = part(7, F)
+    dhc, dhc_at = part(ws, mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", 9), 2 * F)
+    ac, ac_at = part(saved, mb.grouped_mlp_saved_offset(E, R, H, F, "mxfp8", 3), F,
+                     mb.grouped_mlp_saved_offset(E, R, H, F, "mxfp8", 4))
     return (dhr, dhr_s), (dhc, grouped_atoms_to_scales(dhc_at, split, 2 * F)), \
         (ac, grouped_atoms_to_scales(ac_at, split, F))
+
+
+def forward_a(layer, d, split, F, H):
+    """The forward's exact a (fp64 on the same MXFP8 operands) and its fp32 error bound,
+    for the codes the fc1 epilogue quantised along rows."""
+    xc, xs = layer.perm["xp"].cpu().numpy(), layer.perm["xp_scale"].cpu().numpy()
+    w1c, w1s = om.quantize_weights_kmajor(d["w1"], "rows")
+    w2c, w2s = om.quantize_weights_kmajor(d["w2"], "rows")
+    pp = om.f64(layer.perm["probs_perm"].cpu())[:, None]
+    _, _, _, h = om.grouped_mlp_fwd_mxfp8(xc, xs, split, w1c, w1s, w2c, w2s, pp[:, 0])
+    xq = np.abs(oq.dequantize_blocks_last_axis(xc, xs))
+    w1q = np.abs(oq.dequantize_blocks_last_axis(w1c, w1s))
+    sabs = np.zeros((xq.shape[0], 2 * F))
+    s0 = 0
+    for e, n in enumerate(split):
+        sabs[s0:s0 + n] = xq[s0:s0 + n] @ w1q[e].T
+        s0 += n
+    a = om.silu(h[:, :F]) * h[:, F:] * pp
+    return a, swiglu_fp32_error_bound(h[:, :F], h[:, F:], pp, sabs[:, :F], sabs[:, F:], H)
 
 
 def fused_bounds(dy, w2, split, h, pp, F, H):
@@ -95,10 +119,11 @@ def check_fused_backward(layer, d, E, R, H, F):
     b = layer._bwd
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
     dy, xp, pp = b["dy_perm"].cpu(), layer.xp_bf16.cpu(), layer.perm["probs_perm"].cpu()
-    (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(b["ws"], E, R, H, F, split)
+    (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(layer, E, R, H, F, split)
     exact = om.grouped_mlp_bwd_mxfp8(dy, xp, split, d["w1"], d["w2"], pp, h)
-    dh_exact, a_exact = exact[4], exact[5]
-    err_dh, err_a = fused_bounds(dy, d["w2"], split, h, pp, F, H)
+    dh_exact = exact[4]
+    err_dh, _ = fused_bounds(dy, d["w2"], split, h, pp, F, H)
+    a_exact, err_a = forward_a(layer, d, split, F, H)
     assert_boundary_flips(dhr, dhr_s, dh_exact, "dh along 2F", err=err_dh)
     for name, (c, sc), ex, er in (("dh along rows", (dhc, dhc_s), dh_exact, err_dh),
                                   ("a along rows", (ac, ac_s), a_exact, err_a)):

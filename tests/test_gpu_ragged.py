@@ -108,7 +108,7 @@ def test_mxfp8_backward_ragged_expert_sizes():
     R = T
     b = layer._bwd
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
-    (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(b["ws"], E, R, H, F, split)
+    (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(layer, E, R, H, F, split)
     ref = om.grouped_mlp_bwd_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
                                    layer.perm["probs_perm"].cpu(), h,
                                    dh=oq.dequantize_blocks_last_axis(dhr, dhr_s),
