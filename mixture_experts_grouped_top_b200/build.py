@@ -17,7 +17,7 @@ LIB = os.path.join(PKG, "libmoe_grouped.so")
 SOURCES = ["moe_api.cu"]
 HEADERS = ["ptx_sm100.cuh", "token_kernels.cuh", "grouped_gemm_sm100.cuh", "grouped_gemm_mxf8_sm100.cuh",
            "grouped_gemm_pair_sm100.cuh", "grouped_gemm_mxf8_pair_sm100.cuh",
-           "grouped_gemm_kgroup_pair_sm100.cuh"]
+           "grouped_gemm_kgroup_pair_sm100.cuh", "grouped_gemm_mxf8_kgroup_pair_sm100.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -1,25 +1,26 @@
-// Persistent grouped GEMM for MXFP8 operands on sm_100a: E4M3 A and B, one E8M0 scale
-// per 32 consecutive K values of every row, fp32 accumulation in tensor memory
-// (tcgen05.mma kind::mxf8f6f4.block_scale, M=128, N=256, K=32 per instruction).
+// MXFP8 pieces shared by the block-scaled grouped GEMMs on sm_100a: E4M3 (or E5M2) A and
+// B with one E8M0 scale per 32 consecutive K values, fp32 accumulation in tensor memory
+// (tcgen05.mma kind::mxf8f6f4.block_scale, K=32 per instruction): the parameter block, the
+// warp-level quantisers and the fused epilogues that drain a 128-row x 256-column
+// accumulator.
 //
 // Pages: "Efficient MoE training for biological foundation models" (news.bpdata.com
 // section 2: MXFP8 keeps one scale per block of 32 consecutive values and Blackwell
 // tensor cores consume it directly; section 3: the fused GroupedLinear -> ScaledSwiGLU ->
 // GroupedLinear chain with quantisation fused into it).
 //
-// The library runs its M-grouped MXFP8 GEMMs on CTA pairs (grouped_gemm_mxf8_pair_sm100.cuh,
-// which reuses the epilogues below) and this kernel for the K-grouped weight gradients.
-// Same tile walk and warp roles as the BF16 kernels (grouped_gemm_sm100.cuh). What is
-// specific to block scaling:
+// The kernels live in grouped_gemm_mxf8_pair_sm100.cuh (M-grouped: fc1, fc2 and the two
+// data gradients) and grouped_gemm_mxf8_kgroup_pair_sm100.cuh (K-grouped weight
+// gradients), both on CTA pairs. What is specific to block scaling:
 //   * scales are 512-byte atoms per 128-wide k-block (128 rows x 4 scale bytes, row r of
 //     the group at word (r % 32) * 4 + r / 32, the layout tcgen05.cp expects), already
 //     arranged so in global memory (mma_scale_offset), a row group's atoms for
 //     consecutive k-blocks contiguous: they travel on a two-slot ring of their own, one
-//     bulk copy per row group (A, and B's two 128-row halves) per four k-blocks, since a
-//     copy costs the copy engine about the same whatever its size;
+//     copy per row group (A, and B's two 128-row halves) per four k-blocks, since a copy
+//     costs the copy engine about the same whatever its size;
 //   * the MMA thread moves the atoms into tensor memory with tcgen05.cp (32 lanes x 16 B,
 //     replicated to the four sub-partitions), then issues the four K=32 MMAs of the
-//     stage, selecting scale byte kk of each word through the scale-factor ids;
+//     k-block, selecting scale byte kk of each word through the scale-factor ids;
 //   * two 256-column accumulators plus 12 scale columns exceed the 512 tensor-memory
 //     columns, so the accumulators overlap: acc0 = columns [0, 256), acc1 = [224, 480),
 //     scales at [480, 492). The epilogue drains the shared 32-column strip first and
@@ -32,26 +33,11 @@
 namespace moe {
 
 namespace mx {
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;                       // fp8: 128 bytes of K per row (one swizzle span)
-constexpr int kStages = 4;
-constexpr int kThreads = 384;                 // 4 control warps + 8 epilogue warps
-constexpr int kABytes = BM * BK;              // 16 KB
-constexpr int kBBytes = BN * BK;              // 32 KB
-constexpr int kSfaBytes = 512;                // 128 rows x 4 scale bytes
-constexpr int kSfbBytes = 1024;               // 256 rows x 4 scale bytes
-constexpr int kSfKb = 4;                      // k-blocks per scale copy
-constexpr int kSfGroupBytes = kSfKb * 512;    // one row group's atoms for kSfKb k-blocks
-constexpr int kSfSlotBytes = 3 * kSfGroupBytes;   // A group, B lower group, B upper group
-constexpr int kSfSlots = 2;
-constexpr int kMaxE = 1024;
-constexpr int kTmemCols = 512;
-constexpr uint32_t kAcc1Col = 224;
-constexpr uint32_t kSfaCol = 480;
-constexpr uint32_t kSfbCol = 484;
-constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kSfSlots * kSfSlotBytes + 1024 +
-                           4 * (kMaxE + 1) * 4;
+// tensor-memory layout shared by the MXFP8 pair kernels (columns of each CTA's 512)
+constexpr int BN = 256;                       // accumulator columns per tile
+constexpr uint32_t kAcc1Col = 224;            // acc0 = [0, 256), acc1 = [224, 480)
+constexpr uint32_t kSfaCol = 480;             // A scales: 4 columns
+constexpr uint32_t kSfbCol = 484;             // B scales: 2 x 4 columns
 }  // namespace mx
 
 enum MxEpiKind : int {
@@ -579,324 +565,6 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     }
   }
   return sc_word;
-}
-
-template <bool KGROUP, int EPI>
-__global__ void __launch_bounds__(mx::kThreads, 1)
-    grouped_gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const MxGemmParams mp) {
-  using namespace mx;
-  const GemmParams& p = mp.g;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + kStages * kABytes;
-  uint8_t* sSf = sB + kStages * kBBytes;     // scale ring: kSfSlots slots of three 2 KB groups
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSf + kSfSlots * kSfSlotBytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = bars + 2 * kStages + 2;
-  uint64_t* tovl = bars + 2 * kStages + 4;
-  uint64_t* sfull = bars + 2 * kStages + 5;
-  uint64_t* sempty = sfull + kSfSlots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSfSlots);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
-  int32_t* tile_off = row_off + (kMaxE + 1);
-  int32_t* kg_off = tile_off + (kMaxE + 1);   // K-grouped: k-groups (128 rows) of earlier experts
-  int32_t* order = kg_off + (kMaxE + 1);      // K-grouped: experts by decreasing row count
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = p.E;
-  const int NT = mx_swiglu(EPI) ? (p.N / 128) : (p.N + BN - 1) / BN;
-  const int MT = KGROUP ? (p.M + BM - 1) / BM : 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
-    }
-    mbar_init(tovl, 256);
-    for (int s2 = 0; s2 < kSfSlots; ++s2) {
-      mbar_init(&sfull[s2], 1);
-      mbar_init(&sempty[s2], 1);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 3) {
-    int carry_r = 0, carry_t = 0, carry_k = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      const int n = (e < E) ? p.split_sizes[e] : 0;
-      const int tiles = (e < E) ? (KGROUP ? MT * NT : ((n + BM - 1) / BM) * NT) : 0;
-      const int kgs = (n + BK - 1) / BK;
-      int ir = n, it = tiles, ik = kgs;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
-        const int yt = __shfl_up_sync(0xffffffffu, it, o);
-        const int yk = __shfl_up_sync(0xffffffffu, ik, o);
-        if (lane >= o) {
-          ir += yr;
-          it += yt;
-          ik += yk;
-        }
-      }
-      if (e < E) {
-        row_off[e] = carry_r + ir - n;
-        tile_off[e] = carry_t + it - tiles;
-        kg_off[e] = carry_k + ik - kgs;
-      }
-      carry_r += __shfl_sync(0xffffffffu, ir, 31);
-      carry_t += __shfl_sync(0xffffffffu, it, 31);
-      carry_k += __shfl_sync(0xffffffffu, ik, 31);
-    }
-    if (lane == 0) {
-      row_off[E] = carry_r;
-      tile_off[E] = carry_t;
-      kg_off[E] = carry_k;
-    }
-  }
-  if (warp == 2) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  if (KGROUP) {
-    rank_experts_by_rows(row_off, E, order);
-    __syncthreads();
-  }
-
-  TileWalker<KGROUP> walk{row_off, tile_off, E, MT, NT, p.K, order};
-  // the walker's k-block count assumes 64-wide blocks; MXFP8 uses 128-wide ones
-  auto kblocks = [&](const TileInfo& ti) { return KGROUP ? (ti.rows + BK - 1) / BK : p.K / BK; };
-  const int total = walk.total();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      int stage = 0, sslot = 0;
-      uint32_t phase = 0, sphase = 0;
-      int issued = 0, sissued = 0;
-      bool ok = true;
-      const int KB4 = KGROUP ? 0 : p.K / 128;
-      const int bgroups = mp.b_rows / 128;
-      for (int t = blockIdx.x; t < total && ok && !p.stall_loads; t += gridDim.x) {
-        const TileInfo ti = walk.decode(t);
-        const int num_kb = kblocks(ti);
-        const int n0 = mx_swiglu(EPI) ? ti.n_blk * 128 : ti.n_blk * BN;
-        size_t ga, gb0, gb1;   // first atom of A's and of B's two 128-row halves (k-group 0)
-        if (KGROUP) {
-          const size_t kg = (size_t)(ti.rows + BK - 1) / BK;
-          ga = (size_t)kg_off[ti.e] * (p.M / 128) + (size_t)ti.m_blk * kg;
-          gb0 = (size_t)kg_off[ti.e] * (p.N / 128) + (size_t)(n0 / 128) * kg;
-          gb1 = (n0 + 128 < p.N) ? gb0 + kg : gb0;
-        } else {
-          ga = (size_t)(tile_off[ti.e] / NT + ti.m_blk) * KB4;          // A row group (expert tile)
-          gb0 = ((size_t)ti.e * bgroups + n0 / 128) * KB4;
-          gb1 = ((size_t)ti.e * bgroups + (mx_swiglu(EPI) ? (p.F + n0) / 128 : n0 / 128 + 1)) * KB4;
-          if (!mx_swiglu(EPI) && n0 + 128 >= mp.b_rows) gb1 = gb0;   // past N: codes are zero-filled
-        }
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if ((kb & (kSfKb - 1)) == 0) {
-            // scale atoms of k-blocks [kb, kb + n): each row group's atoms for consecutive
-            // k-blocks are contiguous, so one copy per group (never past this tile's last atom)
-            if (!mbar_wait_bounded(&sempty[sslot], sphase ^ 1, abort_flag, p.timeout_ns)) {
-              ok = false;
-              break;
-            }
-            const uint32_t n = (uint32_t)min(kSfKb, num_kb - kb) * 512;
-            uint8_t* sd = sSf + sslot * kSfSlotBytes;
-            mbar_arrive_expect_tx(&sfull[sslot], 3 * n);
-            bulk_load(sd, mp.a_atoms + (ga + kb) * 512, n, &sfull[sslot]);
-            bulk_load(sd + kSfGroupBytes, mp.b_atoms + (gb0 + kb) * 512, n, &sfull[sslot]);
-            bulk_load(sd + 2 * kSfGroupBytes, mp.b_atoms + (gb1 + kb) * 512, n, &sfull[sslot]);
-            ++sissued;
-            if (++sslot == kSfSlots) {
-              sslot = 0;
-              sphase ^= 1;
-            }
-          }
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          const int k0 = kb * BK;
-          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes);
-          uint8_t* b_dst = sB + stage * kBBytes;
-          if (KGROUP) {
-            // MN-major codes: box {128 columns, 128 rows} at the expert's k-th row block
-            tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], ti.m_blk * BM, ti.row0 + k0, 0);
-            // both 128-column chunks of B in one copy (chunked view, box {128, 128 k rows, 2, 1})
-            tma_load_4d(b_dst, &tmB, &full[stage], 0, ti.row0 + k0, n0 / 128, 0);
-          } else {
-            tma_load_3d(sA + stage * kABytes, &tmA, &full[stage], k0, ti.row0, 0);
-            tma_load_3d(b_dst, &tmB, &full[stage], k0, n0, ti.e);
-            tma_load_3d(b_dst + BM * BK, &tmB, &full[stage], k0, mx_swiglu(EPI) ? p.F + n0 : n0 + 128, ti.e);
-          }
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      if (!ok) {
-        int st = stage, ph = phase;
-        for (int i = 0; i < min(issued, kStages); ++i) {
-          if (--st < 0) {
-            st = kStages - 1;
-            ph ^= 1;
-          }
-          mbar_wait_drain(&full[st], ph, p.timeout_ns);
-        }
-        // and the scale copies still in flight
-        int ss = sslot, sp = sphase;
-        for (int i = 0; i < min(sissued, kSfSlots); ++i) {
-          if (--ss < 0) {
-            ss = kSfSlots - 1;
-            sp ^= 1;
-          }
-          mbar_wait_drain(&sfull[ss], sp, p.timeout_ns);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA issuer
-    int stage = 0, sslot = 0;
-    uint32_t phase = 0, sphase = 0;
-    int lt = 0;
-    bool ok = true;
-    const uint32_t sfa_t = tmem_base + kSfaCol;
-    const uint32_t sfb_t = tmem_base + kSfbCol;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
-      const TileInfo ti = walk.decode(t);
-      const int num_kb = kblocks(ti);
-      const int acc = lt & 1;
-      if (!mbar_wait_bounded(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
-      if (lt > 0 && !mbar_wait_bounded(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + (acc ? kAcc1Col : 0u);
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if ((kb & (kSfKb - 1)) == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        int ksteps = BK / 32;   // K=32 MMAs of this stage
-        if (KGROUP && (kb + 1) * BK > ti.rows) {
-          // clip the contraction at the expert's last row: MMAs only over the expert's
-          // K-rows; inside the last, partial 32-row step zero the rows >= valid of the
-          // three operand blocks (A, two halves of B; 128-byte lines)
-          const int valid = ti.rows - kb * BK;
-          ksteps = (valid + 31) / 32;
-          const int zr = ksteps * 32 - valid;   // 0..31 rows
-          if (zr > 0) {
-            for (int i = lane; i < 3 * zr * 8; i += 32) {
-              const int v = i & 7, rb = i >> 3;
-              const int blk = rb / zr, r = rb - blk * zr;
-              uint8_t* base = (blk == 0) ? sA + stage * kABytes : sB + stage * kBBytes + (blk - 1) * BM * BK;
-              *reinterpret_cast<uint4*>(base + (valid + r) * 128 + v * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-          }
-          __syncwarp();
-        }
-        if (lane == 0) {
-          // this k-block's atoms: entry kb % kSfKb of each group of the current scale slot
-          const uint32_t sf_s = smem_u32(sSf + sslot * kSfSlotBytes) + (uint32_t)(kb & (kSfKb - 1)) * 512;
-          tmem_cp_32x128b_warpx4(sfa_t, make_sdesc(sf_s, 0, 128, 0));
-          tmem_cp_32x128b_warpx4(sfb_t, make_sdesc(sf_s + kSfGroupBytes, 0, 128, 0));
-          tmem_cp_32x128b_warpx4(sfb_t + 4, make_sdesc(sf_s + 2 * kSfGroupBytes, 0, 128, 0));
-          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
-#pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk) {
-            if (kk >= ksteps) break;
-            // K-major: next 32 K values are 32 bytes further in each 128-byte row;
-            // MN-major: 32 rows further (4 x 8-row swizzle atoms), halves of B 16 KB apart
-            const uint64_t adesc = KGROUP ? make_sdesc(a_addr + kk * 4096, BM * BK, 1024, 2)
-                                          : make_sdesc(a_addr + kk * 32, 16, 1024, 2);
-            const uint64_t bdesc = KGROUP ? make_sdesc(b_addr + kk * 4096, BM * BK, 1024, 2)
-                                          : make_sdesc(b_addr + kk * 32, 16, 1024, 2);
-            const uint32_t idesc = make_idesc_mxf8(BM, BN, KGROUP, KGROUP, kk, kk) | mp.ab_fmt;
-            mma_mxf8_ss(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30),
-                        (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&empty[stage]);
-          // the slot's last k-block: release it once these MMAs have read their scales
-          if ((kb & (kSfKb - 1)) == kSfKb - 1 || kb == num_kb - 1) mma_commit(&sempty[sslot]);
-        }
-        __syncwarp();
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if ((kb & (kSfKb - 1)) == kSfKb - 1 || kb == num_kb - 1) {
-          if (++sslot == kSfSlots) {
-            sslot = 0;
-            sphase ^= 1;
-          }
-        }
-      }
-      if (!ok) break;
-      if (lane == 0) {
-        if (num_kb > 0)
-          mma_commit(&tfull[acc]);
-        else
-          mbar_arrive(&tfull[acc]);
-      }
-      __syncwarp();
-    }
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;               // TMEM lane quadrant
-    const int half = (warp - 4) >> 2;     // half of the tile's columns this warp drains
-    const int r_local = q * 32 + lane;
-    int lt = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
-      const TileInfo ti = walk.decode(t);
-      const int acc = lt & 1;
-      if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
-      tc_fence_after();
-      const uint32_t t_row = tmem_base + (acc ? kAcc1Col : 0u) + ((uint32_t)(q * 32) << 16);
-      const uint32_t sc_word =
-          mxf8_epilogue_tile<EPI>(mp, ti, t_row, acc, half, r_local, BM, [&] { mbar_arrive(tovl); });
-      if (EPI == MXEPI_SWIGLU_Q) {
-        // this half's two scale bytes (chunks 2*half, 2*half+1); rows past the expert store 0
-        const size_t g = (size_t)(tile_off[ti.e] / NT + ti.m_blk);
-        *reinterpret_cast<uint16_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk + 2 * half,
-                                                                     p.N / 128)) =
-            (uint16_t)(sc_word >> (16 * half));
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 2) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
-  }
 }
 
 }  // namespace moe

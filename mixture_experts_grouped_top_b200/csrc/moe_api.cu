@@ -10,6 +10,7 @@
 
 #include "moe_grouped.h"
 #include "grouped_gemm_kgroup_pair_sm100.cuh"
+#include "grouped_gemm_mxf8_kgroup_pair_sm100.cuh"
 #include "grouped_gemm_mxf8_pair_sm100.cuh"
 #include "grouped_gemm_mxf8_sm100.cuh"
 #include "grouped_gemm_pair_sm100.cuh"
@@ -172,11 +173,6 @@ int launch_wgrad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPa
   return launch_status();
 }
 
-// E4M3 codes [batch, rows, cols] as a TMA source with box {128 bytes of K, box_rows}.
-int tmap_u8_3d(CUtensorMap* m, const void* ptr, uint64_t batch, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, cols, rows, batch, cols, rows * cols, 128, box_rows);
-}
-
 // MMA scale atoms [groups, kb4 atoms of 512 bytes] as a TMA source: uint32 tensor
 // {128 words, kb4, groups}, boxes of mx2::kSfKb consecutive atoms of one group (unswizzled).
 int tmap_atoms(CUtensorMap* m, const void* atoms, uint64_t groups, uint64_t kb4) {
@@ -212,17 +208,48 @@ int launch_gemm_mx_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   return launch_status();
 }
 
-template <bool KG, int EPI>
-int launch_gemm_mx(const CUtensorMap& ta, const CUtensorMap& tb, const MxGemmParams& p, cudaStream_t st) {
-  auto kern = grouped_gemm_mxf8_kernel<KG, EPI>;
+// Grouped scale atoms (K-grouped operands: n_atoms of 512 bytes) as a TMA source: uint32
+// tensor {128 words, n_atoms, 1}, boxes of mkp::kSfKg consecutive atoms (unswizzled).
+int tmap_atoms_flat(CUtensorMap* m, const void* atoms, uint64_t n_atoms) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, atoms, 128, n_atoms, 1, 512, n_atoms * 512, 128, mkp::kSfKg,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// MXFP8 weight-gradient GEMM dW[e] = A_e^T B_e on CTA pairs. A codes [R, M], B codes
+// [R, N] (MN-major), their grouped atoms (a_atoms / b_atoms hold at least a_n / b_n atoms).
+int launch_wgrad_mx_pair(const uint8_t* a, const uint8_t* a_atoms, uint64_t a_n, const uint8_t* b,
+                         const uint8_t* b_atoms, uint64_t b_n, int R, const MxGemmParams& p, cudaStream_t st) {
+  auto kern = grouped_wgrad_mxf8_pair_kernel;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
+  static int pairs = 0;
   std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mx::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mkp::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(device_props().sm_count, 1, 1);
+    cfg.blockDim = dim3(mkp::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = mkp::kSmemBytes;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_props().sm_count / 2;
+    pairs = std::min(n, device_props().sm_count / 2);
+    cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  const int grid = device_props().sm_count;
-  kern<<<grid, mx::kThreads, mx::kSmemBytes, st>>>(ta, tb, p);
+  if ((p.g.M % 128) || (p.g.N % 128)) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap ta, tb, tsa, tsb;
+  int rc;
+  if ((rc = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, p.g.M, R, 1, p.g.M, (uint64_t)R * p.g.M, 128,
+                      mkp::BK)))
+    return rc;
+  if ((rc = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, p.g.N, R, 1, p.g.N, (uint64_t)R * p.g.N, 128,
+                      mkp::BK)))
+    return rc;
+  if ((rc = tmap_atoms_flat(&tsa, a_atoms, a_n))) return rc;
+  if ((rc = tmap_atoms_flat(&tsb, b_atoms, b_n))) return rc;
+  kern<<<2 * pairs, mkp::kThreads, mkp::kSmemBytes, st>>>(ta, tb, tsa, tsb, p);
   count_launch();
   return launch_status();
 }
@@ -1178,8 +1205,7 @@ int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, 
   if ((rc = fp8_scale_launch(amax, 1, 1, s_dh, st))) return rc;
   if ((rc = fp8_cast_launch(dh, 1, (long long)R * 2 * F, s_dh, 1, dhq, st))) return rc;
   // fc2 wgrad: dw2[e] = a_e^T dy_e, A = a codes (E4M3) [R, F], B = dy codes (E5M2) [R, H]
-  if ((rc = tmap_u8_3d(&ta, a_codes, 1, R, F, mx::BM))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyq, 1, R, H, 1, mx::BK, 2))) return rc;
+  const uint64_t n_unit = fp8_unit_atoms_bytes(E, R, H, F) / 512;
   p = MxGemmParams{};
   p.g = base_params(split_sizes, E);
   p.g.M = F;
@@ -1193,7 +1219,7 @@ int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, 
   p.ab_fmt = B_E5M2;
   p.deq_a = a_scale;
   p.deq_b = s_dy;
-  if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
+  if ((rc = launch_wgrad_mx_pair(a_codes, unit, n_unit, dyq, unit, n_unit, R, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T, A = dh codes (E5M2) [R, 2F], B = w1 codes [E, H, 2F]
   if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhq, 1, R, 2 * F, 1, 128, mx2::kChunks))) return rc;
   if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1, 128, mx2::kChunks))) return rc;
@@ -1214,8 +1240,6 @@ int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, 
   p.deq_b = s_w1;
   if ((rc = launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e, A = xp codes (E4M3) [R, H], B = dh codes (E5M2)
-  if ((rc = tmap_u8_3d(&ta, xq, 1, R, H, mx::BM))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhq, 1, R, 2 * F, 1, mx::BK, 2))) return rc;
   p = MxGemmParams{};
   p.g = base_params(split_sizes, E);
   p.g.M = H;
@@ -1229,7 +1253,7 @@ int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, 
   p.ab_fmt = B_E5M2;
   p.deq_a = s_x;
   p.deq_b = s_dh;
-  return launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st);
+  return launch_wgrad_mx_pair(xq, unit, n_unit, dhq, unit, n_unit, R, p, st);
 }
 
 int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
@@ -1306,8 +1330,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   // xp along its rows for the fc1 weight gradient
   if ((rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc, xc_a, st))) return rc;
   // fc2 wgrad: dw2[e] = a_e^T dy_e (MN-major codes, contraction over the expert's rows)
-  if ((rc = tmap_u8_3d(&ta, ac, 1, R, F, mx::BM))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyc, 1, R, H, 1, mx::BK, 2))) return rc;
+  const uint64_t kgs = (uint64_t)R / 128 + E;   // bound on the experts' 128-row k-groups
   p.g = base_params(split_sizes, E);
   p.g.M = F;
   p.g.N = H;
@@ -1317,7 +1340,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.a_atoms = ac_a;
   p.b_atoms = dyc_a;
   p.b_rows = H;
-  if ((rc = launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st))) return rc;
+  if ((rc = launch_wgrad_mx_pair(ac, ac_a, kgs * (F / 128), dyc, dyc_a, kgs * (H / 128), R, p, st))) return rc;
   // fc1 dgrad: dxp = dh w1[e]^T. A = dh codes [R, 2F], B = w1 codes [E, H, 2F] (N = H)
   if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhr, 1, R, 2 * F, 1, 128, mx2::kChunks))) return rc;
   if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w1q, E, H, 2 * F, 1, 128, mx2::kChunks))) return rc;
@@ -1334,8 +1357,6 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   if ((rc = tmap_atoms(&tsb, w1a, (uint64_t)E * H / 128, 2 * F / 128))) return rc;
   if ((rc = launch_gemm_mx_pair<MXEPI_STORE>(ta, tb, tsa, tsb, p, st))) return rc;
   // fc1 wgrad: dw1[e] = xp_e^T dh_e
-  if ((rc = tmap_u8_3d(&ta, xc, 1, R, H, mx::BM))) return rc;
-  if ((rc = tmap_chunks(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, dhc, 1, R, 2 * F, 1, mx::BK, 2))) return rc;
   p.g = base_params(split_sizes, E);
   p.g.M = H;
   p.g.N = 2 * F;
@@ -1345,7 +1366,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   p.a_atoms = xc_a;
   p.b_atoms = dhc_a;
   p.b_rows = 2 * F;
-  return launch_gemm_mx<true, MXEPI_WGRAD>(ta, tb, p, st);
+  return launch_wgrad_mx_pair(xc, xc_a, kgs * (H / 128), dhc, dhc_a, kgs * (2 * F / 128), R, p, st);
 }
 
 }  // namespace
