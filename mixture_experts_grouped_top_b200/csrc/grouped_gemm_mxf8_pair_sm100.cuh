@@ -19,6 +19,11 @@
 //     tensor memory, so both CTAs fetch both B groups). The leader copies a k-block's
 //     atoms into both CTAs' tensor memory (tcgen05.cp.cta_group::2) before its MMAs.
 //
+// The SwiGLU backward's epilogue also needs the saved h = [g | u] of every row it drains:
+// warp 3 of each CTA copies it with TMA into a shared-memory ring of 32-column strips,
+// ahead of the epilogue, which reads its row from there (coalesced copies instead of one
+// 16-byte load per row and lane from global memory).
+//
 // Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [224, 480),
 // A scales at 480, B scales at 484..491; `tovl` and `tempty` live in the leader and count
 // one arrival per epilogue warp of both CTAs. Waits are bounded like in every other
@@ -55,36 +60,54 @@ static_assert(kChunks == 1 || kChunks == 2, "one or two k-chunks per stage");
 
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes =
-    1024 + kStages * kStageBytes + kSfSlots * kSfSlotBytes + 1024 + 3 * (kMaxE + 1) * 4;
+// SwiGLU backward: the saved h reaches the epilogue through shared memory, a ring of
+// 32-column strips (g and u of the CTA's 128 rows, 64-byte swizzled: 16 KB) per column
+// half; its 64 KB come out of the operand ring, which keeps two stages (the K = H
+// mainloop of that GEMM is shorter than its epilogue).
+constexpr int kHSlotBytes = 2 * 128 * 64;
+constexpr int kHSlots = 2;                    // per half
+__host__ __device__ constexpr bool stages_h(int epi) { return epi == MXEPI_DSWIGLU; }
+__host__ __device__ constexpr int stages_for(int epi) { return stages_h(epi) ? 2 : kStages; }
+__host__ __device__ constexpr int smem_bytes(int epi) {
+  return 1024 + stages_for(epi) * kStageBytes + kSfSlots * kSfSlotBytes + (stages_h(epi) ? 2 * kHSlots * kHSlotBytes : 0) +
+         1024 + 3 * (kMaxE + 1) * 4;
+}
+static_assert(smem_bytes(MXEPI_DSWIGLU) <= 232448 && smem_bytes(MXEPI_STORE) <= 232448, "shared memory per CTA");
 }  // namespace mx2
 
 // tmA / tmB: E4M3 codes [rows, K] / [E][b_rows][K] as {128, rows, K/128 chunks, batch},
 // box {128, 128, 2, 1}. tmSa / tmSb: scale atoms as uint32 tensors {128 words, K/128
 // k-blocks, row groups} with a box of four atoms (no swizzle); A's row groups are the
 // experts' 128-row tiles in order, B's are e * (b_rows / 128) + row / 128.
+// tmH (SwiGLU backward only): the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128},
+// 64-byte swizzle.
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     grouped_gemm_mxf8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                   const __grid_constant__ CUtensorMap tmSa, const __grid_constant__ CUtensorMap tmSb,
-                                  const MxGemmParams mp) {
+                                  const __grid_constant__ CUtensorMap tmH, const MxGemmParams mp) {
   using namespace mx2;
+  constexpr int kSt = stages_for(EPI);
+  constexpr bool kH = stages_h(EPI);
   const GemmParams& p = mp.g;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + kStages * kABytes;
-  uint8_t* sSf = sB + kStages * kBBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSf + kSfSlots * kSfSlotBytes);
+  uint8_t* sB = sA + kSt * kABytes;
+  uint8_t* sSf = sB + kSt * kBBytes;
+  uint8_t* sH = sSf + kSfSlots * kSfSlotBytes;  // 1024-byte aligned: kSfSlots * kSfSlotBytes = 12 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sH + (kH ? 2 * kHSlots * kHSlotBytes : 0));
   uint64_t* full = bars;                      // used in the leader
-  uint64_t* empty = bars + kStages;           // both CTAs
-  uint64_t* tfull = bars + 2 * kStages;       // both CTAs
-  uint64_t* tempty = bars + 2 * kStages + 2;  // used in the leader
-  uint64_t* tovl = bars + 2 * kStages + 4;    // used in the leader
-  uint64_t* sfull = bars + 2 * kStages + 5;   // scale ring: used in the leader
+  uint64_t* empty = bars + kSt;               // both CTAs
+  uint64_t* tfull = bars + 2 * kSt;           // both CTAs
+  uint64_t* tempty = bars + 2 * kSt + 2;      // used in the leader
+  uint64_t* tovl = bars + 2 * kSt + 4;        // used in the leader
+  uint64_t* sfull = bars + 2 * kSt + 5;       // scale ring: used in the leader
   uint64_t* sempty = sfull + kSfSlots;        // scale ring: both CTAs
   uint64_t* drained = sempty + kSfSlots;      // used in the second CTA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  uint64_t* hfull = drained + 1;              // h ring (half * kHSlots + slot): both CTAs
+  uint64_t* hempty = hfull + 2 * kHSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 2 * kHSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -98,9 +121,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   const int NT = mx_swiglu(EPI) ? (p.N / 128) : (p.N + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2 * kHSlots; ++b) {
+      mbar_init(&hfull[b], 1);
+      mbar_init(&hempty[b], 4);   // the four epilogue warps of a half
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -120,6 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSa);
     tma_prefetch_desc(&tmSb);
+    if (kH) tma_prefetch_desc(&tmH);
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0, carry_g = 0;
@@ -221,14 +249,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
           tma_load_4d_pair(sA + stage * kABytes, &tmA, &full[stage], 0, a_row, kChunks * st, 0);
           tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b_row, kChunks * st, ti.e);
 
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
       // no copy may still be landing when either CTA leaves
-      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kStages, ring, sfull, kSfSlots, &sring);
+      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kSt, ring, sfull, kSfSlots, &sring);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
@@ -283,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             if (st % kStPerSf == kStPerSf - 1 || st == num_st - 1) mma_commit_pair(&sempty[sslot]);
           }
           __syncwarp();
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1;
           }
@@ -299,6 +327,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
         __syncwarp();
       }
     }
+  } else if (kH && warp == 3) {
+    // ------------------------- h loader (both CTAs; SwiGLU backward): for every tile, the
+    // saved g and u of this CTA's 128 rows, one 32-column strip at a time, into each
+    // half's ring in the order that half's epilogue warps drain the strips
+    if (lane == 0) {
+      ArmedRing hring;   // slots half * kHSlots + slot
+      int hs[2] = {0, 0};
+      uint32_t hph[2] = {0, 0};
+      bool ok = true;
+      int lt = 0;
+      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+        const TileInfo ti = walk.decode(t);
+        const int acc = lt & 1;
+        const int r0 = ti.row0 + BMC * (int)rank;   // past R: zero-filled; past the expert: unused
+        const int n0 = ti.n_blk * BN;
+        for (int it = 0; it < 4 && ok; ++it) {
+          for (int hf = 0; hf < 2; ++hf) {
+            const bool owner = acc ? (hf == 0) : (hf == 1);
+            const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * hf + it;
+            const int b = hf * kHSlots + hs[hf];
+            if (!mbar_wait_bounded(&hempty[b], hph[hf] ^ 1, abort_flag, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&hfull[b], kHSlotBytes);
+            hring.arm(b, hph[hf]);
+            uint8_t* dst = sH + b * kHSlotBytes;
+            tma_load_3d(dst, &tmH, &hfull[b], n0 + 32 * c, r0, 0);
+            tma_load_3d(dst + kHSlotBytes / 2, &tmH, &hfull[b], p.F + n0 + 32 * c, r0, 0);
+            if (++hs[hf] == kHSlots) {
+              hs[hf] = 0;
+              hph[hf] ^= 1;
+            }
+          }
+        }
+      }
+      // no copy may still be landing when the CTA leaves
+      hring.drain(hfull, 2 * kHSlots, p.timeout_ns);
+    }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
@@ -306,6 +373,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     const int r_local = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
     const uint32_t tovl_leader = map_to_rank(smem_u32(tovl), 0);
+    // SwiGLU backward: this half's position in its h ring; a thread reads its row's 64
+    // bytes of g and of u (16-byte chunk j of row r at r * 64 + 16 * (j ^ ((r >> 1) & 3)))
+    int hs = 0;
+    uint32_t hph = 0;
+    auto h_fetch = [&](uint4 (&g)[4], uint4 (&u)[4]) {
+      const int b = half * kHSlots + hs;
+      const bool ok = mbar_wait_bounded(&hfull[b], hph, abort_flag, p.timeout_ns);
+      const uint8_t* base = sH + b * kHSlotBytes + r_local * 64;
+      const int sw = (r_local >> 1) & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        g[j] = *reinterpret_cast<const uint4*>(base + ((j ^ sw) << 4));
+        u[j] = *reinterpret_cast<const uint4*>(base + kHSlotBytes / 2 + ((j ^ sw) << 4));
+      }
+      // the slot's next fill is a TMA (async-proxy) write: order these generic-proxy reads
+      // before it, or the copy can land under reads still in flight (seen as
+      // run-to-run differences in a few strips without this fence)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hempty[b]);
+      if (++hs == kHSlots) {
+        hs = 0;
+        hph ^= 1;
+      }
+      return ok;
+    };
     int lt = 0;
     for (int t = pair; t < total; t += npairs, ++lt) {
       const TileInfo ti = walk.decode(t);
@@ -319,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tovl_leader);
           },
-          grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e]);
+          grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e], h_fetch);
       if (EPI == MXEPI_SWIGLU_Q && BMC * (int)rank < ti.rows) {
         // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`; rows
         // past the expert in it store 0 (a CTA entirely past the expert writes nothing)

@@ -43,7 +43,7 @@ constexpr uint32_t kSfbCol = 484;             // B scales: 2 x 4 columns
 enum MxEpiKind : int {
   MXEPI_STORE = 0,      // out[row, col] = bf16(acc) (fp32 with out_f32)
   MXEPI_SWIGLU_Q = 1,   // a = SiLU(g) * u * p quantised to MXFP8 along the columns (+ bf16 h)
-  MXEPI_DSWIGLU = 2,    // SwiGLU backward from da = acc and the saved h: dh, recomputed a (bf16), dprob partials
+  MXEPI_DSWIGLU = 2,    // SwiGLU backward from da = acc and the saved h: dh (MXFP8, both axes), dprob partials
   MXEPI_WGRAD = 3,      // K-grouped: out[e, m, n] = bf16(acc), zeros for an expert without rows
   MXEPI_SWIGLU_F8 = 4,  // per-tensor FP8 fc1: a = SiLU(g) * u * p stored bf16 (+ bf16 h), max |a| kept
   MXEPI_DSWIGLU_F8 = 5, // per-tensor FP8 fc2 dgrad: dh stored bf16, max |dh| kept, dprob partials
@@ -62,8 +62,10 @@ struct MxGemmParams {
   int b_rows;                 // rows of each expert's B (2F for fc1, H for fc2)
   uint8_t* out_atoms;         // MXEPI_SWIGLU_Q: scales of `a` as atoms for the next GEMM (K = F)
   // MXEPI_DSWIGLU: the MXFP8 operands of the backward's remaining GEMMs, quantised in the
-  // epilogue: dh = [dg | du] along its columns (codes [R, 2F], tile atoms, K = 2F), dh and
-  // the recomputed a along each expert's rows (codes [R, 2F] / [R, F], grouped atoms)
+  // epilogue: dh = [dg | du] along its columns (codes [R, 2F], tile atoms, K = 2F) and
+  // along each expert's rows (codes [R, 2F], grouped atoms).
+  // MXEPI_SWIGLU_Q in training: a along each expert's rows (codes [R, F], grouped atoms)
+  // for the fc2 weight gradient.
   uint8_t* dh_rows;
   uint8_t* dh_rows_atoms;
   uint8_t* dh_cols;
@@ -139,12 +141,19 @@ __device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]
 // strip that acc0 and acc1 share is drained first by its owning half, which then calls
 // `strip_done()`; the other half calls it before reading anything (warp-uniform calls, so
 // the callee may signal once per warp). Returns the SwiGLU_Q row's four scale bytes.
-// DSWIGLU also takes the expert's first 128-row group (grp0: groups of earlier experts)
-// and its row count n_e, which place its scale atoms.
-template <int EPI, class StripDone>
+// DSWIGLU also takes the expert's first 128-row group (grp0: groups of earlier experts),
+// its row count n_e, which place its scale atoms, and `h_fetch(g, u)`, which hands this
+// thread the saved h of its row for the next 32-column strip in the order the strips are
+// drained (the caller stages h in shared memory ahead of the epilogue).
+struct NoHFetch {
+  __device__ bool operator()(uint4 (&)[4], uint4 (&)[4]) const { return false; }
+};
+
+template <int EPI, class StripDone, class HFetch = NoHFetch>
 __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, const TileInfo& ti, uint32_t t_row,
                                                        int acc, int half, int r_local, int tile_bm,
-                                                       StripDone&& strip_done, int grp0 = 0, int n_e = 0) {
+                                                       StripDone&& strip_done, int grp0 = 0, int n_e = 0,
+                                                       const HFetch& h_fetch = HFetch{}) {
   using mx::BN;
   const GemmParams& p = mp.g;
   const bool row_ok = r_local < ti.rows;
@@ -220,16 +229,15 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     // MxGemmParams): along its columns (this row's 32-column blocks) and along the
     // expert's rows (32-row blocks = this warp's lanes: a pair tile starts at a multiple
     // of 256 rows of its expert, so the blocks restart at every expert; lanes past the
-    // expert's end count as zeros). With a_cols set, a = SiLU(g) u p is recomputed and
-    // quantised along rows too (the layer's forward normally does that itself).
+    // expert's end count as zeros).
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
     const int n0 = ti.n_blk * BN;
     const int F = p.F, F2 = 2 * p.F;
     const int lane = threadIdx.x & 31;
     const int cta = r_local >> 7;                              // which 128-row group of the tile
     const bool grp_ok = 128 * cta < ti.rows;                   // it holds rows of this expert
     const bool half_ok = n0 + 128 * half < p.N;                // F % 128 == 0: halves are whole
+    const bool live = grp_ok && half_ok;                       // warp-uniform
     const int KG = (n_e + 127) / 128;                          // the expert's 128-row groups
     const int jb = 8 * ti.m_blk + (r_local >> 5);              // this warp's 32-row block of the expert
     const bool owner = acc ? (half == 0) : (half == 1);
@@ -240,22 +248,12 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     for (int it = 0; it < 4; ++it) {
       const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
       const int col = n0 + c * 32;
-      const bool live = grp_ok && half_ok;                     // warp-uniform
-      // the saved h of these 32 columns is requested first, so its global latency overlaps
-      // the tensor-memory loads and their wait
+      // the saved h of these 32 columns, staged in shared memory (every strip is taken,
+      // live or not, so that the staging ring advances in step). Taken before the
+      // tensor-memory loads: nothing may run between a tcgen05.ld and its wait that
+      // could move the registers it is still filling.
       uint4 gva[4], uva[4];
-      if (live && row_ok) {
-        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + col);
-        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + F + col);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          gva[i] = gp[i];
-          uva[i] = up[i];
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) gva[i] = uva[i] = make_uint4(0, 0, 0, 0);
-      }
+      h_fetch(gva, uva);
       uint32_t v0[16], v1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
@@ -265,7 +263,11 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         strip_done();
       }
       if (!live) continue;
-      float dg[32], du[32], av[32];
+      if (!row_ok) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) gva[i] = uva[i] = make_uint4(0, 0, 0, 0);
+      }
+      float dg[32], du[32];
       const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva);
       const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva);
 #pragma unroll
@@ -281,15 +283,13 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
           const float sl = gs[j] * sg;
           dg[k] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
           du[k] = da * pr * sl;
-          av[k] = sl * us[j] * pr;   // zero for lanes without a row (h was zero-filled)
           dp = fmaf(da, sl * us[j], dp);
         }
       }
-      // along the expert's rows (warp-wide blocks): dh for fc1 wgrad, a for fc2 wgrad
+      // along the expert's rows (warp-wide blocks): dh for the fc1 weight gradient
       uint32_t w[8];
       const size_t gcol_dh = (size_t)grp0 * (F2 / 128) + (size_t)KG * (col / 128);
       const size_t gcol_du = (size_t)grp0 * (F2 / 128) + (size_t)KG * ((F + col) / 128);
-      const size_t gcol_a = (size_t)grp0 * (F / 128) + (size_t)KG * (col / 128);
       uint32_t sc = quant_cols_warp32(dg, w, lane);
       mp.dh_cols_atoms[mma_scale_offset(gcol_dh, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
       if (row_ok) {
@@ -303,15 +303,6 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         uint4* d = reinterpret_cast<uint4*>(mp.dh_cols + row * F2 + F + col);
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      }
-      if (mp.a_cols) {
-        sc = quant_cols_warp32(av, w, lane);
-        mp.a_cols_atoms[mma_scale_offset(gcol_a, (col + lane) % 128, jb, 1)] = (uint8_t)sc;
-        if (row_ok) {
-          uint4* d = reinterpret_cast<uint4*>(mp.a_cols + row * F + col);
-          d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          d[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
       }
       // along this row's columns: dh for fc1 dgrad (K = 2F)
       sg_word |= quant_row32(dg, w) << (8 * (c & 3));
@@ -327,7 +318,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
     }
-    if (grp_ok && half_ok) {
+    if (live) {
       // this CTA's 128 rows are row group grp0 + 2 m_blk + cta of dh's tile atoms; rows
       // past the expert store zero scales (their codes are never read)
       const size_t g = (size_t)grp0 + 2 * ti.m_blk + cta;

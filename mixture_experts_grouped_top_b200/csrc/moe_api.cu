@@ -181,20 +181,22 @@ int tmap_atoms(CUtensorMap* m, const void* atoms, uint64_t groups, uint64_t kb4)
 }
 
 // MXFP8 CTA-pair kernels: as many 2-CTA clusters as can be resident at once.
+// th: the saved h for the SwiGLU backward (any map otherwise: unused).
 template <int EPI>
 int launch_gemm_mx_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
-                        const MxGemmParams& p, cudaStream_t st) {
+                        const MxGemmParams& p, cudaStream_t st, const CUtensorMap* th = nullptr) {
   auto kern = grouped_gemm_mxf8_pair_kernel<EPI>;
+  constexpr int kSmem = mx2::smem_bytes(EPI);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int pairs = 0;
   std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mx2::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(device_props().sm_count, 1, 1);
     cfg.blockDim = dim3(mx2::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = mx2::kSmemBytes;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
     int n = 0;
@@ -203,7 +205,7 @@ int launch_gemm_mx_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  kern<<<2 * pairs, mx2::kThreads, mx2::kSmemBytes, st>>>(ta, tb, tsa, tsb, p);
+  kern<<<2 * pairs, mx2::kThreads, kSmem, st>>>(ta, tb, tsa, tsb, th ? *th : ta, p);
   count_launch();
   return launch_status();
 }
@@ -1320,7 +1322,12 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   CUtensorMap tsa, tsb;
   if ((rc = tmap_atoms(&tsa, dyr_a, (uint64_t)R / 128 + E, H / 128))) return rc;
   if ((rc = tmap_atoms(&tsb, w2a, (uint64_t)E * F / 128, H / 128))) return rc;
-  if ((rc = launch_gemm_mx_pair<MXEPI_DSWIGLU>(ta, tb, tsa, tsb, p, st))) return rc;
+  // the saved h, staged into shared memory for the epilogue by TMA (32-column strips)
+  CUtensorMap th;
+  if ((rc = make_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h_saved, 2 * F, R, 1, (uint64_t)4 * F,
+                      (uint64_t)R * 4 * F, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B)))
+    return rc;
+  if ((rc = launch_gemm_mx_pair<MXEPI_DSWIGLU>(ta, tb, tsa, tsb, p, st, &th))) return rc;
   if (dprobs_perm) {
     const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
     reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
