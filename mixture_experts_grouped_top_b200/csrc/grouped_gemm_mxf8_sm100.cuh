@@ -279,7 +279,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         for (int j = 0; j < 2; ++j) {
           const int k = 2 * i + j;
           const float da = row_ok ? __uint_as_float(k < 16 ? v0[k] : v1[k - 16]) : 0.f;
-          const float sg = __frcp_rn(1.0f + expf(-gs[j]));   // the correctly rounded 1 / x
+          const float sg = sigmoid_f(gs[j]);
           const float sl = gs[j] * sg;
           dg[k] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
           du[k] = da * pr * sl;
@@ -382,7 +382,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const float da = __uint_as_float(hh ? v1[2 * i + j] : v0[2 * i + j]) * deq;
-              const float sg = __frcp_rn(1.0f + expf(-gs[j]));
+              const float sg = sigmoid_f(gs[j]);
               const float sl = gs[j] * sg;
               dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
               du[j] = da * pr * sl;

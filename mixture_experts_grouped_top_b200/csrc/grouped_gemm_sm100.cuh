@@ -327,7 +327,7 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const float da = __uint_as_float(v[2 * i + j]);
-              const float sg = __frcp_rn(1.0f + expf(-gs[j]));   // the correctly rounded 1 / x
+              const float sg = sigmoid_f(gs[j]);
               const float sl = gs[j] * sg;
               dg[j] = da * pr * us[j] * (sg * (1.0f + gs[j] * (1.0f - sg)));
               du[j] = da * pr * sl;

@@ -378,7 +378,12 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
 }
 
 // --------------------------------------------------------------- small numerics
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + expf(-g)); }
+// The logistic sigmoid 1 / (1 + e^-g) in fp32 with the fast exponential and divide
+// intrinsics (their error: 2 + floor(1.173 |x|) ulp and 2 ulp); the SwiGLU epilogues
+// evaluate it per element, where the accurate expf and a correctly rounded reciprocal
+// cost a sixth of the fc2-dgrad epilogue's time.
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 // 16 fp32 values -> 16 E4M3 codes (round to nearest even, saturating), packed in 4 words.
 __device__ __forceinline__ void pack_e4m3x16(const float* v, uint32_t (&w)[4]) {

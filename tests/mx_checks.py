@@ -25,40 +25,59 @@ from oracle import mxfp8 as oq
 E4M3 = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
 
 
+U = 2.0 ** -24
+
+
+def sigmoid_terms(g):
+    """s = 1 / (1 + e^-g) and a bound on the relative error of the kernels' fp32 value of
+    it. The kernels take e^-g from the fast exponential intrinsic (CUDA documents at most
+    2 + floor(1.173 |x|) ulp), round 1 + e once and divide with the fast divide (at most
+    2 ulp). An ulp of a float is at most 2 U of its value (U = 2^-24), and a relative
+    error of e reaches s scaled by e / (1 + e) = 1 - s:
+        rel(s) <= (1 - s) (4 + 2.346 |g|) U + U + 4 U."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-g))
+    return s, (1.0 - s) * (4.0 + 2.346 * np.abs(g)) * U + 5.0 * U
+
+
 def swiglu_fp32_error_bound(g, u, p, sum_abs_g, sum_abs_u, K: int):
     """Bound on |a_fp32 - a| for a = SiLU(g) * u * p when g and u are K-term dot products
     accumulated in fp32 by the tensor cores: each K=32 MMA step adds its partial sum into
     the fp32 accumulator, so K/32 + 1 roundings of at most u = 2**-24 times the running
     magnitude (at most sum_k |x_k w_k|) each; a factor 4 covers the MMA's internal
-    alignment of its 32 products. The epilogue's own fp32 work (sigmoid, products) adds a
-    few ulps of |a|."""
-    U = 2.0 ** -24
+    alignment of its 32 products. The epilogue's own fp32 work: the sigmoid's relative
+    error (sigmoid_terms) plus a few roundings of the products."""
     n_add = K // 32 + 1
     eps_g = 4.0 * n_add * U * np.asarray(sum_abs_g, dtype=np.float64)
     eps_u = 4.0 * n_add * U * np.asarray(sum_abs_u, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     u = np.asarray(u, dtype=np.float64)
-    s = 1.0 / (1.0 + np.exp(-g))
+    s, rel_s = sigmoid_terms(g)
     silu = g * s
     dsilu = s * (1.0 + g * (1.0 - s))
-    return np.abs(dsilu * u * p) * eps_g + np.abs(silu * p) * eps_u + 16.0 * U * np.abs(silu * u * p)
+    return np.abs(dsilu * u * p) * eps_g + np.abs(silu * p) * eps_u + (rel_s + 12.0 * U) * np.abs(silu * u * p)
 
 
 def dswiglu_fp32_error_bounds(g, u, p, sum_abs_da, K: int):
     """Bounds on |x_fp32 - x| for the SwiGLU backward's dg, du and the recomputed a, when
     da is a K-term dot product accumulated in fp32 by the tensor cores (the bound of
-    swiglu_fp32_error_bound on da) and g, u, p are exact inputs; the epilogue's own fp32
-    work adds a few ulps of each value (|da| is at most sum |dy w|)."""
-    U = 2.0 ** -24
+    swiglu_fp32_error_bound on da) and g, u, p are exact inputs (|da| is at most
+    sum |dy w|). The epilogue's own fp32 work: the sigmoid's error (sigmoid_terms) moves
+    SiLU'(g) = s (1 + g (1 - s)) by |1 + g - 2 g s| s rel(s) and SiLU(g) by |g| s rel(s),
+    plus a few roundings of each step."""
     eps_da = 4.0 * (K // 32 + 1) * U * np.asarray(sum_abs_da, dtype=np.float64)
+    da_max = np.abs(np.asarray(sum_abs_da, dtype=np.float64))
     g = np.asarray(g, dtype=np.float64)
     u = np.asarray(u, dtype=np.float64)
-    s = 1.0 / (1.0 + np.exp(-g))
+    s, rel_s = sigmoid_terms(g)
     silu = g * s
     dsilu = s * (1.0 + g * (1.0 - s))
-    return (np.abs(p * u * dsilu) * eps_da + 16.0 * U * np.abs(p * u * dsilu) * np.abs(sum_abs_da),
-            np.abs(p * silu) * eps_da + 16.0 * U * np.abs(p * silu) * np.abs(sum_abs_da),
-            16.0 * U * np.abs(silu * u * p))
+    err_dsilu = np.abs(1.0 + g - 2.0 * g * s) * s * rel_s + 8.0 * U * (s + np.abs(g) * s * (1.0 - s))
+    err_silu = np.abs(g) * s * rel_s + 2.0 * U * np.abs(silu)
+    return (np.abs(p * u * dsilu) * eps_da + np.abs(p * u) * da_max * (err_dsilu + 8.0 * U * np.abs(dsilu)),
+            np.abs(p * silu) * eps_da + np.abs(p) * da_max * (err_silu + 8.0 * U * np.abs(silu)),
+            (rel_s + 12.0 * U) * np.abs(silu * u * p))
 
 
 def boundary_flips_grouped_rows(codes, scales, exact, split, err=None, **tol):
