@@ -29,8 +29,9 @@
 // weight-gradient pair kernel, for that one stage both CTAs load with the 1-SM form onto
 // their own barriers; the second CTA's warp 1 zeroes and signals the leader's `rready`.
 //
-// Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [224, 480),
-// A scales at 480, B scales at 484..491 (the M-grouped MXFP8 layout). Waits are bounded.
+// Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [192, 448),
+// four scale sets at 448..495 that warp 2 of the leader fills ahead of the MMA thread
+// (the M-grouped MXFP8 layout, ScaleCopier). Waits are bounded.
 #pragma once
 #include "grouped_gemm_mxf8_pair_sm100.cuh"
 
@@ -100,7 +101,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
   uint64_t* sfull = tovl + 1;                  // scale ring: leader
   uint64_t* sempty = sfull + kSfSlots;         // scale ring: both CTAs
   uint64_t* drained = sempty + kSfSlots;       // second CTA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  uint64_t* setfull = drained + 1;             // tensor-memory scale sets: leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(setfull + mx::kSfSets);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -131,6 +133,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
       mbar_init(&sempty[s2], 1);
     }
     mbar_init(drained, 1);
+    for (int b = 0; b < mx::kSfSets; ++b) {
+      mbar_init(&setfull[b], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -285,12 +290,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
-    int stage = 0, sslot = 0;
-    uint32_t phase = 0, sphase = 0, rmask = 0;
+    int stage = 0;
+    uint32_t phase = 0, rmask = 0;
     int lt = 0;
     bool ok = true;
-    const uint32_t sfa_t = tmem_base + mx::kSfaCol;
-    const uint32_t sfb_t = tmem_base + mx::kSfbCol;
+    ScaleSets sets{setfull, tmem_base};
     for (int t = pair; t < total && ok; t += npairs, ++lt) {
       const TileInfo ti = walk.decode(t);
       const int nst = stages_of(ti);
@@ -299,11 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
       if (lt > 0 && !mbar_wait_bounded<true>(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (acc ? mx::kAcc1Col : 0u);
-      for (int st = 0; st < nst; ++st) {
-        if (st % kStPerSf == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
+      for (int st = 0; st < nst && ok; ++st) {
         if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
           ok = false;
           break;
@@ -323,46 +323,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
           rmask ^= 1u << stage;
           tc_fence_after();
         }
-        if (lane == 0) {
-          const uint32_t sf_s = smem_u32(sSf + sslot * kSfSlotBytes);
-          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+        const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+        const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+        for (int c = 0; c < kGroupsPerStage; ++c) {
+          if (4 * c >= ksteps) break;
+          // this k-group's scale atoms, copied into tensor memory by the scale warp
+          if (!sets.wait(abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sfa = sets.sfa(), sfb = sets.sfb();
 #pragma unroll
-          for (int c = 0; c < kGroupsPerStage; ++c) {
-            if (4 * c < ksteps) {
-              // this k-group's atoms: entry kg % 4 of each 2 KB group of the slot
-              const uint32_t q = (uint32_t)((kGroupsPerStage * st + c) & (kSfKg - 1)) * 512;
-              tmem_cp_32x128b_warpx4_pair(sfa_t, make_sdesc(sf_s + q, 0, 128, 0));
-              tmem_cp_32x128b_warpx4_pair(sfb_t, make_sdesc(sf_s + kSfGroupBytes + q, 0, 128, 0));
-              tmem_cp_32x128b_warpx4_pair(sfb_t + 4, make_sdesc(sf_s + 2 * kSfGroupBytes + q, 0, 128, 0));
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                if (4 * c + kk < ksteps) {
-                  // MN-major: 32 k rows = 4096 bytes further (four 8-row swizzle atoms)
-                  const uint32_t off = (uint32_t)(4 * c + kk) * 4096;
-                  const uint64_t adesc = make_sdesc(a_addr + off, kABytes, 1024, 2);
-                  const uint64_t bdesc = make_sdesc(b_addr + off, kBBytes, 1024, 2);
-                  const uint32_t idesc = make_idesc_mxf8(BM, BN, true, true, kk, kk) | mp.ab_fmt;
-                  mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30),
-                                sfb_t | ((uint32_t)kk << 30), (st > 0 || c > 0 || kk > 0) ? 1u : 0u);
-                }
+            for (int kk = 0; kk < 4; ++kk) {
+              if (4 * c + kk < ksteps) {
+                // MN-major: 32 k rows = 4096 bytes further (four 8-row swizzle atoms)
+                const uint32_t off = (uint32_t)(4 * c + kk) * 4096;
+                const uint64_t adesc = make_sdesc(a_addr + off, kABytes, 1024, 2);
+                const uint64_t bdesc = make_sdesc(b_addr + off, kBBytes, 1024, 2);
+                const uint32_t idesc = make_idesc_mxf8(BM, BN, true, true, kk, kk) | mp.ab_fmt;
+                mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
+                              (st > 0 || c > 0 || kk > 0) ? 1u : 0u);
               }
             }
           }
-          mma_commit_pair(&empty[stage]);
-          // the slot's last stage: release it once these MMAs have read their scales
-          if (st % kStPerSf == kStPerSf - 1 || st == nst - 1) mma_commit_pair(&sempty[sslot]);
+          sets.next();
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) mma_commit_pair(&empty[stage]);
         __syncwarp();
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;
-        }
-        if (st % kStPerSf == kStPerSf - 1 || st == nst - 1) {
-          if (++sslot == kSfSlots) {
-            sslot = 0;
-            sphase ^= 1;
-          }
         }
       }
       if (!ok) break;
@@ -370,6 +364,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mkp::kThreads, 1)
       // done and the epilogue writes zeros)
       if (lane == 0) mma_commit_pair(&tfull[acc]);
       __syncwarp();
+    }
+  } else if (warp == 2) {
+    // ------------------------------------ scale copies (pair leader): every k-group's
+    // atoms into the next tensor-memory scale set, ahead of the MMA thread
+    if (leader && lane == 0) {
+      ScaleCopier<kSfKg> cp{sfull, sempty, setfull, empty, kStages, sSf, kSfSlots, tmem_base, abort_flag, p.timeout_ns};
+      bool ok = true;
+      int g0 = 0;   // global stage of the tile's first k-group
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileInfo ti = walk.decode(t);
+        const int nkg = (ti.rows + 127) / 128;   // k-groups holding the expert's rows
+        for (int kg = 0; kg < nkg && ok; ++kg) ok = cp.copy(kg, kg == nkg - 1, g0 + kg / kGroupsPerStage);
+        g0 += stages_of(ti);
+      }
+      cp.drain();
     }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue (both CTAs)

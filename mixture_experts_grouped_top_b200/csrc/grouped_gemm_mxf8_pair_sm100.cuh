@@ -16,16 +16,17 @@
 //   * scale atoms travel on their own two-slot ring, four k-blocks per copy (2 KB): per
 //     two stages, one copy for this CTA's A rows and two for the B tile's two 128-row
 //     groups (the block-scaled pair MMA reads every N column's scales from each CTA's own
-//     tensor memory, so both CTAs fetch both B groups). The leader copies a k-block's
-//     atoms into both CTAs' tensor memory (tcgen05.cp.cta_group::2) before its MMAs.
+//     tensor memory, so both CTAs fetch both B groups). Warp 2 of the leader copies each
+//     k-block's atoms into both CTAs' tensor memory (tcgen05.cp.cta_group::2), into the
+//     next of four scale sets, ahead of the MMA thread (ScaleCopier).
 //
 // The SwiGLU backward's epilogue also needs the saved h = [g | u] of every row it drains:
 // warp 3 of each CTA copies it with TMA into a shared-memory ring of 32-column strips,
 // ahead of the epilogue, which reads its row from there (coalesced copies instead of one
 // 16-byte load per row and lane from global memory).
 //
-// Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [224, 480),
-// A scales at 480, B scales at 484..491; `tovl` and `tempty` live in the leader and count
+// Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [192, 448),
+// four scale sets at 448..495; `tovl` and `tempty` live in the leader and count
 // one arrival per epilogue warp of both CTAs. Waits are bounded like in every other
 // kernel of this library.
 #pragma once
@@ -107,7 +108,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   uint64_t* drained = sempty + kSfSlots;      // used in the second CTA
   uint64_t* hfull = drained + 1;              // h ring (half * kHSlots + slot): both CTAs
   uint64_t* hempty = hfull + 2 * kHSlots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 2 * kHSlots);
+  uint64_t* setfull = hempty + 2 * kHSlots;   // tensor-memory scale sets: used in the leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(setfull + mx::kSfSets);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* row_off = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
@@ -128,6 +130,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     for (int b = 0; b < 2 * kHSlots; ++b) {
       mbar_init(&hfull[b], 1);
       mbar_init(&hempty[b], 4);   // the four epilogue warps of a half
+    }
+    for (int b = 0; b < mx::kSfSets; ++b) {
+      mbar_init(&setfull[b], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -261,71 +266,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
     if (leader) {
-      int stage = 0, sslot = 0;
-      uint32_t phase = 0, sphase = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       int lt = 0;
       bool ok = true;
-      const uint32_t sfa_t = tmem_base + mx::kSfaCol;
-      const uint32_t sfb_t = tmem_base + mx::kSfbCol;
+      ScaleSets sets{setfull, tmem_base};
       for (int t = pair; t < total && ok; t += npairs, ++lt) {
         const int acc = lt & 1;
         if (!mbar_wait_bounded<true>(&tempty[acc], ((lt >> 1) & 1) ^ 1, abort_flag, p.timeout_ns)) break;
         if (lt > 0 && !mbar_wait_bounded<true>(tovl, (lt - 1) & 1, abort_flag, p.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc ? mx::kAcc1Col : 0u);
-        for (int st = 0; st < num_st; ++st) {
-          if (st % kStPerSf == 0 && !mbar_wait_bounded(&sfull[sslot], sphase, abort_flag, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
+        for (int st = 0; st < num_st && ok; ++st) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sf_s = smem_u32(sSf + sslot * kSfSlotBytes);
-            const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-            const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-              const int kb = kChunks * st + c;
-              if (kb < kblocks) {
-                // this k-block's atoms: entry kb % 4 of each 2 KB group of the slot
-                const uint32_t q = (uint32_t)(kb & (kSfKb - 1)) * 512;
-                tmem_cp_32x128b_warpx4_pair(sfa_t, make_sdesc(sf_s + q, 0, 128, 0));
-                tmem_cp_32x128b_warpx4_pair(sfb_t, make_sdesc(sf_s + kSfGroupBytes + q, 0, 128, 0));
-                tmem_cp_32x128b_warpx4_pair(sfb_t + 4, make_sdesc(sf_s + 2 * kSfGroupBytes + q, 0, 128, 0));
+          for (int c = 0; c < kChunks; ++c) {
+            const int kb = kChunks * st + c;
+            if (kb >= kblocks) break;
+            // this k-block's scale atoms, copied into tensor memory by the scale warp
+            if (!sets.wait(abort_flag, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t sfa = sets.sfa(), sfb = sets.sfb();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t adesc = make_sdesc(a_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
-                  const uint64_t bdesc = make_sdesc(b_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
-                  const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk) | mp.ab_fmt;
-                  mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | ((uint32_t)kk << 30),
-                                sfb_t | ((uint32_t)kk << 30), (kb > 0 || kk > 0) ? 1u : 0u);
-                }
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = make_sdesc(a_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
+                const uint64_t bdesc = make_sdesc(b_addr + c * kChunkBytes + kk * 32, 16, 1024, 2);
+                const uint32_t idesc = make_idesc_mxf8(BM, BN, false, false, kk, kk) | mp.ab_fmt;
+                mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa | ((uint32_t)kk << 30), sfb | ((uint32_t)kk << 30),
+                              (kb > 0 || kk > 0) ? 1u : 0u);
               }
             }
-            mma_commit_pair(&empty[stage]);
-            // the slot's last stage: release it once these MMAs have read their scales
-            if (st % kStPerSf == kStPerSf - 1 || st == num_st - 1) mma_commit_pair(&sempty[sslot]);
+            sets.next();
+            __syncwarp();
           }
+          if (!ok) break;
+          if (lane == 0) mma_commit_pair(&empty[stage]);
           __syncwarp();
           if (++stage == kSt) {
             stage = 0;
             phase ^= 1;
-          }
-          if (st % kStPerSf == kStPerSf - 1 || st == num_st - 1) {
-            if (++sslot == kSfSlots) {
-              sslot = 0;
-              sphase ^= 1;
-            }
           }
         }
         if (!ok) break;
         if (lane == 0) mma_commit_pair(&tfull[acc]);
         __syncwarp();
       }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------ scale copies (pair leader): every k-block's
+    // atoms into the next tensor-memory scale set, ahead of the MMA thread
+    if (leader && lane == 0) {
+      ScaleCopier<kSfKb> cp{sfull, sempty, setfull, empty, kSt, sSf, kSfSlots, tmem_base, abort_flag, p.timeout_ns};
+      bool ok = true;
+      int g0 = 0;   // global stage of the tile's first k-block
+      for (int t = pair; t < total && ok; t += npairs, g0 += num_st)
+        for (int kb = 0; kb < kblocks && ok; ++kb) ok = cp.copy(kb, kb == kblocks - 1, g0 + kb / kChunks);
+      cp.drain();
     }
   } else if (kH && warp == 3) {
     // ------------------------- h loader (both CTAs; SwiGLU backward): for every tile, the
@@ -344,8 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
         const int n0 = ti.n_blk * BN;
         for (int it = 0; it < 4 && ok; ++it) {
           for (int hf = 0; hf < 2; ++hf) {
-            const bool owner = acc ? (hf == 0) : (hf == 1);
-            const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * hf + it;
+            const int c = strip8(acc, hf, it);
             const int b = hf * kHSlots + hs[hf];
             if (!mbar_wait_bounded(&hempty[b], hph[hf] ^ 1, abort_flag, p.timeout_ns)) {
               ok = false;
@@ -414,12 +418,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
           },
           grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e], h_fetch);
       if (EPI == MXEPI_SWIGLU_Q && BMC * (int)rank < ti.rows) {
-        // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`; rows
-        // past the expert in it store 0 (a CTA entirely past the expert writes nothing)
+        // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`: the bytes
+        // of this half's two a-strips (rows past the expert store 0; a CTA entirely past
+        // the expert writes nothing)
         const size_t g = (size_t)(grp_off[ti.e] + 2 * ti.m_blk + (int)rank);
-        *reinterpret_cast<uint16_t*>(mp.out_atoms + mma_scale_offset(g, r_local, 4 * ti.n_blk + 2 * half,
-                                                                     p.N / 128)) =
-            (uint16_t)(sc_word >> (16 * half));
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int c = strip4(acc, half, it);
+          mp.out_atoms[mma_scale_offset(g, r_local, 4 * ti.n_blk + c, p.N / 128)] = (uint8_t)(sc_word >> (8 * c));
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -18,14 +18,20 @@
 //     consecutive k-blocks contiguous: they travel on a two-slot ring of their own, one
 //     copy per row group (A, and B's two 128-row halves) per four k-blocks, since a copy
 //     costs the copy engine about the same whatever its size;
-//   * the MMA thread moves the atoms into tensor memory with tcgen05.cp (32 lanes x 16 B,
-//     replicated to the four sub-partitions), then issues the four K=32 MMAs of the
-//     k-block, selecting scale byte kk of each word through the scale-factor ids;
-//   * two 256-column accumulators plus 12 scale columns exceed the 512 tensor-memory
-//     columns, so the accumulators overlap: acc0 = columns [0, 256), acc1 = [224, 480),
-//     scales at [480, 492). The epilogue drains the shared 32-column strip first and
-//     signals `tovl`; the next tile's MMAs wait for that strip (and for the full drain
-//     of the tile two back) instead of the whole previous epilogue.
+//   * a warp of its own moves each k-block's atoms into tensor memory with tcgen05.cp
+//     (32 lanes x 16 B, replicated to the four sub-partitions), into the next of four
+//     scale sets, ahead of the MMA thread, which issues the four K=32 MMAs of the k-block
+//     from that set, selecting scale byte kk of each word through the scale-factor ids.
+//     Copies issued by the MMA thread itself, right before its MMAs, held its tensor-core
+//     stream (tensor pipe active 65% with them, 82% with the copies on another warp: fc2 of
+//     the Mixtral MXFP8 forward, 2048 tokens), and with only two sets the handoff between
+//     the warps left the MMA thread waiting (56%); see ScaleCopier;
+//   * two 256-column accumulators plus the scale sets exceed the 512 tensor-memory
+//     columns, so the accumulators overlap: acc0 = columns [0, 256), acc1 = [192, 448),
+//     four 12-column scale sets at [448, 496). The epilogue drains the two shared 32-column
+//     strips first (one per half, strip8 / strip4) and signals `tovl`; the next tile's MMAs
+//     wait for them (and for the full drain of the tile two back) instead of the whole
+//     previous epilogue.
 #pragma once
 #include "grouped_gemm_sm100.cuh"
 #include "token_kernels.cuh"
@@ -35,9 +41,11 @@ namespace moe {
 namespace mx {
 // tensor-memory layout shared by the MXFP8 pair kernels (columns of each CTA's 512)
 constexpr int BN = 256;                       // accumulator columns per tile
-constexpr uint32_t kAcc1Col = 224;            // acc0 = [0, 256), acc1 = [224, 480)
-constexpr uint32_t kSfaCol = 480;             // A scales: 4 columns
-constexpr uint32_t kSfbCol = 484;             // B scales: 2 x 4 columns
+constexpr uint32_t kAcc1Col = 192;            // acc0 = [0, 256), acc1 = [192, 448)
+constexpr uint32_t kSfaCol = 448;             // A scales of set 0: 4 columns
+constexpr uint32_t kSfbCol = 452;             // B scales of set 0: 2 x 4 columns
+constexpr uint32_t kSfSetCols = 12;           // set s at 448 + 12 s
+constexpr int kSfSets = 4;                    // [448, 496)
 }  // namespace mx
 
 enum MxEpiKind : int {
@@ -136,11 +144,110 @@ __device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]
   return (uint32_t)code;
 }
 
+// Scale-set handoff between the scale-copy warp and the MMA thread of a CTA pair (both in
+// the leader). The copier takes k-block kb's atoms from the scale ring in shared memory
+// (slots of kPerSlot k-blocks, 3 groups of kPerSlot atoms: A, B lower, B upper) into the
+// next of mx::kSfSets tensor-memory sets, round robin, and commits `setfull[set]`; the
+// MMA thread waits for it and issues the k-block's MMAs from that set. A set is free again
+// once the MMAs of the k-block that used it before are done: the copier learns that from
+// the operand ring's `empty` barrier of that k-block's stage, which the MMA thread commits
+// anyway (an extra commit per k-block held the MMA thread's stream, like the copies
+// themselves). The copier releases a scale-ring slot (`sempty`) once the copies of its
+// last k-block are done. Bounded waits; all barriers count one arrival.
+template <int kPerSlot>
+struct ScaleCopier {
+  uint64_t* sfull;
+  uint64_t* sempty;
+  uint64_t* setfull;
+  uint64_t* empty;            // the operand ring's stage barriers (nstages slots)
+  int nstages;
+  const uint8_t* ring;        // slot s at ring + s * 3 * kPerSlot * 512
+  int nslots;
+  uint32_t tmem_base;
+  volatile int* abort;
+  uint64_t timeout_ns;
+  int slot = 0, set = 0;
+  uint32_t sphase = 0;
+  uint32_t par = 0;           // bit s: parity of the copies committed into set s so far
+  uint32_t used = 0;          // bit s: set s received copies
+  int q0 = -1, q1 = -1, q2 = -1, q3 = -1;   // global stages of the last four k-blocks copied
+
+  // the atoms of k-block kb of the current tile, whose operands are global stage `gstage`
+  // of the operand ring; `last`: the tile's last k-block
+  __device__ __forceinline__ bool copy(int kb, bool last, int gstage) {
+    static_assert(mx::kSfSets == 4, "the stage history below holds four k-blocks");
+    const int q = kb % kPerSlot;
+    if (q == 0 && !mbar_wait_bounded(&sfull[slot], sphase, abort, timeout_ns)) return false;
+    // the set's previous k-block (four copies back): its stage's MMAs must be done
+    if (q0 >= 0 && !mbar_wait_bounded(&empty[q0 % nstages], (uint32_t)(q0 / nstages) & 1u, abort, timeout_ns))
+      return false;
+    q0 = q1;
+    q1 = q2;
+    q2 = q3;
+    q3 = gstage;
+    tc_fence_after();
+    const uint32_t src = smem_u32(ring + (size_t)slot * 3 * kPerSlot * 512) + (uint32_t)q * 512;
+    const uint32_t sfa = tmem_base + mx::kSfaCol + (uint32_t)set * mx::kSfSetCols;
+    const uint32_t sfb = tmem_base + mx::kSfbCol + (uint32_t)set * mx::kSfSetCols;
+    tmem_cp_32x128b_warpx4_pair(sfa, make_sdesc(src, 0, 128, 0));
+    tmem_cp_32x128b_warpx4_pair(sfb, make_sdesc(src + kPerSlot * 512, 0, 128, 0));
+    tmem_cp_32x128b_warpx4_pair(sfb + 4, make_sdesc(src + 2 * kPerSlot * 512, 0, 128, 0));
+    mma_commit_pair(&setfull[set]);
+    if (q == kPerSlot - 1 || last) {
+      mma_commit_pair(&sempty[slot]);
+      if (++slot == nslots) {
+        slot = 0;
+        sphase ^= 1u;
+      }
+    }
+    par ^= 1u << set;
+    used |= 1u << set;
+    set = (set + 1) % mx::kSfSets;
+    return true;
+  }
+  // on the way out: wait (bounded) until the last copies into each set have landed (the
+  // last commit into set s completed phase parity ((par >> s) & 1) ^ 1)
+  __device__ __forceinline__ void drain() const {
+    for (int s_ = 0; s_ < mx::kSfSets; ++s_)
+      if ((used >> s_) & 1u) mbar_wait_drain(&setfull[s_], ((par >> s_) & 1u) ^ 1u, timeout_ns);
+  }
+};
+
+// The MMA thread's side of the handoff: which set the next k-block reads.
+struct ScaleSets {
+  uint64_t* setfull;
+  uint32_t tmem_base;
+  int set = 0;
+  uint32_t par = 0;           // bit s: parity of the next fill of set s to wait for
+  __device__ __forceinline__ bool wait(volatile int* abort, uint64_t timeout_ns) const {
+    return mbar_wait_bounded(&setfull[set], (par >> set) & 1u, abort, timeout_ns);
+  }
+  __device__ __forceinline__ uint32_t sfa() const { return tmem_base + mx::kSfaCol + (uint32_t)set * mx::kSfSetCols; }
+  __device__ __forceinline__ uint32_t sfb() const { return tmem_base + mx::kSfbCol + (uint32_t)set * mx::kSfSetCols; }
+  // after the k-block's MMAs are issued (every lane advances)
+  __device__ __forceinline__ void next() {
+    par ^= 1u << set;
+    set = (set + 1) % mx::kSfSets;
+  }
+};
+
+// The 32-column strips of a 256-column accumulator that the two halves of the epilogue
+// warps drain, in order: half h takes strips h, h+2, h+4, h+6 (SwiGLU epilogues: a-strips
+// h and h+2, a-strip c reading gate strip c and up strip 4 + c). acc0 and acc1 share 64
+// columns, acc0's strips 6 and 7 and acc1's strips 0 and 1, one per half: each half
+// drains its shared strip first, so that the next tile's MMAs may start writing there.
+__host__ __device__ constexpr int strip8(int acc, int half, int it) {
+  return acc ? half + 2 * it : (it == 0 ? 6 + half : half + 2 * (it - 1));
+}
+__host__ __device__ constexpr int strip4(int acc, int half, int it) {
+  return acc ? half + 2 * it : (it == 0 ? 2 + half : half);
+}
+
 // Drains one 128-row x 256-column accumulator (this thread's row: lane quadrant of
-// `t_row`, row r_local of the output tile) and runs the epilogue EPI on it. The 32-column
-// strip that acc0 and acc1 share is drained first by its owning half, which then calls
-// `strip_done()`; the other half calls it before reading anything (warp-uniform calls, so
-// the callee may signal once per warp). Returns the SwiGLU_Q row's four scale bytes.
+// `t_row`, row r_local of the output tile) and runs the epilogue EPI on it, strip by strip
+// (strip8 / strip4); after its first strip every warp calls `strip_done()` (warp-uniform
+// calls, so the callee may signal once per warp). Returns the SwiGLU_Q row's scale bytes
+// (byte c: a-strip c; the bytes of the other half's strips are 0).
 // DSWIGLU also takes the expert's first 128-row group (grp0: groups of earlier experts),
 // its row count n_e, which place its scale atoms, and `h_fetch(g, u)`, which hands this
 // thread the saved h of its row for the next 32-column strip in the order the strips are
@@ -175,19 +282,15 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
       ok_row = row_ok;
       orow = row * p.ldo;
     }
-    // the 32-column strip shared with the other accumulator: chunk 7 of acc0 (upper
-    // half), chunk 0 of acc1 (lower half); its owner drains it first, then signals
-    const bool owner = acc ? (half == 0) : (half == 1);
-    if (!owner) strip_done();
     const float deq = mx_deq_factor(mp, EPI == MXEPI_WGRAD ? 0 : ti.e);
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
-      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      const int c = strip8(acc, half, it);
       uint32_t v0[16], v1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
       tmem_wait_ld();
-      if (owner && it == 0) {
+      if (it == 0) {
         tc_fence_before();
         strip_done();
       }
@@ -236,18 +339,16 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     const int lane = threadIdx.x & 31;
     const int cta = r_local >> 7;                              // which 128-row group of the tile
     const bool grp_ok = 128 * cta < ti.rows;                   // it holds rows of this expert
-    const bool half_ok = n0 + 128 * half < p.N;                // F % 128 == 0: halves are whole
-    const bool live = grp_ok && half_ok;                       // warp-uniform
     const int KG = (n_e + 127) / 128;                          // the expert's 128-row groups
     const int jb = 8 * ti.m_blk + (r_local >> 5);              // this warp's 32-row block of the expert
-    const bool owner = acc ? (half == 0) : (half == 1);
-    if (!owner) strip_done();
+    // this CTA's 128 rows are row group grp0 + 2 m_blk + cta of dh's tile atoms
+    const size_t g_rows = (size_t)grp0 + 2 * ti.m_blk + cta;
     float dp = 0.f;
-    uint32_t sg_word = 0, su_word = 0;   // this row's scale codes of its four dg / du blocks
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
-      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      const int c = strip8(acc, half, it);
       const int col = n0 + c * 32;
+      const bool live = grp_ok && col < p.N;                   // warp-uniform
       // the saved h of these 32 columns, staged in shared memory (every strip is taken,
       // live or not, so that the staging ring advances in step). Taken before the
       // tensor-memory loads: nothing may run between a tcgen05.ld and its wait that
@@ -258,7 +359,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
       tmem_wait_ld();
-      if (owner && it == 0) {
+      if (it == 0) {
         tc_fence_before();
         strip_done();
       }
@@ -304,29 +405,22 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
-      // along this row's columns: dh for fc1 dgrad (K = 2F)
-      sg_word |= quant_row32(dg, w) << (8 * (c & 3));
+      // along this row's columns: dh for fc1 dgrad (K = 2F); rows past the expert store
+      // zero scales (their codes are never read)
+      uint32_t code = quant_row32(dg, w);
+      mp.dh_rows_atoms[mma_scale_offset(g_rows, r_local & 127, col / 32, F2 / 128)] = row_ok ? (uint8_t)code : 0;
       if (row_ok) {
         uint4* d = reinterpret_cast<uint4*>(mp.dh_rows + row * F2 + col);
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
-      su_word |= quant_row32(du, w) << (8 * (c & 3));
+      code = quant_row32(du, w);
+      mp.dh_rows_atoms[mma_scale_offset(g_rows, r_local & 127, (F + col) / 32, F2 / 128)] = row_ok ? (uint8_t)code : 0;
       if (row_ok) {
         uint4* d = reinterpret_cast<uint4*>(mp.dh_rows + row * F2 + F + col);
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
-    }
-    if (live) {
-      // this CTA's 128 rows are row group grp0 + 2 m_blk + cta of dh's tile atoms; rows
-      // past the expert store zero scales (their codes are never read)
-      const size_t g = (size_t)grp0 + 2 * ti.m_blk + cta;
-      const int kb_g = (n0 + 128 * half) / 32, kb_u = (F + n0 + 128 * half) / 32;
-      *reinterpret_cast<uint32_t*>(mp.dh_rows_atoms + mma_scale_offset(g, r_local & 127, kb_g, F2 / 128)) =
-          row_ok ? sg_word : 0u;
-      *reinterpret_cast<uint32_t*>(mp.dh_rows_atoms + mma_scale_offset(g, r_local & 127, kb_u, F2 / 128)) =
-          row_ok ? su_word : 0u;
     }
     if (row_ok) p.dprob_part[(long long)(2 * ti.n_blk + half) * p.M + row] = dp;
   } else if (EPI == MXEPI_DSWIGLU_F8) {
@@ -338,12 +432,10 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
     const int n0 = ti.n_blk * BN;
     const float deq = mx_deq_factor(mp, ti.e);
-    const bool owner = acc ? (half == 0) : (half == 1);
-    if (!owner) strip_done();
     float dp = 0.f, amax = 0.f;
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
-      const int c = owner ? (acc ? it : (it == 0 ? 7 : 3 + it)) : 4 * half + it;
+      const int c = strip8(acc, half, it);
       const int col = n0 + c * 32;
       const bool cols_ok = row_ok && col < p.N;
       uint4 gva[4], uva[4];
@@ -360,7 +452,7 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
       tmem_ld_32x32b_x16(t_row + c * 32, v0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, v1);
       tmem_wait_ld();
-      if (owner && it == 0) {
+      if (it == 0) {
         tc_fence_before();
         strip_done();
       }
@@ -414,19 +506,17 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     const float deq = mx_deq_factor(mp, ti.e);
     __nv_bfloat16* a_out = reinterpret_cast<__nv_bfloat16*>(p.out);
     __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
-    const bool owner = acc ? (half == 0) : (half == 1);
-    if (!owner) strip_done();
     float amax = 0.f;
 #pragma unroll 1
     for (int it = 0; it < 2; ++it) {
-      const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
+      const int c = strip4(acc, half, it);
       uint32_t g0[16], g1[16], u0[16], u1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, g0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
       tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
       tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
       tmem_wait_ld();
-      if (owner && it == 0) {
+      if (it == 0) {
         tc_fence_before();
         strip_done();
       }
@@ -475,20 +565,18 @@ __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, c
     const int jb = 8 * ti.m_blk + (r_local >> 5);            // this warp's 32-row block of the expert
     uint8_t* a_codes = reinterpret_cast<uint8_t*>(p.out);
     __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(p.out2);
-    // output chunk 3 of acc0 (its up columns are the shared strip) belongs to the
-    // upper half, chunk 0 of acc1 (gate columns) to the lower half
-    const bool owner = acc ? (half == 0) : (half == 1);
-    if (!owner) strip_done();
+    // a-strips in strip4 order: acc0 shares the up columns of a-strips 2 and 3, acc1 the
+    // gate columns of a-strips 0 and 1, one of each per half
 #pragma unroll 1
     for (int it = 0; it < 2; ++it) {
-      const int c = owner ? (acc ? it : 3 - it) : 2 * half + it;
+      const int c = strip4(acc, half, it);
       uint32_t g0[16], g1[16], u0[16], u1[16];
       tmem_ld_32x32b_x16(t_row + c * 32, g0);
       tmem_ld_32x32b_x16(t_row + c * 32 + 16, g1);
       tmem_ld_32x32b_x16(t_row + 128 + c * 32, u0);
       tmem_ld_32x32b_x16(t_row + 128 + c * 32 + 16, u1);
       tmem_wait_ld();
-      if (owner && it == 0) {
+      if (it == 0) {
         tc_fence_before();
         strip_done();
       }

@@ -874,6 +874,7 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __
                                                          uint8_t* __restrict__ codes,
                                                          uint8_t* __restrict__ scales) {
   __shared__ __align__(16) uint8_t tile[32][256 + 16];
+  __shared__ __align__(16) __nv_bfloat16 in_tile[32][256];
   const int b = blockIdx.z;
   const int r0 = blockIdx.y * 32;
   const int c0 = blockIdx.x * 256;
@@ -884,7 +885,23 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __
   uint8_t* sdst = scales + (size_t)b * (rows / 32) * cols;
   float f[32];
   float amax = 0.f;
-  if (c < cols) {
+  if ((cols & 7) == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0) {
+    // the 32 x 256 input tile with 16-byte loads (a warp reads one 512-byte row segment),
+    // then each thread takes its column from shared memory
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = j + 256 * i, row = idx >> 5, cv = (idx & 31) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (c0 + cv < cols) v = *reinterpret_cast<const uint4*>(src + (size_t)(r0 + row) * cols + c0 + cv);
+      *reinterpret_cast<uint4*>(&in_tile[row][cv]) = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      f[i] = __bfloat162float(in_tile[i][j]);
+      amax = fmaxf(amax, fabsf(f[i]));
+    }
+  } else if (c < cols) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       f[i] = __bfloat162float(src[(size_t)(r0 + i) * cols + c]);

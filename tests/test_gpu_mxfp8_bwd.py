@@ -178,3 +178,35 @@ def test_mxfp8_backward_close_to_bf16_definition():
         err = np.max(np.abs(g.float().cpu().numpy() - r)) / np.max(np.abs(r))
         print(f"MXFP8 backward {name}: rel err vs unquantised definition {err:.3e}")
         assert err <= 0.25   # MXFP8 rounding of the method itself (dw2 contracts over ~128 rows here)
+
+
+def test_mxfp8_layer_bitwise_deterministic():
+    """Two forward+backward passes over the same inputs give the same bits, fused codes
+    included. A race between a producer and a consumer inside a kernel (for instance the
+    staging of the saved h for the fc2-dgrad epilogue) shows up here as run-to-run
+    differences in a few strips long before it breaks a tolerance; the size gives each
+    CTA pair tens of tiles."""
+    T, H, F, E, k = 16384, 2048, 4096, 8, 2
+    g = torch.Generator(device=DEV)
+    g.manual_seed(7)
+    x = torch.randn(T, H, device=DEV, generator=g).to(torch.bfloat16)
+    logits = torch.randn(T, E, device=DEV, generator=g)
+    w1 = (torch.randn(E, H, 2 * F, device=DEV, generator=g) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(E, F, H, device=DEV, generator=g) * 0.02).to(torch.bfloat16)
+    gy = torch.randn(T, H, device=DEV, generator=g).to(torch.bfloat16)
+    layer = mb.MoEExpertLayer(T, H, F, E, k, precision="mxfp8", training=True)
+    layer.set_weights(w1, w2)
+    R = T * k
+    parts = [mb.grouped_mlp_bwd_workspace_offset(E, R, H, F, "mxfp8", i) for i in (8, 9)]
+    runs = []
+    for _ in range(2):
+        out = layer.forward(x, logits).clone()
+        dx, dw1, dw2, dprob = (t.clone() for t in layer.backward(gy))
+        ws = layer._bwd["ws"]
+        codes = [ws[o: o + R * 2 * F].clone() for o in parts]
+        runs.append([out, dx, dw1, dw2, dprob, layer.saved.clone()] + codes)
+        assert mb.moe_device_status() == 0
+    names = ["out", "dx", "dw1", "dw2", "dprob", "saved", "dh codes (2F)", "dh codes (rows)"]
+    for name, a, b in zip(names, *runs):
+        assert torch.equal(a.view(torch.uint8) if a.dtype != torch.uint8 else a,
+                           b.view(torch.uint8) if b.dtype != torch.uint8 else b), f"{name} differs between runs"
