@@ -252,10 +252,6 @@ __host__ __device__ constexpr int strip4(int acc, int half, int it) {
 // its row count n_e, which place its scale atoms, and `h_fetch(g, u)`, which hands this
 // thread the saved h of its row for the next 32-column strip in the order the strips are
 // drained (the caller stages h in shared memory ahead of the epilogue).
-struct NoHFetch {
-  __device__ bool operator()(uint4 (&)[4], uint4 (&)[4]) const { return false; }
-};
-
 template <int EPI, class StripDone, class HFetch = NoHFetch>
 __device__ __forceinline__ uint32_t mxf8_epilogue_tile(const MxGemmParams& mp, const TileInfo& ti, uint32_t t_row,
                                                        int acc, int half, int r_local, int tile_bm,

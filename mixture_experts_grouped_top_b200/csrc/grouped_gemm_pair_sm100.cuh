@@ -20,6 +20,11 @@
 // For fc1 the leader's half of B is the gate columns [n0, n0+128) and the other CTA's
 // the up columns [F+n0, F+n0+128), so each CTA's accumulator holds [gate | up] for its
 // rows and the ScaledSwiGLU epilogue stays thread-local.
+//
+// SwiGLU backward: warp 3 of each CTA copies the saved h of the rows being drained with
+// TMA into a shared-memory ring of 32-column strips, ahead of the epilogue, which reads its
+// row from there instead of one 16-byte global load per row and lane (as in the MXFP8
+// pair kernel).
 #pragma once
 #include "grouped_gemm_sm100.cuh"
 
@@ -38,29 +43,49 @@ constexpr int kChunkBytes = 128 * 64 * 2;     // one 64-element chunk of 128 row
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024 + 2 * (kMaxE + 1) * 4;
+// SwiGLU backward: the saved h reaches the epilogue through shared memory, a two-slot
+// ring of 32-column strips (g and u of the CTA's 128 rows, 64-byte swizzled: 16 KB) per
+// column half; its 64 KB come out of the operand ring, which keeps two stages there.
+constexpr int kHSlotBytes = 2 * 128 * 64;
+constexpr int kHSlots = 2;
+__host__ __device__ constexpr bool stages_h(int epi) { return epi == EPI_DSWIGLU; }
+__host__ __device__ constexpr int stages_for(int epi) { return stages_h(epi) ? 2 : kStages; }
+__host__ __device__ constexpr int smem_bytes(int epi) {
+  return 1024 + stages_for(epi) * kStageBytes + (stages_h(epi) ? 2 * kHSlots * kHSlotBytes : 0) + 1024 +
+         2 * (kMaxE + 1) * 4;
+}
+constexpr int kSmemBytes = smem_bytes(EPI_STORE);
+static_assert(smem_bytes(EPI_DSWIGLU) <= 232448 && smem_bytes(EPI_STORE) <= 232448, "shared memory per CTA");
 }  // namespace g2
 
 // tmA: A [rows, K] as {64, rows, K/64 chunks, 1}; tmB: B_MN ? [E][K rows][N] as
 // {64, K, N/64 chunks, E} : [E][N rows][K] as {64, N, K/64 chunks, E}; boxes {64, 128, 2, 1}.
+// tmH (SwiGLU backward only): the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128},
+// 64-byte swizzle.
 template <bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                  const GemmParams p) {
+                                  const __grid_constant__ CUtensorMap tmH, const GemmParams p) {
   using namespace g2;
+  constexpr int kSt = stages_for(EPI);
+  constexpr bool kH = stages_h(EPI);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* sB = smem + kSt * kABytes;
+  uint8_t* sH = smem + kSt * kStageBytes;     // 1024-byte aligned
+  uint8_t* bar_base = sH + (kH ? 2 * kHSlots * kHSlotBytes : 0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bar_base);
   uint64_t* full = bars;                      // used in the leader
-  uint64_t* empty = bars + kStages;           // both CTAs
-  uint64_t* tfull = bars + 2 * kStages;       // both CTAs
-  uint64_t* tempty = bars + 2 * kStages + 2;  // used in the leader
-  uint64_t* drained = bars + 2 * kStages + 4; // used in the second CTA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* empty = bars + kSt;               // both CTAs
+  uint64_t* tfull = bars + 2 * kSt;           // both CTAs
+  uint64_t* tempty = bars + 2 * kSt + 2;      // used in the leader
+  uint64_t* drained = bars + 2 * kSt + 4;     // used in the second CTA
+  uint64_t* hfull = bars + 2 * kSt + 5;       // h ring (half * kHSlots + slot): both CTAs
+  uint64_t* hempty = hfull + 2 * kHSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 2 * kHSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
+  int32_t* row_off = reinterpret_cast<int32_t*>(bar_base + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -71,9 +96,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
   const int NT = (EPI == EPI_SWIGLU) ? (p.N / 128) : (p.N + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2 * kHSlots; ++b) {
+      mbar_init(&hfull[b], 1);
+      mbar_init(&hempty[b], 4);   // the four epilogue warps of a half
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -86,6 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (kH) tma_prefetch_desc(&tmH);
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0;
@@ -156,14 +186,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
             tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, kb * BK, b0 / 64, ti.e);
           else
             tma_load_4d_pair(sB + stage * kBBytes, &tmB, &full[stage], 0, b0, 2 * kb, ti.e);
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
       // no copy may still be landing when either CTA leaves
-      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kStages, ring);
+      pair_producer_drain(leader, ok, drained, p.timeout_ns, full, kSt, ring);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (pair leader)
@@ -201,7 +231,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
             mma_commit_pair(&empty[stage]);
           }
           __syncwarp();
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1;
           }
@@ -211,12 +241,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
         __syncwarp();
       }
     }
+  } else if (kH && warp == 3) {
+    // ------------------------- h loader (both CTAs; SwiGLU backward): for every tile, the
+    // saved g and u of this CTA's 128 rows, one 32-column strip at a time, into each
+    // half's ring in the order the half drains them (half h: strips 4h, 4h+1, ...)
+    if (lane == 0) {
+      ArmedRing hring;   // slots half * kHSlots + slot
+      int hs[2] = {0, 0};
+      uint32_t hph[2] = {0, 0};
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileInfo ti = walk.decode(t);
+        const int r0 = ti.row0 + BMC * (int)rank;   // past R: zero-filled; past the expert: unused
+        const int n0 = ti.n_blk * BN;
+        for (int it = 0; it < 4 && ok; ++it) {
+          for (int hf = 0; hf < 2; ++hf) {
+            const int c = 4 * hf + it;
+            const int b = hf * kHSlots + hs[hf];
+            if (!mbar_wait_bounded(&hempty[b], hph[hf] ^ 1, abort_flag, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&hfull[b], kHSlotBytes);
+            hring.arm(b, hph[hf]);
+            uint8_t* dst = sH + b * kHSlotBytes;
+            tma_load_3d(dst, &tmH, &hfull[b], n0 + 32 * c, r0, 0);
+            tma_load_3d(dst + kHSlotBytes / 2, &tmH, &hfull[b], p.F + n0 + 32 * c, r0, 0);
+            if (++hs[hf] == kHSlots) {
+              hs[hf] = 0;
+              hph[hf] ^= 1;
+            }
+          }
+        }
+      }
+      // no copy may still be landing when the CTA leaves
+      hring.drain(hfull, 2 * kHSlots, p.timeout_ns);
+    }
   } else if (warp >= 4) {
     // -------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
     const int r_local = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
+    // SwiGLU backward: this half's position in its h ring; a thread reads its row's 64
+    // bytes of g and of u (16-byte chunk j of row r at r * 64 + 16 * (j ^ ((r >> 1) & 3)))
+    int hs = 0;
+    uint32_t hph = 0;
+    auto h_fetch = [&](uint4 (&g)[4], uint4 (&u)[4]) {
+      const int b = half * kHSlots + hs;
+      const bool ok = mbar_wait_bounded(&hfull[b], hph, abort_flag, p.timeout_ns);
+      const uint8_t* base = sH + b * kHSlotBytes + r_local * 64;
+      const int sw = (r_local >> 1) & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        g[j] = *reinterpret_cast<const uint4*>(base + ((j ^ sw) << 4));
+        u[j] = *reinterpret_cast<const uint4*>(base + kHSlotBytes / 2 + ((j ^ sw) << 4));
+      }
+      // the slot's next fill is a TMA (async-proxy) write: order these reads before it
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hempty[b]);
+      if (++hs == kHSlots) {
+        hs = 0;
+        hph ^= 1;
+      }
+      return ok;
+    };
     int lt = 0;
     for (int t = pair; t < total; t += npairs, ++lt) {
       const TileInfo ti = walk.decode(t);
@@ -224,7 +314,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM);
+      if (kH)
+        bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM, h_fetch);
+      else
+        bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);

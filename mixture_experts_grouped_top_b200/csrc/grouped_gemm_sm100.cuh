@@ -174,9 +174,16 @@ __device__ __forceinline__ void rank_experts_by_rows(const int32_t* row_off, int
 
 // Drain one BF16 accumulator tile: this thread owns row `tile_row` of the tile (its TMEM
 // lane is folded into t_row) and the columns of `half`; applies the fused epilogue EPI.
-template <int EPI>
+// A SwiGLU-backward epilogue takes the saved h of its row strip by strip from `h_fetch(g,
+// u)` (32 columns of the gate and of the up half, staged in shared memory by the caller in
+// the order the strips are drained); other epilogues take none.
+struct NoHFetch {
+  __device__ bool operator()(uint4 (&)[4], uint4 (&)[4]) const { return false; }
+};
+
+template <int EPI, class HFetch = NoHFetch>
 __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const TileInfo& ti, uint32_t t_row, int half,
-                                                   int tile_row, int tile_bm) {
+                                                   int tile_row, int tile_bm, const HFetch& h_fetch = HFetch{}) {
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
 
   if (EPI == EPI_STORE || EPI == EPI_WGRAD) {
@@ -279,31 +286,18 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
     const bool row_ok = tile_row < ti.rows;
     const long long row = ti.row0 + tile_row;
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(p.aux);
     __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
     const int n0 = ti.n_blk * gg::BN;
     float dp = 0.f;
 #pragma unroll 1
     for (int c0 = half * (gg::BN / 2); c0 < (half + 1) * (gg::BN / 2); c0 += 32) {
-      // 32 columns per round: the saved h of the round is requested first, so its global
-      // latency overlaps the two tensor-memory loads and their wait
+      // 32 columns per round; the saved h of the round comes from shared memory (every
+      // round takes its strip, so that the staging ring advances in step), before the
+      // tensor-memory loads: nothing may run between a tcgen05.ld and its wait
       uint4 gva[4], uva[4];
       const bool cols_ok0 = row_ok && n0 + c0 < p.N;
       const bool cols_ok1 = row_ok && n0 + c0 + 16 < p.N;
-      if (cols_ok0) {
-        const uint4* gp = reinterpret_cast<const uint4*>(h + row * p.ld_aux + n0 + c0);
-        const uint4* up = reinterpret_cast<const uint4*>(h + row * p.ld_aux + p.F + n0 + c0);
-        gva[0] = gp[0];
-        gva[1] = gp[1];
-        uva[0] = up[0];
-        uva[1] = up[1];
-        if (cols_ok1) {
-          gva[2] = gp[2];
-          gva[3] = gp[3];
-          uva[2] = up[2];
-          uva[3] = up[3];
-        }
-      }
+      h_fetch(gva, uva);
       uint32_t vv[2][16];
       tmem_ld_32x32b_x16(t_row + c0, vv[0]);
       tmem_ld_32x32b_x16(t_row + c0 + 16, vv[1]);

@@ -121,19 +121,22 @@ int tmap_chunks(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_
 
 // CTA-pair kernels: launch as many 2-CTA clusters as can be resident at once (a
 // persistent grid larger than that would leave some pairs waiting for others to finish).
+// th: the saved h for the SwiGLU backward (any map otherwise: unused).
 template <bool B_MN, int EPI>
-int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st,
+                     const CUtensorMap* th = nullptr) {
   auto kern = grouped_gemm_bf16_pair_kernel<B_MN, EPI>;
+  constexpr int kSmem = g2::smem_bytes(EPI);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int pairs = 0;
   std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g2::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(device_props().sm_count, 1, 1);
     cfg.blockDim = dim3(g2::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = g2::kSmemBytes;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.attrs = nullptr;   // the kernel declares its 2-CTA cluster at compile time
     cfg.numAttrs = 0;
     int n = 0;
@@ -142,7 +145,7 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
     cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  kern<<<2 * pairs, g2::kThreads, g2::kSmemBytes, st>>>(ta, tb, p);
+  kern<<<2 * pairs, g2::kThreads, kSmem, st>>>(ta, tb, th ? *th : ta, p);
   count_launch();
   return launch_status();
 }
@@ -1426,7 +1429,12 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.ld_aux = 2 * F;
   p.dprob_part = dpart;
   p.F = F;
-  if ((rc = launch_gemm_pair<false, EPI_DSWIGLU>(ta, tb, p, st))) return rc;
+  // the saved h, staged into shared memory for the epilogue by TMA (32-column strips)
+  CUtensorMap th;
+  if ((rc = make_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h_buf, 2 * F, R, 1, (uint64_t)4 * F,
+                      (uint64_t)R * 4 * F, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B)))
+    return rc;
+  if ((rc = launch_gemm_pair<false, EPI_DSWIGLU>(ta, tb, p, st, &th))) return rc;
   if (dprobs_perm) {
     const int grid = std::min((R + 255) / 256, device_props().sm_count * 4);
     reduce_dprob_kernel<<<grid, 256, 0, st>>>(dpart, nparts, R, dprobs_perm);
