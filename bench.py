@@ -325,13 +325,20 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
                 layer._alloc_bwd()
             b = layer._bwd
             if prec == "mxfp8":
+                # xp along the expert rows, dy both ways: permuted and quantised in one pass
                 layer.permute_for_backward(x)
-            mb.moe_permute_rows(grad, layer.perm["row_map"], cfg.k, out=b["dy_perm"])
-            mark(5)
-            xp_b = layer.perm["xp"] if prec == "bf16" else layer.xp_bf16
-            mb.grouped_mlp_bwd(b["dy_perm"], layer.perm["split_sizes"], xp_b, w1, w2,
-                               layer.perm["probs_perm"], layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"], dw2=b["dw2"],
-                               dprobs_perm=b["dprobs_perm"], workspace=b["ws"])
+                layer.permute_grad(grad)
+                mark(5)
+                mb.grouped_mlp_bwd(None, layer.perm["split_sizes"], None, w1, w2, layer.perm["probs_perm"],
+                                   layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"], dw2=b["dw2"],
+                                   dprobs_perm=b["dprobs_perm"], workspace=b["ws"], operands=layer.bwd_operands(),
+                                   shape=(cfg.R, cfg.H, cfg.F))
+            else:
+                mb.moe_permute_rows(grad, layer.perm["row_map"], cfg.k, out=b["dy_perm"])
+                mark(5)
+                mb.grouped_mlp_bwd(b["dy_perm"], layer.perm["split_sizes"], layer.perm["xp"], w1, w2,
+                                   layer.perm["probs_perm"], layer.saved, prec, dxp=b["dxp"], dw1=b["dw1"],
+                                   dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"])
             mark(6)
             if world > 1:
                 # data-parallel replicas: the weight gradients are summed over the ranks
@@ -418,11 +425,12 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
         "clocks": clocks.summary(),
     }
     if quant_ms:
-        wq_bytes = (d["w1"].numel() + d["w2"].numel()) * (2 + 1 + 1 / 32)
+        both = training and prec == "mxfp8"
+        wq_bytes = (d["w1"].numel() + d["w2"].numel()) * (2 + (2 if both else 1) * (1 + 1 / 32))
         res["bandwidth"]["weight_quant"] = {
             "GB/s": round(wq_bytes / (quant_ms * 1e-3) / 1e9, 1), "ms": round(quant_ms, 4), "bytes": wq_bytes,
-            "note": "forward orientation of w1 and w2 (the backward's other-axis copies run inside "
-                    "grouped_mlp_bwd)"}
+            "note": ("both orientations of w1 and w2 in one pass (mxfp8_quantize_weights: the forward's and the "
+                     "backward's operands)" if both else "the forward orientation of w1 and w2")}
 
     if with_e2e:
         # every step: pinned host -> device copies of the step's inputs, the path, and a

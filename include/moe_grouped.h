@@ -219,6 +219,30 @@ MOE_API int moe_permute_capacity(const uint16_t* x, const int32_t* idx, const fl
  */
 MOE_API int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, int k, uint16_t* dst, void* stream);
 
+/* Bytes of scratch moe_permute_rows_mxfp8 needs: the token of every permuted row. */
+MOE_API size_t moe_permute_rows_mxfp8_workspace_size(int T, int k);
+
+/*
+ * moe_permute_rows_mxfp8 — moe_permute_rows fused with the MXFP8 quantisation of the
+ * permuted rows (news.bpdata.com section 2: one scale per 32 consecutive values along a
+ * GEMM's contraction axis) in the two forms the backward GEMMs read, so that the bf16
+ * permuted tensor is never written:
+ *   rows form (rows_codes, rows_atoms): codes [R, H], blocks of 32 along H, scale atoms
+ *     grouped per 128-row expert tile (the layout of grouped_mlp_fwd's xp_scale, and of
+ *     moe_mxfp8_bwd_operands.dy_rows);
+ *   cols form (cols_codes, cols_atoms): codes [R, H], blocks of 32 rows restarting at every
+ *     expert's first row, atoms in mxfp8_quantize_grouped's layout (dy_cols, xp_cols).
+ * Row row_map[t*k + j] of both is src[t] (a dropless row_map: R = T*k rows, every row
+ * owned by one slot). split_sizes [E] on the device (sum = R). Either output pair may be
+ * NULL. Each atom buffer holds mxfp8_grouped_atoms_bytes(E, R, H) bytes and is zeroed
+ * first (bytes of rows or blocks past an expert's end stay 0). H % 128 == 0.
+ * workspace: moe_permute_rows_mxfp8_workspace_size(T, k) bytes.
+ */
+MOE_API int moe_permute_rows_mxfp8(const uint16_t* src, const int32_t* row_map, int T, int H, int k,
+                                   const int32_t* split_sizes, int E, uint8_t* rows_codes, uint8_t* rows_atoms,
+                                   uint8_t* cols_codes, uint8_t* cols_atoms, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /*
  * moe_unpermute — combine of the k expert outputs of every token.
  * Pages: sitech.ge "Grouped experts instead of a Python loop": the routing weights are
@@ -390,9 +414,9 @@ MOE_API size_t grouped_mlp_bwd_workspace_offset(int E, int R, int H, int F, int 
  * stored in bf16 by the fc2-dgrad epilogue (with its max) before its quantisation.
  * MOE_MXFP8: all four GEMMs run on MXFP8 operands quantised along their own contraction
  * axis (blocks of 32): dy and dh along columns for the data gradients, and dy, a
- * (recomputed from h), dh and xp along rows — in 32-row blocks restarting at every
+ * (from the forward), dh and xp along rows — in 32-row blocks restarting at every
  * expert's first row — for the weight gradients; the weights are re-quantised along
- * their other axis. dh is quantised (both ways) by the fc2-dgrad kernel that computes
+ * their other axis (grouped_mlp_bwd_mxfp8_operands takes operands already quantised). dh is quantised (both ways) by the fc2-dgrad kernel that computes
  * it, from fp32, and never exists at 16 bits; a along rows comes from the forward (its
  * fc1 epilogue quantises a both ways in training). Requires H % 128 == 0 for MOE_MXFP8.
  */
@@ -400,6 +424,55 @@ MOE_API int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int
                             const void* xp, const void* w1, const void* w2, const float* probs_perm, int precision,
                             const void* saved, uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* Operands of the MXFP8 backward that the caller has already quantised, each a pair (E4M3
+ * codes, scale atoms). A pair left NULL is quantised by the call from its bf16 source. */
+typedef struct moe_mxfp8_bwd_operands {
+  /* dy along H, codes [R, H]; atoms grouped per 128-row expert tile (the layout of
+   * grouped_mlp_fwd's xp_scale) */
+  const uint8_t* dy_rows;
+  const uint8_t* dy_rows_atoms;
+  /* dy along the expert's rows, codes [R, H]; atoms in mxfp8_quantize_grouped's layout */
+  const uint8_t* dy_cols;
+  const uint8_t* dy_cols_atoms;
+  /* xp along the expert's rows, codes [R, H]; atoms in mxfp8_quantize_grouped's layout */
+  const uint8_t* xp_cols;
+  const uint8_t* xp_cols_atoms;
+  /* w1 along 2F, codes [E, H, 2F]; w2 along H, codes [E, F, H]: mxfp8_quantize_weights'
+   * codes_r / atoms_r */
+  const uint8_t* w1_rows;
+  const uint8_t* w1_rows_atoms;
+  const uint8_t* w2_rows;
+  const uint8_t* w2_rows_atoms;
+} moe_mxfp8_bwd_operands;
+
+/*
+ * grouped_mlp_bwd_mxfp8_operands — grouped_mlp_bwd(..., MOE_MXFP8, ...) with some of its
+ * operands already quantised (q, see moe_mxfp8_bwd_operands; q may be NULL). dy_perm may
+ * be NULL when both of dy's forms are given, xp when xp_cols is, w1 / w2 when their rows
+ * forms are. Same results, outputs and workspace as grouped_mlp_bwd with MOE_MXFP8.
+ */
+MOE_API int grouped_mlp_bwd_mxfp8_operands(const moe_mxfp8_bwd_operands* q, const void* dy_perm,
+                                           const int32_t* split_sizes, int E, int R, int H, int F, const void* xp,
+                                           const void* w1, const void* w2, const float* probs_perm, const void* saved,
+                                           uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/*
+ * mxfp8_quantize_weights — both MXFP8 forms of expert weights in one pass over the bf16
+ * masters, which a training step re-quantises after every optimizer step (news.bpdata.com
+ * section 2: one scale per 32 consecutive values along the contraction axis):
+ *   w [batch, rows, cols] bf16 (w1: [E, H, 2F]; w2: [E, F, H]); rows, cols multiples of 128;
+ *   codes_t [batch, cols, rows] E4M3, blocks of 32 along `rows` (the forward GEMM's K),
+ *     transposed, and atoms_t their scale atoms: the same bytes as mxfp8_quantize(w, batch,
+ *     rows, cols, axis 1, transpose_out, MOE_SCALES_MMA);
+ *   codes_r [batch, rows, cols] E4M3, blocks of 32 along `cols` (the data-gradient GEMM's
+ *     K), and atoms_r their scale atoms: the same bytes as mxfp8_quantize of w viewed as
+ *     [batch * rows, cols], axis 0, MOE_SCALES_MMA.
+ * Sizes: codes_t, codes_r batch*rows*cols bytes; atoms_t, atoms_r batch*rows*cols/32 bytes.
+ */
+MOE_API int mxfp8_quantize_weights(const uint16_t* w, int batch, int rows, int cols, uint8_t* codes_t,
+                                   uint8_t* atoms_t, uint8_t* codes_r, uint8_t* atoms_r, void* stream);
 
 /*
  * mxfp8_quantize_grouped — MXFP8 quantisation of expert-contiguous rows along the rows:

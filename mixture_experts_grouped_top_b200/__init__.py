@@ -292,6 +292,57 @@ def mxfp8_quantize(x, axis: int = 0, transpose_out: bool = False, codes=None, sc
     return codes, scales
 
 
+def moe_permute_rows_mxfp8(src, row_map, k, split_sizes, rows=True, cols=True, out=None, workspace=None,
+                           stream=None):
+    """moe_permute_rows fused with the MXFP8 quantisation of the permuted rows in the rows
+    form (along H, tile atoms) and / or the cols form (along each expert's rows, grouped
+    atoms). Returns a dict with "rows", "rows_atoms", "cols", "cols_atoms" (None where not
+    asked for); ``out`` may hold preallocated tensors under those names."""
+    _need(src, torch.bfloat16, "src")
+    T, H = src.shape
+    R = T * k
+    E = split_sizes.numel()
+    dev = src.device
+    out = {} if out is None else out
+    nat = int(lib().mxfp8_grouped_atoms_bytes(E, R, H))
+    for name, want, shape in (("rows", rows, (R, H)), ("cols", cols, (R, H))):
+        if want:
+            if out.get(name) is None:
+                out[name] = torch.empty(shape, dtype=torch.uint8, device=dev)
+            if out.get(name + "_atoms") is None:
+                out[name + "_atoms"] = torch.empty(max(nat, 1), dtype=torch.uint8, device=dev)
+        else:
+            out[name] = out[name + "_atoms"] = None
+    if workspace is None:
+        workspace = torch.empty(int(lib().moe_permute_rows_mxfp8_workspace_size(T, k)), dtype=torch.uint8,
+                                device=dev)
+    rc = lib().moe_permute_rows_mxfp8(_p(src), _p(row_map), T, H, k, _p(split_sizes), E, _p(out["rows"]),
+                                      _p(out["rows_atoms"]), _p(out["cols"]), _p(out["cols_atoms"]), _p(workspace),
+                                      workspace.numel(), _stream(stream))
+    _check("moe_permute_rows_mxfp8", rc)
+    return out
+
+
+def mxfp8_quantize_weights(w, codes_t=None, atoms_t=None, codes_r=None, atoms_r=None, stream=None):
+    """Both MXFP8 forms of bf16 weights [batch, rows, cols] in one pass: (codes_t
+    [batch, cols, rows], atoms_t) blocked along rows (the forward's K-major operand, as
+    mxfp8_quantize(axis=1, transpose_out=True, mma_scales=True)) and (codes_r
+    [batch, rows, cols], atoms_r) blocked along cols (the backward's data-gradient
+    operand). Returns (codes_t, atoms_t, codes_r, atoms_r)."""
+    _need(w, torch.bfloat16, "w")
+    B, rows, cols = w.shape
+    dev = w.device
+    n = B * rows * cols
+    codes_t = torch.empty((B, cols, rows), dtype=torch.uint8, device=dev) if codes_t is None else codes_t
+    codes_r = torch.empty((B, rows, cols), dtype=torch.uint8, device=dev) if codes_r is None else codes_r
+    atoms_t = torch.empty(n // 32, dtype=torch.uint8, device=dev) if atoms_t is None else atoms_t
+    atoms_r = torch.empty(n // 32, dtype=torch.uint8, device=dev) if atoms_r is None else atoms_r
+    rc = lib().mxfp8_quantize_weights(_p(w), B, rows, cols, _p(codes_t), _p(atoms_t), _p(codes_r), _p(atoms_r),
+                                      _stream(stream))
+    _check("mxfp8_quantize_weights", rc)
+    return codes_t, atoms_t, codes_r, atoms_r
+
+
 def fp8_quantize(x, fmt="e4m3", transpose_out=False, codes=None, scales=None, stream=None):
     """Per-tensor FP8 (current scaling) of bf16 [batch, rows, cols] (or [rows, cols]): one
     fp32 scale per batch matrix. Returns (codes uint8, scales fp32 [batch])."""
@@ -400,14 +451,20 @@ def grouped_mlp_bwd_workspace_offset(E, R, H, F, precision, part) -> int:
 
 
 def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precision="bf16", dxp=None, dw1=None,
-                    dw2=None, dprobs_perm=None, workspace=None, stream=None):
+                    dw2=None, dprobs_perm=None, workspace=None, stream=None, operands=None, shape=None):
     """Backward of grouped_mlp_fwd. Returns (dxp, dw1, dw2, dprobs_perm). xp, w1 and w2
-    are bf16 on both paths (the MXFP8 path quantises what it needs)."""
+    are bf16 on both paths (the MXFP8 path quantises what it needs). MXFP8 only:
+    ``operands`` maps names of moe_mxfp8_bwd_operands ("w1_rows", "w1_rows_atoms", ...,
+    "dy_rows", "dy_cols", "xp_cols" and their atoms) to tensors already quantised; their
+    bf16 sources may then be None, and ``shape`` = (R, H, F) names the sizes."""
     prec = _PREC[precision]
-    R, H = dy_perm.shape
+    if shape is not None:
+        R, H, F = shape
+    else:
+        R, H = dy_perm.shape
+        F = w2.shape[1]
     E = split_sizes.numel()
-    F = w2.shape[1]
-    dev = dy_perm.device
+    dev = split_sizes.device
     dxp = torch.empty((R, H), dtype=torch.bfloat16, device=dev) if dxp is None else dxp
     dw1 = torch.empty((E, H, 2 * F), dtype=torch.bfloat16, device=dev) if dw1 is None else dw1
     dw2 = torch.empty((E, F, H), dtype=torch.bfloat16, device=dev) if dw2 is None else dw2
@@ -416,10 +473,20 @@ def grouped_mlp_bwd(dy_perm, split_sizes, xp, w1, w2, probs_perm, saved, precisi
     ws_bytes = grouped_mlp_bwd_workspace_size(E, R, H, F, precision)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    rc = lib().grouped_mlp_bwd(_p(dy_perm), _p(split_sizes), E, R, H, F, _p(xp), _p(w1), _p(w2), _p(probs_perm),
-                               prec, _p(saved), _p(dxp), _p(dw1), _p(dw2), _p(dprobs_perm), _p(workspace),
-                               workspace.numel(), _stream(stream))
-    _check("grouped_mlp_bwd", rc)
+    if operands:
+        if prec != MXFP8:
+            raise ValueError("pre-quantised operands are for the MXFP8 backward")
+        q = _lib.MxBwdOperands(**{k: (v.data_ptr() if v is not None else None) for k, v in operands.items()})
+        rc = lib().grouped_mlp_bwd_mxfp8_operands(ctypes.byref(q), _p(dy_perm), _p(split_sizes), E, R, H, F, _p(xp),
+                                                  _p(w1), _p(w2), _p(probs_perm), _p(saved), _p(dxp), _p(dw1),
+                                                  _p(dw2), _p(dprobs_perm), _p(workspace), workspace.numel(),
+                                                  _stream(stream))
+        _check("grouped_mlp_bwd_mxfp8_operands", rc)
+    else:
+        rc = lib().grouped_mlp_bwd(_p(dy_perm), _p(split_sizes), E, R, H, F, _p(xp), _p(w1), _p(w2),
+                                   _p(probs_perm), prec, _p(saved), _p(dxp), _p(dw1), _p(dw2), _p(dprobs_perm),
+                                   _p(workspace), workspace.numel(), _stream(stream))
+        _check("grouped_mlp_bwd", rc)
     return dxp, dw1, dw2, dprobs_perm
 
 

@@ -28,6 +28,8 @@ SIGNATURES = {
     "moe_permute_capacity": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                   _vp]),
     "moe_permute_rows": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_permute_rows_mxfp8_workspace_size": (_sz, [_i, _i]),
+    "moe_permute_rows_mxfp8": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_unpermute": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "mxfp8_quantize": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "fp8_quantize_workspace_size": (_sz, [_i]),
@@ -43,10 +45,19 @@ SIGNATURES = {
     "grouped_mlp_bwd": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                              _vp]),
     "grouped_mlp_bwd_workspace_offset": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "grouped_mlp_bwd_mxfp8_operands": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, _vp, _sz, _vp]),
+    "mxfp8_quantize_weights": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "mxfp8_quantize_grouped": (_i, [_vp, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "mxfp8_grouped_atoms_bytes": (_sz, [_i, _i, _i]),
     "moe_gather_slots": (_i, [_vp, _vp, _i, _vp, _vp]),
 }
+
+class MxBwdOperands(ctypes.Structure):
+    """moe_mxfp8_bwd_operands: (codes, atoms) pointer pairs, NULL where not given."""
+    _fields_ = [(name, _vp) for name in ("dy_rows", "dy_rows_atoms", "dy_cols", "dy_cols_atoms", "xp_cols",
+                                        "xp_cols_atoms", "w1_rows", "w1_rows_atoms", "w2_rows", "w2_rows_atoms")]
+
 
 _lock = threading.Lock()
 _handle = None

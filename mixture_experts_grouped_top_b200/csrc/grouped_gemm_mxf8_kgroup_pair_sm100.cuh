@@ -58,6 +58,8 @@ constexpr int kTmemCols = 512;
 constexpr int kSmemBytes =
     1024 + kStages * kStageBytes + kSfSlots * kSfSlotBytes + 1024 + 4 * (kMaxE + 1) * 4;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+// ScaleCopier's look-back of mx::kSfSets k-groups must stay within the operand ring
+static_assert(mx::kSfSets <= kStages * kGroupsPerStage, "operand ring too short for the scale-set look-back");
 }  // namespace mkp
 
 // Zero rows [valid, end) of this CTA's A and B blocks of one stage (128-byte rows), one

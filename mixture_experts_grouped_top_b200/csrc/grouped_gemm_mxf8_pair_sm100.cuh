@@ -63,12 +63,14 @@ constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
 // SwiGLU backward: the saved h reaches the epilogue through shared memory, a ring of
 // 32-column strips (g and u of the CTA's 128 rows, 64-byte swizzled: 16 KB) per column
-// half; its 64 KB come out of the operand ring, which keeps two stages (the K = H
-// mainloop of that GEMM is shorter than its epilogue).
+// half; its 64 KB come out of the operand ring, which keeps the stages that remain (the
+// K = H mainloop of that GEMM is shorter than its epilogue).
 constexpr int kHSlotBytes = 2 * 128 * 64;
 constexpr int kHSlots = 2;                    // per half
 __host__ __device__ constexpr bool stages_h(int epi) { return epi == MXEPI_DSWIGLU; }
-__host__ __device__ constexpr int stages_for(int epi) { return stages_h(epi) ? 2 : kStages; }
+__host__ __device__ constexpr int stages_for(int epi) {
+  return stages_h(epi) ? kStages - (2 * kHSlots * kHSlotBytes + kStageBytes - 1) / kStageBytes : kStages;
+}
 __host__ __device__ constexpr int smem_bytes(int epi) {
   return 1024 + stages_for(epi) * kStageBytes + kSfSlots * kSfSlotBytes + (stages_h(epi) ? 2 * kHSlots * kHSlotBytes : 0) +
          1024 + 3 * (kMaxE + 1) * 4;
@@ -90,6 +92,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   using namespace mx2;
   constexpr int kSt = stages_for(EPI);
   constexpr bool kH = stages_h(EPI);
+  // ScaleCopier waits for the `empty` phase of the stage kSfSets k-blocks back; the MMA
+  // thread can complete at most kSfSets / kChunks - 1 later stages meanwhile, which must
+  // stay below the ring's kSt (else that slot's barrier could be two phases ahead)
+  static_assert(mx::kSfSets <= kSt * kChunks, "operand ring too short for the scale-set look-back");
   const GemmParams& p = mp.g;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

@@ -103,47 +103,6 @@ __device__ __forceinline__ void warp_amax_to(unsigned int* out, float v) {
   if ((threadIdx.x & 31) == 0 && m) atomicMax(out, m);
 }
 
-// E4M3 codes of 32 fp32 values (one lane's row) quantised along the 32 LANES of the warp:
-// for each column j the block maximum is the warp-wide max of |v[j]| (one redux: the bits
-// of a non-negative float order like the float), E8M0 code max(exp(amax) - 8, 0), element
-// scaled by 2^(127 - code) exactly and rounded to nearest even with saturation. Lanes
-// that hold no row pass zeros. Every lane of the warp must call this together. Returns
-// the codes in `w` (byte j = column j) and, in lane j, the scale code of column j.
-__device__ __forceinline__ uint32_t quant_cols_warp32(const float (&v)[32], uint32_t (&w)[8], int lane) {
-  uint32_t mine = 0;
-#pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
-    const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + 1])));
-    const int c0 = max((int)(m0 >> 23) - 8, 0), c1 = max((int)(m1 >> 23) - 8, 0);
-    const float i0 = __uint_as_float((uint32_t)(254 - c0) << 23), i1 = __uint_as_float((uint32_t)(254 - c1) << 23);
-    const uint32_t pair =
-        (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v[j] * i0, v[j + 1] * i1), __NV_SATFINITE, __NV_E4M3);
-    if ((j & 2) == 0)
-      w[j >> 2] = pair;
-    else
-      w[j >> 2] |= pair << 16;
-    if (lane == j) mine = (uint32_t)c0;
-    if (lane == j + 1) mine = (uint32_t)c1;
-  }
-  return mine;
-}
-
-// E4M3 codes of 32 fp32 values of one row quantised as one block along the row; returns
-// the block's scale code.
-__device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
-  const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] *= inv;
-  pack_e4m3x16(v, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
-  pack_e4m3x16(v + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
-  return (uint32_t)code;
-}
-
 // Scale-set handoff between the scale-copy warp and the MMA thread of a CTA pair (both in
 // the leader). The copier takes k-block kb's atoms from the scale ring in shared memory
 // (slots of kPerSlot k-blocks, 3 groups of kPerSlot atoms: A, B lower, B upper) into the
@@ -152,8 +111,10 @@ __device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]
 // once the MMAs of the k-block that used it before are done: the copier learns that from
 // the operand ring's `empty` barrier of that k-block's stage, which the MMA thread commits
 // anyway (an extra commit per k-block held the MMA thread's stream, like the copies
-// themselves). The copier releases a scale-ring slot (`sempty`) once the copies of its
-// last k-block are done. Bounded waits; all barriers count one arrival.
+// themselves). That phase is the last one the stage's slot completed as long as the
+// MMA thread cannot finish another kSt stages first: kernels assert kSfSets <= kSt *
+// (k-blocks per stage). The copier releases a scale-ring slot (`sempty`) once the copies
+// of its last k-block are done. Bounded waits; all barriers count one arrival.
 template <int kPerSlot>
 struct ScaleCopier {
   uint64_t* sfull;

@@ -509,6 +509,46 @@ int moe_permute_rows(const uint16_t* src, const int32_t* row_map, int T, int H, 
   return launch_status();
 }
 
+size_t moe_permute_rows_mxfp8_workspace_size(int T, int k) {
+  if (T < 0 || k < 1) return 0;
+  return ((size_t)T * k * 4 + 255) / 256 * 256 + 256;
+}
+
+int moe_permute_rows_mxfp8(const uint16_t* src, const int32_t* row_map, int T, int H, int k,
+                           const int32_t* split_sizes, int E, uint8_t* rows_codes, uint8_t* rows_atoms,
+                           uint8_t* cols_codes, uint8_t* cols_atoms, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (T < 0 || H < 128 || k < 1 || k > 32 || E < 1 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (H % 128) return MOE_ERR_UNSUPPORTED;
+  const long long R = (long long)T * k;
+  if (R > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if ((rows_codes == nullptr) != (rows_atoms == nullptr) || (cols_codes == nullptr) != (cols_atoms == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (R == 0 || (!rows_codes && !cols_codes)) return MOE_OK;
+  if (!src || !row_map || !split_sizes || !workspace) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe_permute_rows_mxfp8_workspace_size(T, k)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(rows_codes) |
+       reinterpret_cast<uintptr_t>(cols_codes)) & 15)
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  int32_t* row_token = reinterpret_cast<int32_t*>(workspace);
+  row_token_kernel<<<std::min((int)((R + 255) / 256), device_props().sm_count * 8), 256, 0, st>>>(row_map, (int)R, k,
+                                                                                               row_token);
+  count_launch();
+  int rc;
+  if ((rc = launch_status())) return rc;
+  const size_t atoms = mma_atoms_bytes(E, (int)R, H);
+  if (rows_atoms && cudaMemsetAsync(rows_atoms, 0, atoms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cols_atoms && cudaMemsetAsync(cols_atoms, 0, atoms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const int blocks32 = (int)std::min<long long>(R / 32 + E, (long long)device_props().sm_count * 8);
+  dim3 grid(blocks32, (H + 255) / 256);
+  permute_quant_both_kernel<<<grid, 256, 3 * (E + 1) * sizeof(int32_t), st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(src), H, row_token, split_sizes, E, rows_codes, rows_atoms, cols_codes,
+      cols_atoms);
+  count_launch();
+  return launch_status();
+}
+
 namespace {
 int permute_rows_from_counts(const uint16_t* x, const int32_t* idx, const float* prob, int T, int H, int E, int k,
                              int precision, void* xp, uint8_t* xp_scale, int32_t* row_map, float* probs_perm,
@@ -753,6 +793,24 @@ int mxfp8_quantize(const uint16_t* in, int batch, int rows, int cols, int axis, 
     quant_cols_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in), rows, cols, transpose_out,
                                             scale_layout == MOE_SCALES_MMA, codes, scales);
   }
+  count_launch();
+  return launch_status();
+}
+
+int mxfp8_quantize_weights(const uint16_t* w, int batch, int rows, int cols, uint8_t* codes_t, uint8_t* atoms_t,
+                           uint8_t* codes_r, uint8_t* atoms_r, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+  if ((rows % 128) || (cols % 128)) return MOE_ERR_UNSUPPORTED;
+  if ((long long)batch * rows * cols == 0) return MOE_OK;
+  if (!w || !codes_t || !atoms_t || !codes_r || !atoms_r) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(codes_t) | reinterpret_cast<uintptr_t>(codes_r)) &
+      15)
+    return MOE_ERR_INVALID_ARG;
+  if (batch > 65535 || rows / 32 > 65535) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  dim3 grid((cols + 255) / 256, rows / 32, batch);
+  quant_weights_both_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, codes_t,
+                                                  atoms_t, codes_r, atoms_r);
   count_launch();
   return launch_status();
 }
@@ -1261,24 +1319,41 @@ int grouped_mlp_bwd_fp8(const void* dy_perm, const int32_t* split_sizes, int E, 
   return launch_wgrad_mx_pair(xq, unit, n_unit, dhq, unit, n_unit, R, p, st);
 }
 
-int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E, int R, int H, int F,
-                          const void* xp, const void* w1, const void* w2, const float* probs_perm, const void* saved,
-                          uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm, void* ws,
-                          cudaStream_t st) {
+// q: operands the caller quantised already (NULL pairs, or q == NULL: quantised here into
+// the workspace from dy_perm, xp, w1, w2).
+int grouped_mlp_bwd_mxfp8(const moe_mxfp8_bwd_operands* q, const void* dy_perm, const int32_t* split_sizes, int E,
+                          int R, int H, int F, const void* xp, const void* w1, const void* w2, const float* probs_perm,
+                          const void* saved, uint16_t* dxp, uint16_t* dw1, uint16_t* dw2, float* dprobs_perm,
+                          void* ws, cudaStream_t st) {
   if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  const moe_mxfp8_bwd_operands none{};
+  if (!q) q = &none;
+  const bool have_w2 = q->w2_rows && q->w2_rows_atoms, have_w1 = q->w1_rows && q->w1_rows_atoms;
+  const bool have_dyr = q->dy_rows && q->dy_rows_atoms, have_dyc = q->dy_cols && q->dy_cols_atoms;
+  const bool have_xc = q->xp_cols && q->xp_cols_atoms;
+  if ((!have_w2 && !w2) || (!have_w1 && !w1) || ((!have_dyr || !have_dyc) && !dy_perm) || (!have_xc && !xp))
+    return MOE_ERR_INVALID_ARG;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   auto part = [&](int i) { return base + bwd_part_offset(i, E, R, H, F, MOE_MXFP8); };
   float* dpart = reinterpret_cast<float*>(part(2));
   const size_t efh = (size_t)E * F * H;
-  uint8_t* w2q = part(3);
-  uint8_t* w2a = w2q + align_up(efh, 256);
-  uint8_t* w1q = part(4);
-  uint8_t* w1a = w1q + align_up(efh * 2, 256);
-  uint8_t* dyr = part(5);
-  uint8_t* dyr_s = dyr + align_up((size_t)R * H, 256);
-  uint8_t* dyr_a = dyr_s + align_up((size_t)R * H / 32, 256);
-  uint8_t* dyc = part(6);
-  uint8_t* dyc_a = dyc + align_up((size_t)R * H, 256);
+  uint8_t* w2q_ws = part(3);
+  uint8_t* w2a_ws = w2q_ws + align_up(efh, 256);
+  uint8_t* w1q_ws = part(4);
+  uint8_t* w1a_ws = w1q_ws + align_up(efh * 2, 256);
+  uint8_t* dyr_ws = part(5);
+  uint8_t* dyr_s = dyr_ws + align_up((size_t)R * H, 256);
+  uint8_t* dyr_a_ws = dyr_s + align_up((size_t)R * H / 32, 256);
+  uint8_t* dyc_ws = part(6);
+  uint8_t* dyc_a_ws = dyc_ws + align_up((size_t)R * H, 256);
+  const uint8_t* w2q = have_w2 ? q->w2_rows : w2q_ws;
+  const uint8_t* w2a = have_w2 ? q->w2_rows_atoms : w2a_ws;
+  const uint8_t* w1q = have_w1 ? q->w1_rows : w1q_ws;
+  const uint8_t* w1a = have_w1 ? q->w1_rows_atoms : w1a_ws;
+  const uint8_t* dyr = have_dyr ? q->dy_rows : dyr_ws;
+  const uint8_t* dyr_a = have_dyr ? q->dy_rows_atoms : dyr_a_ws;
+  const uint8_t* dyc = have_dyc ? q->dy_cols : dyc_ws;
+  const uint8_t* dyc_a = have_dyc ? q->dy_cols_atoms : dyc_a_ws;
   // a along the expert's rows: quantised by the forward's fc1 epilogue into `saved`
   const uint8_t* ac = reinterpret_cast<const uint8_t*>(saved) + align_up((size_t)R * 2 * F * 2, 256) +
                       align_up((size_t)R * F, 256) + mma_atoms_bytes(E, R, F);
@@ -1287,18 +1362,22 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
   uint8_t* dhr_a = dhr + align_up((size_t)R * 2 * F, 256);
   uint8_t* dhc = part(9);
   uint8_t* dhc_a = dhc + align_up((size_t)R * 2 * F, 256);
-  uint8_t* xc = part(10);
-  uint8_t* xc_a = xc + align_up((size_t)R * H, 256);
+  uint8_t* xc_ws = part(10);
+  uint8_t* xc_a_ws = xc_ws + align_up((size_t)R * H, 256);
+  const uint8_t* xc = have_xc ? q->xp_cols : xc_ws;
+  const uint8_t* xc_a = have_xc ? q->xp_cols_atoms : xc_a_ws;
   const uint16_t* h_saved = reinterpret_cast<const uint16_t*>(saved);
   const int nparts = 2 * ((F + gg::BN - 1) / gg::BN);   // one partial per N-tile half
   int rc;
   // weights along their other axis (the masters change every optimizer step)
-  if ((rc = quant_rows_launch(w2, (long long)E * F, H, 1, w2q, w2a, st))) return rc;
-  if ((rc = quant_rows_launch(w1, (long long)E * H, 2 * F, 1, w1q, w1a, st))) return rc;
+  if (!have_w2 && (rc = quant_rows_launch(w2, (long long)E * F, H, 1, w2q_ws, w2a_ws, st))) return rc;
+  if (!have_w1 && (rc = quant_rows_launch(w1, (long long)E * H, 2 * F, 1, w1q_ws, w1a_ws, st))) return rc;
   // dy along H (fc2 dgrad) and along rows (fc2 wgrad)
-  if ((rc = quant_rows_launch(dy_perm, R, H, 0, dyr, dyr_s, st))) return rc;
-  if ((rc = scales_to_atoms_launch(dyr_s, split_sizes, E, R, H, dyr_a, st))) return rc;
-  if ((rc = quant_cols_grouped_launch(dy_perm, R, H, split_sizes, E, dyc, dyc_a, st))) return rc;
+  if (!have_dyr) {
+    if ((rc = quant_rows_launch(dy_perm, R, H, 0, dyr_ws, dyr_s, st))) return rc;
+    if ((rc = scales_to_atoms_launch(dyr_s, split_sizes, E, R, H, dyr_a_ws, st))) return rc;
+  }
+  if (!have_dyc && (rc = quant_cols_grouped_launch(dy_perm, R, H, split_sizes, E, dyc_ws, dyc_a_ws, st))) return rc;
   CUtensorMap ta, tb;
   // fc2 dgrad + SwiGLU backward: A = dy codes [R, H], B = w2 codes [E, F, H] (N = F)
   if ((rc = tmap_chunks(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, dyr, 1, R, H, 1, 128, mx2::kChunks))) return rc;
@@ -1338,7 +1417,7 @@ int grouped_mlp_bwd_mxfp8(const void* dy_perm, const int32_t* split_sizes, int E
     if ((rc = launch_status())) return rc;
   }
   // xp along its rows for the fc1 weight gradient
-  if ((rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc, xc_a, st))) return rc;
+  if (!have_xc && (rc = quant_cols_grouped_launch(xp, R, H, split_sizes, E, xc_ws, xc_a_ws, st))) return rc;
   // fc2 wgrad: dw2[e] = a_e^T dy_e (MN-major codes, contraction over the expert's rows)
   const uint64_t kgs = (uint64_t)R / 128 + E;   // bound on the experts' 128-row k-groups
   p.g = base_params(split_sizes, E);
@@ -1401,7 +1480,7 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
     return MOE_OK;
   }
   if (precision == MOE_MXFP8)
-    return grouped_mlp_bwd_mxfp8(dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
+    return grouped_mlp_bwd_mxfp8(nullptr, dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
                                  dprobs_perm, ws, st);
   if (precision == MOE_FP8)
     return grouped_mlp_bwd_fp8(dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
@@ -1471,6 +1550,26 @@ int grouped_mlp_bwd(const void* dy_perm, const int32_t* split_sizes, int E, int 
   p.ldo = 2 * F;
   p.out_batch = (long long)H * 2 * F;
   return launch_wgrad_pair(ta, tb, p, st);
+}
+
+int grouped_mlp_bwd_mxfp8_operands(const moe_mxfp8_bwd_operands* q, const void* dy_perm, const int32_t* split_sizes,
+                                   int E, int R, int H, int F, const void* xp, const void* w1, const void* w2,
+                                   const float* probs_perm, const void* saved, uint16_t* dxp, uint16_t* dw1,
+                                   uint16_t* dw2, float* dprobs_perm, void* ws, size_t ws_bytes, void* stream) {
+  if (E < 1 || E > gg::kMaxE || R < 0 || H < 128 || F < 128) return MOE_ERR_INVALID_ARG;
+  if ((H % 128) || (F % 128)) return MOE_ERR_UNSUPPORTED;
+  if (!split_sizes || !dw1 || !dw2) return MOE_ERR_INVALID_ARG;
+  if (R > 0 && (!saved || !dxp || !ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < grouped_mlp_bwd_workspace_size(E, R, H, F, MOE_MXFP8)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (R == 0) {
+    if (cudaMemsetAsync(dw1, 0, (size_t)E * H * 2 * F * 2, st) != cudaSuccess ||
+        cudaMemsetAsync(dw2, 0, (size_t)E * F * H * 2, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  return grouped_mlp_bwd_mxfp8(q, dy_perm, split_sizes, E, R, H, F, xp, w1, w2, probs_perm, saved, dxp, dw1, dw2,
+                               dprobs_perm, ws, st);
 }
 
 }  // extern "C"

@@ -729,6 +729,47 @@ __global__ void __launch_bounds__(256) scales_to_atoms_kernel(const uint8_t* __r
 }
 
 // ------------------------------------------------------------ MXFP8 quantiser
+// E4M3 codes of 32 fp32 values (one lane's row) quantised along the 32 LANES of the warp:
+// for each column j the block maximum is the warp-wide max of |v[j]| (one redux: the bits
+// of a non-negative float order like the float), E8M0 code max(exp(amax) - 8, 0), element
+// scaled by 2^(127 - code) exactly and rounded to nearest even with saturation. Lanes
+// that hold no row pass zeros. Every lane of the warp must call this together. Returns
+// the codes in `w` (byte j = column j) and, in lane j, the scale code of column j.
+__device__ __forceinline__ uint32_t quant_cols_warp32(const float (&v)[32], uint32_t (&w)[8], int lane) {
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
+    const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + 1])));
+    const int c0 = max((int)(m0 >> 23) - 8, 0), c1 = max((int)(m1 >> 23) - 8, 0);
+    const float i0 = __uint_as_float((uint32_t)(254 - c0) << 23), i1 = __uint_as_float((uint32_t)(254 - c1) << 23);
+    const uint32_t pair =
+        (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v[j] * i0, v[j + 1] * i1), __NV_SATFINITE, __NV_E4M3);
+    if ((j & 2) == 0)
+      w[j >> 2] = pair;
+    else
+      w[j >> 2] |= pair << 16;
+    if (lane == j) mine = (uint32_t)c0;
+    if (lane == j + 1) mine = (uint32_t)c1;
+  }
+  return mine;
+}
+
+// E4M3 codes of 32 fp32 values of one row quantised as one block along the row; returns
+// the block's scale code.
+__device__ __forceinline__ uint32_t quant_row32(float (&v)[32], uint32_t (&w)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
+  const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= inv;
+  pack_e4m3x16(v, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
+  pack_e4m3x16(v + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
+  return (uint32_t)code;
+}
+
 // axis 0: blocks of 32 along the columns of each row. 4 lanes per block.
 __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ in, long long nvec, int cols,
                                                          int mma_scales, uint8_t* __restrict__ codes,
@@ -951,6 +992,209 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __
       const int n = min(32, cols - cc);
       uint8_t* o = dst + (size_t)(r0 + row) * cols + cc;
       for (int i = 0; i < n; ++i) o[i] = tile[row][part * 32 + i];
+    }
+  }
+}
+
+// Both MXFP8 forms of a weight tensor [batch, rows, cols] bf16 in one pass (one read):
+//   T: blocks of 32 along the rows of each column, codes transposed to [batch, cols, rows]
+//      with scale atoms of the transposed matrix (the K-major operand of a GEMM whose K is
+//      `rows`: fc1 and fc2 forward);
+//   R: blocks of 32 along the columns of each row, codes [batch, rows, cols] with atoms of
+//      the [batch * rows, cols] matrix (the K-major operand of a GEMM whose K is `cols`:
+//      the data-gradient GEMMs of the backward).
+// The same rule as every quantiser here: E8M0 code max(biased_exp(amax) - 8, 0), elements
+// times 2^(127 - code), round to nearest even, saturating. A block of 256 threads loads a
+// 32 x 256 tile with 16-byte loads into shared memory (row pitch 528 bytes: the column
+// reads of T and the 32-column row reads of R are both free of bank conflicts); thread j
+// then quantises column c0 + j (T) and row j % 32 of the 32-column block j / 32 (R).
+// rows and cols are multiples of 128 (a matrix's last 256-column tile may be half empty).
+__global__ void __launch_bounds__(256) quant_weights_both_kernel(const __nv_bfloat16* __restrict__ in, int rows,
+                                                                 int cols, uint8_t* __restrict__ codes_t,
+                                                                 uint8_t* __restrict__ atoms_t,
+                                                                 uint8_t* __restrict__ codes_r,
+                                                                 uint8_t* __restrict__ atoms_r) {
+  constexpr int kPitch = 264;   // bf16 per shared row: 256 + 8
+  __shared__ __align__(16) __nv_bfloat16 tile[32 * kPitch];
+  const int b = blockIdx.z;
+  const int r0 = blockIdx.y * 32;
+  const int c0 = blockIdx.x * 256;
+  const int j = threadIdx.x;
+  const __nv_bfloat16* src = in + (size_t)b * rows * cols;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = j + 256 * i, row = idx >> 5, cv = (idx & 31) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c0 + cv < cols) v = *reinterpret_cast<const uint4*>(src + (size_t)(r0 + row) * cols + c0 + cv);
+    *reinterpret_cast<uint4*>(&tile[row * kPitch + cv]) = v;
+  }
+  __syncthreads();
+  float f[32];
+  // T: column c0 + j over the 32 rows (the last tile of a matrix may be half empty)
+  if (c0 + j < cols) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      f[i] = __bfloat162float(tile[i * kPitch + j]);
+      amax = fmaxf(amax, fabsf(f[i]));
+    }
+    const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
+    const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] *= inv;
+    uint32_t w[8];
+    pack_e4m3x16(f, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
+    pack_e4m3x16(f + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
+    const int c = c0 + j;
+    uint4* o = reinterpret_cast<uint4*>(codes_t + (size_t)b * rows * cols + (size_t)c * rows + r0);
+    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    atoms_t[mma_scale_offset((size_t)b * (cols / 128) + c / 128, c % 128, r0 / 32, rows / 128)] = (uint8_t)code;
+  }
+  // R: row r0 + (j % 32), columns [c0 + 32 (j / 32), +32)
+  if (c0 + 32 * (j >> 5) < cols) {
+    const int row = j & 31, blk = j >> 5;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(&tile[row * kPitch + blk * 32 + 8 * i]);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 p2 = __bfloat1622float2(h2[q]);
+        f[8 * i + 2 * q] = p2.x;
+        f[8 * i + 2 * q + 1] = p2.y;
+        amax = fmaxf(amax, fmaxf(fabsf(p2.x), fabsf(p2.y)));
+      }
+    }
+    const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
+    const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] *= inv;
+    uint32_t w[8];
+    pack_e4m3x16(f, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
+    pack_e4m3x16(f + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
+    const size_t grow = (size_t)b * rows + r0 + row;
+    const int c = c0 + 32 * blk;
+    uint4* o = reinterpret_cast<uint4*>(codes_r + grow * cols + c);
+    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    atoms_r[mma_scale_offset(grow >> 7, (int)(grow & 127), c / 32, cols / 128)] = (uint8_t)code;
+  }
+}
+
+// Gather rows into expert order and quantise them both ways, for the two GEMMs that read
+// a permuted activation or gradient in the backward (dy: fc2 dgrad along H, fc2 wgrad
+// along the expert's rows; x: fc1 wgrad along the rows):
+//   rows form: codes [R, C] in blocks of 32 along C, scale atoms grouped per 128-row
+//     expert tile (row group sum_{e'<e} ceil(n_e'/128) + m for rows [off_e + 128 m, +128));
+//   cols form: codes [R, C] in blocks of 32 rows restarting at each expert's first row,
+//     scale atoms in mxfp8_quantize_grouped's layout.
+// Row r of the output is src[row_token[r]]. blockIdx.x walks the 32-row blocks of all
+// experts, blockIdx.y tiles of 256 columns; warp w takes 32 columns, lane l row 32 j + l
+// of the expert (rows past its end count as zeros and store nothing). The atom buffers
+// are zeroed by the caller (bytes of rows or blocks past an expert's end stay 0).
+__global__ void __launch_bounds__(256) permute_quant_both_kernel(const __nv_bfloat16* __restrict__ src, int C,
+                                                                 const int32_t* __restrict__ row_token,
+                                                                 const int32_t* __restrict__ split_sizes, int E,
+                                                                 uint8_t* __restrict__ rcodes,
+                                                                 uint8_t* __restrict__ ratoms,
+                                                                 uint8_t* __restrict__ ccodes,
+                                                                 uint8_t* __restrict__ catoms) {
+  extern __shared__ int32_t tabs[];   // [E+1] row offsets, [E+1] 32-row block offsets, [E+1] 128-row group offsets
+  int32_t* roff = tabs;
+  int32_t* boff = tabs + (E + 1);
+  int32_t* koff = tabs + 2 * (E + 1);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int cr = 0, cb = 0, ck = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int n = (e < E) ? split_sizes[e] : 0;
+      const int nb = (n + 31) / 32, nk = (n + 127) / 128;
+      int ir = n, ib = nb, ik = nk;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yr = __shfl_up_sync(0xffffffffu, ir, o);
+        const int yb = __shfl_up_sync(0xffffffffu, ib, o);
+        const int yk = __shfl_up_sync(0xffffffffu, ik, o);
+        if (lane >= o) {
+          ir += yr;
+          ib += yb;
+          ik += yk;
+        }
+      }
+      if (e < E) {
+        roff[e] = cr + ir - n;
+        boff[e] = cb + ib - nb;
+        koff[e] = ck + ik - nk;
+      }
+      cr += __shfl_sync(0xffffffffu, ir, 31);
+      cb += __shfl_sync(0xffffffffu, ib, 31);
+      ck += __shfl_sync(0xffffffffu, ik, 31);
+    }
+    if (lane == 0) {
+      roff[E] = cr;
+      boff[E] = cb;
+      koff[E] = ck;
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.y * 256 + warp * 32;   // this warp's 32 columns
+  if (c >= C) return;                           // warp-uniform; no block-wide sync follows
+  const int CG = C / 128;
+  for (int blk = blockIdx.x; blk < boff[E]; blk += gridDim.x) {
+    int lo = 0, hi = E - 1;   // expert owning 32-row block `blk`
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (boff[mid] <= blk) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int j = blk - boff[e];                 // block index inside the expert
+    const int n = roff[e + 1] - roff[e];
+    const int rl = 32 * j + lane;                // this lane's row inside the expert
+    const bool live = rl < n;
+    const long long r = (long long)roff[e] + rl;
+    float v[32];
+    const int tok = live ? row_token[r] : -1;
+    if (tok >= 0) {
+      const uint4* sp = reinterpret_cast<const uint4*>(src + (size_t)tok * C + c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 q = __ldg(sp + i);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f2 = __bfloat1622float2(h2[t]);
+          v[8 * i + 2 * t] = f2.x;
+          v[8 * i + 2 * t + 1] = f2.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    }
+    uint32_t w[8];
+    if (ccodes) {
+      // along the expert's rows: the warp's 32 lanes are rows 32 j .. 32 j + 31
+      const int KG = (n + 127) / 128;
+      const uint32_t sc = quant_cols_warp32(v, w, lane);
+      catoms[mma_scale_offset((size_t)koff[e] * CG + (size_t)KG * (c / 128), (c + lane) % 128, j, 1)] =
+          (uint8_t)sc;
+      if (live) {
+        uint4* d = reinterpret_cast<uint4*>(ccodes + r * C + c);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+    if (rcodes && live) {
+      // along this row's 32 columns (quant_row32 scales v in place: after the cols form)
+      const uint32_t code = quant_row32(v, w);
+      ratoms[mma_scale_offset((size_t)koff[e] + rl / 128, rl % 128, c / 32, CG)] = (uint8_t)code;
+      uint4* d = reinterpret_cast<uint4*>(rcodes + r * C + c);
+      d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
 }

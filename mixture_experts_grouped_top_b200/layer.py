@@ -3,6 +3,10 @@
 forward:  moe_route_permute (route + permutation) -> grouped_mlp_fwd -> moe_unpermute
 backward: moe_permute_rows(grad_out) -> grouped_mlp_bwd -> moe_unpermute(dxp) -> moe_gather_slots
           -> moe_route_bwd (dlogits)
+MXFP8 training: the weights are quantised in both orientations at once (mxfp8_quantize_weights),
+the forward also quantises the permuted x along the expert rows and the backward permutes and
+quantises grad_out both ways (moe_permute_rows_mxfp8), so grouped_mlp_bwd gets every operand
+already quantised (grouped_mlp_bwd_mxfp8_operands) and no bf16 permuted copy is written.
 
 All arithmetic runs in libmoe_grouped.so; this module only owns buffers and call order.
 """
@@ -12,7 +16,13 @@ import torch
 
 from . import (BF16, FP8, MXFP8, _PREC, fp8_quantize, grouped_mlp_bwd, grouped_mlp_bwd_workspace_size, grouped_mlp_fwd,
                grouped_mlp_fwd_combine, grouped_mlp_fwd_combine_workspace_size, grouped_mlp_saved_size, grouped_mlp_workspace_size, moe_gather_slots, moe_permute_rows,
-               moe_permute_workspace_size, moe_route_bwd, moe_route_permute, moe_unpermute, mxfp8_quantize)
+               moe_permute_rows_mxfp8, moe_permute_workspace_size, moe_route_bwd, moe_route_permute, moe_unpermute,
+               mxfp8_quantize, mxfp8_quantize_weights)
+
+
+def lib_ws_bytes(T: int, k: int) -> int:
+    from . import lib
+    return max(int(lib().moe_permute_rows_mxfp8_workspace_size(T, k)), 1)
 
 
 class MoEExpertLayer:
@@ -57,7 +67,10 @@ class MoEExpertLayer:
                       if training else None)
         self.w1 = self.w2 = None
         self.w1_scale = self.w2_scale = None
-        self.xp_bf16 = None
+        self.w_rows = None
+        self.xp_cols = None
+        self._perm_q_ws = (torch.empty(int(lib_ws_bytes(T, k)), dtype=u8, device=dev)
+                           if training and self.prec == MXFP8 else None)
         self._bwd = None
 
     # --------------------------------------------------------------- weights
@@ -71,6 +84,12 @@ class MoEExpertLayer:
             # one E4M3 scale per expert, codes K-major for the forward GEMMs
             self.w1, self.w1_scale = fp8_quantize(w1, "e4m3", transpose_out=True, stream=stream)
             self.w2, self.w2_scale = fp8_quantize(w2, "e4m3", transpose_out=True, stream=stream)
+        elif self.training:
+            # both MXFP8 forms in one pass: K-major along H / F for the forward, along the
+            # other axis for the backward's data-gradient GEMMs
+            self.w1, self.w1_scale, w1r, w1ra = mxfp8_quantize_weights(w1, stream=stream)
+            self.w2, self.w2_scale, w2r, w2ra = mxfp8_quantize_weights(w2, stream=stream)
+            self.w_rows = {"w1_rows": w1r, "w1_rows_atoms": w1ra, "w2_rows": w2r, "w2_rows_atoms": w2ra}
         else:
             self.w1, self.w1_scale = mxfp8_quantize(w1, axis=1, transpose_out=True, mma_scales=True, stream=stream)
             self.w2, self.w2_scale = mxfp8_quantize(w2, axis=1, transpose_out=True, mma_scales=True, stream=stream)
@@ -101,18 +120,40 @@ class MoEExpertLayer:
             self.permute_for_backward(x, stream=stream)
         return self.out
 
+    def bwd_operands(self):
+        """MXFP8 backward operands this layer already holds quantised (None otherwise)."""
+        if self.prec != MXFP8 or self.w_rows is None:
+            return None
+        ops = dict(self.w_rows)
+        if self.xp_cols is not None:
+            ops.update(xp_cols=self.xp_cols["cols"], xp_cols_atoms=self.xp_cols["cols_atoms"])
+        if self._bwd is not None and self._bwd.get("dyq") is not None:
+            q = self._bwd["dyq"]
+            ops.update(dy_rows=q["rows"], dy_rows_atoms=q["rows_atoms"], dy_cols=q["cols"],
+                       dy_cols_atoms=q["cols_atoms"])
+        return ops
+
     def permute_for_backward(self, x: torch.Tensor, stream=None):
-        """The MXFP8 weight gradient re-quantises xp along its rows: keep a bf16 copy."""
-        if self.xp_bf16 is None:
-            self.xp_bf16 = torch.empty((self.R, self.H), dtype=torch.bfloat16, device=self.device)
-        moe_permute_rows(x, self.perm["row_map"], self.k, out=self.xp_bf16, stream=stream)
+        """The MXFP8 fc1 weight gradient reads xp quantised along each expert's rows:
+        permute and quantise x that way (no bf16 copy of the permuted rows)."""
+        if self.xp_cols is None:
+            self.xp_cols = {}
+            self._perm_q_ws = None
+        self.xp_cols = moe_permute_rows_mxfp8(x, self.perm["row_map"], self.k, self.perm["split_sizes"], rows=False,
+                                              cols=True, out=self.xp_cols, workspace=self._perm_q_ws, stream=stream)
+
+    def permute_grad(self, grad_out: torch.Tensor, stream=None):
+        """The MXFP8 backward's dy in both forms (along H and along each expert's rows)."""
+        b = self._bwd
+        b["dyq"] = moe_permute_rows_mxfp8(grad_out, self.perm["row_map"], self.k, self.perm["split_sizes"],
+                                          out=b.get("dyq"), workspace=self._perm_q_ws, stream=stream)
 
     # -------------------------------------------------------------- backward
     def _alloc_bwd(self):
         T, H, F, E, R = self.T, self.H, self.F, self.E, self.R
         dev, bf = self.device, torch.bfloat16
         self._bwd = {
-            "dy_perm": torch.empty((R, H), dtype=bf, device=dev),
+            "dy_perm": torch.empty((R, H), dtype=bf, device=dev) if self.prec != MXFP8 else None,
             "dxp": torch.empty((R, H), dtype=bf, device=dev),
             "dw1": torch.empty((E, H, 2 * F), dtype=bf, device=dev),
             "dw2": torch.empty((E, F, H), dtype=bf, device=dev),
@@ -132,11 +173,18 @@ class MoEExpertLayer:
         if self._bwd is None:
             self._alloc_bwd()
         b = self._bwd
-        moe_permute_rows(grad_out, self.perm["row_map"], self.k, out=b["dy_perm"], stream=stream)
-        xp = self.xp_bf16 if self.prec == MXFP8 else self.perm["xp"]
-        grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], xp, self.w1_master, self.w2_master,
-                        self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"], dw1=b["dw1"],
-                        dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream)
+        if self.prec == MXFP8:
+            self.permute_grad(grad_out, stream=stream)
+            grouped_mlp_bwd(None, self.perm["split_sizes"], None, self.w1_master, self.w2_master,
+                            self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"], dw1=b["dw1"],
+                            dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"], stream=stream,
+                            operands=self.bwd_operands(), shape=(self.R, self.H, self.F))
+        else:
+            moe_permute_rows(grad_out, self.perm["row_map"], self.k, out=b["dy_perm"], stream=stream)
+            grouped_mlp_bwd(b["dy_perm"], self.perm["split_sizes"], self.perm["xp"], self.w1_master,
+                            self.w2_master, self.perm["probs_perm"], self.saved, self.precision, dxp=b["dxp"],
+                            dw1=b["dw1"], dw2=b["dw2"], dprobs_perm=b["dprobs_perm"], workspace=b["ws"],
+                            stream=stream)
         moe_unpermute(b["dxp"], self.perm["row_map"], self.T, self.k, out=b["dx"], stream=stream)
         moe_gather_slots(b["dprobs_perm"], self.perm["row_map"], out=b["dprob"].view(-1), stream=stream)
         if router:

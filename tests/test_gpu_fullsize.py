@@ -14,6 +14,7 @@ import mixture_experts_grouped_top_b200 as mb
 from oracle import moe as om
 import workloads
 from oracle import mxfp8 as oq
+from tests.gather import permuted
 from tests.mx_checks import assert_boundary_flips, dswiglu_fp32_error_bounds, swiglu_fp32_error_bound
 from tests.mx_layout import grouped_atoms_to_scales, tile_atoms_to_plain
 
@@ -173,13 +174,15 @@ def test_genomic_mxfp8_full_size_fwd_bwd():
     rng = np.random.default_rng(9)
     cols = (np.sort(rng.choice(F, 16, replace=False)), np.sort(rng.choice(H, 16, replace=False)),
             np.sort(rng.choice(H, 16, replace=False)), np.sort(rng.choice(2 * F, 16, replace=False)))
-    ref = om.bwd_sampled_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
+    row_map = layer.perm["row_map"]
+    dy_cpu = permuted(d["grad_out"], row_map, cfg.k)   # the bf16 rows the fused quantiser read
+    ref = om.bwd_sampled_mxfp8(dy_cpu, permuted(d["x"], row_map, cfg.k), split, d["w1"], d["w2"],
                                layer.perm["probs_perm"].cpu(), h, RowsDeq(), ColsDeq(ac, ac_s), rows,
                                [small, large], cols, dh_wgrad=ColsDeq(dhc, dhc_s))
     # dh along 2F at the sampled rows: only rounding-boundary flips against the exact dh;
     # the fp32 error bound takes |da| magnitudes from the oracle's fc2-dgrad operands
     sabs = np.zeros((rows.size, F))
-    dyq = np.abs(oq.dequantize(*oq.quantize(om.f64(b["dy_perm"][torch.as_tensor(rows, device=DEV)].cpu()), axis=0),
+    dyq = np.abs(oq.dequantize(*oq.quantize(om.f64(dy_cpu[torch.as_tensor(rows)]), axis=0),
                                axis=0))
     for e in (small, large):
         sel = (rows >= offs[e]) & (rows < offs[e + 1])

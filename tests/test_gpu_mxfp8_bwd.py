@@ -18,6 +18,7 @@ from oracle import mxfp8 as oq
 import workloads
 from tests.mx_checks import (assert_boundary_flips, boundary_flips_grouped_rows, dswiglu_fp32_error_bounds,
                              swiglu_fp32_error_bound)
+from tests.gather import permuted
 from tests.mx_layout import grouped_atoms_to_scales, grouped_scales_to_atoms, tile_atoms_to_plain
 
 pytestmark = pytest.mark.gpu
@@ -118,7 +119,9 @@ def check_fused_backward(layer, d, E, R, H, F):
     split = layer.perm["split_sizes"].cpu().numpy()
     b = layer._bwd
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
-    dy, xp, pp = b["dy_perm"].cpu(), layer.xp_bf16.cpu(), layer.perm["probs_perm"].cpu()
+    row_map = layer.perm["row_map"]
+    dy, xp = permuted(d["grad_out"], row_map, layer.k), permuted(d["x"], row_map, layer.k)
+    pp = layer.perm["probs_perm"].cpu()
     (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(layer, E, R, H, F, split)
     exact = om.grouped_mlp_bwd_mxfp8(dy, xp, split, d["w1"], d["w2"], pp, h)
     dh_exact = exact[4]
@@ -210,3 +213,70 @@ def test_mxfp8_layer_bitwise_deterministic():
     for name, a, b in zip(names, *runs):
         assert torch.equal(a.view(torch.uint8) if a.dtype != torch.uint8 else a,
                            b.view(torch.uint8) if b.dtype != torch.uint8 else b), f"{name} differs between runs"
+
+
+@pytest.mark.parametrize("batch,rows,cols", [(3, 256, 384), (2, 384, 256), (1, 128, 128)])
+def test_quantize_weights_both_forms_bit_exact(batch, rows, cols):
+    """mxfp8_quantize_weights' two forms are the bytes of the two one-orientation
+    quantisers (whose codes and scales the oracle pins bit for bit)."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(rows + cols)
+    w = (torch.randn(batch, rows, cols, device=DEV, generator=g) *
+         torch.exp(torch.randn(batch, 1, cols, device=DEV, generator=g) * 3)).to(torch.bfloat16)
+    ct, at, cr, ar = mb.mxfp8_quantize_weights(w)
+    ct_ref, at_ref = mb.mxfp8_quantize(w, axis=1, transpose_out=True, mma_scales=True)
+    cr_ref, ar_ref = mb.mxfp8_quantize(w.reshape(batch * rows, cols), axis=0, mma_scales=True)
+    assert mb.moe_device_status() == 0
+    assert torch.equal(ct, ct_ref) and torch.equal(at, at_ref)
+    assert torch.equal(cr.reshape(batch * rows, cols), cr_ref) and torch.equal(ar, ar_ref)
+    # and the oracle's quantisation along each axis, on one matrix
+    rc, rs = oq.quantize(om.f64(w[0].cpu()), axis=1)
+    assert np.array_equal(ct[0].cpu().numpy(), rc.T)
+
+
+def test_mxfp8_backward_with_prequantised_operands_is_identical():
+    """The layer's backward (grouped_mlp_bwd_mxfp8_operands on the weights quantised both
+    ways at once, xp and dy permuted and quantised in one pass) gives the same bits as
+    grouped_mlp_bwd quantising the bf16 masters and bf16 permuted tensors itself."""
+    T, H, F, E, k = 600, 256, 384, 5, 2
+    d = workloads.small_layer(T, H, F, E, k, seed=41, with_grad=True)
+    layer = mb.MoEExpertLayer(T, H, F, E, k, precision="mxfp8", training=True)
+    layer.set_weights(d["w1"].to(DEV), d["w2"].to(DEV))
+    layer.forward(d["x"].to(DEV), d["logits"].to(DEV))
+    dx, dw1, dw2, dprob = (t.clone() for t in layer.backward(d["grad_out"].to(DEV)))
+    b = layer._bwd
+    row_map = layer.perm["row_map"]
+    dy_perm = mb.moe_permute_rows(d["grad_out"].to(DEV), row_map, k)
+    xp = mb.moe_permute_rows(d["x"].to(DEV), row_map, k)
+    ref = mb.grouped_mlp_bwd(dy_perm, layer.perm["split_sizes"], xp, layer.w1_master, layer.w2_master,
+                             layer.perm["probs_perm"], layer.saved, "mxfp8")
+    assert mb.moe_device_status() == 0
+    for got, want in zip((b["dxp"], dw1, dw2, b["dprobs_perm"]), ref):
+        assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("T,H,E,k,empty", [(300, 256, 5, 2, (3,)), (257, 384, 4, 1, (0, 2)), (96, 128, 8, 4, ())])
+def test_permute_rows_mxfp8_both_forms_bit_exact(T, H, E, k, empty):
+    """moe_permute_rows_mxfp8: the permuted rows quantised along H (tile atoms) and along
+    each expert's rows (grouped atoms), bit for bit against the oracle's quantisers of the
+    gathered bf16 rows; empty experts and ragged expert ends included."""
+    bias = np.zeros(E)
+    bias[list(empty)] = -1e4
+    d = workloads.small_layer(T, H, 256, E, k, seed=T + H, with_grad=True, logits_bias=bias)
+    ridx, _ = om.route(d["logits"], k)
+    row_map, split, _ = om.permute_index(ridx, E)
+    rm = torch.from_numpy(row_map.astype(np.int32)).to(DEV)
+    sp = torch.from_numpy(split.astype(np.int32)).to(DEV)
+    out = mb.moe_permute_rows_mxfp8(d["grad_out"].to(DEV), rm, k, sp)
+    assert mb.moe_device_status() == 0
+    dyp = om.f64(permuted(d["grad_out"], row_map, k))
+    # rows form: blocks of 32 along H; atoms per 128-row expert tile
+    rc, rs = oq.quantize(dyp, axis=0)
+    assert np.array_equal(out["rows"].cpu().numpy(), rc)
+    got_s, _, _ = tile_atoms_to_plain(out["rows_atoms"].cpu().numpy(), split, H // 32)
+    assert np.array_equal(got_s, rs)
+    # cols form: blocks of 32 rows restarting at every expert
+    cc, cs = oq.quantize_grouped_rows(dyp, split)
+    assert np.array_equal(out["cols"].cpu().numpy(), cc)
+    ref_atoms = grouped_scales_to_atoms(cs, split, H)
+    assert np.array_equal(out["cols_atoms"].cpu().numpy()[: ref_atoms.size], ref_atoms)

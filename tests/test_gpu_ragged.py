@@ -109,7 +109,10 @@ def test_mxfp8_backward_ragged_expert_sizes():
     b = layer._bwd
     h = layer.saved[: R * 2 * F * 2].view(torch.bfloat16).view(R, 2 * F).cpu()
     (dhr, dhr_s), (dhc, dhc_s), (ac, ac_s) = fused_operands(layer, E, R, H, F, split)
-    ref = om.grouped_mlp_bwd_mxfp8(b["dy_perm"].cpu(), layer.xp_bf16.cpu(), split, d["w1"], d["w2"],
+    from tests.gather import permuted
+    row_map = layer.perm["row_map"]
+    ref = om.grouped_mlp_bwd_mxfp8(permuted(d["grad_out"], row_map, layer.k), permuted(d["x"], row_map, layer.k),
+                                   split, d["w1"], d["w2"],
                                    layer.perm["probs_perm"].cpu(), h,
                                    dh=oq.dequantize_blocks_last_axis(dhr, dhr_s),
                                    a=oq.dequantize_grouped_rows(ac, ac_s, split),
