@@ -806,11 +806,19 @@ int mxfp8_quantize_weights(const uint16_t* w, int batch, int rows, int cols, uin
   if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(codes_t) | reinterpret_cast<uintptr_t>(codes_r)) &
       15)
     return MOE_ERR_INVALID_ARG;
-  if (batch > 65535 || rows / 32 > 65535) return MOE_ERR_UNSUPPORTED;
+  if (batch > 65535) return MOE_ERR_UNSUPPORTED;
   cudaStream_t st = as_stream(stream);
-  dim3 grid((cols + 255) / 256, rows / 32, batch);
-  quant_weights_both_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, codes_t,
-                                                  atoms_t, codes_r, atoms_r);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, []() {
+    attr_err = cudaFuncSetAttribute(quant_weights_both_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    qw::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
+  if (rows / 128 > 65535) return MOE_ERR_UNSUPPORTED;
+  dim3 grid(cols / 128, rows / 128, batch);
+  quant_weights_both_kernel<<<grid, 256, qw::kSmemBytes, st>>>(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols,
+                                                               codes_t, atoms_t, codes_r, atoms_r);
   count_launch();
   return launch_status();
 }

@@ -1004,60 +1004,73 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(const __nv_bfloat16* __
 //      the [batch * rows, cols] matrix (the K-major operand of a GEMM whose K is `cols`:
 //      the data-gradient GEMMs of the backward).
 // The same rule as every quantiser here: E8M0 code max(biased_exp(amax) - 8, 0), elements
-// times 2^(127 - code), round to nearest even, saturating. A block of 256 threads loads a
-// 32 x 256 tile with 16-byte loads into shared memory (row pitch 528 bytes: the column
-// reads of T and the 32-column row reads of R are both free of bank conflicts); thread j
-// then quantises column c0 + j (T) and row j % 32 of the 32-column block j / 32 (R).
-// rows and cols are multiples of 128 (a matrix's last 256-column tile may be half empty).
+// times 2^(127 - code), round to nearest even, saturating. A block of 256 threads takes a
+// 128 x 128 tile: 16-byte loads into shared memory, each thread quantises two 32-value
+// blocks of each form into shared staging tiles, and both 128 x 128 code tiles leave as
+// whole 128-byte lines (a 32-byte piece per output row scattered the stores). Row pitches
+// of 272 / 144 bytes keep the column reads, the 32-value row reads and the staging stores
+// free of bank conflicts. rows and cols are multiples of 128.
+namespace qw {
+constexpr int kInPitch = 136;    // bf16 per input row: 128 + 8
+constexpr int kOutPitch = 144;   // bytes per staged code row: 128 + 16
+constexpr int kSmemBytes = 128 * kInPitch * 2 + 2 * 128 * kOutPitch;
+}  // namespace qw
+
 __global__ void __launch_bounds__(256) quant_weights_both_kernel(const __nv_bfloat16* __restrict__ in, int rows,
                                                                  int cols, uint8_t* __restrict__ codes_t,
                                                                  uint8_t* __restrict__ atoms_t,
                                                                  uint8_t* __restrict__ codes_r,
                                                                  uint8_t* __restrict__ atoms_r) {
-  constexpr int kPitch = 264;   // bf16 per shared row: 256 + 8
-  __shared__ __align__(16) __nv_bfloat16 tile[32 * kPitch];
+  using namespace qw;
+  extern __shared__ __align__(16) uint8_t qw_smem[];
+  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(qw_smem);
+  uint8_t* st_t = qw_smem + 128 * kInPitch * 2;   // [128 columns][128 rows] codes of T
+  uint8_t* st_r = st_t + 128 * kOutPitch;         // [128 rows][128 columns] codes of R
   const int b = blockIdx.z;
-  const int r0 = blockIdx.y * 32;
-  const int c0 = blockIdx.x * 256;
+  const int r0 = blockIdx.y * 128;
+  const int c0 = blockIdx.x * 128;
   const int j = threadIdx.x;
   const __nv_bfloat16* src = in + (size_t)b * rows * cols;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int idx = j + 256 * i, row = idx >> 5, cv = (idx & 31) * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c0 + cv < cols) v = *reinterpret_cast<const uint4*>(src + (size_t)(r0 + row) * cols + c0 + cv);
-    *reinterpret_cast<uint4*>(&tile[row * kPitch + cv]) = v;
+  for (int i = 0; i < 8; ++i) {
+    const int idx = j + 256 * i, row = idx >> 4, cv = (idx & 15) * 8;
+    *reinterpret_cast<uint4*>(&tile[row * kInPitch + cv]) =
+        *reinterpret_cast<const uint4*>(src + (size_t)(r0 + row) * cols + c0 + cv);
   }
   __syncthreads();
   float f[32];
-  // T: column c0 + j over the 32 rows (the last tile of a matrix may be half empty)
-  if (c0 + j < cols) {
+  uint32_t w[8];
+#pragma unroll 1
+  for (int it = 0; it < 2; ++it) {
+    // T: column c (a warp: 32 consecutive columns), rows [32 rb, +32)
+    const int item = j + 256 * it, c = item & 127, rb = item >> 7;
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      f[i] = __bfloat162float(tile[i * kPitch + j]);
+      f[i] = __bfloat162float(tile[(32 * rb + i) * kInPitch + c]);
       amax = fmaxf(amax, fabsf(f[i]));
     }
     const int code = max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 8, 0);
     const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
 #pragma unroll
     for (int i = 0; i < 32; ++i) f[i] *= inv;
-    uint32_t w[8];
     pack_e4m3x16(f, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
     pack_e4m3x16(f + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
-    const int c = c0 + j;
-    uint4* o = reinterpret_cast<uint4*>(codes_t + (size_t)b * rows * cols + (size_t)c * rows + r0);
+    uint4* o = reinterpret_cast<uint4*>(st_t + c * kOutPitch + 32 * rb);
     o[0] = make_uint4(w[0], w[1], w[2], w[3]);
     o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    atoms_t[mma_scale_offset((size_t)b * (cols / 128) + c / 128, c % 128, r0 / 32, rows / 128)] = (uint8_t)code;
+    const int cg = c0 + c;
+    atoms_t[mma_scale_offset((size_t)b * (cols / 128) + cg / 128, cg % 128, (r0 + 32 * rb) / 32, rows / 128)] =
+        (uint8_t)code;
   }
-  // R: row r0 + (j % 32), columns [c0 + 32 (j / 32), +32)
-  if (c0 + 32 * (j >> 5) < cols) {
-    const int row = j & 31, blk = j >> 5;
+#pragma unroll 1
+  for (int it = 0; it < 2; ++it) {
+    // R: row r (a warp: 32 consecutive rows), columns [32 cb, +32)
+    const int item = j + 256 * it, r = item & 127, cb = item >> 7;
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(&tile[row * kPitch + blk * 32 + 8 * i]);
+      const uint4 v = *reinterpret_cast<const uint4*>(&tile[r * kInPitch + 32 * cb + 8 * i]);
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -1071,15 +1084,23 @@ __global__ void __launch_bounds__(256) quant_weights_both_kernel(const __nv_bflo
     const float inv = __uint_as_float((uint32_t)(254 - code) << 23);
 #pragma unroll
     for (int i = 0; i < 32; ++i) f[i] *= inv;
-    uint32_t w[8];
     pack_e4m3x16(f, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
     pack_e4m3x16(f + 16, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
-    const size_t grow = (size_t)b * rows + r0 + row;
-    const int c = c0 + 32 * blk;
-    uint4* o = reinterpret_cast<uint4*>(codes_r + grow * cols + c);
+    uint4* o = reinterpret_cast<uint4*>(st_r + r * kOutPitch + 32 * cb);
     o[0] = make_uint4(w[0], w[1], w[2], w[3]);
     o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    atoms_r[mma_scale_offset(grow >> 7, (int)(grow & 127), c / 32, cols / 128)] = (uint8_t)code;
+    const size_t grow = (size_t)b * rows + r0 + r;
+    atoms_r[mma_scale_offset(grow >> 7, (int)(grow & 127), (c0 + 32 * cb) / 32, cols / 128)] = (uint8_t)code;
+  }
+  __syncthreads();
+  // both 128 x 128 code tiles out as whole lines: 8 threads per 128-byte line
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = j + 256 * i, line = idx >> 3, part = (idx & 7) * 16;
+    *reinterpret_cast<uint4*>(codes_t + (size_t)b * rows * cols + (size_t)(c0 + line) * rows + r0 + part) =
+        *reinterpret_cast<const uint4*>(st_t + line * kOutPitch + part);
+    *reinterpret_cast<uint4*>(codes_r + ((size_t)b * rows + r0 + line) * cols + c0 + part) =
+        *reinterpret_cast<const uint4*>(st_r + line * kOutPitch + part);
   }
 }
 
