@@ -735,24 +735,38 @@ __global__ void __launch_bounds__(256) scales_to_atoms_kernel(const uint8_t* __r
 // scaled by 2^(127 - code) exactly and rounded to nearest even with saturation. Lanes
 // that hold no row pass zeros. Every lane of the warp must call this together. Returns
 // the codes in `w` (byte j = column j) and, in lane j, the scale code of column j.
+// The scale factor's bits come straight from the maximum's exponent field e:
+// (254 - max(e - 8, 0)) << 23 = min((262 - e) << 23, 254 << 23), unsigned. Lane j's own
+// column maximum is picked from the 32 (warp-uniform) maxima by a select tree on the bits
+// of j, built as the columns go (31 selects, not a compare and a select per column).
 __device__ __forceinline__ uint32_t quant_cols_warp32(const float (&v)[32], uint32_t (&w)[8], int lane) {
-  uint32_t mine = 0;
+  uint32_t lv[5];   // pending select-tree nodes, one per level
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
     const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
     const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + 1])));
-    const int c0 = max((int)(m0 >> 23) - 8, 0), c1 = max((int)(m1 >> 23) - 8, 0);
-    const float i0 = __uint_as_float((uint32_t)(254 - c0) << 23), i1 = __uint_as_float((uint32_t)(254 - c1) << 23);
+    const float i0 = __uint_as_float(min(0x83000000u - (m0 & 0x7F800000u), 0x7F000000u));
+    const float i1 = __uint_as_float(min(0x83000000u - (m1 & 0x7F800000u), 0x7F000000u));
     const uint32_t pair =
         (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v[j] * i0, v[j + 1] * i1), __NV_SATFINITE, __NV_E4M3);
     if ((j & 2) == 0)
       w[j >> 2] = pair;
     else
       w[j >> 2] |= pair << 16;
-    if (lane == j) mine = (uint32_t)c0;
-    if (lane == j + 1) mine = (uint32_t)c1;
+    // the tree: node of pair i = j / 2 at level 0, merged upwards while i's low bits are 1
+    uint32_t node = (lane & 1) ? m1 : m0;
+    const int i = j >> 1;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      if (((i >> l) & 1) == 0) {
+        lv[l] = node;
+        break;
+      }
+      node = ((lane >> (l + 1)) & 1) ? node : lv[l];
+    }
+    if (i == 15) lv[4] = node;
   }
-  return mine;
+  return (uint32_t)max((int)(lv[4] >> 23) - 8, 0);
 }
 
 // E4M3 codes of 32 fp32 values of one row quantised as one block along the row; returns
