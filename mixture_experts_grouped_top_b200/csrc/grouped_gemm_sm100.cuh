@@ -91,10 +91,7 @@ struct TileInfo {
 
 template <bool KGROUP, int TBM = gg::BM>
 struct TileWalker {
-#ifndef MOE_GROUP_M
-#define MOE_GROUP_M 8
-#endif
-  static constexpr int kGroupM = MOE_GROUP_M;   // M-grouped: m-blocks per band of the tile order
+  static constexpr int kGroupM = 12;   // M-grouped: bound on the m-blocks of a band
   const int32_t* row_off;   // smem [E+1]
   const int32_t* tile_off;  // smem [E+1]
   int E, MT, NT, K;
@@ -121,14 +118,19 @@ struct TileWalker {
       const int n_e = row_off[ti.e + 1] - row_off[ti.e];
       const int mt = (n_e + TBM - 1) / TBM;
       const int local = t - tile_off[ti.e];
-      // grouped order: bands of kGroupM m-blocks; inside a band every n-block in turn,
-      // the band's m-blocks fastest. The tiles in flight at once (one per CTA or pair)
-      // then share a few A row blocks and a few B column blocks, which stay in L2, where
-      // an m-fastest walk over a large expert streams all of its A rows once per n-block.
-      const int band = local / (kGroupM * NT);
-      const int gm = min(kGroupM, mt - band * kGroupM);
-      const int r = local - band * kGroupM * NT;
-      ti.m_blk = band * kGroupM + r % gm;
+      // grouped order: the expert's m-blocks split into equal bands of at most kGroupM;
+      // inside a band every n-block in turn, the band's m-blocks fastest. The tiles in
+      // flight at once (one per pair, ~74) then cover about a band's A row blocks and as
+      // many B column blocks, which stay in L2 while they are shared, and B streams once
+      // per band. An m-fastest walk over a large expert streams all of its A rows once
+      // per n-block; fixed bands of 8 left a band of one or two m-blocks at the end of an
+      // expert (a Mixtral expert has 8-9) that streamed all of B again for them.
+      const int nbands = (mt + kGroupM - 1) / kGroupM;
+      const int gsz = (mt + nbands - 1) / nbands;
+      const int band = local / (gsz * NT);
+      const int gm = min(gsz, mt - band * gsz);
+      const int r = local - band * gsz * NT;
+      ti.m_blk = band * gsz + r % gm;
       ti.n_blk = r / gm;
       ti.row0 = row_off[ti.e] + ti.m_blk * TBM;
       ti.rows = min(TBM, n_e - ti.m_blk * TBM);
