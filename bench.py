@@ -145,7 +145,7 @@ class ClockSampler:
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["ptx_sm100.cuh", "token_kernels.cuh", "grouped_gemm_sm100.cuh", "grouped_gemm_mxf8_sm100.cuh",
                   "grouped_gemm_pair_sm100.cuh", "grouped_gemm_mxf8_pair_sm100.cuh",
-                  "grouped_gemm_kgroup_pair_sm100.cuh", "moe_api.cu"]
+                  "grouped_gemm_kgroup_pair_sm100.cuh", "grouped_gemm_mxf8_kgroup_pair_sm100.cuh", "moe_api.cu"]
 
 
 def kernel_sources_sha256() -> str:
@@ -408,8 +408,8 @@ def run_workload(cfg, args, world, rank, local, steps, warmup, with_e2e=True, fu
                          % ((d["w1"].numel() + d["w2"].numel()) * 2 / 1e9),
                    "parallelism": (f"dp{world} replicas" + (", dw1/dw2 all-reduced (NCCL) every step" if training
                                                               else "")) if world > 1 else "single GPU"},
-        "roofline": {"kernel": ("grouped_mlp_fwd + grouped_mlp_bwd (the six tcgen05 grouped GEMMs and the "
-                                "backward's quantisation passes)" if training else
+        "roofline": {"kernel": ("grouped_mlp_fwd + grouped_mlp_bwd (the six tcgen05 grouped GEMMs; MXFP8: the "
+                                "backward's operands come quantised from their producers)" if training else
                                 "grouped_mlp_fwd (fc1 gate|up + ScaledSwiGLU, fc2: two tcgen05 grouped GEMMs)"),
                      "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_note} (timed region {wall:.2f} s)",

@@ -650,16 +650,19 @@ int moe_route_permute(const float* logits, const uint16_t* x, int T, int H, int 
   if (cudaMemsetAsync(done, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
   const int P = std::max(1, 1024 / E);
   const size_t smem = (size_t)std::max(E, (P + 1) * E) * sizeof(int32_t);
-#define MOE_ROUTE_INDEX_CASE(V)                                                                             \
-  case V:                                                                                                   \
-    route_index_kernel<V><<<nblk, 1024, smem, st>>>(logits, T, E, k, renorm, idx, prob, counts, nblk, split_sizes, \
-                                                    offsets, done);                                         \
+#define MOE_ROUTE_INDEX_CASE(C, V, W)                                                                          \
+  case C:                                                                                                      \
+    route_index_kernel<V, W><<<nblk, 1024, smem, st>>>(logits, T, E, k, renorm, idx, prob, counts, nblk,         \
+                                                       split_sizes, offsets, done);                             \
     break;
-  switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : 8) {
-    MOE_ROUTE_INDEX_CASE(1)
-    MOE_ROUTE_INDEX_CASE(2)
-    MOE_ROUTE_INDEX_CASE(4)
-    MOE_ROUTE_INDEX_CASE(8)
+  // up to 8 or 16 experts: 8 or 16 lanes per token
+  switch (E <= 8 ? 0 : E <= 16 ? 1 : vpl <= 1 ? 2 : vpl <= 2 ? 3 : vpl <= 4 ? 4 : 5) {
+    MOE_ROUTE_INDEX_CASE(0, 1, 8)
+    MOE_ROUTE_INDEX_CASE(1, 1, 16)
+    MOE_ROUTE_INDEX_CASE(2, 1, 32)
+    MOE_ROUTE_INDEX_CASE(3, 2, 32)
+    MOE_ROUTE_INDEX_CASE(4, 4, 32)
+    MOE_ROUTE_INDEX_CASE(5, 8, 32)
   }
 #undef MOE_ROUTE_INDEX_CASE
   count_launch();

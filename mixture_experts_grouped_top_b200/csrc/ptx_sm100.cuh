@@ -383,6 +383,15 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
 // evaluate it per element, where the accurate expf and a correctly rounded reciprocal
 // cost a sixth of the fc2-dgrad epilogue's time.
 __device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+
+// max |v| over the 32 lanes of a full warp, as the bits of the fp32 result (sm_100a's
+// floating-point redux with the absolute-value modifier; for finite inputs the same bits
+// as an integer max over the lanes' |v| bit patterns)
+__device__ __forceinline__ uint32_t warp_max_abs_bits(float v) {
+  uint32_t r;
+  asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=r"(r) : "f"(v));
+  return r;
+}
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 // 16 fp32 values -> 16 E4M3 codes (round to nearest even, saturating), packed in 4 words.

@@ -77,6 +77,51 @@ __device__ __forceinline__ void route_one_token(const float* __restrict__ row, i
   p_out = renorm ? pk / psum : pk;
 }
 
+// The same routing with W lanes per token (E <= W <= 32, W a power of two), so that a
+// warp routes 32 / W tokens at once; lane `sub` of its group holds logit v of expert sub
+// (-inf past E). The results are those of route_one_token bit for bit: there, lanes past
+// E enter the max, sum and arg-max trees as -inf, exact zeros and (-inf, no expert) and
+// change nothing, and the trees over the first W lanes use the same xor steps.
+template <int W>
+__device__ __forceinline__ void route_one_token_narrow(float v, int E, int k, int renorm, int sub, int& e_out,
+                                                       float& p_out) {
+  float m = v;
+#pragma unroll
+  for (int o = W / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o, W));
+  float s = (sub < E) ? expf(v - m) : 0.f;
+#pragma unroll
+  for (int o = W / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, W);
+  bool taken = false;
+  float psum = 0.f, pk = 0.f;
+  int ek = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    if (sub < E && !taken && (v > bv || (v == bv && sub < be))) {
+      bv = v;
+      be = sub;
+    }
+#pragma unroll
+    for (int o = W / 2; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o, W);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o, W);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if (be == sub) taken = true;
+    const float p = expf(bv - m) / s;
+    psum += p;
+    if (sub == j) {
+      pk = p;
+      ek = be;
+    }
+  }
+  e_out = ek;
+  p_out = renorm ? pk / psum : pk;
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int renorm, int32_t* __restrict__ idx,
@@ -289,7 +334,9 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
 // chunk b — and writes that chunk's expert histogram; the last block to finish (a
 // device-wide counter, zeroed before the launch and reset by that block) then runs the
 // scan of pass 2. Replaces the route, histogram and scan launches of the unfused path.
-template <int VPL>
+// W < 32 (E <= W, VPL = 1): W lanes per token, 32 / W tokens per warp at a time (every
+// block routes its 1024/k tokens whatever T is, so its latency sets the launch's).
+template <int VPL, int W = 32>
 __global__ void __launch_bounds__(1024, 1) route_index_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                               int renorm, int32_t* __restrict__ idx,
                                                               float* __restrict__ prob, int32_t* __restrict__ counts,
@@ -304,14 +351,36 @@ __global__ void __launch_bounds__(1024, 1) route_index_kernel(const float* __res
   const int t0 = blockIdx.x * tpb, t1 = min(T, t0 + tpb);
   for (int e = threadIdx.x; e < E; e += blockDim.x) sm[e] = 0;
   __syncthreads();
-  for (int t = t0 + warp; t < t1; t += (int)(blockDim.x >> 5)) {
-    int e;
-    float p;
-    route_one_token<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, p);
-    if (lane < k) {
-      idx[(size_t)t * k + lane] = e;
-      prob[(size_t)t * k + lane] = p;
-      atomicAdd(&sm[e], 1);
+  if (W < 32) {
+    constexpr int G = 32 / W;   // tokens per warp at a time
+    const int sub = lane % W, grp = lane / W;
+    const int step = (int)(blockDim.x >> 5) * G;
+    auto load = [&](int t) { return (t < t1 && sub < E) ? __ldg(logits + (size_t)t * E + sub) : -INFINITY; };
+    float vn = load(t0 + warp * G + grp);   // the next tokens' logits are loaded a round ahead
+    for (int tb = t0 + warp * G; tb < t1; tb += step) {   // warp-uniform bound
+      const int t = tb + grp;
+      const bool ok = t < t1;
+      const float v = vn;
+      vn = load(t + step);
+      int e;
+      float p;
+      route_one_token_narrow<W>(v, E, k, renorm, sub, e, p);
+      if (ok && sub < k) {
+        idx[(size_t)t * k + sub] = e;
+        prob[(size_t)t * k + sub] = p;
+        atomicAdd(&sm[e], 1);
+      }
+    }
+  } else {
+    for (int t = t0 + warp; t < t1; t += (int)(blockDim.x >> 5)) {
+      int e;
+      float p;
+      route_one_token<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, p);
+      if (lane < k) {
+        idx[(size_t)t * k + lane] = e;
+        prob[(size_t)t * k + lane] = p;
+        atomicAdd(&sm[e], 1);
+      }
     }
   }
   __syncthreads();
@@ -730,8 +799,8 @@ __global__ void __launch_bounds__(256) scales_to_atoms_kernel(const uint8_t* __r
 
 // ------------------------------------------------------------ MXFP8 quantiser
 // E4M3 codes of 32 fp32 values (one lane's row) quantised along the 32 LANES of the warp:
-// for each column j the block maximum is the warp-wide max of |v[j]| (one redux: the bits
-// of a non-negative float order like the float), E8M0 code max(exp(amax) - 8, 0), element
+// for each column j the block maximum is the warp-wide max of |v[j]| (one floating-point
+// redux with the absolute-value modifier), E8M0 code max(exp(amax) - 8, 0), element
 // scaled by 2^(127 - code) exactly and rounded to nearest even with saturation. Lanes
 // that hold no row pass zeros. Every lane of the warp must call this together. Returns
 // the codes in `w` (byte j = column j) and, in lane j, the scale code of column j.
@@ -743,8 +812,8 @@ __device__ __forceinline__ uint32_t quant_cols_warp32(const float (&v)[32], uint
   uint32_t lv[5];   // pending select-tree nodes, one per level
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
-    const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + 1])));
+    const uint32_t m0 = warp_max_abs_bits(v[j]);
+    const uint32_t m1 = warp_max_abs_bits(v[j + 1]);
     const float i0 = __uint_as_float(min(0x83000000u - (m0 & 0x7F800000u), 0x7F000000u));
     const float i1 = __uint_as_float(min(0x83000000u - (m1 & 0x7F800000u), 0x7F000000u));
     const uint32_t pair =

@@ -89,8 +89,12 @@ def test_route_bwd_bad_index_sets_device_error():
 
 
 FUSED_CASES = [
-    (256, 128, 4, 2, "bf16"),       # fused
-    (8192, 64, 8, 2, "bf16"),       # fused, several blocks
+    (256, 128, 4, 2, "bf16"),       # fused (8 lanes per token)
+    (8192, 64, 8, 2, "bf16"),       # fused, several blocks (8 lanes per token)
+    (3001, 64, 5, 4, "mxfp8"),      # fused, 8 lanes per token, k = 4, ragged last block
+    (4096, 64, 16, 4, "bf16"),      # fused, 16 lanes per token
+    (2000, 64, 13, 2, "mxfp8"),     # fused, 16 lanes per token, E not a power of two
+    (600, 64, 32, 4, "bf16"),       # fused, a warp per token
     (16384, 64, 128, 8, "bf16"),    # fused, Qwen3's routing shape
     (3000, 96, 256, 16, "mxfp8"),   # fused, largest E of the fused launch, ragged last block
     (1, 32, 1, 1, "bf16"),          # fused, one token
@@ -110,6 +114,10 @@ def test_route_permute_matches_oracle(T, H, E, k, prec):
         assert mb.moe_device_status() == 0
         ridx, rprob = om.route(lg, k)
         assert np.array_equal(o["idx"].cpu().numpy(), ridx)
+        # the fused launch routes 32 / W tokens per warp for E <= 16: the same bits as the
+        # warp-per-token routing kernel
+        uidx, uprob = mb.moe_route(torch.from_numpy(lg).to(DEV), k, True)
+        assert torch.equal(uidx, o["idx"]) and torch.equal(uprob, o["prob"])
         assert np.max(np.abs(o["prob"].cpu().numpy() - rprob)) <= 1e-6
         row_map, split, offsets = om.permute_index(ridx, E)
         assert np.array_equal(o["row_map"].cpu().numpy(), row_map)
@@ -121,3 +129,21 @@ def test_route_permute_matches_oracle(T, H, E, k, prec):
         assert torch.equal(sep["xp"], o["xp"])
         if prec == "mxfp8":
             assert torch.equal(sep["xp_scale"], o["xp_scale"])
+
+
+@pytest.mark.parametrize("T,E,k", [(2048, 8, 2), (999, 13, 3), (64, 2, 2)])
+def test_route_permute_no_renorm_narrow(T, E, k):
+    """Fused routing with 8 / 16 lanes per token and renorm off: idx bit-exact and prob
+    within 1e-6 of the oracle, and the same bits as the warp-per-token routing kernel."""
+    rng = np.random.default_rng(T + E)
+    lg = rng.standard_normal((T, E), dtype=np.float32)
+    lg[: T // 4] = np.round(lg[: T // 4])            # exact ties between experts
+    x = torch.from_numpy(rng.standard_normal((T, 64), dtype=np.float32)).to(torch.bfloat16)
+    ws = torch.empty(mb.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
+    o = mb.moe_route_permute(torch.from_numpy(lg).to(DEV), x.to(DEV), k, False, "bf16", workspace=ws)
+    assert mb.moe_device_status() == 0
+    ridx, rprob = om.route(lg, k, renorm=False)
+    assert np.array_equal(o["idx"].cpu().numpy(), ridx)
+    assert np.max(np.abs(o["prob"].cpu().numpy() - rprob)) <= 1e-6
+    uidx, uprob = mb.moe_route(torch.from_numpy(lg).to(DEV), k, False)
+    assert torch.equal(uidx, o["idx"]) and torch.equal(uprob, o["prob"])
