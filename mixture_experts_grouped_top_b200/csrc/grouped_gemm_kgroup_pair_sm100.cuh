@@ -38,8 +38,61 @@ constexpr int kBBytes = 2 * kChunkBytes;      // this CTA's 128 columns of B
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kMaxE = 1024;
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024 + 3 * (kMaxE + 1) * 4;
+constexpr int kStgBytes = 32 * 64;            // an epilogue warp's staging tile: 32 rows x 32 bf16
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 8 * kStgBytes + 1024 + 3 * (kMaxE + 1) * 4;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 }  // namespace kp
+
+// Epilogue of one dW tile for one warp: its 32 rows (m_row0.. of dW[e]) x this half's 128
+// columns, in 32-column strips: tensor memory -> bf16 -> the warp's staging tile (64-byte
+// swizzle: 16-byte chunk j of row r at r*64 + 16*(j ^ ((r>>1)&3))) -> one TMA store per
+// strip, issued and waited on by lane 0 (a strip reuses the tile once the previous
+// store has read it). Each lane storing its own row 16 bytes at a time made 32 separate
+// L2 requests per instruction, which held back the tiles of experts with few rows. A
+// strip that is not wholly inside [M, N) of dW[e] is stored by the lanes instead.
+__device__ __forceinline__ void kp_wgrad_epilogue(const GemmParams& p, const CUtensorMap* tmO, uint8_t* stg,
+                                                  const TileInfo& ti, uint32_t t_row, int half, int m_row0, int lane) {
+  const bool zero = (ti.num_kb == 0);
+  const int n0 = ti.n_blk * kp::BN;
+  const int m = m_row0 + lane;
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+  for (int s = 0; s < 4; ++s) {
+    const int c = half * (kp::BN / 2) + 32 * s;
+    uint32_t v0[16], v1[16];
+    tmem_ld_32x32b_x16(t_row + c, v0);
+    tmem_ld_32x32b_x16(t_row + c + 16, v1);
+    tmem_wait_ld();
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+      w[8 + i] = zero ? 0u : pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+    }
+    const int col = n0 + c;
+    if (col + 32 <= p.N && m_row0 + 32 <= p.M) {   // warp-uniform
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+      uint8_t* row = stg + lane * 64;
+      const int sw = (lane >> 1) & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(row + 16 * (j ^ sw)) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmO, stg, col, m_row0, ti.e);
+        bulk_commit_group();
+      }
+    } else if (m < p.M) {
+      __nv_bfloat16* o = out + (long long)ti.e * p.out_batch + (long long)m * p.ldo + col;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (col + 8 * j < p.N)
+          *reinterpret_cast<uint4*>(o + 8 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    }
+  }
+}
 
 // Zero rows [valid, end) of the four 64-column chunks (A 2, B 2) of one stage of this
 // CTA, one warp; then make the stores visible to the tensor cores' reads.
@@ -58,16 +111,18 @@ __device__ __forceinline__ void kp_zero_rows(uint8_t* a_st, uint8_t* b_st, int v
 }
 
 // tmA: A [R rows, M] as {64, R, M/64 chunks, 1}; tmB: B [R, N] as {64, R, N/64, 1};
-// boxes {64, 128 k rows, 2 chunks, 1}. Output dW[e] [M, N] bf16 at p.out + e * p.out_batch.
+// boxes {64, 128 k rows, 2 chunks, 1}. Output dW[e] [M, N] bf16 at p.out + e * p.out_batch;
+// tmO: dW as {N, M, E}, boxes {32, 32, 1}, 64-byte swizzle.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
     grouped_wgrad_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                   const GemmParams p) {
+                                   const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
   using namespace kp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* stg = smem + kStages * kStageBytes;   // 8 epilogue warps' staging tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + 8 * kStgBytes);
   uint64_t* full = bars;                       // leader: 2-SM copies, and its own copies of a ragged stage
   uint64_t* empty = bars + kStages;            // both CTAs
   uint64_t* pfull = bars + 2 * kStages;        // second CTA: its own copies of a ragged stage
@@ -77,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
   uint64_t* drained = bars + 4 * kStages + 4;  // second CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* row_off = reinterpret_cast<int32_t*>(smem + kStages * kStageBytes + 1024);
+  int32_t* row_off = reinterpret_cast<int32_t*>(stg + 8 * kStgBytes + 1024);
   int32_t* tile_off = row_off + (kMaxE + 1);
   int32_t* order = tile_off + (kMaxE + 1);
 
@@ -106,6 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0;
@@ -292,11 +348,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kp::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      bf16_epilogue_tile<EPI_WGRAD>(p, ti, t_row, half, BMC * (int)rank + r_local, BM);
+      kp_wgrad_epilogue(p, &tmO, stg + (warp - 4) * kStgBytes, ti, t_row, half,
+                        ti.m_blk * BM + BMC * (int)rank + q * 32, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
     }
+    // the tile stores must have completed before the CTA (and its shared memory) goes
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -152,6 +152,11 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
 
 // BF16 weight-gradient GEMMs on CTA pairs: as many 2-CTA clusters as can be resident.
 int launch_wgrad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+  // dW [E, M, N] bf16 as the epilogue's TMA store target: {N, M, E}, boxes {32, 32}
+  CUtensorMap to;
+  if (int rc = make_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, p.E, (uint64_t)p.ldo * 2,
+                         (uint64_t)p.out_batch * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return rc;
   auto kern = grouped_wgrad_bf16_pair_kernel;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -171,7 +176,7 @@ int launch_wgrad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPa
     cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  kern<<<2 * pairs, kp::kThreads, kp::kSmemBytes, st>>>(ta, tb, p);
+  kern<<<2 * pairs, kp::kThreads, kp::kSmemBytes, st>>>(ta, tb, to, p);
   count_launch();
   return launch_status();
 }
