@@ -48,24 +48,80 @@ constexpr int kTmemCols = 512;
 // column half; its 64 KB come out of the operand ring, which keeps two stages there.
 constexpr int kHSlotBytes = 2 * 128 * 64;
 constexpr int kHSlots = 2;
+// STORE: a 2 KB staging tile (32 rows x 32 bf16) per epilogue warp for TMA stores
+constexpr int kStgBytes = 32 * 64;
 __host__ __device__ constexpr bool stages_h(int epi) { return epi == EPI_DSWIGLU; }
 __host__ __device__ constexpr int stages_for(int epi) { return stages_h(epi) ? 2 : kStages; }
+__host__ __device__ constexpr int side_bytes(int epi) {
+  return stages_h(epi) ? 2 * kHSlots * kHSlotBytes : (epi == EPI_STORE ? 8 * kStgBytes : 0);
+}
 __host__ __device__ constexpr int smem_bytes(int epi) {
-  return 1024 + stages_for(epi) * kStageBytes + (stages_h(epi) ? 2 * kHSlots * kHSlotBytes : 0) + 1024 +
-         2 * (kMaxE + 1) * 4;
+  return 1024 + stages_for(epi) * kStageBytes + side_bytes(epi) + 1024 + 2 * (kMaxE + 1) * 4;
 }
 constexpr int kSmemBytes = smem_bytes(EPI_STORE);
 static_assert(smem_bytes(EPI_DSWIGLU) <= 232448 && smem_bytes(EPI_STORE) <= 232448, "shared memory per CTA");
 }  // namespace g2
 
+// STORE epilogue of one warp through TMA: its 32 rows (tile rows row0.., all inside the
+// expert) x this half's 128 columns, in 32-column strips: tensor memory -> bf16 -> the
+// warp's staging tile (64-byte swizzle: 16-byte chunk j of row r at r*64 +
+// 16*(j ^ ((r>>1)&3))) -> one TMA store per strip by lane 0, which first waits until the
+// previous strip's store has read the tile. A strip past N is stored by the lanes.
+// Lane stores of 16 bytes per row made 32 separate L2 requests per instruction.
+__device__ __forceinline__ void g2_store_tma(const GemmParams& p, const CUtensorMap* tmO, uint8_t* stg,
+                                             const TileInfo& ti, uint32_t t_row, int half, long long row0,
+                                             int lane) {
+  const bool zero = (ti.num_kb == 0);
+  const int n0 = ti.n_blk * g2::BN;
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+  for (int s = 0; s < 4; ++s) {
+    const int c = half * (g2::BN / 2) + 32 * s;
+    const int col = n0 + c;
+    if (col >= p.N) break;   // warp-uniform; the rest of the half is past N too
+    uint32_t v0[16], v1[16];
+    tmem_ld_32x32b_x16(t_row + c, v0);
+    tmem_ld_32x32b_x16(t_row + c + 16, v1);
+    tmem_wait_ld();
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[i] = zero ? 0u : pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+      w[8 + i] = zero ? 0u : pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+    }
+    if (col + 32 <= p.N) {
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+      uint8_t* row = stg + lane * 64;
+      const int sw = (lane >> 1) & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(row + 16 * (j ^ sw)) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(tmO, stg, col, (int)row0, 0);
+        bulk_commit_group();
+      }
+    } else {
+      __nv_bfloat16* o = out + (row0 + lane) * p.ldo + col;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (col + 8 * j < p.N)
+          *reinterpret_cast<uint4*>(o + 8 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    }
+  }
+}
+
 // tmA: A [rows, K] as {64, rows, K/64 chunks, 1}; tmB: B_MN ? [E][K rows][N] as
 // {64, K, N/64 chunks, E} : [E][N rows][K] as {64, N, K/64 chunks, E}; boxes {64, 128, 2, 1}.
-// tmH (SwiGLU backward only): the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128},
-// 64-byte swizzle.
+// tmX: SwiGLU backward: the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128}, 64-byte
+// swizzle; STORE with p.tma_out: the output [R, N] bf16 as {N, R, 1}, box {32, 32},
+// 64-byte swizzle; otherwise unused.
 template <bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                  const __grid_constant__ CUtensorMap tmH, const GemmParams p) {
+                                  const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
   using namespace g2;
   constexpr int kSt = stages_for(EPI);
   constexpr bool kH = stages_h(EPI);
@@ -73,8 +129,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kSt * kABytes;
-  uint8_t* sH = smem + kSt * kStageBytes;     // 1024-byte aligned
-  uint8_t* bar_base = sH + (kH ? 2 * kHSlots * kHSlotBytes : 0);
+  uint8_t* sH = smem + kSt * kStageBytes;     // 1024-byte aligned: the h ring, or STORE's staging tiles
+  uint8_t* bar_base = sH + side_bytes(EPI);
   uint64_t* bars = reinterpret_cast<uint64_t*>(bar_base);
   uint64_t* full = bars;                      // used in the leader
   uint64_t* empty = bars + kSt;               // both CTAs
@@ -115,7 +171,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (kH) tma_prefetch_desc(&tmH);
+    if (kH || (EPI == EPI_STORE && p.tma_out)) tma_prefetch_desc(&tmX);
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0;
@@ -265,8 +321,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
             mbar_arrive_expect_tx(&hfull[b], kHSlotBytes);
             hring.arm(b, hph[hf]);
             uint8_t* dst = sH + b * kHSlotBytes;
-            tma_load_3d(dst, &tmH, &hfull[b], n0 + 32 * c, r0, 0);
-            tma_load_3d(dst + kHSlotBytes / 2, &tmH, &hfull[b], p.F + n0 + 32 * c, r0, 0);
+            tma_load_3d(dst, &tmX, &hfull[b], n0 + 32 * c, r0, 0);
+            tma_load_3d(dst + kHSlotBytes / 2, &tmX, &hfull[b], p.F + n0 + 32 * c, r0, 0);
             if (++hs[hf] == kHSlots) {
               hs[hf] = 0;
               hph[hf] ^= 1;
@@ -314,14 +370,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       if (!mbar_wait_bounded(&tfull[acc], (lt >> 1) & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
+      const int w_row = BMC * (int)rank + q * 32;   // this warp's first row of the tile
       if (kH)
         bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM, h_fetch);
+      else if (EPI == EPI_STORE && p.tma_out && w_row + 32 <= ti.rows)
+        g2_store_tma(p, &tmX, sH + (warp - 4) * kStgBytes, ti, t_row, half, (long long)ti.row0 + w_row, lane);
       else
         bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
     }
+    // the tile stores must have completed before the CTA (and its shared memory) goes
+    if (EPI == EPI_STORE && lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -67,6 +67,9 @@ struct GemmParams {
   // out32[row_token[r]] instead of being stored (out32 [T, ldo] fp32, zeroed beforehand)
   const int32_t* row_token;
   float* out32;
+  // STORE (bf16 out): the kernel's output tensor map is valid, so whole 32-row strips
+  // inside the expert may be stored by TMA
+  int tma_out;
 };
 
 // Adds 16 fp32 accumulator values (raw bits) to out32[0..16) with four 16-byte vector

@@ -145,7 +145,16 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
     cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  kern<<<2 * pairs, g2::kThreads, kSmem, st>>>(ta, tb, th ? *th : ta, p);
+  GemmParams q = p;
+  CUtensorMap to = ta;
+  if (EPI == EPI_STORE && p.out && p.M > 0 && p.N > 0 && !p.out_f32 && !p.row_token) {
+    // bf16 output [M rows, N] as the epilogue's TMA store target: {N, M, 1}, boxes {32, 32}
+    if (int rc = make_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 1, (uint64_t)p.ldo * 2,
+                           (uint64_t)p.ldo * 2 * p.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return rc;
+    q.tma_out = 1;
+  }
+  kern<<<2 * pairs, g2::kThreads, kSmem, st>>>(ta, tb, th ? *th : to, q);
   count_launch();
   return launch_status();
 }
