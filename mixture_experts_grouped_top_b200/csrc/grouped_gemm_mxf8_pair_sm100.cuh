@@ -71,9 +71,15 @@ __host__ __device__ constexpr bool stages_h(int epi) { return epi == MXEPI_DSWIG
 __host__ __device__ constexpr int stages_for(int epi) {
   return stages_h(epi) ? kStages - (2 * kHSlots * kHSlotBytes + kStageBytes - 1) / kStageBytes : kStages;
 }
+// SwiGLU backward: a 1 KB staging tile (32 rows x 32 codes) per epilogue warp for the TMA
+// stores of dh's code tiles
+constexpr int kCodeStgBytes = 32 * 32;
+__host__ __device__ constexpr int side_bytes(int epi) {
+  return stages_h(epi) ? 2 * kHSlots * kHSlotBytes + 8 * kCodeStgBytes : 0;
+}
 __host__ __device__ constexpr int smem_bytes(int epi) {
-  return 1024 + stages_for(epi) * kStageBytes + kSfSlots * kSfSlotBytes + (stages_h(epi) ? 2 * kHSlots * kHSlotBytes : 0) +
-         1024 + 3 * (kMaxE + 1) * 4;
+  return 1024 + stages_for(epi) * kStageBytes + kSfSlots * kSfSlotBytes + side_bytes(epi) + 1024 +
+         3 * (kMaxE + 1) * 4;
 }
 static_assert(smem_bytes(MXEPI_DSWIGLU) <= 232448 && smem_bytes(MXEPI_STORE) <= 232448, "shared memory per CTA");
 }  // namespace mx2
@@ -83,12 +89,14 @@ static_assert(smem_bytes(MXEPI_DSWIGLU) <= 232448 && smem_bytes(MXEPI_STORE) <= 
 // k-blocks, row groups} with a box of four atoms (no swizzle); A's row groups are the
 // experts' 128-row tiles in order, B's are e * (b_rows / 128) + row / 128.
 // tmH (SwiGLU backward only): the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128},
-// 64-byte swizzle.
+// 64-byte swizzle; tmDc / tmDr (SwiGLU backward only): dh_cols / dh_rows codes [R, 2F] as
+// {2F, R, 1}, box {32, 32}, 32-byte swizzle.
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     grouped_gemm_mxf8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                   const __grid_constant__ CUtensorMap tmSa, const __grid_constant__ CUtensorMap tmSb,
-                                  const __grid_constant__ CUtensorMap tmH, const MxGemmParams mp) {
+                                  const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDc,
+                                  const __grid_constant__ CUtensorMap tmDr, const MxGemmParams mp) {
   using namespace mx2;
   constexpr int kSt = stages_for(EPI);
   constexpr bool kH = stages_h(EPI);
@@ -103,7 +111,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
   uint8_t* sB = sA + kSt * kABytes;
   uint8_t* sSf = sB + kSt * kBBytes;
   uint8_t* sH = sSf + kSfSlots * kSfSlotBytes;  // 1024-byte aligned: kSfSlots * kSfSlotBytes = 12 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sH + (kH ? 2 * kHSlots * kHSlotBytes : 0));
+  uint8_t* sStg = sH + (kH ? 2 * kHSlots * kHSlotBytes : 0);   // SwiGLU backward: code staging tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sH + side_bytes(EPI));
   uint64_t* full = bars;                      // used in the leader
   uint64_t* empty = bars + kSt;               // both CTAs
   uint64_t* tfull = bars + 2 * kSt;           // both CTAs
@@ -158,7 +167,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSa);
     tma_prefetch_desc(&tmSb);
-    if (kH) tma_prefetch_desc(&tmH);
+    if (kH) {
+      tma_prefetch_desc(&tmH);
+      tma_prefetch_desc(&tmDc);
+      tma_prefetch_desc(&tmDr);
+    }
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0, carry_g = 0;
@@ -422,7 +435,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tovl_leader);
           },
-          grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e], h_fetch);
+          grp_off[ti.e], row_off[ti.e + 1] - row_off[ti.e], h_fetch,
+          kH ? CodeStager{sStg + (warp - 4) * kCodeStgBytes, &tmDc, &tmDr} : CodeStager{});
       if (EPI == MXEPI_SWIGLU_Q && BMC * (int)rank < ti.rows) {
         // this CTA's 128 rows form scale group grp_off[e] + 2 m_blk + rank of `a`: the bytes
         // of this half's two a-strips (rows past the expert store 0; a CTA entirely past
@@ -438,6 +452,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mx2::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
     }
+    // the code tiles' stores must have completed before the CTA (and its shared memory) goes
+    if (kH && lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();

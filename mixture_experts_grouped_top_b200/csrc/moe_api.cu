@@ -222,7 +222,19 @@ int launch_gemm_mx_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     cudaGetLastError();
   });
   if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-  kern<<<2 * pairs, mx2::kThreads, kSmem, st>>>(ta, tb, tsa, tsb, th ? *th : ta, p);
+  CUtensorMap tdc = ta, tdr = ta;
+  if (EPI == MXEPI_DSWIGLU) {
+    // dh's code arrays [R, 2F] as the epilogue's TMA store targets: {2F, R, 1}, boxes {32, 32}
+    const uint64_t F2 = 2 * (uint64_t)p.g.F, R = (uint64_t)p.g.M;
+    if (R == 0) return MOE_OK;
+    int rc;
+    if ((rc = make_tmap(&tdc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.dh_cols, F2, R, 1, F2, F2 * R, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_32B)) ||
+        (rc = make_tmap(&tdr, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.dh_rows, F2, R, 1, F2, F2 * R, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_32B)))
+      return rc;
+  }
+  kern<<<2 * pairs, mx2::kThreads, kSmem, st>>>(ta, tb, tsa, tsb, th ? *th : ta, tdc, tdr, p);
   count_launch();
   return launch_status();
 }
