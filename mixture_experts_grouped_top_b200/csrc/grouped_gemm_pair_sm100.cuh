@@ -53,7 +53,8 @@ constexpr int kStgBytes = 32 * 64;
 __host__ __device__ constexpr bool stages_h(int epi) { return epi == EPI_DSWIGLU; }
 __host__ __device__ constexpr int stages_for(int epi) { return stages_h(epi) ? 2 : kStages; }
 __host__ __device__ constexpr int side_bytes(int epi) {
-  return stages_h(epi) ? 2 * kHSlots * kHSlotBytes : (epi == EPI_STORE ? 8 * kStgBytes : 0);
+  // SwiGLU backward: the h ring, then a staging tile per epilogue warp for dh
+  return stages_h(epi) ? 2 * kHSlots * kHSlotBytes + 8 * kStgBytes : (epi == EPI_STORE ? 8 * kStgBytes : 0);
 }
 __host__ __device__ constexpr int smem_bytes(int epi) {
   return 1024 + stages_for(epi) * kStageBytes + side_bytes(epi) + 1024 + 2 * (kMaxE + 1) * 4;
@@ -117,11 +118,13 @@ __device__ __forceinline__ void g2_store_tma(const GemmParams& p, const CUtensor
 // {64, K, N/64 chunks, E} : [E][N rows][K] as {64, N, K/64 chunks, E}; boxes {64, 128, 2, 1}.
 // tmX: SwiGLU backward: the saved h [R, 2F] bf16 as {2F, R, 1}, box {32, 128}, 64-byte
 // swizzle; STORE with p.tma_out: the output [R, N] bf16 as {N, R, 1}, box {32, 32},
-// 64-byte swizzle; otherwise unused.
+// 64-byte swizzle; otherwise unused. tmY (SwiGLU backward only): dh [R, 2F] bf16 as
+// {2F, R, 1}, box {32, 32}, 64-byte swizzle.
 template <bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                  const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
+                                  const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                                  const GemmParams p) {
   using namespace g2;
   constexpr int kSt = stages_for(EPI);
   constexpr bool kH = stages_h(EPI);
@@ -172,6 +175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (kH || (EPI == EPI_STORE && p.tma_out)) tma_prefetch_desc(&tmX);
+    if (kH) tma_prefetch_desc(&tmY);
   }
   if (warp == 3) {
     int carry_r = 0, carry_t = 0;
@@ -372,7 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
       const int w_row = BMC * (int)rank + q * 32;   // this warp's first row of the tile
       if (kH)
-        bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM, h_fetch);
+        bf16_epilogue_tile<EPI>(p, ti, t_row, half, BMC * (int)rank + r_local, BM, h_fetch,
+                                Bf16Stager{sH + 2 * kHSlots * kHSlotBytes + (warp - 4) * kStgBytes, &tmY});
       else if (EPI == EPI_STORE && p.tma_out && w_row + 32 <= ti.rows)
         g2_store_tma(p, &tmX, sH + (warp - 4) * kStgBytes, ti, t_row, half, (long long)ti.row0 + w_row, lane);
       else
@@ -382,7 +387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
     }
     // the tile stores must have completed before the CTA (and its shared memory) goes
-    if (EPI == EPI_STORE && lane == 0) bulk_wait_group0();
+    if ((EPI == EPI_STORE || kH) && lane == 0) bulk_wait_group0();
     __syncwarp();
   }
 

@@ -186,9 +186,38 @@ struct NoHFetch {
   __device__ bool operator()(uint4 (&)[4], uint4 (&)[4]) const { return false; }
 };
 
+// EPI_DSWIGLU: where a warp's dh tiles go by TMA (null stg: lane stores). stg: the warp's
+// 2 KB staging tile; tm: dh [R, 2F] bf16 as {2F, R, 1}, boxes {32, 32}, 64-byte swizzle.
+struct Bf16Stager {
+  uint8_t* stg = nullptr;
+  const CUtensorMap* tm = nullptr;
+};
+
+// A warp's 32 rows x 32 bf16 (w: this lane's row, starting at global row y) to column x
+// by one TMA store through the warp's staging tile (64-byte swizzle: 16-byte chunk j of
+// row r at r*64 + 16*(j ^ ((r>>1)&3))); lane 0 first waits until the tile's previous
+// store has read it.
+__device__ __forceinline__ void store_bf16_tile_tma(uint8_t* stg, const CUtensorMap* tm, int x, int y,
+                                                    const uint32_t (&w)[16], int lane) {
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
+  uint8_t* row = stg + lane * 64;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(row + 16 * (j ^ sw)) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(tm, stg, x, y, 0);
+    bulk_commit_group();
+  }
+}
+
 template <int EPI, class HFetch = NoHFetch>
 __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const TileInfo& ti, uint32_t t_row, int half,
-                                                   int tile_row, int tile_bm, const HFetch& h_fetch = HFetch{}) {
+                                                   int tile_row, int tile_bm, const HFetch& h_fetch = HFetch{},
+                                                   const Bf16Stager& bs = Bf16Stager{}) {
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
 
   if (EPI == EPI_STORE || EPI == EPI_WGRAD) {
@@ -293,6 +322,10 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
     const float pr = (row_ok && p.probs) ? p.probs[row] : 1.0f;
     __nv_bfloat16* dh = reinterpret_cast<__nv_bfloat16*>(p.out2);
     const int n0 = ti.n_blk * gg::BN;
+    const int lane = threadIdx.x & 31;
+    // the warp's 32 rows all belong to the expert: its dg / du tiles go by TMA
+    const int w_row = tile_row - lane;
+    const bool tma = bs.stg != nullptr && w_row + 32 <= ti.rows;   // warp-uniform
     float dp = 0.f;
 #pragma unroll 1
     for (int c0 = half * (gg::BN / 2); c0 < (half + 1) * (gg::BN / 2); c0 += 32) {
@@ -307,16 +340,13 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
       tmem_ld_32x32b_x16(t_row + c0, vv[0]);
       tmem_ld_32x32b_x16(t_row + c0 + 16, vv[1]);
       tmem_wait_ld();
+      uint32_t ogw[16], ouw[16];   // this row's 32 dg and 32 du, bf16 pairs
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
-        const int c = c0 + 16 * jj;
         const uint32_t* v = vv[jj];
         if (jj == 0 ? cols_ok0 : cols_ok1) {
           const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gva + 2 * jj);
           const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uva + 2 * jj);
-          uint4 og[2], ou[2];
-          uint32_t* ogw = reinterpret_cast<uint32_t*>(og);
-          uint32_t* ouw = reinterpret_cast<uint32_t*>(ou);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float2 gg2 = __bfloat1622float2(g2[i]);
@@ -332,15 +362,25 @@ __device__ __forceinline__ void bf16_epilogue_tile(const GemmParams& p, const Ti
               du[j] = da * pr * sl;
               dp = fmaf(da, sl * us[j], dp);
             }
-            ogw[i] = pack_bf16x2(dg[0], dg[1]);
-            ouw[i] = pack_bf16x2(du[0], du[1]);
+            ogw[8 * jj + i] = pack_bf16x2(dg[0], dg[1]);
+            ouw[8 * jj + i] = pack_bf16x2(du[0], du[1]);
           }
+        }
+      }
+      if (tma && n0 + c0 + 32 <= p.N) {   // warp-uniform
+        store_bf16_tile_tma(bs.stg, bs.tm, n0 + c0, (int)(ti.row0 + w_row), ogw, lane);
+        store_bf16_tile_tma(bs.stg, bs.tm, p.F + n0 + c0, (int)(ti.row0 + w_row), ouw, lane);
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          if (!(jj == 0 ? cols_ok0 : cols_ok1)) continue;
+          const int c = c0 + 16 * jj;
           uint4* dg_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + n0 + c);
-          dg_dst[0] = og[0];
-          dg_dst[1] = og[1];
+          dg_dst[0] = make_uint4(ogw[8 * jj], ogw[8 * jj + 1], ogw[8 * jj + 2], ogw[8 * jj + 3]);
+          dg_dst[1] = make_uint4(ogw[8 * jj + 4], ogw[8 * jj + 5], ogw[8 * jj + 6], ogw[8 * jj + 7]);
           uint4* du_dst = reinterpret_cast<uint4*>(dh + row * p.ldo2 + p.F + n0 + c);
-          du_dst[0] = ou[0];
-          du_dst[1] = ou[1];
+          du_dst[0] = make_uint4(ouw[8 * jj], ouw[8 * jj + 1], ouw[8 * jj + 2], ouw[8 * jj + 3]);
+          du_dst[1] = make_uint4(ouw[8 * jj + 4], ouw[8 * jj + 5], ouw[8 * jj + 6], ouw[8 * jj + 7]);
         }
       }
     }

@@ -154,7 +154,15 @@ int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPar
       return rc;
     q.tma_out = 1;
   }
-  kern<<<2 * pairs, g2::kThreads, kSmem, st>>>(ta, tb, th ? *th : to, q);
+  CUtensorMap ty = ta;
+  if (EPI == EPI_DSWIGLU) {
+    // dh [R, 2F] bf16 as the epilogue's TMA store target: {2F, R, 1}, boxes {32, 32}
+    if (p.M == 0) return MOE_OK;
+    if (int rc = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out2, 2 * (uint64_t)p.F, p.M, 1,
+                           (uint64_t)p.ldo2 * 2, (uint64_t)p.ldo2 * 2 * p.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return rc;
+  }
+  kern<<<2 * pairs, g2::kThreads, kSmem, st>>>(ta, tb, th ? *th : to, ty, q);
   count_launch();
   return launch_status();
 }
