@@ -19,6 +19,9 @@
  *     Every call only enqueues work on it and returns; nothing synchronises the host.
  *   - bf16 tensors are passed as uint16_t* (raw bfloat16 bits); all tensors are dense
  *     row-major with the logical shapes given below.
+ *   - The grouped GEMMs read and write their operands and outputs with TMA and 16-byte
+ *     vector accesses: those buffers start on 16-byte boundaries (a misaligned one is
+ *     an argument error, MOE_ERR_INVALID_ARG).
  *   - Return value: a moe_status_t. Argument errors are reported synchronously before
  *     anything is launched. Errors found by kernels (bad expert index, split sizes that
  *     do not add up, a wait that ran out of time) set a device error word that
