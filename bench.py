@@ -149,11 +149,16 @@ KERNEL_SOURCES = ["ptx_sm100.cuh", "token_kernels.cuh", "grouped_gemm_sm100.cuh"
 
 
 def kernel_sources_sha256() -> str:
+    """sha256 of the kernel sources without their comment-only and blank lines (a comment
+    edit does not change what the counters measured; any code change does)."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "mixture_experts_grouped_top_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+            for line in f.read().decode().splitlines():
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(line.encode() + b"\n")
     return h.hexdigest()
 
 

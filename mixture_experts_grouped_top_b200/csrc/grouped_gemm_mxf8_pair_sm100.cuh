@@ -25,6 +25,10 @@
 // ahead of the epilogue, which reads its row from there (coalesced copies instead of one
 // 16-byte load per row and lane from global memory).
 //
+// Its dh code tiles (32 rows x 32 codes, in both quantised forms) leave through a 1 KB
+// shared-memory staging tile per epilogue warp with one TMA store each, for warps whose
+// rows all belong to the tile's expert.
+//
 // Tensor memory per CTA: overlapping accumulators acc0 = [0, 256) and acc1 = [192, 448),
 // four scale sets at 448..495; `tovl` and `tempty` live in the leader and count
 // one arrival per epilogue warp of both CTAs. Waits are bounded like in every other

@@ -25,6 +25,11 @@
 // TMA into a shared-memory ring of 32-column strips, ahead of the epilogue, which reads its
 // row from there instead of one 16-byte global load per row and lane (as in the MXFP8
 // pair kernel).
+//
+// Outputs: a warp whose 32 rows all belong to the tile's expert sends its bf16 results
+// (STORE: the output; SwiGLU backward: dg and du) through a 2 KB shared-memory staging
+// tile with one TMA store per 32x32 strip instead of 16-byte stores of 32 different rows
+// per instruction; the other warps, the fused combine and fp32 outputs store per lane.
 #pragma once
 #include "grouped_gemm_sm100.cuh"
 
